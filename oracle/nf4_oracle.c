@@ -1,0 +1,447 @@
+/*
+ * nf4_oracle.c -- plain, slow CPU oracle for the QLoRA linear layer
+ * (NF4-quantized frozen weight plus a LoRA branch).
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing in the product path may link, load or
+ * call this file: only the test suite, the package entry point's smoke check
+ * and the benchmark's CPU-baseline leg use it. It shares no code, header,
+ * table or constant with the CUDA library; the two are compared against each
+ * other on identical seeded inputs.
+ *
+ * Build: gcc -O2 -std=c11 -fno-fast-math -ffp-contract=off -fopenmp -shared -fPIC
+ * (no contraction, no fast math: every float operation below is one IEEE-754
+ * operation in the precision written).
+ *
+ * Sources (web pages; cited by title and section):
+ *   [P1] "QLoRA Finetuner -- Juan Martos", sections "1. Low-Rank Adaptation
+ *        (LoRA)" and "2. Block-by-Block NormalFloat4 (NF4) Quantization".
+ *   [P2] "QLoRA Specification for EMEP Fine-Tuning", "NF4 Quantization" and
+ *        "Hyperparameters" table.
+ *   [P3] "QLoRA explained: fine-tuning in 4-bit precision", sections
+ *        "Double quantization", "The LoRA adapter path" and "Common
+ *        misconceptions" (the NF4 lookup table).
+ *   [P4] "How Fine-Tuning LLMs with LoRA and QLoRA Works", "Merging and
+ *        Deployment Strategies".
+ *   [P5] "Parameter-Efficient Fine-Tuning: From LoRA to QLoRA", sections
+ *        "Vanilla Uniform Quantization", "Block-Wise (Chunking) Quantization",
+ *        "Pillar 1: 4-bit NormalFloat (NF4) Quantization" (level table and the
+ *        numerical step-by-step example) and "Pillar 2: Double Quantization".
+ *
+ * Readings taken where the pages are silent (each is listed in the design
+ * notes of the repository):
+ *   R1  normalisation w' = fl32(w / s), one IEEE fp32 division.
+ *   R2  nearest level by |w' - c_j| over the 16 levels; an exact tie goes to
+ *       the lower index (the more negative level).
+ *   R3  an all-zero block stores s = 0 and every code is 7 (the exact zero).
+ *   R4  double quantisation: groups of 256 consecutive blocks; c_g = max s_i
+ *       over the group; q8_i = RNE(fl32(fl32(s_i / c_g) * 127)); dequantised
+ *       scale fl32(q8_i * fl32(c_g / 127)); c_g = 0 gives q8 = 0.
+ *   R5  NF4 codes are always computed against the unquantised fp32 s_i.
+ *   R6  the matmul operand is RNE_bf16(fl32(scale * c[q])).
+ *   R7  W0 is stored [n_out, k_in] row-major; x is [M, k_in]; A is [r, k_in];
+ *       B is [n_out, r]; h = x W~^T + (alpha/r) (x A^T) B^T.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------ */
+/* NF4 levels as printed, to 16 digits, in [P3] "Common misconceptions"     */
+/* (the NF4 lookup table). Every printed value is an exact fp32 number.     */
+/* Index 0 = -1, index 7 = 0, index 15 = +1 (order as in [P5] level table). */
+/* ------------------------------------------------------------------------ */
+static const float NF4_LEVELS[16] = {
+    -1.0f,
+    -0.6961928009986877f,
+    -0.5250730514526367f,
+    -0.39491748809814453f,
+    -0.28444138169288635f,
+    -0.18477343022823334f,
+    -0.09105003625154495f,
+    0.0f,
+    0.07958029955625534f,
+    0.16093020141124725f,
+    0.24611230194568634f,
+    0.33791524171829224f,
+    0.44070982933044434f,
+    0.5626170039176941f,
+    0.7229568362236023f,
+    1.0f,
+};
+
+enum {
+    ORACLE_OK = 0,
+    ORACLE_ERR_ARG = 1,
+    ORACLE_ERR_NONFINITE = 4,
+};
+
+void oracle_nf4_levels(float out[16]) { memcpy(out, NF4_LEVELS, sizeof NF4_LEVELS); }
+
+/* Nearest of the 16 levels to a normalised value ([P1] section 2,
+ * "Normalization"; [P5] Pillar 1 "Map to Closest NF4 Bin").
+ * Distances are taken in fp64. For fp32 w' and fp32 levels the difference is
+ * exact whenever two candidate distances are close enough for rounding to
+ * matter (near a midpoint both operands have comparable exponents), so the
+ * argmin is the exact one. Strict '<' keeps the lower index on a tie (R2). */
+int oracle_nearest_level(float wn)
+{
+    int best = 0;
+    double best_d = fabs((double)wn - (double)NF4_LEVELS[0]);
+    for (int j = 1; j < 16; ++j) {
+        double d = fabs((double)wn - (double)NF4_LEVELS[j]);
+        if (d < best_d) {
+            best_d = d;
+            best = j;
+        }
+    }
+    return best;
+}
+
+/* Blockwise NF4 quantisation with optional double quantisation.
+ *   W       numel fp32 values, flattened row-major ([P5] "Block-Wise
+ *           (Chunking) Quantization": slice the flattened tensor into
+ *           contiguous chunks).
+ *   block   block size (64 in the layer; any even size here, e.g. 6 for the
+ *           [P5] numerical example).
+ *   codes   numel/2 bytes; element 2j in the HIGH nibble of byte j
+ *           ([P5] Pillar 1 "Byte Packing": [1,8] -> 24).
+ *   absmax  numel/block fp32 scales s_i = max_j |w_ij| ([P1] section 2,
+ *           "Absmax Scale").
+ *   dq      when nonzero, also writes q8 (one byte per block) and cg (one fp32
+ *           per group of dq_group blocks) per reading R4 ([P5] Pillar 2;
+ *           [P3] "Double quantization"; the int8 absmax formula of [P5]
+ *           "Vanilla Uniform Quantization").
+ * Returns ORACLE_ERR_NONFINITE if any input is NaN or infinite. */
+int oracle_nf4_quantize(const float *W, int64_t numel, int32_t block, int32_t dq,
+                        int32_t dq_group, uint8_t *codes, float *absmax,
+                        uint8_t *q8, float *cg)
+{
+    if (block <= 0 || (block % 2) != 0 || numel < 0 || (numel % block) != 0)
+        return ORACLE_ERR_ARG;
+    if (dq && dq_group <= 0)
+        return ORACLE_ERR_ARG;
+    for (int64_t i = 0; i < numel; ++i)
+        if (!isfinite(W[i]))
+            return ORACLE_ERR_NONFINITE;
+
+    const int64_t nb = numel / block;
+    memset(codes, 0, (size_t)(numel / 2));
+
+    /* First pass: absmax, normalise, nearest level, pack. Blocks are
+     * independent (an even block size never splits a byte), so they are
+     * spread over threads. */
+#pragma omp parallel for schedule(static)
+    for (int64_t b = 0; b < nb; ++b) {
+        const float *w = W + b * block;
+        float s = 0.0f;
+        for (int32_t j = 0; j < block; ++j) {
+            float a = fabsf(w[j]);
+            if (a > s)
+                s = a;
+        }
+        absmax[b] = s;
+        for (int32_t j = 0; j < block; ++j) {
+            int q;
+            if (s == 0.0f) {
+                q = 7; /* R3 */
+            } else {
+                float wn = w[j] / s; /* R1: one fp32 division */
+                q = oracle_nearest_level(wn);
+            }
+            int64_t e = b * block + j;
+            if ((e & 1) == 0)
+                codes[e / 2] |= (uint8_t)(q << 4);
+            else
+                codes[e / 2] |= (uint8_t)q;
+        }
+    }
+
+    /* Second pass: 8-bit quantisation of the scales in groups (R4, R5). */
+    if (dq) {
+        const int64_t ng = (nb + dq_group - 1) / dq_group;
+        for (int64_t g = 0; g < ng; ++g) {
+            int64_t b0 = g * dq_group;
+            int64_t b1 = b0 + dq_group < nb ? b0 + dq_group : nb;
+            float c = 0.0f;
+            for (int64_t b = b0; b < b1; ++b)
+                if (absmax[b] > c)
+                    c = absmax[b];
+            cg[g] = c;
+            for (int64_t b = b0; b < b1; ++b) {
+                if (c == 0.0f) {
+                    q8[b] = 0;
+                } else {
+                    float t = absmax[b] / c;   /* fl32(s / c) */
+                    float u = t * 127.0f;      /* fl32(. * 127) */
+                    q8[b] = (uint8_t)nearbyintf(u); /* round half to even */
+                }
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* Dequantised scale of block b: s_b itself, or fl32(q8_b * fl32(c_g / 127))
+ * with double quantisation (R4). */
+static float oracle_block_scale(int64_t b, const float *absmax, const uint8_t *q8,
+                                const float *cg, int32_t dq, int32_t dq_group)
+{
+    if (!dq)
+        return absmax[b];
+    float kg = cg[b / dq_group] / 127.0f;
+    return (float)q8[b] * kg;
+}
+
+void oracle_block_scales(int64_t nb, const float *absmax, const uint8_t *q8,
+                         const float *cg, int32_t dq, int32_t dq_group, float *out)
+{
+    for (int64_t b = 0; b < nb; ++b)
+        out[b] = oracle_block_scale(b, absmax, q8, cg, dq, dq_group);
+}
+
+/* w~ = fl32(scale * NF4[q]) ([P1] section 2, "On-the-Fly Dequantization";
+ * [P1] flowchart "Dynamic Dequantization"). */
+void oracle_nf4_dequantize(const uint8_t *codes, const float *absmax,
+                           const uint8_t *q8, const float *cg, int64_t numel,
+                           int32_t block, int32_t dq, int32_t dq_group, float *out)
+{
+    for (int64_t e = 0; e < numel; ++e) {
+        uint8_t byte = codes[e / 2];
+        int q = (e & 1) == 0 ? (byte >> 4) : (byte & 15);
+        float s = oracle_block_scale(e / block, absmax, q8, cg, dq, dq_group);
+        out[e] = s * NF4_LEVELS[q];
+    }
+}
+
+/* Round an fp32 value to bf16 (round to nearest, ties to even), returned as
+ * the 16 stored bits. Written from the definition: keep the top 16 bits of
+ * the fp32 encoding after adding half an ulp of bf16 plus the tie bias. */
+uint16_t oracle_f32_to_bf16(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7f800000u) == 0x7f800000u && (u & 0x007fffffu) != 0)
+        return (uint16_t)((u >> 16) | 0x0040u); /* quiet NaN */
+    uint32_t lsb = (u >> 16) & 1u;
+    u += 0x7fffu + lsb;
+    return (uint16_t)(u >> 16);
+}
+
+double oracle_bf16_to_f64(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+void oracle_f32_to_bf16_array(const float *in, int64_t n, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = oracle_f32_to_bf16(in[i]);
+}
+
+/* Widen a bf16 array to fp64. */
+static double *widen_bf16(const uint16_t *p, int64_t n)
+{
+    double *d = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+    if (!d)
+        return NULL;
+    for (int64_t i = 0; i < n; ++i)
+        d[i] = oracle_bf16_to_f64(p[i]);
+    return d;
+}
+
+/* Dequantised weight as the bf16 matmul operand (R6), held as fp32 (every
+ * bf16 value is exact in fp32) and widened to fp64 where it is used:
+ * Wt[n][k] = RNE_bf16(fl32(scale * NF4[q])). */
+static float *dequant_operand(const uint8_t *codes, const float *absmax,
+                               const uint8_t *q8, const float *cg, int64_t N,
+                               int64_t K, int32_t dq)
+{
+    int64_t numel = N * K;
+    float *w = (float *)malloc(sizeof(float) * (size_t)numel);
+    if (!w)
+        return NULL;
+    oracle_nf4_dequantize(codes, absmax, q8, cg, numel, 64, dq, 256, w);
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < numel; ++i)
+        w[i] = (float)oracle_bf16_to_f64(oracle_f32_to_bf16(w[i]));
+    return w;
+}
+
+/* Forward of the layer for a subset of token rows ([P1] section 1, forward
+ * step h = W0 x + (alpha/r) B(A(dropout x)) with dropout p = 0; [P3] "The
+ * LoRA adapter path": base = x W^T, lora = (x A^T) B^T * scale). Everything in
+ * fp64 from the bf16 inputs and the bf16 dequantised operand.
+ *   rows[i]     token index of output row i (0 <= rows[i] < M)
+ *   h_out       nrows x N fp64
+ *   u_out       nrows x r fp64 (u = x A^T), may be NULL
+ * Returns 0, or ORACLE_ERR_ARG on allocation failure / bad shapes. */
+int oracle_qlora_fwd_rows(const uint8_t *codes, const float *absmax, const uint8_t *q8,
+                          const float *cg, int32_t dq, int64_t N, int64_t K,
+                          const uint16_t *x, int64_t M, const uint16_t *A,
+                          const uint16_t *B, int32_t r, double alpha,
+                          const int64_t *rows, int64_t nrows, double *h_out, double *u_out)
+{
+    if (N <= 0 || K <= 0 || K % 64 != 0 || r <= 0 || M < 0)
+        return ORACLE_ERR_ARG;
+    float *Wt = dequant_operand(codes, absmax, q8, cg, N, K, dq);
+    double *Ad = widen_bf16(A, (int64_t)r * K);
+    double *Bd = widen_bf16(B, N * r);
+    if (!Wt || !Ad || !Bd) {
+        free(Wt); free(Ad); free(Bd);
+        return ORACLE_ERR_ARG;
+    }
+    const double s = alpha / (double)r;
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < nrows; ++i) {
+        int64_t m = rows[i];
+        if (m < 0 || m >= M) {
+            err = 1;
+            continue;
+        }
+        double *xr = widen_bf16(x + m * K, K);
+        double *u = (double *)malloc(sizeof(double) * (size_t)r);
+        if (!xr || !u) {
+            free(xr); free(u);
+            err = 1;
+            continue;
+        }
+        for (int32_t j = 0; j < r; ++j) {           /* u = x A^T */
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                acc += xr[k] * Ad[(int64_t)j * K + k];
+            u[j] = acc;
+            if (u_out)
+                u_out[i * r + j] = acc;
+        }
+        for (int64_t n = 0; n < N; ++n) {
+            double base = 0.0;                       /* x W~^T */
+            for (int64_t k = 0; k < K; ++k)
+                base += xr[k] * (double)Wt[n * K + k];
+            double lora = 0.0;                       /* (x A^T) B^T */
+            for (int32_t j = 0; j < r; ++j)
+                lora += u[j] * Bd[n * r + j];
+            h_out[i * N + n] = base + s * lora;
+        }
+        free(xr);
+        free(u);
+    }
+    free(Wt); free(Ad); free(Bd);
+    return err ? ORACLE_ERR_ARG : ORACLE_OK;
+}
+
+/* Backward of the layer (chain rule; the frozen weight gets no gradient:
+ * [P3] "The LoRA adapter path", the dequantised base weight is a constant in
+ * backprop; [P4] "Mathematical Foundation", W frozen, only A and B trained):
+ *   v  = dY B                      (M x r)
+ *   u  = x A^T                     (M x r)
+ *   dX = dY W~ + s v A             (rows listed in dx_rows only)
+ *   dA = s v^T x                   (r x K, full)
+ *   dB = s dY^T u                  (N x r, full)
+ * All in fp64 from bf16 inputs. dx_out is ndx x K; dA_out r x K; dB_out N x r.
+ * Any output pointer may be NULL to skip it. */
+int oracle_qlora_bwd(const uint8_t *codes, const float *absmax, const uint8_t *q8,
+                     const float *cg, int32_t dq, int64_t N, int64_t K,
+                     const uint16_t *x, int64_t M, const uint16_t *A,
+                     const uint16_t *B, int32_t r, double alpha, const uint16_t *dY,
+                     const int64_t *dx_rows, int64_t ndx, double *dx_out,
+                     double *dA_out, double *dB_out)
+{
+    if (N <= 0 || K <= 0 || K % 64 != 0 || r <= 0 || M < 0)
+        return ORACLE_ERR_ARG;
+    const double s = alpha / (double)r;
+    double *Ad = widen_bf16(A, (int64_t)r * K);
+    double *Bd = widen_bf16(B, N * r);
+    double *v = (double *)calloc((size_t)(M * r + 1), sizeof(double));
+    double *u = (double *)calloc((size_t)(M * r + 1), sizeof(double));
+    if (!Ad || !Bd || !v || !u) {
+        free(Ad); free(Bd); free(v); free(u);
+        return ORACLE_ERR_ARG;
+    }
+
+    /* v[m][j] = sum_n dY[m][n] B[n][j];  u[m][j] = sum_k x[m][k] A[j][k] */
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            double g = oracle_bf16_to_f64(dY[m * N + n]);
+            for (int32_t j = 0; j < r; ++j)
+                v[m * r + j] += g * Bd[n * r + j];
+        }
+        for (int32_t j = 0; j < r; ++j) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                acc += oracle_bf16_to_f64(x[m * K + k]) * Ad[(int64_t)j * K + k];
+            u[m * r + j] = acc;
+        }
+    }
+
+    int err = 0;
+    if (dx_out && ndx > 0) {
+        float *Wt = dequant_operand(codes, absmax, q8, cg, N, K, dq);
+        if (!Wt) {
+            err = 1;
+        } else {
+#pragma omp parallel for schedule(dynamic, 1)
+            for (int64_t i = 0; i < ndx; ++i) {
+                int64_t m = dx_rows[i];
+                if (m < 0 || m >= M) {
+                    err = 1;
+                    continue;
+                }
+                double *row = dx_out + i * K;
+                for (int64_t k = 0; k < K; ++k)
+                    row[k] = 0.0;
+                for (int64_t n = 0; n < N; ++n) {    /* dY W~ */
+                    double g = oracle_bf16_to_f64(dY[m * N + n]);
+                    for (int64_t k = 0; k < K; ++k)
+                        row[k] += g * (double)Wt[n * K + k];
+                }
+                for (int64_t k = 0; k < K; ++k) {    /* + s v A */
+                    double acc = 0.0;
+                    for (int32_t j = 0; j < r; ++j)
+                        acc += v[m * r + j] * Ad[(int64_t)j * K + k];
+                    row[k] += s * acc;
+                }
+            }
+            free(Wt);
+        }
+    }
+
+    if (dA_out) {
+        /* dA[j][k] = s sum_m v[m][j] x[m][k] */
+#pragma omp parallel for schedule(static)
+        for (int64_t k = 0; k < K; ++k) {
+            for (int32_t j = 0; j < r; ++j) {
+                double acc = 0.0;
+                for (int64_t m = 0; m < M; ++m)
+                    acc += v[m * r + j] * oracle_bf16_to_f64(x[m * K + k]);
+                dA_out[(int64_t)j * K + k] = s * acc;
+            }
+        }
+    }
+
+    if (dB_out) {
+        /* dB[n][j] = s sum_m dY[m][n] u[m][j]; each thread owns a range of n
+         * and walks m in order, so every sum runs over m = 0..M-1. */
+        for (int64_t i = 0; i < N * r; ++i)
+            dB_out[i] = 0.0;
+#pragma omp parallel for schedule(static)
+        for (int64_t n = 0; n < N; ++n) {
+            double *acc = dB_out + n * r;
+            for (int64_t m = 0; m < M; ++m) {
+                double g = oracle_bf16_to_f64(dY[m * N + n]);
+                for (int32_t j = 0; j < r; ++j)
+                    acc[j] += g * u[m * r + j];
+            }
+            for (int32_t j = 0; j < r; ++j)
+                acc[j] *= s;
+        }
+    }
+
+    free(Ad); free(Bd); free(v); free(u);
+    return err ? ORACLE_ERR_ARG : ORACLE_OK;
+}

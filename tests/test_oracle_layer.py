@@ -1,0 +1,148 @@
+"""Pins for the oracle's QLoRA forward and backward: the merged-weight
+identity, B = 0 and W0 = 0 special cases, exact central differences on
+dyadic inputs, an independent fp64 autograd opinion, and the pages'
+parameter-count arithmetic."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from conftest import read_golden_kv
+
+
+def dyadic_bf16(rng, shape, scale_pow=2):
+    """Small integers times 2^-scale_pow: exact in bf16 and in fp64 sums."""
+    vals = rng.integers(-2, 3, size=shape).astype(np.float32) * np.float32(2.0 ** -scale_pow)
+    return oracle.f32_to_bf16(vals)
+
+
+def random_layer(rng, N, K, M, r, dq, sigma=0.02):
+    W = rng.normal(0, sigma, size=(N, K)).astype(np.float32)
+    qw = oracle.quantize(W.reshape(-1), dq=dq)
+    x = oracle.f32_to_bf16(rng.normal(size=(M, K)).astype(np.float32))
+    A = oracle.f32_to_bf16(rng.uniform(-K ** -0.5, K ** -0.5, size=(r, K)).astype(np.float32))
+    B = oracle.f32_to_bf16(rng.normal(0, 0.01, size=(N, r)).astype(np.float32))
+    dY = oracle.f32_to_bf16(rng.normal(size=(M, N)).astype(np.float32))
+    return qw, x, A, B, dY
+
+
+def operand(qw, N, K):
+    """The bf16 matmul operand RNE(w~) as fp64, via the oracle's codec."""
+    return oracle.bf16_to_f64(oracle.f32_to_bf16(oracle.dequantize(qw))).reshape(N, K)
+
+
+def f64(a):
+    return oracle.bf16_to_f64(a)
+
+
+@pytest.mark.parametrize("dq", [False, True])
+def test_forward_equals_merged_weight(dq):
+    rng = np.random.default_rng(21)
+    N, K, M, r, alpha = 96, 192, 7, 8, 16.0
+    qw, x, A, B, _ = random_layer(rng, N, K, M, r, dq)
+    h, u = oracle.qlora_fwd_rows(qw, N, K, x, A, B, r, alpha)
+    s = alpha / r
+    merged = operand(qw, N, K) + s * f64(B) @ f64(A)        # W~ + (alpha/r) B A
+    ref = f64(x) @ merged.T
+    assert np.max(np.abs(h - ref)) <= 1e-12 * np.sqrt(np.mean(ref ** 2))
+    assert np.allclose(u, f64(x) @ f64(A).T, rtol=0, atol=1e-13)
+    # a subset of rows is the same as those rows of the full result
+    h2, _ = oracle.qlora_fwd_rows(qw, N, K, x, A, B, r, alpha, rows=[6, 0, 3])
+    assert np.array_equal(h2, h[[6, 0, 3]])
+
+
+def test_b_zero_gives_base_output():
+    rng = np.random.default_rng(22)
+    N, K, M, r = 64, 128, 5, 16
+    qw, x, A, B, _ = random_layer(rng, N, K, M, r, True)
+    B0 = np.zeros_like(B)
+    h, _ = oracle.qlora_fwd_rows(qw, N, K, x, A, B0, r, 32.0)
+    assert np.array_equal(h, np.asarray(f64(x) @ operand(qw, N, K).T)) or \
+        np.max(np.abs(h - f64(x) @ operand(qw, N, K).T)) < 1e-13
+
+
+def test_w0_zero_gives_lora_only():
+    rng = np.random.default_rng(23)
+    N, K, M, r, alpha = 64, 128, 5, 8, 16.0
+    qw = oracle.quantize(np.zeros(N * K, dtype=np.float32), dq=True)
+    assert np.all(qw.codes == 0x77) and np.all(qw.absmax == 0)
+    _, x, A, B, _ = random_layer(rng, N, K, M, r, True)
+    h, _ = oracle.qlora_fwd_rows(qw, N, K, x, A, B, r, alpha)
+    ref = (alpha / r) * (f64(x) @ f64(A).T) @ f64(B).T
+    assert np.max(np.abs(h - ref)) <= 1e-13 * np.max(np.abs(ref))
+    assert np.max(np.abs(ref)) > 0
+
+
+def loss(qw, N, K, x, A, B, r, alpha, dY):
+    h, _ = oracle.qlora_fwd_rows(qw, N, K, x, A, B, r, alpha)
+    return float(np.sum(f64(dY) * h))
+
+
+def test_backward_equals_exact_central_differences():
+    """L = sum(dY * h) is linear in each of x, A, B; with dyadic inputs and a
+    dyadic step the central difference is the exact partial derivative."""
+    rng = np.random.default_rng(24)
+    N, K, M, r, alpha = 16, 64, 3, 4, 8.0
+    W = rng.normal(0, 0.02, size=(N, K)).astype(np.float32)
+    qw = oracle.quantize(W.reshape(-1), dq=True)
+    x, A, B, dY = (dyadic_bf16(rng, s) for s in [(M, K), (r, K), (N, r), (M, N)])
+    dX, dA, dB = oracle.qlora_bwd(qw, N, K, x, A, B, r, alpha, dY)
+    delta = np.float32(0.25)
+
+    def fd(which, idx):
+        arrs = {"x": x, "A": A, "B": B}
+        base = f64(arrs[which]).astype(np.float32)
+        plus, minus = base.copy(), base.copy()
+        plus[idx] += delta
+        minus[idx] -= delta
+        lp = dict(arrs); lp[which] = oracle.f32_to_bf16(plus)
+        lm = dict(arrs); lm[which] = oracle.f32_to_bf16(minus)
+        assert np.array_equal(f64(lp[which]).astype(np.float32), plus)
+        Lp = loss(qw, N, K, lp["x"], lp["A"], lp["B"], r, alpha, dY)
+        Lm = loss(qw, N, K, lm["x"], lm["A"], lm["B"], r, alpha, dY)
+        return (Lp - Lm) / (2 * float(delta))
+
+    for idx in [(0, 0), (1, 17), (2, 63), (0, 31)]:
+        assert fd("x", idx) == pytest.approx(dX[idx], rel=1e-12, abs=1e-12)
+    for idx in [(0, 0), (3, 63), (1, 5), (2, 40)]:
+        assert fd("A", idx) == pytest.approx(dA[idx], rel=1e-12, abs=1e-12)
+    for idx in [(0, 0), (15, 3), (7, 1), (9, 2)]:
+        assert fd("B", idx) == pytest.approx(dB[idx], rel=1e-12, abs=1e-12)
+    # the gradients are not trivially zero
+    assert np.abs(dX).max() > 0 and np.abs(dA).max() > 0 and np.abs(dB).max() > 0
+
+
+@pytest.mark.parametrize("dq", [False, True])
+def test_backward_matches_fp64_autograd(dq):
+    rng = np.random.default_rng(25)
+    N, K, M, r, alpha = 48, 128, 9, 8, 16.0
+    qw, x, A, B, dY = random_layer(rng, N, K, M, r, dq)
+    dX, dA, dB = oracle.qlora_bwd(qw, N, K, x, A, B, r, alpha, dY)
+    Wt = torch.from_numpy(operand(qw, N, K))
+    xt = torch.from_numpy(f64(x)).requires_grad_(True)
+    At = torch.from_numpy(f64(A)).requires_grad_(True)
+    Bt = torch.from_numpy(f64(B)).requires_grad_(True)
+    h = xt @ Wt.T + (alpha / r) * (xt @ At.T) @ Bt.T
+    (torch.from_numpy(f64(dY)) * h).sum().backward()
+    for got, ref in [(dX, xt.grad), (dA, At.grad), (dB, Bt.grad)]:
+        ref = ref.numpy()
+        assert np.max(np.abs(got - ref)) <= 1e-12 * max(1e-30, np.sqrt(np.mean(ref ** 2)))
+    # dX rows subset
+    dX2, _, _ = oracle.qlora_bwd(qw, N, K, x, A, B, r, alpha, dY, dx_rows=[8, 2],
+                                 want_dA=False, want_dB=False)
+    assert np.array_equal(dX2, dX[[8, 2]])
+
+
+def test_adapter_gradient_sizes_match_parameter_count():
+    g = read_golden_kv("lora_param_count.txt")
+    d, k, r = int(g["d"]), int(g["k"]), int(g["r"])
+    rng = np.random.default_rng(26)
+    qw = oracle.quantize(np.zeros(k * d, dtype=np.float32), dq=True)
+    x = oracle.f32_to_bf16(rng.normal(size=(1, d)).astype(np.float32))
+    A = np.zeros((r, d), dtype=np.uint16)
+    B = np.zeros((k, r), dtype=np.uint16)
+    dY = np.zeros((1, k), dtype=np.uint16)
+    _, dA, dB = oracle.qlora_bwd(qw, k, d, x, A, B, r, 32.0, dY, dx_rows=[])
+    assert dA.size + dB.size == int(g["per_matrix"])
+    assert 4 * (dA.size + dB.size) == int(g["per_layer"])
+    assert round(int(g["layers"]) * 4 * (dA.size + dB.size) / 1e6, 1) == float(g["total_millions"])
