@@ -1,0 +1,436 @@
+#!/usr/bin/env python
+"""Benchmark of the QLoRA linear layer (NF4 frozen weight + LoRA adapters) on B200.
+
+One step = the layer's forward and backward on one batch of synthetic tokens,
+i.e. h = x W~^T + (alpha/r)(x A^T)B^T, then dX, dA, dB (with the adapter
+gradients all-reduced across ranks when N > 1). Workload: the LLaMA-13B-like
+attention projection (W0 5120x5120 NF4 with double quantisation, 2048 tokens,
+r = 16, alpha = 32). value = algorithmic fwd+bwd FLOP/s over all ranks.
+
+Alongside it the same run reports, on rank 0: the decode-shaped forward
+(W0 13824x5120, M in {1,4,16}) as GB/s of 4-bit weight codes, the full-weight
+quantisation of the Llama-2-70B-like MLP weight (28672x8192) as GB/s moved,
+the CPU oracle's speed on a bounded sample, and the end-to-end speed through
+the public API with host buffers.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+       (N > 1: launch under torch.distributed.run, one rank per GPU)
+"""
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "QLoRA linear fwd+bwd TFLOP/s (large M) & NF4 weight GB/s (decode) vs roofline"
+MAIN = "llama13b_attn_5120"
+DECODE = "decode_mlp_up_13824x5120"
+QUANT = "llama2_70b_mlp_28672x8192"
+L2_FLUSH_BYTES = 512 << 20
+
+
+def layer_flops(M, N, K, r):
+    """Algorithmic FLOPs of one forward and one backward of the layer."""
+    fwd = 2 * M * N * K + 2 * M * r * (K + N)
+    bwd = 2 * M * N * K + 4 * M * N * r + 4 * M * K * r
+    return fwd, bwd
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# --------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only)
+# --------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index, period_s=0.01):
+        self.samples, self.reasons = [], 0
+        self.period = period_s
+        self.ok = False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            handle = None
+            try:
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+                if not uuid.startswith("GPU-"):
+                    uuid = "GPU-" + uuid
+                handle = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            except Exception:
+                handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.h = handle
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML missing: report that instead of clocks
+            self.err = str(e)
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                try:
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except Exception:
+                    r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.reasons |= int(r)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"error": getattr(self, "err", "nvml unavailable")}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "samples": len(self.samples), "reasons": names}
+
+
+# --------------------------------------------------------------------------
+# CPU oracle on a bounded sample (the reported baseline and the reference arm)
+# --------------------------------------------------------------------------
+def oracle_sample_step(w, inp, tokens):
+    """Oracle forward+backward on the first `tokens` tokens of the workload.
+    Returns (flops, seconds)."""
+    import oracle
+    bits = workloads.bf16_bits
+    qw = oracle.quantize(inp["W0"].numpy().reshape(-1), dq=w.double_quant)
+    x, A, B = bits(inp["x"][:tokens]), bits(inp["A"]), bits(inp["B"])
+    dY = bits(inp["dY"][:tokens])
+    t0 = time.perf_counter()
+    oracle.qlora_fwd_rows(qw, w.N, w.K, x, A, B, w.r, w.alpha)
+    oracle.qlora_bwd(qw, w.N, w.K, x, A, B, w.r, w.alpha, dY)
+    dt = time.perf_counter() - t0
+    f, b = layer_flops(tokens, w.N, w.K, w.r)
+    return f + b, dt
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count()
+
+
+def run_reference(args, rank, world):
+    """The oracle as it stands, timed on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    w = workloads.WORKLOADS[MAIN]
+    tokens = 4
+    inp = workloads.make_inputs(w, M=tokens)
+    for _ in range(args.warmup):
+        oracle_sample_step(w, inp, tokens)
+    tot_f, tot_t = 0, 0.0
+    for _ in range(args.steps):
+        f, t = oracle_sample_step(w, inp, tokens)
+        tot_f += f
+        tot_t += t
+    value = tot_f / tot_t / 1e12
+    sample = (f"{tokens} of the {w.M} tokens per step: full forward and backward of those "
+              f"tokens (h, dX rows, and their dA/dB contributions), W0 dequantised each step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{MAIN}: W0 5120x5120 NF4 double-quant, x {w.M}x5120 bf16, "
+                               f"r=16, alpha=32, forward+backward", "parallelism": "cpu-oracle"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--skip-extras", action="store_true",
+                    help="only the main fwd+bwd line (no decode/quantize/oracle/e2e legs)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import bit_nf4_quantized_05_b200 as q
+    from bit_nf4_quantized_05_b200 import dp
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    peaks = load_peaks()
+
+    w = workloads.WORKLOADS[MAIN]
+    M, N, K, r, alpha = w.M, w.N, w.K, w.r, w.alpha
+    inp = workloads.make_inputs(w)
+    qw = q.nf4_quantize(inp["W0"].to(dev), double_quant=w.double_quant)
+    x, A, B, dY = (inp[k].to(dev) for k in ("x", "A", "B", "dY"))
+    h = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    u = torch.empty(M, r, dtype=torch.float32, device=dev)
+    dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    flat, dA, dB = dp.grad_buffer(r, K, N, device=dev)
+    ws_f = torch.empty(q.fwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(q.bwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(xx=x, dYY=dY):
+        q.qlora_linear_fwd(qw, xx, A, B, alpha, h=h, u=u, workspace=ws_f)
+        q.qlora_linear_bwd(qw, xx, A, B, alpha, dYY, u=u, workspace=ws_b, outs=(dX, dA, dB))
+        dp.allreduce_adapter_grads(flat, world)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = q.device_status(dev)
+    if st != q.NF4_OK:
+        raise RuntimeError(f"device status after warm-up: {q.status_string(st)}")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    q.profiling(True)
+    with ClockSampler(local_rank) as clk:
+        for i in range(args.steps):
+            flush.zero_()                      # L2 flush between timed steps (untimed)
+            starts[i].record()
+            step()
+            ends[i].record()
+        torch.cuda.synchronize()
+    barrier()
+    q.profiling(False)
+    prof = q.profile_read()
+    per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms = statistics.mean(per_step)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    f_fwd, f_bwd = layer_flops(M, N, K, r)
+    value = world * (f_fwd + f_bwd) / (ms * 1e-3) / 1e12
+
+    # roofline of the dominant kernel: the fused dequant-GEMM (forward + dgrad launches)
+    g_launch = sum(prof.get(k, (0, 0.0))[0] for k in ("qlora_gemm_fwd", "qlora_gemm_dgrad"))
+    g_ms = sum(prof.get(k, (0, 0.0))[1] for k in ("qlora_gemm_fwd", "qlora_gemm_dgrad"))
+    g_flops = args.steps * ((2 * M * N * K + 2 * M * N * r) + (2 * M * N * K + 2 * M * K * r))
+    g_tflops = g_flops / (g_ms * 1e-3) / 1e12 if g_ms > 0 else None
+    roofline = {"bound": "tensor", "achieved": g_tflops, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": (g_tflops / peaks["bf16_tflops"]) if g_tflops else None,
+                "traffic": None, "kernel": "qlora_gemm (forward + dgrad launches)",
+                "peak_source": peaks["source"] + " bf16 burst",
+                "avg_launch_us": 1e3 * g_ms / max(g_launch, 1)}
+    kernels = {k: {"launches": n, "avg_us": 1e3 * t / max(n, 1), "share": t / max(
+        sum(v[1] for v in prof.values()), 1e-12)} for k, (n, t) in prof.items()}
+    gpu_launches = sum(n for n, _ in prof.values())
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"{MAIN}: W0 {N}x{K} NF4 (blocks of 64, double quant), "
+                               f"x {M}x{K} bf16 per rank, r={r}, alpha={alpha:g}, fwd+bwd",
+                   "global_batch_tokens": M * world, "parallelism": f"dp{world}",
+                   "l2": "512 MiB buffer written before every timed step (outside the events)"},
+        "roofline": roofline,
+        "gpu_launches": gpu_launches,
+        "clocks": clk.summary(),
+        "kernels": kernels,
+    }
+
+    if rank == 0 and not args.skip_extras:
+        line["e2e"] = e2e_leg(q, dp, qw, inp, w, args, dev, world)
+        line["decode"] = decode_leg(q, dev, peaks)
+        line["quantize"] = quantize_leg(q, dev, peaks)
+        line["cpu_baseline"] = cpu_baseline_leg(w, inp)
+    elif not args.skip_extras:
+        e2e_leg(q, dp, qw, inp, w, args, dev, world)  # same collectives on every rank
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def e2e_leg(q, dp, qw, inp, w, args, dev, world):
+    """Same metric through the public API with host buffers: every step copies
+    x and dY in from pinned host memory and h, dX, dA, dB back out."""
+    M, N, K, r, alpha = w.M, w.N, w.K, w.r, w.alpha
+    hx = inp["x"].pin_memory()
+    hdY = inp["dY"].pin_memory()
+    oh = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
+    odX = torch.empty(M, K, dtype=torch.bfloat16).pin_memory()
+    ograd = torch.empty(r * K + N * r, dtype=torch.bfloat16).pin_memory()
+    A, B = inp["A"].to(dev), inp["B"].to(dev)
+    x = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    dY = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    flat, dA, dB = dp.grad_buffer(r, K, N, device=dev)
+
+    def step():
+        x.copy_(hx, non_blocking=True)
+        dY.copy_(hdY, non_blocking=True)
+        h, u = q.qlora_linear_fwd(qw, x, A, B, alpha)
+        dX, _, _ = q.qlora_linear_bwd(qw, x, A, B, alpha, dY, u=u, outs=(torch.empty_like(x), dA, dB))
+        dp.allreduce_adapter_grads(flat, world)
+        oh.copy_(h, non_blocking=True)
+        odX.copy_(dX, non_blocking=True)
+        ograd.copy_(flat, non_blocking=True)
+
+    steps = max(5, min(args.steps, 20))
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        step()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    f, b = layer_flops(M, N, K, r)
+    return {"value": world * (f + b) / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "ms_per_step": ms, "h2d_bytes_per_step": hx.nbytes + hdY.nbytes,
+            "d2h_bytes_per_step": oh.nbytes + odX.nbytes + ograd.nbytes}
+
+
+def decode_leg(q, dev, peaks):
+    """Decode-shaped forward, GB/s counted on the 4-bit code bytes; 8 weight
+    copies are rotated so that no call finds its weight in L2."""
+    w = workloads.WORKLOADS[DECODE]
+    W0 = workloads.make_weight(w).to(dev)
+    copies = [q.nf4_quantize(W0, double_quant=True) for _ in range(8)]
+    del W0
+    code_bytes = w.N * w.K // 2
+    out = {"workload": f"{DECODE}: W0 {w.N}x{w.K} NF4 double quant (0.1% x20 outliers), "
+                       f"r={w.r}; forward only", "code_bytes": code_bytes,
+           "peak_gbs": peaks["hbm_gbs"]}
+    for M in (1, 4, 16):
+        inp = workloads.make_inputs(w, M=M, with_dy=False)
+        x, A, B = (inp[k].to(dev) for k in ("x", "A", "B"))
+        h = torch.empty(M, w.N, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(q.fwd_workspace_bytes(M, w.N, w.K, w.r), dtype=torch.uint8, device=dev)
+        for i in range(8):
+            q.qlora_linear_fwd(copies[i], x, A, B, w.alpha, save_u=False, h=h, workspace=ws)
+        torch.cuda.synchronize()
+        iters = 64
+        q.profiling(True)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for i in range(iters):
+            q.qlora_linear_fwd(copies[i % 8], x, A, B, w.alpha, save_u=False, h=h, workspace=ws)
+        e.record()
+        torch.cuda.synchronize()
+        q.profiling(False)
+        prof = q.profile_read()
+        call_us = 1e3 * s.elapsed_time(e) / iters
+        kern = {k: 1e3 * t / max(n, 1) for k, (n, t) in prof.items()}
+        main_us = kern.get("qlora_gemm_fwd") or kern.get("qlora_decode")
+        out[f"M{M}"] = {"call_us": call_us, "gbs_call": code_bytes / (call_us * 1e-6) / 1e9,
+                        "kernel_us": kern,
+                        "gbs_kernel": code_bytes / (main_us * 1e-6) / 1e9 if main_us else None,
+                        "frac_kernel": (code_bytes / (main_us * 1e-6) / 1e9 / peaks["hbm_gbs"])
+                        if main_us else None}
+    del copies
+    torch.cuda.empty_cache()
+    return out
+
+
+def quantize_leg(q, dev, peaks):
+    """Full-weight nf4_quantize of the 28672x8192 fp32 weight (double quant)."""
+    w = workloads.WORKLOADS[QUANT]
+    W0 = workloads.make_weight(w).to(dev)
+    qw = q.nf4_quantize(W0, double_quant=True)
+    torch.cuda.synchronize()
+    nb = w.N * w.K // 64
+    moved = w.N * w.K * 4 + w.N * w.K // 2 + nb * 4 + nb + ((nb + 255) // 256) * 4
+    iters = 10
+    q.profiling(True)
+    for _ in range(iters):
+        q.nf4_quantize(W0, double_quant=True, out=qw)
+    torch.cuda.synchronize()
+    q.profiling(False)
+    n, t = q.profile_read()["nf4_quantize"]
+    us = 1e3 * t / n
+    gbs = moved / (us * 1e-6) / 1e9
+    del W0, qw
+    torch.cuda.empty_cache()
+    return {"workload": f"{QUANT}: W0 {w.N}x{w.K} fp32 -> NF4 + double quant",
+            "bytes_moved": moved, "kernel_us": us, "gbs": gbs, "frac": gbs / peaks["hbm_gbs"],
+            "peak_gbs": peaks["hbm_gbs"]}
+
+
+def cpu_baseline_leg(w, inp):
+    tokens = 16
+    f, t = oracle_sample_step(w, inp, tokens)
+    return {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"{tokens} of {w.M} tokens: oracle forward+backward of those tokens "
+                      f"({t:.1f} s on the host)"}
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,246 @@
+"""Python binding of the sm_100a QLoRA linear-layer library (libqlora_nf4.so).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels; this module allocates outputs and workspace with torch, passes raw
+device pointers and the current CUDA stream through the C ABI declared in
+include/qlora_nf4.h, and turns status codes into exceptions. Importing the
+package loads the shared library and fails loudly if it has not been built.
+
+Layouts (see the C header): W0 [n, k] fp32; x [M, k] bf16; A [r, k] bf16;
+B [n, r] bf16; h [M, n] bf16; dY [M, n] bf16; dX [M, k]; dA [r, k];
+dB [n, r] (bf16).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_lib", "libqlora_nf4.so")
+
+# status codes (mirror of nf4_status)
+NF4_OK = 0
+NF4_ERR_INVALID_ARG = 1
+NF4_ERR_UNSUPPORTED_SHAPE = 2
+NF4_ERR_ALIGNMENT = 3
+NF4_ERR_NONFINITE = 4
+NF4_ERR_TIMEOUT = 5
+NF4_ERR_CUDA = 6
+NF4_ERR_WORKSPACE = 7
+
+BLOCK_SIZE = 64
+DQ_GROUP = 256
+
+
+class NF4Error(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} (status {code})")
+
+
+class NF4WeightStruct(ctypes.Structure):
+    _fields_ = [
+        ("n", ctypes.c_int64),
+        ("k", ctypes.c_int64),
+        ("block_size", ctypes.c_int32),
+        ("double_quant", ctypes.c_int32),
+        ("codes", ctypes.c_void_p),
+        ("absmax", ctypes.c_void_p),
+        ("absmax_q8", ctypes.c_void_p),
+        ("absmax_c", ctypes.c_void_p),
+    ]
+
+
+class NF4KernelTime(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char_p), ("launches", ctypes.c_int64), ("total_ms", ctypes.c_double)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m bit_nf4_quantized_05_b200.build` "
+            "(nvcc, sm_100a). There is no fallback implementation.")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32, f32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    W = ctypes.POINTER(NF4WeightStruct)
+    sig = {
+        "nf4_quantize": ([vp, W, vp], ctypes.c_int),
+        "nf4_dequantize": ([W, vp, i32, vp], ctypes.c_int),
+        "qlora_fwd_workspace_bytes": ([i64, i64, i64, i32], sz),
+        "qlora_linear_fwd": ([W, vp, i64, vp, vp, i32, f32, vp, vp, vp, sz, vp], ctypes.c_int),
+        "qlora_bwd_workspace_bytes": ([i64, i64, i64, i32], sz),
+        "qlora_linear_bwd": ([W, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, vp, vp, sz, vp],
+                             ctypes.c_int),
+        "nf4_device_status": ([vp], ctypes.c_int),
+        "nf4_status_string": ([ctypes.c_int], ctypes.c_char_p),
+        "nf4_profiling": ([i32], ctypes.c_int),
+        "nf4_profile_read": ([ctypes.POINTER(NF4KernelTime), i32], ctypes.c_int32),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = res
+    return L
+
+
+lib = _load()
+
+
+def status_string(code: int) -> str:
+    return lib.nf4_status_string(int(code)).decode()
+
+
+def _check(code: int, where: str):
+    if code != NF4_OK:
+        raise NF4Error(code, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need_cuda(*ts: torch.Tensor):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors (the library has no CPU path)")
+
+
+@dataclass
+class QuantizedWeight:
+    """A frozen NF4 weight: device tensors owned by this object."""
+    n: int
+    k: int
+    double_quant: bool
+    codes: torch.Tensor                  # uint8 [n*k/2]
+    absmax: torch.Tensor                 # fp32 [n*k/64]
+    absmax_q8: Optional[torch.Tensor]    # uint8 [n*k/64]
+    absmax_c: Optional[torch.Tensor]     # fp32 [ceil(n*k/64/256)]
+
+    def struct(self) -> NF4WeightStruct:
+        return NF4WeightStruct(self.n, self.k, BLOCK_SIZE, int(self.double_quant),
+                               self.codes.data_ptr(), self.absmax.data_ptr(),
+                               self.absmax_q8.data_ptr() if self.absmax_q8 is not None else None,
+                               self.absmax_c.data_ptr() if self.absmax_c is not None else None)
+
+    @property
+    def device(self) -> torch.device:
+        return self.codes.device
+
+    @staticmethod
+    def empty(n: int, k: int, double_quant: bool, device) -> "QuantizedWeight":
+        nb = n * k // BLOCK_SIZE
+        ng = (nb + DQ_GROUP - 1) // DQ_GROUP
+        dev = torch.device(device)
+        return QuantizedWeight(
+            n, k, double_quant,
+            torch.empty(n * k // 2, dtype=torch.uint8, device=dev),
+            torch.empty(nb, dtype=torch.float32, device=dev),
+            torch.empty(max(nb, 1), dtype=torch.uint8, device=dev) if double_quant else None,
+            torch.empty(max(ng, 1), dtype=torch.float32, device=dev) if double_quant else None)
+
+
+def nf4_quantize(W0: torch.Tensor, double_quant: bool = True,
+                 out: Optional[QuantizedWeight] = None) -> QuantizedWeight:
+    """Blockwise NF4 quantisation of a [n, k] fp32 CUDA tensor."""
+    _need_cuda(W0)
+    if W0.dtype != torch.float32 or W0.dim() != 2 or not W0.is_contiguous():
+        raise ValueError("W0 must be a contiguous 2-D float32 tensor")
+    n, k = W0.shape
+    qw = out if out is not None else QuantizedWeight.empty(n, k, double_quant, W0.device)
+    s = qw.struct()
+    _check(lib.nf4_quantize(_ptr(W0), ctypes.byref(s), _stream(W0.device)), "nf4_quantize")
+    return qw
+
+
+def nf4_dequantize(qw: QuantizedWeight, bf16: bool = True) -> torch.Tensor:
+    out = torch.empty(qw.n, qw.k, dtype=torch.bfloat16 if bf16 else torch.float32, device=qw.device)
+    s = qw.struct()
+    _check(lib.nf4_dequantize(ctypes.byref(s), _ptr(out), int(bf16), _stream(qw.device)),
+           "nf4_dequantize")
+    return out
+
+
+def fwd_workspace_bytes(M: int, n: int, k: int, r: int) -> int:
+    return int(lib.qlora_fwd_workspace_bytes(M, n, k, r))
+
+
+def bwd_workspace_bytes(M: int, n: int, k: int, r: int) -> int:
+    return int(lib.qlora_bwd_workspace_bytes(M, n, k, r))
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def qlora_linear_fwd(qw: QuantizedWeight, x: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
+                     alpha: float, save_u: bool = True, h: Optional[torch.Tensor] = None,
+                     workspace: Optional[torch.Tensor] = None, u: Optional[torch.Tensor] = None
+                     ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """h = x W~^T + (alpha/r)(x A^T) B^T; also returns u = x A^T (fp32) if save_u."""
+    _need_cuda(x, A, B)
+    M = x.shape[0]
+    r = A.shape[0]
+    if h is None:
+        h = torch.empty(M, qw.n, dtype=torch.bfloat16, device=x.device)
+    if u is None and save_u:
+        u = torch.empty(M, r, dtype=torch.float32, device=x.device)
+    nbytes = fwd_workspace_bytes(M, qw.n, qw.k, r)
+    ws = workspace if workspace is not None else _workspace(nbytes, x.device)
+    s = qw.struct()
+    _check(lib.qlora_linear_fwd(ctypes.byref(s), _ptr(x), M, _ptr(A), _ptr(B), r, float(alpha),
+                                _ptr(h), _ptr(u), _ptr(ws), ws.numel(), _stream(x.device)),
+           "qlora_linear_fwd")
+    return h, u
+
+
+def qlora_linear_bwd(qw: QuantizedWeight, x: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
+                     alpha: float, dY: torch.Tensor, u: Optional[torch.Tensor] = None,
+                     need_dX: bool = True, workspace: Optional[torch.Tensor] = None,
+                     outs: Optional[tuple] = None):
+    """(dX, dA, dB) of the layer; dX is None when need_dX is False."""
+    _need_cuda(x, A, B, dY)
+    M = x.shape[0]
+    r = A.shape[0]
+    if outs is not None:
+        dX, dA, dB = outs
+    else:
+        dX = torch.empty(M, qw.k, dtype=torch.bfloat16, device=x.device) if need_dX else None
+        dA = torch.empty(r, qw.k, dtype=torch.bfloat16, device=x.device)
+        dB = torch.empty(qw.n, r, dtype=torch.bfloat16, device=x.device)
+    nbytes = bwd_workspace_bytes(M, qw.n, qw.k, r)
+    ws = workspace if workspace is not None else _workspace(nbytes, x.device)
+    s = qw.struct()
+    _check(lib.qlora_linear_bwd(ctypes.byref(s), _ptr(x), M, _ptr(A), _ptr(B), r, float(alpha),
+                                _ptr(dY), _ptr(u), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws),
+                                ws.numel(), _stream(x.device)),
+           "qlora_linear_bwd")
+    return dX, dA, dB
+
+
+def device_status(device=None) -> int:
+    """Synchronise the current stream and return (and clear) the device status word."""
+    dev = torch.device("cuda" if device is None else device)
+    return int(lib.nf4_device_status(_stream(dev)))
+
+
+def profiling(enable: bool) -> None:
+    """Enable (and clear) or disable per-kernel event timing inside the library."""
+    _check(lib.nf4_profiling(int(enable)), "nf4_profiling")
+
+
+def profile_read() -> dict:
+    """{kernel kind: (launches, total milliseconds)} for the launches recorded
+    since profiling was last enabled (synchronises the recorded events)."""
+    buf = (NF4KernelTime * 32)()
+    n = lib.nf4_profile_read(buf, 32)
+    if n < 0:
+        raise NF4Error(NF4_ERR_CUDA, "nf4_profile_read")
+    return {buf[i].name.decode(): (int(buf[i].launches), float(buf[i].total_ms)) for i in range(n)}

@@ -1,0 +1,273 @@
+// nf4_common.cuh -- shared device helpers of the sm_100a QLoRA library:
+// the NF4 level table, the device status word, and thin wrappers over the
+// PTX of mbarriers, TMA and tcgen05 (tensor memory + 5th-gen tensor cores).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/qlora_nf4.h"
+
+namespace nf4 {
+
+// ---------------------------------------------------------------------------
+// NF4 levels: the 16-value lookup table printed in "QLoRA explained:
+// fine-tuning in 4-bit precision" (section "Common misconceptions"), index
+// order as in the level table of "Parameter-Efficient Fine-Tuning: From LoRA
+// to QLoRA" (Pillar 1). Written as hex floats; every value is an exact fp32.
+// ---------------------------------------------------------------------------
+#define NF4_LEVEL_LIST                                                          \
+    -0x1.000000p+0f, -0x1.647362p-1f, -0x1.0cd660p-1f, -0x1.946540p-2f,         \
+    -0x1.23449ap-2f, -0x1.7a6a7ep-3f, -0x1.74f0e2p-4f, 0x0.0p+0f,               \
+    0x1.45f5fep-4f, 0x1.4995c6p-3f, 0x1.f809bap-3f, 0x1.5a0674p-2f,            \
+    0x1.c34970p-2f, 0x1.200f56p-1f, 0x1.722766p-1f, 0x1.000000p+0f
+
+__constant__ float c_levels[16] = {NF4_LEVEL_LIST};
+
+constexpr int kBlock = 64;       // elements per NF4 block
+constexpr int kGroup = 256;      // blocks per double-quant group
+
+// ---------------------------------------------------------------------------
+// Device status word (first error wins). Read and cleared by the host.
+// ---------------------------------------------------------------------------
+__device__ unsigned int g_status;
+
+__device__ __forceinline__ void record_status(unsigned int code) {
+    atomicCAS(&g_status, 0u, code);
+}
+
+// Pipeline waits give up after this many SM cycles (about 2 s at the
+// B200's clocks), record NF4_ERR_TIMEOUT and unwind.
+constexpr long long kWaitLimitCycles = 4000000000LL;
+
+// ---------------------------------------------------------------------------
+// Shared-memory addresses, mbarriers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity. Returns false (and
+// raises the CTA's abort flag) when the wait runs out of time or another
+// role of the CTA has already aborted.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (clock64() - t0 > kWaitLimitCycles) {
+            record_status(NF4_ERR_TIMEOUT);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
+// Generic-proxy writes to shared memory become visible to the async proxy
+// (tensor core operand reads, TMA) after this fence.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
+// TMA (cp.async.bulk.tensor), 2-D tiles into shared memory
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar,
+                                            int32_t c0, int32_t c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// tcgen05: tensor memory allocation, MMA, commit, loads
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void umma_bf16_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive once on the mbarrier when every tcgen05 op issued so far by this
+// thread has completed.
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+
+// 32 TMEM lanes x 32 consecutive 32-bit columns; thread i of the warp gets
+// lane (quadrant*32 + i), columns [col, col+32).
+__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor (tcgen05 form): start address, leading and
+// stride byte offsets (16-byte units), descriptor version 1, 128-byte swizzle.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes,
+                                                    uint32_t sbo_bytes) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+    d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1) << 46;   // version
+    d |= static_cast<uint64_t>(2) << 61;   // SWIZZLE_128B
+    return d;
+}
+
+// Instruction descriptor: bf16 x bf16 -> fp32, M x N, A/B major-ness
+// (0 = K-major, 1 = MN-major).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_major, int b_mn_major) {
+    return (1u << 4)                                  // D format fp32
+           | (1u << 7)                                // A bf16
+           | (1u << 10)                               // B bf16
+           | (static_cast<uint32_t>(a_mn_major) << 15)
+           | (static_cast<uint32_t>(b_mn_major) << 16)
+           | (static_cast<uint32_t>(N >> 3) << 17)
+           | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// ---------------------------------------------------------------------------
+// NF4 block dequantisation into packed bf16 pairs (register-resident lookup)
+//
+// A block of 64 codes shares one scale s. The 16 possible outputs
+// bf16(fl32(s * level_j)) are computed once per block and kept as byte planes
+// in 8 registers; each code then selects its output with byte permutes, so
+// no shared-memory lookup (and no bank conflict) is needed per element.
+// ---------------------------------------------------------------------------
+struct BlockLut {
+    uint32_t lo[4];   // lo[q] bytes: low bytes of entries 4q..4q+3
+    uint32_t hi[4];   // hi[q] bytes: high bytes of entries 4q..4q+3
+};
+
+__device__ __forceinline__ BlockLut make_block_lut(float s) {
+    uint32_t pair[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        // fp32 product, then one rounding to bf16 (nearest even); entry 2i in
+        // the low half, 2i+1 in the high half
+        __nv_bfloat162 p = __floats2bfloat162_rn(s * c_levels[2 * i], s * c_levels[2 * i + 1]);
+        pair[i] = *reinterpret_cast<uint32_t *>(&p);
+    }
+    BlockLut L;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        L.lo[q] = __byte_perm(pair[2 * q], pair[2 * q + 1], 0x6420);
+        L.hi[q] = __byte_perm(pair[2 * q], pair[2 * q + 1], 0x7531);
+    }
+    return L;
+}
+
+// PRMT with the selector used as given (a selector nibble with bit 3 set
+// replicates the sign bit of the selected byte across the output byte).
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// Dequantise the 8 codes of one 32-bit word (bytes in memory order; byte b
+// holds element 2b in its high nibble and 2b+1 in its low nibble) into 4
+// packed bf16x2 words, element order preserved (lower element in the low
+// half).
+__device__ __forceinline__ void dequant8(const BlockLut &L, uint32_t w, uint32_t (&out)[4]) {
+    const uint32_t w4 = w << 4;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const uint32_t sel = (half ? (w >> 16) : w) & 0x7777u;
+        // byte mask of codes >= 8, output byte order = nibble order of `sel`
+        const uint32_t m = prmt(w, w4, half ? 0xBFAEu : 0x9D8Cu);
+        const uint32_t la = __byte_perm(L.lo[0], L.lo[1], sel);
+        const uint32_t lb = __byte_perm(L.lo[2], L.lo[3], sel);
+        const uint32_t ha = __byte_perm(L.hi[0], L.hi[1], sel);
+        const uint32_t hb = __byte_perm(L.hi[2], L.hi[3], sel);
+        const uint32_t lo = (la & ~m) | (lb & m);
+        const uint32_t hi = (ha & ~m) | (hb & m);
+        // nibble order in `sel` is (odd, even, odd, even) elements; rebuild
+        // bf16 pairs (even element low)
+        out[2 * half + 0] = __byte_perm(lo, hi, 0x4051);
+        out[2 * half + 1] = __byte_perm(lo, hi, 0x6273);
+    }
+}
+
+}  // namespace nf4

@@ -1,0 +1,481 @@
+// qlora_nf4.cu -- C ABI of the sm_100a QLoRA linear-layer library: argument
+// validation, workspace layout, TMA descriptor set-up and kernel dispatch.
+// The whole library is this one translation unit (the kernels live in the
+// included headers), so the device status word has a single definition.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "codec.cuh"
+#include "gemm_tc.cuh"
+#include "lora_small.cuh"
+
+using namespace nf4;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+#define NF4_TRY_CUDA(expr)                          \
+    do {                                            \
+        if ((expr) != cudaSuccess) return NF4_ERR_CUDA; \
+    } while (0)
+
+// ---------------------------------------------------------------------------
+// Optional per-kernel event timing (nf4_profiling / nf4_profile_read)
+// ---------------------------------------------------------------------------
+enum KernelKind {
+    KK_QUANTIZE, KK_DEQUANTIZE, KK_ROWDOT, KK_COLPROD, KK_COLREDUCE, KK_TRANSPOSE, KK_ZERO,
+    KK_GEMM_FWD, KK_GEMM_DGRAD, KK_COUNT
+};
+const char *const kKindNames[KK_COUNT] = {
+    "nf4_quantize", "nf4_dequantize", "lora_rowdot", "lora_colprod", "lora_colreduce",
+    "lora_transpose", "zero_fill", "qlora_gemm_fwd", "qlora_gemm_dgrad"};
+
+struct ProfRecord {
+    int kind;
+    int device;
+    cudaEvent_t start, stop;
+};
+
+struct Profiler {
+    std::mutex mu;
+    bool on = false;
+    std::vector<ProfRecord> recs;
+    std::vector<ProfRecord> pool;   // spare event pairs (kind unused)
+
+    bool take(int device, cudaEvent_t *a, cudaEvent_t *b) {
+        for (size_t i = 0; i < pool.size(); ++i) {
+            if (pool[i].device == device) {
+                *a = pool[i].start;
+                *b = pool[i].stop;
+                pool.erase(pool.begin() + static_cast<long>(i));
+                return true;
+            }
+        }
+        return cudaEventCreate(a) == cudaSuccess && cudaEventCreate(b) == cudaSuccess;
+    }
+};
+
+Profiler &profiler() {
+    static Profiler p;
+    return p;
+}
+
+// Brackets one launch with events on its stream when profiling is enabled.
+class LaunchTimer {
+  public:
+    LaunchTimer(int kind, cudaStream_t s) : kind_(kind), s_(s) {
+        Profiler &p = profiler();
+        std::lock_guard<std::mutex> g(p.mu);
+        if (!p.on) return;
+        if (cudaGetDevice(&dev_) != cudaSuccess) return;
+        if (!p.take(dev_, &a_, &b_)) return;
+        active_ = cudaEventRecord(a_, s_) == cudaSuccess;
+    }
+    void stop() {
+        if (!active_) return;
+        active_ = false;
+        Profiler &p = profiler();
+        std::lock_guard<std::mutex> g(p.mu);
+        if (cudaEventRecord(b_, s_) == cudaSuccess) p.recs.push_back({kind_, dev_, a_, b_});
+        else p.pool.push_back({kind_, dev_, a_, b_});
+    }
+    ~LaunchTimer() { stop(); }
+
+  private:
+    int kind_;
+    cudaStream_t s_;
+    int dev_ = 0;
+    cudaEvent_t a_{}, b_{};
+    bool active_ = false;
+};
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int current_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    return dev;
+}
+
+int num_sms(int dev) {
+    static int cache[kMaxDevices] = {0};
+    if (dev < 0 || dev >= kMaxDevices) return 148;
+    if (cache[dev] == 0) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+            v = 148;
+        cache[dev] = v;
+    }
+    return cache[dev];
+}
+
+// cuTensorMapEncodeTiled, fetched once from the driver through the runtime.
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D row-major tensor [outer, inner] of `elem` bytes per element.
+bool make_map(CUtensorMap *map, CUtensorMapDataType dt, size_t elem, const void *base,
+              uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer,
+              CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {inner * elem};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+nf4_status check_weight(const nf4_weight *w, bool need_scales) {
+    if (!w) return NF4_ERR_INVALID_ARG;
+    if (w->block_size != kBlock || (w->double_quant != 0 && w->double_quant != 1))
+        return NF4_ERR_INVALID_ARG;
+    if (w->n < 8 || w->k < 64 || (w->n % 8) != 0 || (w->k % 64) != 0) return NF4_ERR_UNSUPPORTED_SHAPE;
+    if (w->n > (int64_t(1) << 31) - 1 || w->k > (int64_t(1) << 31) - 1) return NF4_ERR_UNSUPPORTED_SHAPE;
+    if (!w->codes || !w->absmax) {
+        if (!w->codes || !(w->double_quant || !need_scales)) return NF4_ERR_INVALID_ARG;
+    }
+    if (w->double_quant && (!w->absmax_q8 || !w->absmax_c)) return NF4_ERR_INVALID_ARG;
+    if (!aligned16(w->codes) || (w->absmax && !aligned16(w->absmax)) ||
+        (w->absmax_q8 && !aligned16(w->absmax_q8)) || (w->absmax_c && !aligned16(w->absmax_c)))
+        return NF4_ERR_ALIGNMENT;
+    return NF4_OK;
+}
+
+nf4_status check_layer(const nf4_weight *w, const void *x, int64_t M, const void *A, const void *B,
+                       int32_t r, float alpha) {
+    nf4_status st = check_weight(w, true);
+    if (st != NF4_OK) return st;
+    if (M < 0 || M > (int64_t(1) << 30)) return NF4_ERR_UNSUPPORTED_SHAPE;
+    if (r < 1 || r > 128 || (r % 8) != 0) return NF4_ERR_UNSUPPORTED_SHAPE;
+    if (!std::isfinite(alpha)) return NF4_ERR_INVALID_ARG;
+    if (!A || !B || (M > 0 && !x)) return NF4_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(A) || !aligned16(B)) return NF4_ERR_ALIGNMENT;
+    return NF4_OK;
+}
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// Splits of the M dimension for the column products (dB over n, dA over k).
+int col_splits(int64_t M, int64_t C, int sms) {
+    const int64_t tiles = (C + kColTile - 1) / kColTile;
+    int64_t s = (2 * sms + tiles - 1) / tiles;
+    s = std::max<int64_t>(1, std::min<int64_t>(s, (M + 127) / 128));
+    return static_cast<int>(s);
+}
+
+struct BwdLayout {
+    size_t bt, v, vs, u, part, total;
+    int s_dB, s_dA;
+};
+
+BwdLayout bwd_layout(int64_t M, int64_t n, int64_t k, int32_t r, int sms) {
+    BwdLayout L{};
+    size_t off = 0;
+    L.bt = off;   off = align256(off + size_t(n) * r * 2);
+    L.v = off;    off = align256(off + size_t(M) * r * 4);
+    L.vs = off;   off = align256(off + size_t(M) * r * 2);
+    L.u = off;    off = align256(off + size_t(M) * r * 4);
+    L.s_dB = col_splits(M, n, sms);
+    L.s_dA = col_splits(M, k, sms);
+    L.part = off;
+    off = align256(off + size_t(std::max(int64_t(L.s_dB) * n, int64_t(L.s_dA) * k)) * r * 4);
+    L.total = off;
+    return L;
+}
+
+template <int BN, bool DGRAD>
+nf4_status launch_gemm(const nf4_weight *w, const uint16_t *act, int64_t M, int64_t red,
+                       int64_t out, const uint16_t *la, int32_t r, const uint16_t *lb,
+                       uint16_t *D, cudaStream_t stream) {
+    using Cfg = GemmCfg<BN, DGRAD>;
+    CUtensorMap tm_act, tm_codes, tm_la, tm_lb;
+    const int64_t N = w->n, K = w->k;
+    bool ok = make_map(&tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, act, red, M, kBK, kBM,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!DGRAD)
+        ok = ok && make_map(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, K / 2, N,
+                            kBK / 2, BN, CU_TENSOR_MAP_SWIZZLE_NONE);
+    else
+        ok = ok && make_map(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, K / 2, N,
+                            BN / 2, kBK, CU_TENSOR_MAP_SWIZZLE_NONE);
+    ok = ok && make_map(&tm_la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, la, r, M, kBK, kBM,
+                        CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!DGRAD)  // B [N, r]: rows n, K-major over j
+        ok = ok && make_map(&tm_lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, lb, r, N, kBK, BN,
+                            CU_TENSOR_MAP_SWIZZLE_128B);
+    else         // A [r, K]: rows j, 64 output columns per box (MN-major atoms)
+        ok = ok && make_map(&tm_lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, lb, K, r, 64, kBK,
+                            CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!ok) return NF4_ERR_CUDA;
+
+    GemmArgs a;
+    a.M = static_cast<int>(M);
+    a.red = static_cast<int>(red);
+    a.out = static_cast<int>(out);
+    a.main_steps = static_cast<int>((red + kBK - 1) / kBK);
+    a.lora_steps = (r + kBK - 1) / kBK;
+    a.m_tiles = static_cast<int>((M + kBM - 1) / kBM);
+    a.n_tiles = static_cast<int>((out + BN - 1) / BN);
+    a.Nw = N;
+    a.kblocks = K / kBlock;
+    a.absmax = w->absmax;
+    a.q8 = w->absmax_q8;
+    a.cg = w->absmax_c;
+    a.dq = w->double_quant;
+    a.D = D;
+
+    const int dev = current_device();
+    const int tiles = a.m_tiles * a.n_tiles;
+    const int grid = std::min(tiles, num_sms(dev));
+    auto kern = qlora_gemm_kernel<BN, DGRAD>;
+    NF4_TRY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      Cfg::kSmemBytes));
+    LaunchTimer t(DGRAD ? KK_GEMM_DGRAD : KK_GEMM_FWD, stream);
+    kern<<<grid, kGemmThreads, Cfg::kSmemBytes, stream>>>(tm_act, tm_codes, tm_la, tm_lb, a);
+    t.stop();
+    NF4_TRY_CUDA(cudaGetLastError());
+    return NF4_OK;
+}
+
+nf4_status launch_rowdot(const uint16_t *P, const uint16_t *Q, int64_t M, int64_t Kd, int32_t r,
+                         float *out_f32, uint16_t *out_bf16, float scale, cudaStream_t stream) {
+    if (M == 0) return NF4_OK;
+    const int grid = static_cast<int>((M + kRowdotRows - 1) / kRowdotRows);
+    LaunchTimer t(KK_ROWDOT, stream);
+    rowdot_kernel<<<grid, 256, 0, stream>>>(P, Q, static_cast<int>(M), static_cast<int>(Kd), r,
+                                            out_f32, out_bf16, scale);
+    t.stop();
+    NF4_TRY_CUDA(cudaGetLastError());
+    return NF4_OK;
+}
+
+nf4_status launch_colprod(const uint16_t *P, const float *U, int64_t M, int64_t C, int32_t r,
+                          int S, float *part, float scale, int transposed, uint16_t *out,
+                          cudaStream_t stream) {
+    const int rows_per_split = static_cast<int>((M + S - 1) / S);
+    dim3 grid(static_cast<unsigned>((C + kColTile - 1) / kColTile), static_cast<unsigned>(S));
+    LaunchTimer t1(KK_COLPROD, stream);
+    colprod_partial_kernel<<<grid, 256, 0, stream>>>(P, U, static_cast<int>(M),
+                                                     static_cast<int>(C), r, rows_per_split, part);
+    t1.stop();
+    NF4_TRY_CUDA(cudaGetLastError());
+    const int64_t total = C * r;
+    const int rgrid = static_cast<int>(std::min<int64_t>((total + 255) / 256, 4096));
+    LaunchTimer t2(KK_COLREDUCE, stream);
+    colprod_reduce_kernel<<<rgrid, 256, 0, stream>>>(part, S, static_cast<int>(C), r, scale,
+                                                     transposed, out);
+    t2.stop();
+    NF4_TRY_CUDA(cudaGetLastError());
+    return NF4_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *nf4_status_string(nf4_status s) {
+    switch (s) {
+        case NF4_OK: return "ok";
+        case NF4_ERR_INVALID_ARG: return "invalid argument";
+        case NF4_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+        case NF4_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+        case NF4_ERR_NONFINITE: return "non-finite value in the weight";
+        case NF4_ERR_TIMEOUT: return "device pipeline wait timed out";
+        case NF4_ERR_CUDA: return "CUDA call failed";
+        case NF4_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+nf4_status nf4_profiling(int32_t enable) {
+    Profiler &p = profiler();
+    std::lock_guard<std::mutex> g(p.mu);
+    if (enable) {
+        for (auto &r : p.recs) p.pool.push_back(r);
+        p.recs.clear();
+    }
+    p.on = enable != 0;
+    return NF4_OK;
+}
+
+int32_t nf4_profile_read(nf4_kernel_time *out, int32_t max) {
+    Profiler &p = profiler();
+    std::lock_guard<std::mutex> g(p.mu);
+    int64_t n[KK_COUNT] = {0};
+    double ms[KK_COUNT] = {0};
+    for (auto &r : p.recs) {
+        float t = 0.f;
+        if (cudaEventSynchronize(r.stop) != cudaSuccess ||
+            cudaEventElapsedTime(&t, r.start, r.stop) != cudaSuccess)
+            return -1;
+        n[r.kind] += 1;
+        ms[r.kind] += t;
+    }
+    int32_t cnt = 0;
+    for (int k = 0; k < KK_COUNT; ++k) {
+        if (n[k] == 0) continue;
+        if (out && cnt < max) out[cnt] = {kKindNames[k], n[k], ms[k]};
+        ++cnt;
+    }
+    return cnt;
+}
+
+nf4_status nf4_device_status(void *stream) {
+    NF4_TRY_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+    unsigned int v = 0, zero = 0;
+    NF4_TRY_CUDA(cudaMemcpyFromSymbol(&v, g_status, sizeof v));
+    if (v != 0) NF4_TRY_CUDA(cudaMemcpyToSymbol(g_status, &zero, sizeof zero));
+    return static_cast<nf4_status>(v);
+}
+
+nf4_status nf4_quantize(const float *W0, const nf4_weight *w, void *stream) {
+    nf4_status st = check_weight(w, false);
+    if (st != NF4_OK) return st;
+    if (!W0 || !w->absmax) return NF4_ERR_INVALID_ARG;
+    if (!aligned16(W0)) return NF4_ERR_ALIGNMENT;
+    const int64_t nb = w->n * w->k / kBlock;
+    const int64_t groups = (nb + kGroup - 1) / kGroup;
+    if (groups > 0x7fffffff) return NF4_ERR_UNSUPPORTED_SHAPE;
+    LaunchTimer t(KK_QUANTIZE, static_cast<cudaStream_t>(stream));
+    nf4_quantize_kernel<<<static_cast<unsigned>(groups), kQuantThreads, 0,
+                          static_cast<cudaStream_t>(stream)>>>(
+        W0, nb, w->double_quant, w->codes, w->absmax, w->absmax_q8, w->absmax_c);
+    t.stop();
+    NF4_TRY_CUDA(cudaGetLastError());
+    return NF4_OK;
+}
+
+nf4_status nf4_dequantize(const nf4_weight *w, void *out, int32_t out_bf16, void *stream) {
+    nf4_status st = check_weight(w, true);
+    if (st != NF4_OK) return st;
+    if (!out || (out_bf16 != 0 && out_bf16 != 1)) return NF4_ERR_INVALID_ARG;
+    if (!aligned16(out)) return NF4_ERR_ALIGNMENT;
+    const int64_t nb = w->n * w->k / kBlock;
+    const int dev = current_device();
+    const int grid = static_cast<int>(std::min<int64_t>((nb + 255) / 256, int64_t(num_sms(dev)) * 16));
+    LaunchTimer t(KK_DEQUANTIZE, static_cast<cudaStream_t>(stream));
+    nf4_dequantize_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        w->codes, w->absmax, w->absmax_q8, w->absmax_c, w->double_quant, nb, out_bf16, out);
+    t.stop();
+    NF4_TRY_CUDA(cudaGetLastError());
+    return NF4_OK;
+}
+
+size_t qlora_fwd_workspace_bytes(int64_t M, int64_t n, int64_t k, int32_t r) {
+    (void)n;
+    (void)k;
+    if (M <= 0 || r <= 0) return 256;
+    return align256(size_t(M) * r * 2);
+}
+
+nf4_status qlora_linear_fwd(const nf4_weight *w, const uint16_t *x, int64_t M, const uint16_t *A,
+                            const uint16_t *B, int32_t r, float alpha, uint16_t *h, float *u_out,
+                            void *workspace, size_t ws_bytes, void *stream) {
+    nf4_status st = check_layer(w, x, M, A, B, r, alpha);
+    if (st != NF4_OK) return st;
+    if (M == 0) return NF4_OK;
+    if (!h) return NF4_ERR_INVALID_ARG;
+    if (!aligned16(h) || !aligned16(u_out)) return NF4_ERR_ALIGNMENT;
+    if (!workspace || ws_bytes < qlora_fwd_workspace_bytes(M, w->n, w->k, r)) return NF4_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return NF4_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const float scale = alpha / static_cast<float>(r);
+    uint16_t *u_s = static_cast<uint16_t *>(workspace);
+    st = launch_rowdot(x, A, M, w->k, r, u_out, u_s, scale, s);
+    if (st != NF4_OK) return st;
+    return launch_gemm<256, false>(w, x, M, w->k, w->n, u_s, r, B, h, s);
+}
+
+size_t qlora_bwd_workspace_bytes(int64_t M, int64_t n, int64_t k, int32_t r) {
+    if (M < 0 || n <= 0 || k <= 0 || r <= 0) return 256;
+    const int sms = num_sms(current_device());
+    return bwd_layout(std::max<int64_t>(M, 1), n, k, r, sms).total;
+}
+
+nf4_status qlora_linear_bwd(const nf4_weight *w, const uint16_t *x, int64_t M, const uint16_t *A,
+                            const uint16_t *B, int32_t r, float alpha, const uint16_t *dY,
+                            const float *u, uint16_t *dX, uint16_t *dA, uint16_t *dB,
+                            void *workspace, size_t ws_bytes, void *stream) {
+    nf4_status st = check_layer(w, x, M, A, B, r, alpha);
+    if (st != NF4_OK) return st;
+    if (!dA || !dB || (M > 0 && !dY)) return NF4_ERR_INVALID_ARG;
+    if (!aligned16(dY) || !aligned16(u) || !aligned16(dX) || !aligned16(dA) || !aligned16(dB))
+        return NF4_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t N = w->n, K = w->k;
+    if (M == 0) {
+        LaunchTimer t(KK_ZERO, s);
+        zero_u16_kernel<<<64, 256, 0, s>>>(dA, int64_t(r) * K);
+        zero_u16_kernel<<<64, 256, 0, s>>>(dB, N * r);
+        t.stop();
+        NF4_TRY_CUDA(cudaGetLastError());
+        return NF4_OK;
+    }
+    const int sms = num_sms(current_device());
+    const BwdLayout L = bwd_layout(M, N, K, r, sms);
+    if (!workspace || ws_bytes < L.total) return NF4_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return NF4_ERR_ALIGNMENT;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint16_t *Bt = reinterpret_cast<uint16_t *>(ws + L.bt);
+    float *v = reinterpret_cast<float *>(ws + L.v);
+    uint16_t *v_s = reinterpret_cast<uint16_t *>(ws + L.vs);
+    float *part = reinterpret_cast<float *>(ws + L.part);
+    const float scale = alpha / static_cast<float>(r);
+
+    // v = dY B (fp32) and bf16(s v) for the dgrad LoRA stage
+    {
+        LaunchTimer t(KK_TRANSPOSE, s);
+        transpose_nr_kernel<<<static_cast<int>(std::min<int64_t>((N * r + 255) / 256, 4096)), 256,
+                              0, s>>>(B, static_cast<int>(N), r, Bt);
+        t.stop();
+    }
+    NF4_TRY_CUDA(cudaGetLastError());
+    st = launch_rowdot(dY, Bt, M, N, r, v, v_s, scale, s);
+    if (st != NF4_OK) return st;
+    // u = x A^T unless the forward saved it
+    const float *uu = u;
+    if (!uu) {
+        float *ur = reinterpret_cast<float *>(ws + L.u);
+        st = launch_rowdot(x, A, M, K, r, ur, nullptr, 1.0f, s);
+        if (st != NF4_OK) return st;
+        uu = ur;
+    }
+    // dB = s dY^T u  ([N, r]);  dA = s v^T x  ([r, K])
+    st = launch_colprod(dY, uu, M, N, r, L.s_dB, part, scale, 0, dB, s);
+    if (st != NF4_OK) return st;
+    st = launch_colprod(x, v, M, K, r, L.s_dA, part, scale, 1, dA, s);
+    if (st != NF4_OK) return st;
+    // dX = dY W~ + bf16(s v) A
+    if (dX) return launch_gemm<256, true>(w, dY, M, N, K, v_s, r, A, dX, s);
+    return NF4_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,180 @@
+/*
+ * qlora_nf4.h -- C ABI of the B200 (sm_100a) QLoRA linear-layer library.
+ *
+ * The layer computes, for a frozen weight W0 stored as 4-bit NormalFloat
+ * (NF4) codes with blockwise scales, and trainable low-rank adapters A, B:
+ *
+ *     h = x W~^T + (alpha / r) (x A^T) B^T
+ *
+ * ("QLoRA Finetuner -- Juan Martos", section 1, forward step of the LoRA
+ * layer, and its flowchart "Quantized Base Inference"; "QLoRA explained:
+ * fine-tuning in 4-bit precision", section "The LoRA adapter path").
+ *
+ * Shapes and layouts (all row-major, all device memory owned by the caller):
+ *   W0  [n, k] fp32      n = output features, k = input features. The pages
+ *                        write W0 as d x k with A r x d and B k x r; here
+ *                        d == k (input) and the pages' k == n (output), stored
+ *                        out-by-in like a torch Linear weight.
+ *   x   [M, k] bf16      tokens
+ *   A   [r, k] bf16      down-projection
+ *   B   [n, r] bf16      up-projection
+ *   h   [M, n] bf16
+ *   dY  [M, n] bf16      gradient of the loss w.r.t. h
+ *   dX  [M, k] bf16, dA [r, k] bf16, dB [n, r] bf16
+ * bf16 values travel as uint16_t bit patterns.
+ *
+ * Conventions:
+ *   - The library never allocates device memory. Scratch space is passed in
+ *     (`workspace`, sized by the *_workspace_bytes queries).
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Every
+ *     entry point is asynchronous: NF4_OK means the arguments were valid and
+ *     the kernels were launched. Conditions detected on the device
+ *     (non-finite weight values, a pipeline wait that ran out of time) are
+ *     recorded in a per-device status word read by nf4_device_status().
+ *   - Requirements (violations return an error and launch nothing):
+ *       k % 64 == 0, n % 8 == 0, n >= 8, k >= 64, M >= 0,
+ *       1 <= r <= 128 and r % 8 == 0, alpha finite,
+ *       every pointer 16-byte aligned, block_size == 64.
+ *   - No C++ exception crosses this boundary. Entry points are reentrant;
+ *     calls on one stream are ordered, calls on different streams that share
+ *     output or workspace buffers race.
+ */
+#ifndef QLORA_NF4_H
+#define QLORA_NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QLORA_API __attribute__((visibility("default")))
+#else
+#define QLORA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NF4_OK = 0,
+    NF4_ERR_INVALID_ARG = 1,       /* null pointer where one is required, bad flag */
+    NF4_ERR_UNSUPPORTED_SHAPE = 2, /* a shape requirement above is violated */
+    NF4_ERR_ALIGNMENT = 3,         /* a pointer is not 16-byte aligned */
+    NF4_ERR_NONFINITE = 4,         /* (device) NaN or Inf in the weight to quantise */
+    NF4_ERR_TIMEOUT = 5,           /* (device) a pipeline wait ran out of time */
+    NF4_ERR_CUDA = 6,              /* a CUDA runtime/driver call failed */
+    NF4_ERR_WORKSPACE = 7,         /* workspace missing or smaller than required */
+} nf4_status;
+
+/* A quantised frozen weight. The struct lives in host memory; the arrays it
+ * points to are device memory owned by the caller.
+ *   codes      n*k/2 bytes. Element e of the flattened weight is a 4-bit
+ *              index into the 16 NF4 levels; element 2j is the HIGH nibble of
+ *              byte j ("Parameter-Efficient Fine-Tuning: From LoRA to QLoRA",
+ *              Pillar 1, byte packing step of the numerical example).
+ *   absmax     nb = n*k/64 fp32 block scales s_i = max |w| over each run of
+ *              64 consecutive elements ("QLoRA Finetuner", section 2, absmax
+ *              scale). Always written by nf4_quantize; read by the other
+ *              entry points only when double_quant == 0.
+ *   absmax_q8  nb bytes in [0, 127]: 8-bit codes of the block scales
+ *              (double_quant == 1 only).
+ *   absmax_c   ceil(nb/256) fp32 group constants: the largest s_i in each run
+ *              of 256 consecutive blocks (double_quant == 1 only). The scale
+ *              used by dequantisation is then q8_i * (c_g / 127) in fp32
+ *              ("Parameter-Efficient Fine-Tuning", Pillar 2: 8-bit
+ *              quantisation of the scales in blocks of 256). */
+typedef struct {
+    int64_t n;
+    int64_t k;
+    int32_t block_size;   /* must be 64 */
+    int32_t double_quant; /* 0 or 1 */
+    uint8_t *codes;
+    float *absmax;
+    uint8_t *absmax_q8;
+    float *absmax_c;
+} nf4_weight;
+
+/* Blockwise NF4 quantisation of W0 [n, k] fp32 into w ("QLoRA Finetuner",
+ * section 2: absmax per 64-element block, normalise to [-1, 1], nearest of
+ * the 16 NF4 quantiles; "Parameter-Efficient Fine-Tuning", Pillar 1 and the
+ * numerical step-by-step example; Pillar 2 for double quantisation).
+ * Normalisation is one IEEE fp32 division w / s. A value exactly halfway
+ * between two levels takes the lower level. An all-zero block stores s = 0
+ * and code 7 (the exact zero level). With double_quant, each group of 256
+ * blocks stores c_g = max s_i and q8_i = round_half_even((s_i / c_g) * 127)
+ * in fp32; the NF4 codes are always taken against the unquantised s_i.
+ * A NaN/Inf in W0 sets NF4_ERR_NONFINITE in the device status (the outputs
+ * are then unspecified). Writes codes, absmax, and (if double_quant)
+ * absmax_q8 and absmax_c. */
+QLORA_API nf4_status nf4_quantize(const float *W0, const nf4_weight *w, void *stream);
+
+/* Dequantisation w~ = fl32(scale_i * NF4[q]) for every element ("QLoRA
+ * Finetuner", section 2, on-the-fly dequantization). out is n*k elements:
+ * fp32 when out_bf16 == 0, else bf16 (round to nearest even of the fp32
+ * value). The bf16 result is exactly the operand the layer's matmuls use. */
+QLORA_API nf4_status nf4_dequantize(const nf4_weight *w, void *out, int32_t out_bf16, void *stream);
+
+/* Workspace needed by qlora_linear_fwd for M tokens at rank r. */
+QLORA_API size_t qlora_fwd_workspace_bytes(int64_t M, int64_t n, int64_t k, int32_t r);
+
+/* Forward of the layer: h = x W~^T + (alpha/r) (x A^T) B^T, with W~ the bf16
+ * dequantised weight and fp32 accumulation ("QLoRA explained", section "The
+ * LoRA adapter path"; "QLoRA Finetuner", section 1 with dropout p = 0).
+ * The scaled down-projection (alpha/r)(x A^T) is rounded to bf16 before the
+ * up-projection. u_out (nullable, [M, r] fp32) receives u = x A^T for the
+ * backward. workspace: at least qlora_fwd_workspace_bytes(M, n, k, r) bytes
+ * of device memory, 256-byte aligned. M == 0 is a no-op. */
+QLORA_API nf4_status qlora_linear_fwd(const nf4_weight *w, const uint16_t *x, int64_t M,
+                            const uint16_t *A, const uint16_t *B, int32_t r, float alpha,
+                            uint16_t *h, float *u_out, void *workspace, size_t ws_bytes,
+                            void *stream);
+
+/* Workspace needed by qlora_linear_bwd for M tokens at rank r. */
+QLORA_API size_t qlora_bwd_workspace_bytes(int64_t M, int64_t n, int64_t k, int32_t r);
+
+/* Backward of the layer; the frozen weight gets no gradient ("QLoRA
+ * explained", section "The LoRA adapter path": the dequantised base weight is
+ * a constant in backprop and only the adapters are trained):
+ *     v  = dY B                  (fp32, [M, r])
+ *     dX = dY W~ + s v A         (s = alpha / r; v rounded to bf16 as s*v)
+ *     dA = s v^T x
+ *     dB = s dY^T u,   u = x A^T (taken from `u` when non-null, else recomputed)
+ * dX may be NULL (first layer: no input gradient). dA and dB are required.
+ * M == 0 writes zeros to dA and dB. */
+QLORA_API nf4_status qlora_linear_bwd(const nf4_weight *w, const uint16_t *x, int64_t M,
+                            const uint16_t *A, const uint16_t *B, int32_t r, float alpha,
+                            const uint16_t *dY, const float *u, uint16_t *dX, uint16_t *dA,
+                            uint16_t *dB, void *workspace, size_t ws_bytes, void *stream);
+
+/* Synchronises `stream`, then returns and clears the status word that the
+ * kernels of the current device set (NF4_OK if nothing was recorded). */
+QLORA_API nf4_status nf4_device_status(void *stream);
+
+/* Per-kernel timing, for benchmarks. While enabled, every kernel the library
+ * launches is bracketed by two CUDA events recorded on the stream it is
+ * launched on; nf4_profile_read() synchronises those events and reports, per
+ * kernel kind, the number of launches and their summed duration.
+ * nf4_profiling(1) enables and clears the records, nf4_profiling(0) disables
+ * recording (records are kept until the next enable). Not thread-safe with
+ * respect to concurrent enable/read; launches from several threads are
+ * recorded under a lock. */
+typedef struct {
+    const char *name;   /* static string: kernel kind */
+    int64_t launches;
+    double total_ms;
+} nf4_kernel_time;
+
+QLORA_API nf4_status nf4_profiling(int32_t enable);
+
+/* Fills up to `max` entries and returns how many kernel kinds were recorded
+ * (or -1 if reading an event failed). */
+QLORA_API int32_t nf4_profile_read(nf4_kernel_time *out, int32_t max);
+
+/* Static description of a status code. Never NULL. */
+QLORA_API const char *nf4_status_string(nf4_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_NF4_H */

@@ -1,0 +1,116 @@
+"""The C-ABI library loads, exports every entry point the header declares, and
+rejects bad arguments on the host (these paths make no CUDA call, so they run
+without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "qlora_nf4.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return re.findall(r"QLORA_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)
+
+
+@pytest.fixture(scope="module")
+def q():
+    from bit_nf4_quantized_05_b200 import build
+    build.build()
+    import bit_nf4_quantized_05_b200 as mod
+    return mod
+
+
+def test_header_declares_the_layer_entry_points():
+    names = declared_functions()
+    for n in ["nf4_quantize", "nf4_dequantize", "qlora_linear_fwd", "qlora_linear_bwd",
+              "qlora_fwd_workspace_bytes", "qlora_bwd_workspace_bytes", "nf4_device_status",
+              "nf4_status_string"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(q):
+    lib = ctypes.CDLL(q.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(q):
+    for code in range(8):
+        s = q.status_string(code)
+        assert s and s != "unknown status"
+    assert q.status_string(99) == "unknown status"
+
+
+def test_workspace_queries(q):
+    a = q.fwd_workspace_bytes(16, 1024, 1024, 8)
+    b = q.fwd_workspace_bytes(2048, 1024, 1024, 8)
+    assert 256 <= a <= b and b >= 2048 * 8 * 2 and b % 256 == 0
+    c = q.bwd_workspace_bytes(16, 1024, 1024, 8)
+    d = q.bwd_workspace_bytes(2048, 5120, 5120, 16)
+    assert 256 <= c <= d and d >= 2048 * 16 * (4 + 2 + 4)
+
+
+FAKE = 0x10000  # aligned, never dereferenced: validation fails or M == 0 returns first
+
+
+def weight(q, n=64, k=64, block=64, dq=0, codes=FAKE, absmax=FAKE, q8=FAKE, cg=FAKE):
+    return q.NF4WeightStruct(n, k, block, dq, codes, absmax, q8, cg)
+
+
+def call_fwd(q, w, M=4, r=8, alpha=16.0, x=FAKE, A=FAKE, B=FAKE, h=FAKE, u=None, ws=FAKE,
+             wsb=1 << 20):
+    return q.lib.qlora_linear_fwd(ctypes.byref(w), x, M, A, B, r, alpha, h, u, ws, wsb, None)
+
+
+def test_quantize_argument_checks(q):
+    L = q.lib
+    assert L.nf4_quantize(FAKE, None, None) == q.NF4_ERR_INVALID_ARG
+    assert L.nf4_quantize(FAKE, ctypes.byref(weight(q, block=32)), None) == q.NF4_ERR_INVALID_ARG
+    assert L.nf4_quantize(FAKE, ctypes.byref(weight(q, dq=2)), None) == q.NF4_ERR_INVALID_ARG
+    assert L.nf4_quantize(FAKE, ctypes.byref(weight(q, n=60)), None) == q.NF4_ERR_UNSUPPORTED_SHAPE
+    assert L.nf4_quantize(FAKE, ctypes.byref(weight(q, k=96)), None) == q.NF4_ERR_UNSUPPORTED_SHAPE
+    assert L.nf4_quantize(None, ctypes.byref(weight(q)), None) == q.NF4_ERR_INVALID_ARG
+    assert L.nf4_quantize(FAKE + 4, ctypes.byref(weight(q)), None) == q.NF4_ERR_ALIGNMENT
+    assert L.nf4_quantize(FAKE, ctypes.byref(weight(q, codes=FAKE + 8)), None) == q.NF4_ERR_ALIGNMENT
+    assert L.nf4_quantize(FAKE, ctypes.byref(weight(q, dq=1, q8=None)), None) == q.NF4_ERR_INVALID_ARG
+    assert L.nf4_dequantize(ctypes.byref(weight(q)), FAKE, 2, None) == q.NF4_ERR_INVALID_ARG
+    assert L.nf4_dequantize(ctypes.byref(weight(q)), FAKE + 2, 1, None) == q.NF4_ERR_ALIGNMENT
+
+
+def test_layer_argument_checks(q):
+    w = weight(q)
+    assert call_fwd(q, w, r=7) == q.NF4_ERR_UNSUPPORTED_SHAPE
+    assert call_fwd(q, w, r=0) == q.NF4_ERR_UNSUPPORTED_SHAPE
+    assert call_fwd(q, w, r=136) == q.NF4_ERR_UNSUPPORTED_SHAPE
+    assert call_fwd(q, w, alpha=float("nan")) == q.NF4_ERR_INVALID_ARG
+    assert call_fwd(q, w, alpha=float("inf")) == q.NF4_ERR_INVALID_ARG
+    assert call_fwd(q, w, M=-1) == q.NF4_ERR_UNSUPPORTED_SHAPE
+    assert call_fwd(q, w, A=None) == q.NF4_ERR_INVALID_ARG
+    assert call_fwd(q, w, x=FAKE + 2) == q.NF4_ERR_ALIGNMENT
+    assert call_fwd(q, w, h=None) == q.NF4_ERR_INVALID_ARG
+    assert call_fwd(q, w, ws=None) == q.NF4_ERR_WORKSPACE
+    assert call_fwd(q, w, wsb=16) == q.NF4_ERR_WORKSPACE
+    assert call_fwd(q, w, ws=FAKE + 16) == q.NF4_ERR_ALIGNMENT
+    assert call_fwd(q, w, M=0) == q.NF4_OK              # empty batch: nothing to launch
+    bw = q.lib.qlora_linear_bwd
+    args = lambda **kw: [ctypes.byref(kw.get("w", w)), FAKE, kw.get("M", 4), FAKE, FAKE,
+                         kw.get("r", 8), 16.0, kw.get("dY", FAKE), None, None,
+                         kw.get("dA", FAKE), kw.get("dB", FAKE), kw.get("ws", FAKE),
+                         kw.get("wsb", 16), None]
+    assert bw(*args(r=12)) == q.NF4_ERR_UNSUPPORTED_SHAPE
+    assert bw(*args(dA=None)) == q.NF4_ERR_INVALID_ARG
+    assert bw(*args(dY=None)) == q.NF4_ERR_INVALID_ARG
+    assert bw(*args(dB=FAKE + 4)) == q.NF4_ERR_ALIGNMENT
+    assert bw(*args(wsb=16)) == q.NF4_ERR_WORKSPACE
+
+
+def test_python_binding_refuses_cpu_tensors(q):
+    import torch
+    W = torch.zeros(64, 64)
+    with pytest.raises(ValueError):
+        q.nf4_quantize(W)

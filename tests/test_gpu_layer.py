@@ -1,0 +1,164 @@
+"""GPU parity of the fused QLoRA forward and backward against the CPU oracle.
+
+Bar (per output tensor): max|gpu - oracle| <= 2e-2 * rms(oracle), with the
+oracle in fp64 from the same bf16 inputs and the same NF4 weight (the GPU's
+own quantisation, already checked bit-exact against the oracle's). The LoRA
+branch is also checked alone (W0 = 0) against its own rms, because at large
+shapes it is only a few percent of h."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-2
+
+
+@pytest.fixture(scope="module")
+def q():
+    import bit_nf4_quantized_05_b200 as mod
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    return mod
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def to_f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def rel_err(got: np.ndarray, ref: np.ndarray) -> float:
+    rms = np.sqrt(np.mean(ref ** 2))
+    return float(np.max(np.abs(got - ref)) / max(rms, 1e-300))
+
+
+def oracle_weight(qw):
+    """The GPU's quantised weight as an oracle Quantized record."""
+    return oracle.Quantized(qw.codes.cpu().numpy(), qw.absmax.cpu().numpy(),
+                            qw.absmax_q8.cpu().numpy()[: qw.n * qw.k // 64] if qw.double_quant else None,
+                            qw.absmax_c.cpu().numpy()[: (qw.n * qw.k // 64 + 255) // 256]
+                            if qw.double_quant else None,
+                            64, qw.double_quant, 256, qw.n * qw.k)
+
+
+def run_layer(q, W0, A, B, x, dY, alpha, dq, rows=None, need_bwd=True):
+    dev = "cuda"
+    qw = q.nf4_quantize(W0.to(dev), double_quant=dq)
+    xd, Ad, Bd = x.to(dev), A.to(dev), B.to(dev)
+    h, u = q.qlora_linear_fwd(qw, xd, Ad, Bd, alpha)
+    out = {"qw": qw, "h": h, "u": u}
+    if need_bwd:
+        dX, dA, dB = q.qlora_linear_bwd(qw, xd, Ad, Bd, alpha, dY.to(dev), u=u)
+        out.update(dX=dX, dA=dA, dB=dB)
+    torch.cuda.synchronize()
+    assert q.device_status() == q.NF4_OK
+    return out
+
+
+def check_against_oracle(q, res, A, B, x, dY, alpha, rows=None, need_bwd=True, tag=""):
+    qw = res["qw"]
+    N, K, r, M = qw.n, qw.k, A.shape[0], x.shape[0]
+    ow = oracle_weight(qw)
+    xb, Ab, Bb = bits(x), bits(A), bits(B)
+    rows = np.arange(M) if rows is None else np.asarray(rows)
+    h_ref, u_ref = oracle.qlora_fwd_rows(ow, N, K, xb, Ab, Bb, r, alpha, rows=rows)
+    errs = {"h": rel_err(to_f64(res["h"])[rows], h_ref),
+            "u": rel_err(res["u"].cpu().numpy().astype(np.float64)[rows], u_ref)}
+    if need_bwd:
+        dX_ref, dA_ref, dB_ref = oracle.qlora_bwd(ow, N, K, xb, Ab, Bb, r, alpha, bits(dY),
+                                                  dx_rows=rows)
+        errs.update(dX=rel_err(to_f64(res["dX"])[rows], dX_ref),
+                    dA=rel_err(to_f64(res["dA"]), dA_ref),
+                    dB=rel_err(to_f64(res["dB"]), dB_ref))
+    bad = {k: v for k, v in errs.items() if not v <= TOL}
+    assert not bad, f"{tag} relative errors over {TOL}: {errs}"
+    return errs
+
+
+SMALL = [
+    # (N, K, M, r, alpha, dq)   several tiles in every dimension, ragged tails
+    (384, 512, 300, 16, 32.0, True),
+    (256, 256, 128, 8, 16.0, False),
+    (520, 640, 77, 64, 16.0, True),
+    (264, 192, 1, 128, 32.0, True),
+    (128, 1088, 513, 32, 8.0, False),
+]
+
+
+@pytest.mark.parametrize("N,K,M,r,alpha,dq", SMALL)
+def test_layer_small_shapes(q, N, K, M, r, alpha, dq):
+    w = workloads.LayerWorkload("t", N, K, M, r, alpha, 0.02, dq, 12345 + N + K + M + r)
+    inp = workloads.make_inputs(w)
+    res = run_layer(q, inp["W0"], inp["A"], inp["B"], inp["x"], inp["dY"], alpha, dq)
+    check_against_oracle(q, res, inp["A"], inp["B"], inp["x"], inp["dY"], alpha,
+                         tag=f"{N}x{K} M={M} r={r}")
+
+
+@pytest.mark.parametrize("r", [8, 64])
+def test_lora_branch_alone(q, r):
+    """W0 = 0: every code is the zero level, h and dX are the LoRA terms only."""
+    N, K, M, alpha = 320, 384, 200, 16.0
+    w = workloads.LayerWorkload("t", N, K, M, r, alpha, 0.02, True, 777 + r)
+    inp = workloads.make_inputs(w)
+    W0 = torch.zeros(N, K)
+    res = run_layer(q, W0, inp["A"], inp["B"], inp["x"], inp["dY"], alpha, True)
+    assert torch.all(res["qw"].codes == 0x77)
+    errs = check_against_oracle(q, res, inp["A"], inp["B"], inp["x"], inp["dY"], alpha,
+                                tag="lora-only")
+    assert float(res["h"].float().abs().max()) > 0
+
+
+def test_b_zero_is_base_only(q):
+    N, K, M, r, alpha = 256, 320, 130, 16, 32.0
+    w = workloads.LayerWorkload("t", N, K, M, r, alpha, 0.02, True, 4242)
+    inp = workloads.make_inputs(w)
+    B0 = torch.zeros_like(inp["B"])
+    res = run_layer(q, inp["W0"], inp["A"], B0, inp["x"], inp["dY"], alpha, True)
+    check_against_oracle(q, res, inp["A"], B0, inp["x"], inp["dY"], alpha, tag="B=0")
+    assert float(res["dA"].float().abs().max()) == 0.0   # v = dY B = 0
+
+
+def test_single_1024_workload(q):
+    w = workloads.WORKLOADS["single_1024"]
+    inp = workloads.make_inputs(w)
+    res = run_layer(q, inp["W0"], inp["A"], inp["B"], inp["x"], inp["dY"], w.alpha, w.double_quant)
+    check_against_oracle(q, res, inp["A"], inp["B"], inp["x"], inp["dY"], w.alpha, tag=w.name)
+
+
+def sampled_rows(M, count, seed):
+    rng = np.random.default_rng(seed)
+    rows = rng.choice(M, size=min(count, M), replace=False)
+    rows[:2] = [0, M - 1]
+    return np.sort(rows)
+
+
+def test_llama13b_attention_full_size(q):
+    w = workloads.WORKLOADS["llama13b_attn_5120"]
+    inp = workloads.make_inputs(w)
+    res = run_layer(q, inp["W0"], inp["A"], inp["B"], inp["x"], inp["dY"], w.alpha, w.double_quant)
+    check_against_oracle(q, res, inp["A"], inp["B"], inp["x"], inp["dY"], w.alpha,
+                         rows=sampled_rows(w.M, 48, 1), tag=w.name)
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_decode_workload_full_size(q, M):
+    w = workloads.WORKLOADS["decode_mlp_up_13824x5120"]
+    inp = workloads.make_inputs(w, M=M)
+    res = run_layer(q, inp["W0"], inp["A"], inp["B"], inp["x"], None, w.alpha, w.double_quant,
+                    need_bwd=False)
+    check_against_oracle(q, res, inp["A"], inp["B"], inp["x"], None, w.alpha, need_bwd=False,
+                         tag=f"{w.name} M={M}")
+
+
+@pytest.mark.slow
+def test_llama2_70b_mlp_full_size(q):
+    w = workloads.WORKLOADS["llama2_70b_mlp_28672x8192"]
+    inp = workloads.make_inputs(w)
+    res = run_layer(q, inp["W0"], inp["A"], inp["B"], inp["x"], inp["dY"], w.alpha, w.double_quant)
+    check_against_oracle(q, res, inp["A"], inp["B"], inp["x"], inp["dY"], w.alpha,
+                         rows=sampled_rows(w.M, 12, 2), tag=w.name)
