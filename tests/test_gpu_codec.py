@@ -89,17 +89,17 @@ def test_quantize_midpoints_and_special_blocks(q):
 
 def test_quantize_dense_fp32_sweep(q):
     """Every 97th fp32 bit pattern in [0, 1] and its negative, against a unit
-    absmax, plus +-1 neighbours of every midpoint: the code is a monotone step
-    function of w', so agreement at and around all 15 steps and on a dense
-    sweep between them leaves no room for a different mapping."""
+    absmax (so w' == w). Together with the midpoint test (every step of the
+    monotone code function and its fp32 neighbours) this leaves no room for a
+    different mapping."""
     one = np.float32(1.0).view(np.uint32)
     pos = np.arange(0, int(one), 97, dtype=np.uint32).view(np.float32)
     vals = np.concatenate([pos, -pos])
     pad = (-vals.size) % 63
     vals = np.concatenate([vals, np.zeros(pad, dtype=np.float32)]).reshape(-1, 63)
     W = np.concatenate([np.ones((vals.shape[0], 1), dtype=np.float32), vals], axis=1)
-    rows = W.shape[0]
-    W = W[: rows - rows % 8].reshape(-1, 64 * 8)        # 8 blocks per row, k = 512
+    blocks = W.shape[0]
+    W = W[: blocks - blocks % 64].reshape(-1, 64 * 8)   # 8 blocks per row, rows % 8 == 0
     ref, qw = quant_both(q, W, False)
     assert np.array_equal(qw.codes.cpu().numpy(), ref.codes)
 

@@ -4,7 +4,13 @@ Bar (per output tensor): max|gpu - oracle| <= 2e-2 * rms(oracle), with the
 oracle in fp64 from the same bf16 inputs and the same NF4 weight (the GPU's
 own quantisation, already checked bit-exact against the oracle's). The LoRA
 branch is also checked alone (W0 = 0) against its own rms, because at large
-shapes it is only a few percent of h."""
+shapes it is only a few percent of h.
+
+The outputs are bf16, so rounding the exact result alone costs up to 2^-9 of
+each value. For the edge shapes below (one token, an outer-product dA/dB)
+max|y| / rms(y) exceeds 10 and that rounding by itself reaches the bar, so
+those cases add an element-wise allowance of 2^-8 * |oracle| (one bf16 ulp)
+to it. The named workloads use the bar as stated."""
 import numpy as np
 import pytest
 import torch
@@ -32,9 +38,13 @@ def to_f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
-def rel_err(got: np.ndarray, ref: np.ndarray) -> float:
-    rms = np.sqrt(np.mean(ref ** 2))
-    return float(np.max(np.abs(got - ref)) / max(rms, 1e-300))
+def rel_err(got: np.ndarray, ref: np.ndarray, ulp_allowance: bool = False) -> float:
+    """max over elements of |got - ref| / (TOL-scaled bar); <= TOL passes."""
+    rms = max(np.sqrt(np.mean(ref ** 2)), 1e-300)
+    if not ulp_allowance:
+        return float(np.max(np.abs(got - ref)) / rms)
+    # |got - ref| <= TOL*rms + 2^-8 |ref|  <=>  excess/rms <= TOL
+    return float(np.max(np.abs(got - ref) - 2.0 ** -8 * np.abs(ref)) / rms)
 
 
 def oracle_weight(qw):
@@ -60,21 +70,22 @@ def run_layer(q, W0, A, B, x, dY, alpha, dq, rows=None, need_bwd=True):
     return out
 
 
-def check_against_oracle(q, res, A, B, x, dY, alpha, rows=None, need_bwd=True, tag=""):
+def check_against_oracle(q, res, A, B, x, dY, alpha, rows=None, need_bwd=True, tag="",
+                         edge=False):
     qw = res["qw"]
     N, K, r, M = qw.n, qw.k, A.shape[0], x.shape[0]
     ow = oracle_weight(qw)
     xb, Ab, Bb = bits(x), bits(A), bits(B)
     rows = np.arange(M) if rows is None else np.asarray(rows)
     h_ref, u_ref = oracle.qlora_fwd_rows(ow, N, K, xb, Ab, Bb, r, alpha, rows=rows)
-    errs = {"h": rel_err(to_f64(res["h"])[rows], h_ref),
+    errs = {"h": rel_err(to_f64(res["h"])[rows], h_ref, edge),
             "u": rel_err(res["u"].cpu().numpy().astype(np.float64)[rows], u_ref)}
     if need_bwd:
         dX_ref, dA_ref, dB_ref = oracle.qlora_bwd(ow, N, K, xb, Ab, Bb, r, alpha, bits(dY),
                                                   dx_rows=rows)
-        errs.update(dX=rel_err(to_f64(res["dX"])[rows], dX_ref),
-                    dA=rel_err(to_f64(res["dA"]), dA_ref),
-                    dB=rel_err(to_f64(res["dB"]), dB_ref))
+        errs.update(dX=rel_err(to_f64(res["dX"])[rows], dX_ref, edge),
+                    dA=rel_err(to_f64(res["dA"]), dA_ref, edge),
+                    dB=rel_err(to_f64(res["dB"]), dB_ref, edge))
     bad = {k: v for k, v in errs.items() if not v <= TOL}
     assert not bad, f"{tag} relative errors over {TOL}: {errs}"
     return errs
@@ -96,7 +107,7 @@ def test_layer_small_shapes(q, N, K, M, r, alpha, dq):
     inp = workloads.make_inputs(w)
     res = run_layer(q, inp["W0"], inp["A"], inp["B"], inp["x"], inp["dY"], alpha, dq)
     check_against_oracle(q, res, inp["A"], inp["B"], inp["x"], inp["dY"], alpha,
-                         tag=f"{N}x{K} M={M} r={r}")
+                         tag=f"{N}x{K} M={M} r={r}", edge=M < 16)
 
 
 @pytest.mark.parametrize("r", [8, 64])
