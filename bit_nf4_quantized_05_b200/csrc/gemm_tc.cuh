@@ -23,7 +23,7 @@
 //   warp 1        TMEM owner + MMA issuer (one thread)
 //   warps 4..7    epilogue: TMEM -> registers -> bf16 -> global
 //   warps 8..15   dequantisation
-// Pipelines: kStages shared-memory stages (full / dequantised / empty
+// Pipelines: a ring of shared-memory stages (full / dequantised / empty
 // mbarriers) and two TMEM accumulator buffers (full / empty), so the
 // epilogue of one tile overlaps the main loop of the next.
 #pragma once
@@ -34,7 +34,6 @@ namespace nf4 {
 
 constexpr int kBM = 128;            // tokens per tile = MMA M
 constexpr int kBK = 64;             // reduction per stage = one NF4 block
-constexpr int kStages = 3;
 constexpr int kGemmThreads = 512;
 constexpr int kDequantWarp0 = 8;
 constexpr int kDequantWarps = 8;
@@ -63,11 +62,13 @@ struct GemmCfg {
     static constexpr int kBBytes = BN * kBK * 2;         // BN rows of 128 B
     static constexpr int kCBytes = BN * kBK / 2;         // 4-bit codes of the B tile
     static constexpr int kStageBytes = kABytes + kBBytes + kCBytes;
+    static constexpr int kStages = (220 * 1024) / kStageBytes > 6 ? 6 : (220 * 1024) / kStageBytes;
     static constexpr int kTmemCols = (2 * BN <= 256) ? 256 : 512;
     static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
     static constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, BN, 0, DGRAD ? 1 : 0);
     static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
     static_assert(kStageBytes % 1024 == 0, "stage alignment");
+    static_assert(kStages >= 3, "pipeline depth");
 };
 
 template <int BN, bool DGRAD>
@@ -81,14 +82,14 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red] bf1
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
-    uint8_t *slot_a = smem;                                        // [kStages][kABytes]
-    uint8_t *slot_b = smem + kStages * Cfg::kABytes;               // [kStages][kBBytes]
-    uint8_t *slot_c = slot_b + kStages * Cfg::kBBytes;             // [kStages][kCBytes]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(slot_c + kStages * Cfg::kCBytes);
+    uint8_t *slot_a = smem;                                        // [Cfg::kStages][kABytes]
+    uint8_t *slot_b = smem + Cfg::kStages * Cfg::kABytes;               // [Cfg::kStages][kBBytes]
+    uint8_t *slot_c = slot_b + Cfg::kStages * Cfg::kBBytes;             // [Cfg::kStages][kCBytes]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(slot_c + Cfg::kStages * Cfg::kCBytes);
     uint64_t *full = bars;                   // TMA landed         (count 1 + tx)
-    uint64_t *bfull = bars + kStages;        // B tile ready       (count kDequantWarps)
-    uint64_t *empty = bars + 2 * kStages;    // MMA done with slot (count 1, tcgen05.commit)
-    uint64_t *acc_full = bars + 3 * kStages; // [2] accumulator complete
+    uint64_t *bfull = bars + Cfg::kStages;        // B tile ready       (count kDequantWarps)
+    uint64_t *empty = bars + 2 * Cfg::kStages;    // MMA done with slot (count 1, tcgen05.commit)
+    uint64_t *acc_full = bars + 3 * Cfg::kStages; // [2] accumulator complete
     uint64_t *acc_empty = acc_full + 2;      // [2] accumulator drained (count 4)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -96,7 +97,7 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red] bf1
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < Cfg::kStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&bfull[s], kDequantWarps);
             mbar_init(&empty[s], 1);
@@ -139,10 +140,14 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red] bf1
                 if (it < args.main_steps) {
                     mbar_arrive_expect_tx(&full[st], Cfg::kABytes + Cfg::kCBytes);
                     tma_load_2d(a, &tm_act, &full[st], it * kBK, m0);
-                    if (!DGRAD)
+                    if (!DGRAD) {
                         tma_load_2d(c, &tm_codes, &full[st], it * (kBK / 2), n0);
-                    else
-                        tma_load_2d(c, &tm_codes, &full[st], n0 / 2, it * kBK);
+                    } else {
+#pragma unroll
+                        for (int kb = 0; kb < BN / 64; ++kb)
+                            tma_load_2d(c + kb * 2048, &tm_codes, &full[st], n0 / 2 + kb * 32,
+                                        it * kBK);
+                    }
                 } else {
                     const int ls = it - args.main_steps;
                     mbar_arrive_expect_tx(&full[st], Cfg::kABytes + Cfg::kBBytes);
@@ -155,7 +160,7 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red] bf1
                             tma_load_2d(b + ma * 8192, &tm_lb, &full[st], n0 + ma * 64, ls * kBK);
                     }
                 }
-                if (++st == kStages) { st = 0; ph ^= 1; }
+                if (++st == Cfg::kStages) { st = 0; ph ^= 1; }
             }
         }
     } else if (warp == 1 && lane == 0) {
@@ -183,7 +188,7 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red] bf1
                     umma_bf16_ss(d_tmem, ad, bd, Cfg::kIdesc, (it > 0 || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(&empty[st]);
-                if (++st == kStages) { st = 0; ph ^= 1; }
+                if (++st == Cfg::kStages) { st = 0; ph ^= 1; }
             }
             umma_commit(&acc_full[ab]);
             if (++ab == 2) { ab = 0; aph ^= 1; }
@@ -230,76 +235,91 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red] bf1
         }
     } else if (warp >= kDequantWarp0) {
         // -------------------------------------------------- dequantisation
-        const int i = threadIdx.x - kDequantWarp0 * 32;   // work item of this thread, 0..255
+        // Work item of this thread: forward: W row n0 + i (one block per
+        // stage); dgrad: reduction row r_loc of the stage and output block kb.
+        // Eight consecutive lanes always take eight consecutive rows of one
+        // 8-row swizzle atom, so their 16-byte stores hit distinct banks.
+        const int i = threadIdx.x - kDequantWarp0 * 32;
         const bool active = i < BN;
-        // forward: item = W row (n0 + i), block `it`
-        // dgrad:   item = (reduction row i / (BN/64), output block i % (BN/64))
-        constexpr int kBPR = BN / 64;                     // blocks per dgrad code row
-        const int r_loc = DGRAD ? i / kBPR : i;
-        const int kb = DGRAD ? i % kBPR : 0;
+        constexpr int kBPR = BN / 64;
+        const int kb = DGRAD ? (i / 8) % kBPR : 0;
+        const int r_loc = DGRAD ? (i / (8 * kBPR)) * 8 + (i & 7) : i;
         const uint32_t row_off = DGRAD ? static_cast<uint32_t>(kb * 8192 + r_loc * 128)
                                        : static_cast<uint32_t>(i * 128);
-        const uint32_t code_off = DGRAD ? static_cast<uint32_t>(r_loc * (BN / 2) + kb * 32)
+        // codes tiles carry the 32-byte TMA swizzle: 16-byte chunk h of row j
+        // sits at chunk h ^ ((j >> 2) & 1)
+        const uint32_t code_off = DGRAD ? static_cast<uint32_t>(kb * 2048 + r_loc * 32)
                                         : static_cast<uint32_t>(i * 32);
+        const uint32_t cswz = static_cast<uint32_t>((r_loc >> 2) & 1);
         const uint32_t swz = static_cast<uint32_t>(r_loc & 7);
-        const int hswap = (lane >> 2) & 1;                // spreads code reads over banks
+
+        // raw scale inputs of one (tile, step), loaded one step ahead
+        struct RawScale { uint32_t q8; float v; bool valid; };
+        auto load_scale = [&](int tile, int it) -> RawScale {
+            RawScale rs{0u, 0.0f, false};
+            if (tile >= total_tiles || it >= args.main_steps || !active) return rs;
+            const int n0 = (tile / args.m_tiles) * BN;
+            int64_t wrow, wblk;
+            if (!DGRAD) {
+                wrow = n0 + i;
+                wblk = it;
+            } else {
+                wrow = static_cast<int64_t>(it) * kBK + r_loc;
+                wblk = n0 / 64 + kb;
+            }
+            if (wrow >= args.Nw || wblk >= args.kblocks) return rs;
+            const int64_t b = wrow * args.kblocks + wblk;
+            rs.valid = true;
+            if (args.dq) {
+                rs.q8 = __ldg(args.q8 + b);
+                rs.v = __ldg(args.cg + (b >> 8));
+            } else {
+                rs.v = __ldg(args.absmax + b);
+            }
+            return rs;
+        };
+
         int st = 0;
         uint32_t ph = 0;
-        for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-            const int n0 = (tile / args.m_tiles) * BN;
-            for (int it = 0; it < nsteps; ++it) {
-                const bool main = it < args.main_steps;
-                // issue the scale load before waiting so its latency overlaps the wait
-                float s = 0.0f;
-                bool valid = false;
-                if (main && active) {
-                    int64_t wrow, wblk;
-                    if (!DGRAD) {
-                        wrow = n0 + i;
-                        wblk = it;
-                    } else {
-                        wrow = static_cast<int64_t>(it) * kBK + r_loc;
-                        wblk = n0 / 64 + kb;
-                    }
-                    valid = wrow < args.Nw && wblk < args.kblocks;
-                    if (valid) {
-                        const int64_t b = wrow * args.kblocks + wblk;
-                        if (args.dq) {
-                            const float kg = __fdiv_rn(__ldg(args.cg + (b >> 8)), 127.0f);
-                            s = __fmul_rn(static_cast<float>(__ldg(args.q8 + b)), kg);
-                        } else {
-                            s = __ldg(args.absmax + b);
-                        }
-                    }
-                }
-                if (!mbar_wait(&full[st], ph, abort_flag)) goto done;
-                if (main && active) {
-                    const uint8_t *cp = slot_c + st * Cfg::kCBytes + code_off;
-                    const uint4 h0 = *reinterpret_cast<const uint4 *>(cp + 16 * hswap);
-                    const uint4 h1 = *reinterpret_cast<const uint4 *>(cp + 16 * (hswap ^ 1));
-                    const uint4 c0 = hswap ? h1 : h0, c1 = hswap ? h0 : h1;
-                    const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                    uint8_t *brow = slot_b + st * Cfg::kBBytes + row_off;
-                    if (valid) {
-                        const BlockLut L = make_block_lut(s);
+        int tile = blockIdx.x, it = 0;
+        RawScale nxt = load_scale(tile, it);
+        while (tile < total_tiles) {
+            const RawScale cur = nxt;
+            const bool main = it < args.main_steps;
+            // advance to the next (tile, step) and start its scale load now
+            int ntile = tile, nit = it + 1;
+            if (nit == nsteps) { nit = 0; ntile += gridDim.x; }
+            nxt = load_scale(ntile, nit);
+            if (!mbar_wait(&full[st], ph, abort_flag)) goto done;
+            if (main && active) {
+                const uint8_t *cp = slot_c + st * Cfg::kCBytes + code_off;
+                const uint4 c0 = *reinterpret_cast<const uint4 *>(cp + 16 * cswz);
+                const uint4 c1 = *reinterpret_cast<const uint4 *>(cp + 16 * (cswz ^ 1));
+                const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                uint8_t *brow = slot_b + st * Cfg::kBBytes + row_off;
+                if (cur.valid) {
+                    float s = cur.v;
+                    if (args.dq) s = __fmul_rn(static_cast<float>(cur.q8), __fdiv_rn(cur.v, 127.0f));
+                    const BlockLut L = make_block_lut(s);
 #pragma unroll
-                        for (int ch = 0; ch < 8; ++ch) {
-                            uint32_t o[4];
-                            dequant8(L, words[ch], o);
-                            *reinterpret_cast<uint4 *>(brow + ((ch ^ swz) << 4)) =
-                                make_uint4(o[0], o[1], o[2], o[3]);
-                        }
-                    } else {
-#pragma unroll
-                        for (int ch = 0; ch < 8; ++ch)
-                            *reinterpret_cast<uint4 *>(brow + (ch << 4)) = make_uint4(0, 0, 0, 0);
+                    for (int ch = 0; ch < 8; ++ch) {
+                        uint32_t o[4];
+                        dequant8(L, words[ch], o);
+                        *reinterpret_cast<uint4 *>(brow + ((ch ^ swz) << 4)) =
+                            make_uint4(o[0], o[1], o[2], o[3]);
                     }
-                    fence_proxy_async_smem();
+                } else {
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch)
+                        *reinterpret_cast<uint4 *>(brow + (ch << 4)) = make_uint4(0, 0, 0, 0);
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bfull[st]);
-                if (++st == kStages) { st = 0; ph ^= 1; }
+                fence_proxy_async_smem();
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bfull[st]);
+            if (++st == Cfg::kStages) { st = 0; ph ^= 1; }
+            tile = ntile;
+            it = nit;
         }
     }
 done:

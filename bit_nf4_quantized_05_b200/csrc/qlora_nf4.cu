@@ -15,7 +15,7 @@
 
 #include "codec.cuh"
 #include "gemm_tc.cuh"
-#include "lora_small.cuh"
+#include "skinny_tc.cuh"
 
 using namespace nf4;
 
@@ -32,12 +32,12 @@ constexpr int kMaxDevices = 64;
 // Optional per-kernel event timing (nf4_profiling / nf4_profile_read)
 // ---------------------------------------------------------------------------
 enum KernelKind {
-    KK_QUANTIZE, KK_DEQUANTIZE, KK_ROWDOT, KK_COLPROD, KK_COLREDUCE, KK_TRANSPOSE, KK_ZERO,
-    KK_GEMM_FWD, KK_GEMM_DGRAD, KK_COUNT
+    KK_QUANTIZE, KK_DEQUANTIZE, KK_LORA_U, KK_LORA_V, KK_LORA_DB, KK_LORA_DA, KK_LORA_REDUCE,
+    KK_SCALE, KK_ZERO, KK_GEMM_FWD, KK_GEMM_DGRAD, KK_COUNT
 };
 const char *const kKindNames[KK_COUNT] = {
-    "nf4_quantize", "nf4_dequantize", "lora_rowdot", "lora_colprod", "lora_colreduce",
-    "lora_transpose", "zero_fill", "qlora_gemm_fwd", "qlora_gemm_dgrad"};
+    "nf4_quantize", "nf4_dequantize", "lora_u", "lora_v", "lora_dB", "lora_dA", "lora_reduce",
+    "lora_scale", "zero_fill", "qlora_gemm_fwd", "qlora_gemm_dgrad"};
 
 struct ProfRecord {
     int kind;
@@ -183,32 +183,116 @@ nf4_status check_layer(const nf4_weight *w, const void *x, int64_t M, const void
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
-// Splits of the M dimension for the column products (dB over n, dA over k).
-int col_splits(int64_t M, int64_t C, int sms) {
-    const int64_t tiles = (C + kColTile - 1) / kColTile;
-    int64_t s = (2 * sms + tiles - 1) / tiles;
-    s = std::max<int64_t>(1, std::min<int64_t>(s, (M + 127) / 128));
-    return static_cast<int>(s);
+// Split plan of one rank-r product: P output rows (tiles of 128), Q reduction
+// elements (steps of 64), split so that about two CTAs per SM stream the
+// large operand.
+struct SkinnyPlan {
+    int RN, p_tiles, steps, sps, splits;
+    size_t part_bytes;
+};
+
+SkinnyPlan plan_skinny(int64_t P, int64_t Q, int32_t r, int sms) {
+    SkinnyPlan p{};
+    p.RN = r <= 64 ? 64 : 128;
+    p.p_tiles = static_cast<int>((P + 127) / 128);
+    p.steps = static_cast<int>((Q + 63) / 64);
+    int want = std::max(1, (2 * sms + p.p_tiles - 1) / p.p_tiles);
+    int splits = std::max(1, std::min(want, p.steps));
+    p.sps = (p.steps + splits - 1) / splits;
+    p.splits = std::max(1, (p.steps + p.sps - 1) / p.sps);
+    p.part_bytes = size_t(p.splits) * size_t(P) * p.RN * 4;
+    return p;
+}
+
+struct FwdLayout {
+    size_t us, part, total;
+};
+
+FwdLayout fwd_layout(int64_t M, int64_t n, int64_t k, int32_t r, int sms) {
+    (void)n;
+    FwdLayout L{};
+    size_t off = 0;
+    L.us = off;   off = align256(off + size_t(M) * r * 2);
+    L.part = off; off = align256(off + plan_skinny(M, k, r, sms).part_bytes);
+    L.total = off;
+    return L;
 }
 
 struct BwdLayout {
-    size_t bt, v, vs, u, part, total;
-    int s_dB, s_dA;
+    size_t us, vs, part, total;
 };
 
 BwdLayout bwd_layout(int64_t M, int64_t n, int64_t k, int32_t r, int sms) {
     BwdLayout L{};
     size_t off = 0;
-    L.bt = off;   off = align256(off + size_t(n) * r * 2);
-    L.v = off;    off = align256(off + size_t(M) * r * 4);
+    L.us = off;   off = align256(off + size_t(M) * r * 2);
     L.vs = off;   off = align256(off + size_t(M) * r * 2);
-    L.u = off;    off = align256(off + size_t(M) * r * 4);
-    L.s_dB = col_splits(M, n, sms);
-    L.s_dA = col_splits(M, k, sms);
-    L.part = off;
-    off = align256(off + size_t(std::max(int64_t(L.s_dB) * n, int64_t(L.s_dA) * k)) * r * 4);
+    size_t part = std::max(std::max(plan_skinny(M, k, r, sms).part_bytes,   // u (recompute)
+                                    plan_skinny(M, n, r, sms).part_bytes),  // v
+                           std::max(plan_skinny(n, M, r, sms).part_bytes,   // dB
+                                    plan_skinny(k, M, r, sms).part_bytes)); // dA
+    L.part = off; off = align256(off + part);
     L.total = off;
     return L;
+}
+
+enum class Major { K, MN };
+
+// Rank-r product out[p][j] = sum_q P(p,q) Q(q,j) through the skinny tcgen05
+// kernel, then the ordered split reduction.
+//   a: row-major bf16 [a_rows, a_cols]; K-major: p = row, q = col; MN-major: q = row, p = col
+//   b: row-major bf16 [b_rows, b_cols]; K-major: j = row, q = col; MN-major: q = row, j = col
+nf4_status skinny_product(int kind, const void *a, int64_t a_rows, int64_t a_cols, Major am,
+                          const void *b, int64_t b_rows, int64_t b_cols, Major bm, int32_t r,
+                          float *part, float *out_f32, uint16_t *out_bf16, float scale,
+                          int transposed, cudaStream_t stream) {
+    const int sms = num_sms(current_device());
+    const int64_t P = am == Major::K ? a_rows : a_cols;
+    const int64_t Q = am == Major::K ? a_cols : a_rows;
+    const SkinnyPlan pl = plan_skinny(P, Q, r, sms);
+    CUtensorMap ta, tb;
+    bool ok = am == Major::K
+                  ? make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a, a_cols, a_rows, 64, 128,
+                             CU_TENSOR_MAP_SWIZZLE_128B)
+                  : make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a, a_cols, a_rows, 64, 64,
+                             CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && (bm == Major::K
+                    ? make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, b, b_cols, b_rows, 64,
+                               static_cast<uint32_t>(pl.RN), CU_TENSOR_MAP_SWIZZLE_128B)
+                    : make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, b, b_cols, b_rows, 64, 64,
+                               CU_TENSOR_MAP_SWIZZLE_128B));
+    if (!ok) return NF4_ERR_CUDA;
+    SkinnyArgs args{static_cast<int>(P), pl.steps, pl.sps, part};
+    dim3 grid(static_cast<unsigned>(pl.p_tiles), static_cast<unsigned>(pl.splits));
+    {
+        LaunchTimer t(kind, stream);
+#define NF4_SKINNY_CASE(RN_, AMN, BMN)                                                      \
+    if (pl.RN == RN_ && (am == Major::MN) == AMN && (bm == Major::MN) == BMN) {             \
+        auto kern = skinny_gemm_kernel<RN_, AMN, BMN>;                                      \
+        NF4_TRY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                                          SkCfg<RN_, AMN, BMN>::kSmemBytes));               \
+        kern<<<grid, kSkThreads, SkCfg<RN_, AMN, BMN>::kSmemBytes, stream>>>(ta, tb, args); \
+    }
+        NF4_SKINNY_CASE(64, false, false)
+        NF4_SKINNY_CASE(128, false, false)
+        NF4_SKINNY_CASE(64, false, true)
+        NF4_SKINNY_CASE(128, false, true)
+        NF4_SKINNY_CASE(64, true, true)
+        NF4_SKINNY_CASE(128, true, true)
+#undef NF4_SKINNY_CASE
+        t.stop();
+    }
+    NF4_TRY_CUDA(cudaGetLastError());
+    const int64_t total = P * r;
+    const int rgrid = static_cast<int>(std::min<int64_t>((total + 255) / 256, int64_t(sms) * 8));
+    {
+        LaunchTimer t(KK_LORA_REDUCE, stream);
+        skinny_reduce_kernel<<<rgrid, 256, 0, stream>>>(part, pl.splits, static_cast<int>(P), pl.RN,
+                                                        r, out_f32, out_bf16, scale, transposed);
+        t.stop();
+    }
+    NF4_TRY_CUDA(cudaGetLastError());
+    return NF4_OK;
 }
 
 template <int BN, bool DGRAD>
@@ -220,12 +304,11 @@ nf4_status launch_gemm(const nf4_weight *w, const uint16_t *act, int64_t M, int6
     const int64_t N = w->n, K = w->k;
     bool ok = make_map(&tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, act, red, M, kBK, kBM,
                        CU_TENSOR_MAP_SWIZZLE_128B);
-    if (!DGRAD)
-        ok = ok && make_map(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, K / 2, N,
-                            kBK / 2, BN, CU_TENSOR_MAP_SWIZZLE_NONE);
-    else
-        ok = ok && make_map(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, K / 2, N,
-                            BN / 2, kBK, CU_TENSOR_MAP_SWIZZLE_NONE);
+    // 4-bit codes: one 32-byte block column per box (BN rows forward, 64 rows
+    // dgrad), 32-byte swizzle so that eight lanes reading eight rows hit
+    // distinct banks
+    ok = ok && make_map(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, K / 2, N, kBK / 2,
+                        DGRAD ? kBK : BN, CU_TENSOR_MAP_SWIZZLE_32B);
     ok = ok && make_map(&tm_la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, la, r, M, kBK, kBM,
                         CU_TENSOR_MAP_SWIZZLE_128B);
     if (!DGRAD)  // B [N, r]: rows n, K-major over j
@@ -265,36 +348,30 @@ nf4_status launch_gemm(const nf4_weight *w, const uint16_t *act, int64_t M, int6
     return NF4_OK;
 }
 
-nf4_status launch_rowdot(const uint16_t *P, const uint16_t *Q, int64_t M, int64_t Kd, int32_t r,
-                         float *out_f32, uint16_t *out_bf16, float scale, cudaStream_t stream) {
-    if (M == 0) return NF4_OK;
-    const int grid = static_cast<int>((M + kRowdotRows - 1) / kRowdotRows);
-    LaunchTimer t(KK_ROWDOT, stream);
-    rowdot_kernel<<<grid, 256, 0, stream>>>(P, Q, static_cast<int>(M), static_cast<int>(Kd), r,
-                                            out_f32, out_bf16, scale);
-    t.stop();
-    NF4_TRY_CUDA(cudaGetLastError());
-    return NF4_OK;
+// Output-column tile: the candidate with the smallest (rounds of tiles over
+// the SMs) x (tile width), i.e. the least per-SM time under even tiles.
+int pick_bn(int64_t M, int64_t out, int sms) {
+    const int64_t m_tiles = (M + kBM - 1) / kBM;
+    int best = 256;
+    int64_t best_cost = -1;
+    for (int bn : {256, 192}) {
+        const int64_t tiles = m_tiles * ((out + bn - 1) / bn);
+        const int64_t cost = ((tiles + sms - 1) / sms) * bn;
+        if (best_cost < 0 || cost < best_cost) {
+            best = bn;
+            best_cost = cost;
+        }
+    }
+    return best;
 }
 
-nf4_status launch_colprod(const uint16_t *P, const float *U, int64_t M, int64_t C, int32_t r,
-                          int S, float *part, float scale, int transposed, uint16_t *out,
-                          cudaStream_t stream) {
-    const int rows_per_split = static_cast<int>((M + S - 1) / S);
-    dim3 grid(static_cast<unsigned>((C + kColTile - 1) / kColTile), static_cast<unsigned>(S));
-    LaunchTimer t1(KK_COLPROD, stream);
-    colprod_partial_kernel<<<grid, 256, 0, stream>>>(P, U, static_cast<int>(M),
-                                                     static_cast<int>(C), r, rows_per_split, part);
-    t1.stop();
-    NF4_TRY_CUDA(cudaGetLastError());
-    const int64_t total = C * r;
-    const int rgrid = static_cast<int>(std::min<int64_t>((total + 255) / 256, 4096));
-    LaunchTimer t2(KK_COLREDUCE, stream);
-    colprod_reduce_kernel<<<rgrid, 256, 0, stream>>>(part, S, static_cast<int>(C), r, scale,
-                                                     transposed, out);
-    t2.stop();
-    NF4_TRY_CUDA(cudaGetLastError());
-    return NF4_OK;
+template <bool DGRAD>
+nf4_status launch_gemm_auto(const nf4_weight *w, const uint16_t *act, int64_t M, int64_t red,
+                            int64_t out, const uint16_t *la, int32_t r, const uint16_t *lb,
+                            uint16_t *D, cudaStream_t stream) {
+    if (pick_bn(M, out, num_sms(current_device())) == 192)
+        return launch_gemm<192, DGRAD>(w, act, M, red, out, la, r, lb, D, stream);
+    return launch_gemm<256, DGRAD>(w, act, M, red, out, la, r, lb, D, stream);
 }
 
 }  // namespace
@@ -390,10 +467,8 @@ nf4_status nf4_dequantize(const nf4_weight *w, void *out, int32_t out_bf16, void
 }
 
 size_t qlora_fwd_workspace_bytes(int64_t M, int64_t n, int64_t k, int32_t r) {
-    (void)n;
-    (void)k;
-    if (M <= 0 || r <= 0) return 256;
-    return align256(size_t(M) * r * 2);
+    if (M <= 0 || n <= 0 || k <= 0 || r <= 0) return 256;
+    return fwd_layout(M, n, k, r, num_sms(current_device())).total;
 }
 
 nf4_status qlora_linear_fwd(const nf4_weight *w, const uint16_t *x, int64_t M, const uint16_t *A,
@@ -404,14 +479,19 @@ nf4_status qlora_linear_fwd(const nf4_weight *w, const uint16_t *x, int64_t M, c
     if (M == 0) return NF4_OK;
     if (!h) return NF4_ERR_INVALID_ARG;
     if (!aligned16(h) || !aligned16(u_out)) return NF4_ERR_ALIGNMENT;
-    if (!workspace || ws_bytes < qlora_fwd_workspace_bytes(M, w->n, w->k, r)) return NF4_ERR_WORKSPACE;
+    const FwdLayout L = fwd_layout(M, w->n, w->k, r, num_sms(current_device()));
+    if (!workspace || ws_bytes < L.total) return NF4_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return NF4_ERR_ALIGNMENT;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint16_t *u_s = reinterpret_cast<uint16_t *>(ws + L.us);
+    float *part = reinterpret_cast<float *>(ws + L.part);
     const float scale = alpha / static_cast<float>(r);
-    uint16_t *u_s = static_cast<uint16_t *>(workspace);
-    st = launch_rowdot(x, A, M, w->k, r, u_out, u_s, scale, s);
+    // u = x A^T (fp32, optional) and bf16((alpha/r) u) for the up-projection stage
+    st = skinny_product(KK_LORA_U, x, M, w->k, Major::K, A, r, w->k, Major::K, r, part, u_out, u_s,
+                        scale, 0, s);
     if (st != NF4_OK) return st;
-    return launch_gemm<256, false>(w, x, M, w->k, w->n, u_s, r, B, h, s);
+    return launch_gemm_auto<false>(w, x, M, w->k, w->n, u_s, r, B, h, s);
 }
 
 size_t qlora_bwd_workspace_bytes(int64_t M, int64_t n, int64_t k, int32_t r) {
@@ -444,37 +524,37 @@ nf4_status qlora_linear_bwd(const nf4_weight *w, const uint16_t *x, int64_t M, c
     if (!workspace || ws_bytes < L.total) return NF4_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return NF4_ERR_ALIGNMENT;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    uint16_t *Bt = reinterpret_cast<uint16_t *>(ws + L.bt);
-    float *v = reinterpret_cast<float *>(ws + L.v);
+    uint16_t *u_s = reinterpret_cast<uint16_t *>(ws + L.us);
     uint16_t *v_s = reinterpret_cast<uint16_t *>(ws + L.vs);
     float *part = reinterpret_cast<float *>(ws + L.part);
     const float scale = alpha / static_cast<float>(r);
 
-    // v = dY B (fp32) and bf16(s v) for the dgrad LoRA stage
-    {
-        LaunchTimer t(KK_TRANSPOSE, s);
-        transpose_nr_kernel<<<static_cast<int>(std::min<int64_t>((N * r + 255) / 256, 4096)), 256,
-                              0, s>>>(B, static_cast<int>(N), r, Bt);
+    // bf16(s u), from the saved u or recomputed from x
+    if (u) {
+        LaunchTimer t(KK_SCALE, s);
+        scale_to_bf16_kernel<<<static_cast<int>(std::min<int64_t>((M * r + 255) / 256, 4096)), 256,
+                               0, s>>>(u, M * r, scale, u_s);
         t.stop();
-    }
-    NF4_TRY_CUDA(cudaGetLastError());
-    st = launch_rowdot(dY, Bt, M, N, r, v, v_s, scale, s);
-    if (st != NF4_OK) return st;
-    // u = x A^T unless the forward saved it
-    const float *uu = u;
-    if (!uu) {
-        float *ur = reinterpret_cast<float *>(ws + L.u);
-        st = launch_rowdot(x, A, M, K, r, ur, nullptr, 1.0f, s);
+        NF4_TRY_CUDA(cudaGetLastError());
+    } else {
+        st = skinny_product(KK_LORA_U, x, M, K, Major::K, A, r, K, Major::K, r, part, nullptr, u_s,
+                            scale, 0, s);
         if (st != NF4_OK) return st;
-        uu = ur;
     }
-    // dB = s dY^T u  ([N, r]);  dA = s v^T x  ([r, K])
-    st = launch_colprod(dY, uu, M, N, r, L.s_dB, part, scale, 0, dB, s);
+    // v = dY B  ->  bf16(s v)
+    st = skinny_product(KK_LORA_V, dY, M, N, Major::K, B, N, r, Major::MN, r, part, nullptr, v_s,
+                        scale, 0, s);
     if (st != NF4_OK) return st;
-    st = launch_colprod(x, v, M, K, r, L.s_dA, part, scale, 1, dA, s);
+    // dB = dY^T bf16(s u)   ([N, r])
+    st = skinny_product(KK_LORA_DB, dY, M, N, Major::MN, u_s, M, r, Major::MN, r, part, nullptr, dB,
+                        1.0f, 0, s);
+    if (st != NF4_OK) return st;
+    // dA = (x^T bf16(s v))^T   ([r, K])
+    st = skinny_product(KK_LORA_DA, x, M, K, Major::MN, v_s, M, r, Major::MN, r, part, nullptr, dA,
+                        1.0f, 1, s);
     if (st != NF4_OK) return st;
     // dX = dY W~ + bf16(s v) A
-    if (dX) return launch_gemm<256, true>(w, dY, M, N, K, v_s, r, A, dX, s);
+    if (dX) return launch_gemm_auto<true>(w, dY, M, N, K, v_s, r, A, dX, s);
     return NF4_OK;
 }
 
