@@ -72,6 +72,7 @@ def _load() -> ctypes.CDLL:
         "nf4_dequantize": ([W, vp, i32, vp], ctypes.c_int),
         "qlora_fwd_workspace_bytes": ([i64, i64, i64, i32], sz),
         "qlora_linear_fwd": ([W, vp, i64, vp, vp, i32, f32, vp, vp, vp, sz, vp], ctypes.c_int),
+        "qlora_linear_fwd_noalloc": ([W, vp, i64, vp, vp, i32, f32, vp, vp, vp], ctypes.c_int),
         "qlora_bwd_workspace_bytes": ([i64, i64, i64, i32], sz),
         "qlora_linear_bwd": ([W, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, vp, vp, sz, vp],
                              ctypes.c_int),
@@ -198,6 +199,28 @@ def qlora_linear_fwd(qw: QuantizedWeight, x: torch.Tensor, A: torch.Tensor, B: t
     _check(lib.qlora_linear_fwd(ctypes.byref(s), _ptr(x), M, _ptr(A), _ptr(B), r, float(alpha),
                                 _ptr(h), _ptr(u), _ptr(ws), ws.numel(), _stream(x.device)),
            "qlora_linear_fwd")
+    return h, u
+
+
+def qlora_linear_fwd_noalloc(qw: QuantizedWeight, x: torch.Tensor, A: torch.Tensor,
+                             B: torch.Tensor, alpha: float, save_u: bool = True,
+                             h: Optional[torch.Tensor] = None, u: Optional[torch.Tensor] = None
+                             ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """The forward without a workspace argument: the library uses its own fixed
+    4 MiB device scratch, for callers that cannot allocate device memory while
+    they run (see the C header for the token limit). Pass preallocated `h` and
+    `u` to make the call itself allocation-free."""
+    _need_cuda(x, A, B)
+    M = x.shape[0]
+    r = A.shape[0]
+    if h is None:
+        h = torch.empty(M, qw.n, dtype=torch.bfloat16, device=x.device)
+    if u is None and save_u:
+        u = torch.empty(M, r, dtype=torch.float32, device=x.device)
+    s = qw.struct()
+    _check(lib.qlora_linear_fwd_noalloc(ctypes.byref(s), _ptr(x), M, _ptr(A), _ptr(B), r,
+                                        float(alpha), _ptr(h), _ptr(u), _stream(x.device)),
+           "qlora_linear_fwd_noalloc")
     return h, u
 
 

@@ -191,12 +191,13 @@ struct SkinnyPlan {
     size_t part_bytes;
 };
 
-SkinnyPlan plan_skinny(int64_t P, int64_t Q, int32_t r, int sms) {
+SkinnyPlan plan_skinny(int64_t P, int64_t Q, int32_t r, int sms, int max_splits = 0) {
     SkinnyPlan p{};
     p.RN = r <= 64 ? 64 : 128;
     p.p_tiles = static_cast<int>((P + 127) / 128);
     p.steps = static_cast<int>((Q + 63) / 64);
     int want = std::max(1, (2 * sms + p.p_tiles - 1) / p.p_tiles);
+    if (max_splits > 0) want = std::min(want, max_splits);
     int splits = std::max(1, std::min(want, p.steps));
     p.sps = (p.steps + splits - 1) / splits;
     p.splits = std::max(1, (p.steps + p.sps - 1) / p.sps);
@@ -245,11 +246,11 @@ enum class Major { K, MN };
 nf4_status skinny_product(int kind, const void *a, int64_t a_rows, int64_t a_cols, Major am,
                           const void *b, int64_t b_rows, int64_t b_cols, Major bm, int32_t r,
                           float *part, float *out_f32, uint16_t *out_bf16, float scale,
-                          int transposed, cudaStream_t stream) {
+                          int transposed, cudaStream_t stream, int max_splits = 0) {
     const int sms = num_sms(current_device());
     const int64_t P = am == Major::K ? a_rows : a_cols;
     const int64_t Q = am == Major::K ? a_cols : a_rows;
-    const SkinnyPlan pl = plan_skinny(P, Q, r, sms);
+    const SkinnyPlan pl = plan_skinny(P, Q, r, sms, max_splits);
     CUtensorMap ta, tb;
     bool ok = am == Major::K
                   ? make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a, a_cols, a_rows, 64, 128,
@@ -374,6 +375,32 @@ nf4_status launch_gemm_auto(const nf4_weight *w, const uint16_t *act, int64_t M,
     return launch_gemm<256, DGRAD>(w, act, M, red, out, la, r, lb, D, stream);
 }
 
+// ---------------------------------------------------------------------------
+// Fixed device scratch for qlora_linear_fwd_noalloc. It is part of the
+// library's image: every device that loads the library holds these bytes
+// until the process exits, and every call of that entry point on a device
+// shares them.
+// ---------------------------------------------------------------------------
+constexpr size_t kStaticScratchBytes = size_t(4) << 20;   // 4 MiB
+__device__ __align__(256) uint8_t g_fwd_static_scratch[kStaticScratchBytes];
+
+// Device address of the static scratch on the current device. Host code may
+// not use the array's name as a pointer (it names a host-side stand-in), so
+// the address is looked up once per device with that device current.
+void *static_scratch_on_current_device() {
+    static std::mutex mu;
+    static void *addr[kMaxDevices] = {nullptr};
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> g(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_fwd_static_scratch) != cudaSuccess) return nullptr;
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
 }  // namespace
 
 extern "C" {
@@ -490,6 +517,33 @@ nf4_status qlora_linear_fwd(const nf4_weight *w, const uint16_t *x, int64_t M, c
     // u = x A^T (fp32, optional) and bf16((alpha/r) u) for the up-projection stage
     st = skinny_product(KK_LORA_U, x, M, w->k, Major::K, A, r, w->k, Major::K, r, part, u_out, u_s,
                         scale, 0, s);
+    if (st != NF4_OK) return st;
+    return launch_gemm_auto<false>(w, x, M, w->k, w->n, u_s, r, B, h, s);
+}
+
+nf4_status qlora_linear_fwd_noalloc(const nf4_weight *w, const uint16_t *x, int64_t M,
+                                    const uint16_t *A, const uint16_t *B, int32_t r, float alpha,
+                                    uint16_t *h, float *u_out, void *stream) {
+    nf4_status st = check_layer(w, x, M, A, B, r, alpha);
+    if (st != NF4_OK) return st;
+    if (M == 0) return NF4_OK;
+    if (!h) return NF4_ERR_INVALID_ARG;
+    if (!aligned16(h) || !aligned16(u_out)) return NF4_ERR_ALIGNMENT;
+    // scratch: bf16 (alpha/r) x A^T [M, r], then fp32 partial sums of x A^T
+    // [splits, M, RN] with as many splits as fit (at least one)
+    const size_t us_bytes = align256(size_t(M) * r * 2);
+    const size_t part_row = size_t(M) * (r <= 64 ? 64 : 128) * 4;
+    if (us_bytes >= kStaticScratchBytes || part_row > kStaticScratchBytes - us_bytes)
+        return NF4_ERR_UNSUPPORTED_SHAPE;
+    const int max_splits = static_cast<int>((kStaticScratchBytes - us_bytes) / part_row);
+    uint8_t *ws = static_cast<uint8_t *>(static_scratch_on_current_device());
+    if (!ws) return NF4_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint16_t *u_s = reinterpret_cast<uint16_t *>(ws);
+    float *part = reinterpret_cast<float *>(ws + us_bytes);
+    const float scale = alpha / static_cast<float>(r);
+    st = skinny_product(KK_LORA_U, x, M, w->k, Major::K, A, r, w->k, Major::K, r, part, u_out, u_s,
+                        scale, 0, s, max_splits);
     if (st != NF4_OK) return st;
     return launch_gemm_auto<false>(w, x, M, w->k, w->n, u_s, r, B, h, s);
 }

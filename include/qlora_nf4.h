@@ -129,6 +129,33 @@ QLORA_API nf4_status qlora_linear_fwd(const nf4_weight *w, const uint16_t *x, in
                             uint16_t *h, float *u_out, void *workspace, size_t ws_bytes,
                             void *stream);
 
+/* The forward of qlora_linear_fwd for callers that cannot allocate device
+ * memory at call time: processes that reserve their whole memory budget at
+ * start-up and forbid later allocations (for example a serving process that
+ * has handed every free byte to its own pool), or code that runs inside a
+ * memory allocator's own callback, where calling cudaMalloc would re-enter
+ * it. Instead of a caller-provided workspace it uses a fixed 4 MiB scratch
+ * array that is part of this library's device image: every GPU that loads
+ * the library holds those 4 MiB until the process exits. No pages give this
+ * entry point: it is an interface variant of this library, not part of the
+ * method.
+ *   - Same arguments and results as qlora_linear_fwd, minus the workspace.
+ *   - Limit: M * (2 r + 4 RN) bytes must fit in 4 MiB, with RN = 64 for
+ *     r <= 64 and 128 otherwise (about 14.5 K tokens at r = 16, 10.9 K at
+ *     r = 64, 5.4 K at r = 128); larger M returns
+ *     NF4_ERR_UNSUPPORTED_SHAPE and launches nothing.
+ *   - The first call on a device looks up the scratch array's device address
+ *     (once per device); make that first call before any stream capture.
+ *   - Every call on a device shares the one scratch array, and a call only
+ *     reads scratch it has written itself, so nothing needs clearing between
+ *     calls; calls whose kernels overlap on the GPU (different streams, or
+ *     different host threads) race on it and must be serialised by the
+ *     caller. */
+QLORA_API nf4_status qlora_linear_fwd_noalloc(const nf4_weight *w, const uint16_t *x, int64_t M,
+                                              const uint16_t *A, const uint16_t *B, int32_t r,
+                                              float alpha, uint16_t *h, float *u_out,
+                                              void *stream);
+
 /* Workspace needed by qlora_linear_bwd for M tokens at rank r. */
 QLORA_API size_t qlora_bwd_workspace_bytes(int64_t M, int64_t n, int64_t k, int32_t r);
 
