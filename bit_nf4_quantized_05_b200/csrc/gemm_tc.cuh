@@ -12,20 +12,24 @@
 //            lora_a = bf16((alpha/r) dY B) [M, r], lora_b = A
 //            (chain rule through the frozen dequantised weight)
 // The 4-bit codes stream into shared memory through TMA; dequantisation
-// warps turn each 64-code block into bf16 with a per-block register lookup
-// table and write it directly in the tensor core's 128-byte-swizzled operand
-// layout (K-major for the forward, MN-major for dgrad). The LoRA term is
-// ceil(r/64) extra reduction stages whose operands TMA loads directly (r is
-// zero-padded to 64 by the TMA out-of-bounds fill).
+// warps turn each 64-code block into bf16 (two threads per block, sharing a
+// per-block register lookup table) and write it directly in the tensor
+// core's 128-byte-swizzled operand layout: K-major for the forward, MN-major
+// for dgrad. The LoRA term is ceil(r/64) extra reduction stages (r zero-padded
+// to 64).
 //
-// Warp roles (16 warps, one CTA per SM, persistent over output tiles):
-//   warp 0        TMA producer (one thread)
-//   warp 1        TMEM owner + MMA issuer (one thread)
-//   warps 4..7    epilogue: TMEM -> registers -> bf16 -> global
-//   warps 8..15   dequantisation
-// Pipelines: a ring of shared-memory stages (full / dequantised / empty
-// mbarriers) and two TMEM accumulator buffers (full / empty), so the
-// epilogue of one tile overlaps the main loop of the next.
+// Warp roles (one CTA per SM, persistent over output tiles):
+//   warps 0..3    epilogue: TMEM -> registers -> bf16 -> global (warp w reads
+//                 TMEM lanes 32(w%4)..)
+//   warp 4        TMA producer of activation tiles
+//   warp 5        TMEM owner + MMA issuer (one thread)
+//   warp 6        TMA producer of code tiles
+//   warps 7..     dequantisation (2*BN threads)
+// Three shared-memory rings decouple the producers: activation tiles (freed
+// by the MMA), code tiles (freed as soon as the dequant warps have read them,
+// so they can be fetched far ahead), and dequantised weight tiles (freed by
+// the MMA). Two TMEM accumulator buffers let the epilogue of one tile overlap
+// the main loop of the next.
 #pragma once
 
 #include "nf4_common.cuh"
@@ -34,10 +38,11 @@ namespace nf4 {
 
 constexpr int kBM = 128;            // tokens per tile = MMA M
 constexpr int kBK = 64;             // reduction per stage = one NF4 block
-constexpr int kGemmThreads = 512;
-constexpr int kDequantWarp0 = 8;
-constexpr int kDequantWarps = 8;
-constexpr int kEpiWarp0 = 4;
+constexpr int kEpiWarp0 = 0;
+constexpr int kTmaAWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kTmaCWarp = 6;
+constexpr int kDequantWarp0 = 7;
 
 struct GemmArgs {
     int M;              // tokens
@@ -46,13 +51,16 @@ struct GemmArgs {
     int main_steps;     // ceil(red / 64)
     int lora_steps;     // ceil(r / 64)
     int m_tiles, n_tiles;
+    int r;
     // quantised weight (always the [N, K] weight)
     int64_t Nw;         // rows of W
+    int64_t Kw;         // columns of W
     int64_t kblocks;    // K / 64 (blocks per W row)
     const float *absmax;
     const uint8_t *q8;
     const float *cg;
     int dq;
+    const uint16_t *lora_b;   // forward: B [N, r]; dgrad: A [r, K]
     uint16_t *D;        // [M, out] bf16
 };
 
@@ -61,46 +69,65 @@ struct GemmCfg {
     static constexpr int kABytes = kBM * kBK * 2;        // 16 KB
     static constexpr int kBBytes = BN * kBK * 2;         // BN rows of 128 B
     static constexpr int kCBytes = BN * kBK / 2;         // 4-bit codes of the B tile
-    static constexpr int kStageBytes = kABytes + kBBytes + kCBytes;
-    static constexpr int kStages = (220 * 1024) / kStageBytes > 6 ? 6 : (220 * 1024) / kStageBytes;
+    static constexpr int kSB = BN <= 192 ? 4 : 2;        // dequantised-tile stages (even)
+    static constexpr int kSC = 6;                        // code-tile stages
+    static constexpr int kSA = (220 * 1024 - kSB * kBBytes - kSC * kCBytes) / kABytes > 8
+                                   ? 8
+                                   : (220 * 1024 - kSB * kBBytes - kSC * kCBytes) / kABytes;
+    static constexpr int kGroupWarps = BN / 32;           // warps of one dequant group
+    static constexpr int kDeqWarps = 2 * kGroupWarps;     // two groups take alternate stages
+    static constexpr int kThreads = 32 * (kDequantWarp0 + kDeqWarps);
     static constexpr int kTmemCols = (2 * BN <= 256) ? 256 : 512;
-    static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+    static constexpr int kSmemBytes =
+        kSA * kABytes + kSB * kBBytes + kSC * kCBytes + 1024 /*align*/ + 512 /*barriers*/;
     static constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, BN, 0, DGRAD ? 1 : 0);
     static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN");
-    static_assert(kStageBytes % 1024 == 0, "stage alignment");
-    static_assert(kStages >= 3, "pipeline depth");
+    static_assert(kBBytes % 1024 == 0 && kCBytes % 1024 == 0, "stage alignment");
+    static_assert(kSA >= 3, "pipeline depth");
+    static_assert(kSB % 2 == 0, "the two dequant groups alternate over the weight-tile ring");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
 template <int BN, bool DGRAD>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(GemmCfg<BN, DGRAD>::kThreads, 1)
 qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red] bf16, box {64,128}
-                  const __grid_constant__ CUtensorMap tm_codes,  // [Nw, K/2] u8
+                  const __grid_constant__ CUtensorMap tm_codes,  // [Nw, K/2] u8, box {32, rows}
                   const __grid_constant__ CUtensorMap tm_la,     // [M, r] bf16, box {64,128}
-                  const __grid_constant__ CUtensorMap tm_lb,     // fwd: B [N, r]; dgrad: A [r, K]
                   const GemmArgs args) {
     using Cfg = GemmCfg<BN, DGRAD>;
+    constexpr int SA = Cfg::kSA, SB = Cfg::kSB, SC = Cfg::kSC;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
-    uint8_t *slot_a = smem;                                        // [Cfg::kStages][kABytes]
-    uint8_t *slot_b = smem + Cfg::kStages * Cfg::kABytes;               // [Cfg::kStages][kBBytes]
-    uint8_t *slot_c = slot_b + Cfg::kStages * Cfg::kBBytes;             // [Cfg::kStages][kCBytes]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(slot_c + Cfg::kStages * Cfg::kCBytes);
-    uint64_t *full = bars;                   // TMA landed         (count 1 + tx)
-    uint64_t *bfull = bars + Cfg::kStages;        // B tile ready       (count kDequantWarps)
-    uint64_t *empty = bars + 2 * Cfg::kStages;    // MMA done with slot (count 1, tcgen05.commit)
-    uint64_t *acc_full = bars + 3 * Cfg::kStages; // [2] accumulator complete
-    uint64_t *acc_empty = acc_full + 2;      // [2] accumulator drained (count 4)
+    uint8_t *slot_a = smem;                              // [SA][kABytes]
+    uint8_t *slot_b = slot_a + SA * Cfg::kABytes;        // [SB][kBBytes]
+    uint8_t *slot_c = slot_b + SB * Cfg::kBBytes;        // [SC][kCBytes]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(slot_c + SC * Cfg::kCBytes);
+    uint64_t *a_full = bars;                 // TMA landed            (1 + tx)
+    uint64_t *a_empty = a_full + SA;         // MMA done              (commit)
+    uint64_t *c_full = a_empty + SA;         // TMA landed            (1 + tx)
+    uint64_t *c_empty = c_full + SC;         // codes read            (one dequant group)
+    uint64_t *b_full = c_empty + SC;         // weight tile written   (one dequant group)
+    uint64_t *b_empty = b_full + SB;         // MMA done              (commit)
+    uint64_t *acc_full = b_empty + SB;       // [2] accumulator complete (commit)
+    uint64_t *acc_empty = acc_full + 2;      // [2] accumulator drained  (4 epilogue warps)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < Cfg::kStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&bfull[s], kDequantWarps);
-            mbar_init(&empty[s], 1);
+        for (int s = 0; s < SA; ++s) {
+            mbar_init(&a_full[s], 1);
+            mbar_init(&a_empty[s], 1);
+        }
+        for (int s = 0; s < SC; ++s) {
+            mbar_init(&c_full[s], 1);
+            mbar_init(&c_empty[s], Cfg::kGroupWarps);
+        }
+        for (int s = 0; s < SB; ++s) {
+            mbar_init(&b_full[s], Cfg::kGroupWarps);
+            mbar_init(&b_empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
@@ -111,9 +138,8 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red] bf1
         tma_prefetch_desc(&tm_act);
         tma_prefetch_desc(&tm_codes);
         tma_prefetch_desc(&tm_la);
-        tma_prefetch_desc(&tm_lb);
     }
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tmem_alloc(tmem_slot, Cfg::kTmemCols);
         tmem_relinquish();
     }
@@ -125,75 +151,81 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red] bf1
     const int total_tiles = args.m_tiles * args.n_tiles;
     const int nsteps = args.main_steps + args.lora_steps;
 
-    if (warp == 0 && lane == 0) {
-        // ------------------------------------------------------------ TMA
-        int st = 0;
-        uint32_t ph = 0;
-        for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-            const int m0 = (tile % args.m_tiles) * kBM;
-            const int n0 = (tile / args.m_tiles) * BN;
-            for (int it = 0; it < nsteps; ++it) {
-                if (!mbar_wait(&empty[st], ph ^ 1, abort_flag)) goto done;
-                uint8_t *a = slot_a + st * Cfg::kABytes;
-                uint8_t *b = slot_b + st * Cfg::kBBytes;
-                uint8_t *c = slot_c + st * Cfg::kCBytes;
-                if (it < args.main_steps) {
-                    mbar_arrive_expect_tx(&full[st], Cfg::kABytes + Cfg::kCBytes);
-                    tma_load_2d(a, &tm_act, &full[st], it * kBK, m0);
+    if (warp == kTmaAWarp) {
+        // ------------------------------------------------ TMA: activations
+        if (lane == 0) {
+            int sa = 0;
+            uint32_t pa = 0;
+            for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+                const int m0 = (tile % args.m_tiles) * kBM;
+                for (int it = 0; it < nsteps; ++it) {
+                    if (!mbar_wait(&a_empty[sa], pa ^ 1, abort_flag)) goto done;
+                    mbar_arrive_expect_tx(&a_full[sa], Cfg::kABytes);
+                    if (it < args.main_steps)
+                        tma_load_2d(slot_a + sa * Cfg::kABytes, &tm_act, &a_full[sa], it * kBK, m0);
+                    else
+                        tma_load_2d(slot_a + sa * Cfg::kABytes, &tm_la, &a_full[sa],
+                                    (it - args.main_steps) * kBK, m0);
+                    if (++sa == SA) { sa = 0; pa ^= 1; }
+                }
+            }
+        }
+    } else if (warp == kTmaCWarp) {
+        // ------------------------------------------------ TMA: 4-bit codes
+        if (lane == 0) {
+            int sc = 0;
+            uint32_t pc = 0;
+            for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+                const int n0 = (tile / args.m_tiles) * BN;
+                for (int it = 0; it < args.main_steps; ++it) {
+                    if (!mbar_wait(&c_empty[sc], pc ^ 1, abort_flag)) goto done;
+                    uint8_t *c = slot_c + sc * Cfg::kCBytes;
+                    mbar_arrive_expect_tx(&c_full[sc], Cfg::kCBytes);
                     if (!DGRAD) {
-                        tma_load_2d(c, &tm_codes, &full[st], it * (kBK / 2), n0);
+                        tma_load_2d(c, &tm_codes, &c_full[sc], it * (kBK / 2), n0);
                     } else {
 #pragma unroll
                         for (int kb = 0; kb < BN / 64; ++kb)
-                            tma_load_2d(c + kb * 2048, &tm_codes, &full[st], n0 / 2 + kb * 32,
+                            tma_load_2d(c + kb * 2048, &tm_codes, &c_full[sc], n0 / 2 + kb * 32,
                                         it * kBK);
                     }
-                } else {
-                    const int ls = it - args.main_steps;
-                    mbar_arrive_expect_tx(&full[st], Cfg::kABytes + Cfg::kBBytes);
-                    tma_load_2d(a, &tm_la, &full[st], ls * kBK, m0);
-                    if (!DGRAD) {
-                        tma_load_2d(b, &tm_lb, &full[st], ls * kBK, n0);
-                    } else {
-#pragma unroll
-                        for (int ma = 0; ma < BN / 64; ++ma)
-                            tma_load_2d(b + ma * 8192, &tm_lb, &full[st], n0 + ma * 64, ls * kBK);
-                    }
+                    if (++sc == SC) { sc = 0; pc ^= 1; }
                 }
-                if (++st == Cfg::kStages) { st = 0; ph ^= 1; }
             }
         }
-    } else if (warp == 1 && lane == 0) {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA
-        int st = 0;
-        uint32_t ph = 0;
-        int ab = 0;
-        uint32_t aph = 0;
-        const uint32_t a_base = smem_u32(slot_a), b_base = smem_u32(slot_b);
-        for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-            if (!mbar_wait(&acc_empty[ab], aph ^ 1, abort_flag)) goto done;
-            tc_fence_after();
-            const uint32_t d_tmem = tmem_base + ab * BN;
-            for (int it = 0; it < nsteps; ++it) {
-                if (!mbar_wait(&full[st], ph, abort_flag)) goto done;
-                if (!mbar_wait(&bfull[st], ph, abort_flag)) goto done;
+        if (lane == 0) {
+            int sa = 0, sb = 0, ab = 0;
+            uint32_t pa = 0, pb = 0, aph = 0;
+            const uint32_t a_base = smem_u32(slot_a), b_base = smem_u32(slot_b);
+            for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+                if (!mbar_wait(&acc_empty[ab], aph ^ 1, abort_flag)) goto done;
                 tc_fence_after();
-                const uint32_t a_addr = a_base + st * Cfg::kABytes;
-                const uint32_t b_addr = b_base + st * Cfg::kBBytes;
+                const uint32_t d_tmem = tmem_base + ab * BN;
+                for (int it = 0; it < nsteps; ++it) {
+                    if (!mbar_wait(&a_full[sa], pa, abort_flag)) goto done;
+                    if (!mbar_wait(&b_full[sb], pb, abort_flag)) goto done;
+                    tc_fence_after();
+                    const uint32_t a_addr = a_base + sa * Cfg::kABytes;
+                    const uint32_t b_addr = b_base + sb * Cfg::kBBytes;
 #pragma unroll
-                for (int kk = 0; kk < kBK / 16; ++kk) {
-                    const uint64_t ad = smem_desc_sw128(a_addr + kk * 32, 16, 1024);
-                    const uint64_t bd = DGRAD ? smem_desc_sw128(b_addr + kk * 2048, 8192, 1024)
-                                              : smem_desc_sw128(b_addr + kk * 32, 16, 1024);
-                    umma_bf16_ss(d_tmem, ad, bd, Cfg::kIdesc, (it > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                        const uint64_t ad = smem_desc_sw128(a_addr + kk * 32, 16, 1024);
+                        const uint64_t bd = DGRAD ? smem_desc_sw128(b_addr + kk * 2048, 8192, 1024)
+                                                  : smem_desc_sw128(b_addr + kk * 32, 16, 1024);
+                        umma_bf16_ss(d_tmem, ad, bd, Cfg::kIdesc, (it > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(&a_empty[sa]);
+                    umma_commit(&b_empty[sb]);
+                    if (++sa == SA) { sa = 0; pa ^= 1; }
+                    if (++sb == SB) { sb = 0; pb ^= 1; }
                 }
-                umma_commit(&empty[st]);
-                if (++st == Cfg::kStages) { st = 0; ph ^= 1; }
+                umma_commit(&acc_full[ab]);
+                if (++ab == 2) { ab = 0; aph ^= 1; }
             }
-            umma_commit(&acc_full[ab]);
-            if (++ab == 2) { ab = 0; aph ^= 1; }
         }
-    } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
+    } else if (warp < kEpiWarp0 + 4) {
         // ------------------------------------------------------- epilogue
         const int q = warp - kEpiWarp0;                   // TMEM lane quadrant (== warp % 4)
         int ab = 0;
@@ -233,31 +265,34 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red] bf1
             if (lane == 0) mbar_arrive(&acc_empty[ab]);
             if (++ab == 2) { ab = 0; aph ^= 1; }
         }
-    } else if (warp >= kDequantWarp0) {
+    } else {
         // -------------------------------------------------- dequantisation
-        // Work item of this thread: forward: W row n0 + i (one block per
-        // stage); dgrad: reduction row r_loc of the stage and output block kb.
-        // Eight consecutive lanes always take eight consecutive rows of one
-        // 8-row swizzle atom, so their 16-byte stores hit distinct banks.
-        const int i = threadIdx.x - kDequantWarp0 * 32;
-        const bool active = i < BN;
+        // Two groups of BN threads take alternate stages (group g handles the
+        // stages whose global index is g mod 2), so each thread has two stage
+        // times for one 64-element block. Thread i of a group owns work item i:
+        //   forward: W row n0 + i, block `it` of the stage
+        //   dgrad:   reduction row r_loc of the stage, output block kb
+        // Eight consecutive lanes take eight consecutive rows of one 8-row
+        // swizzle atom, so each 8-lane phase of a 16-byte shared access hits
+        // distinct banks.
+        const int t = threadIdx.x - kDequantWarp0 * 32;
+        const int grp = t / BN;
+        const int i = t % BN;
         constexpr int kBPR = BN / 64;
         const int kb = DGRAD ? (i / 8) % kBPR : 0;
         const int r_loc = DGRAD ? (i / (8 * kBPR)) * 8 + (i & 7) : i;
         const uint32_t row_off = DGRAD ? static_cast<uint32_t>(kb * 8192 + r_loc * 128)
                                        : static_cast<uint32_t>(i * 128);
-        // codes tiles carry the 32-byte TMA swizzle: 16-byte chunk h of row j
-        // sits at chunk h ^ ((j >> 2) & 1)
+        // code tiles carry the 32-byte TMA swizzle: 16-byte chunk hh of row j
+        // sits at chunk hh ^ ((j >> 2) & 1)
         const uint32_t code_off = DGRAD ? static_cast<uint32_t>(kb * 2048 + r_loc * 32)
                                         : static_cast<uint32_t>(i * 32);
         const uint32_t cswz = static_cast<uint32_t>((r_loc >> 2) & 1);
         const uint32_t swz = static_cast<uint32_t>(r_loc & 7);
 
-        // raw scale inputs of one (tile, step), loaded one step ahead
-        struct RawScale { uint32_t q8; float v; bool valid; };
-        auto load_scale = [&](int tile, int it) -> RawScale {
-            RawScale rs{0u, 0.0f, false};
-            if (tile >= total_tiles || it >= args.main_steps || !active) return rs;
+        // block index of (tile, stage) for this item, or -1 outside the weight
+        auto block_of = [&](int tile, int it) -> int64_t {
+            if (tile >= total_tiles || it >= args.main_steps) return -1;
             const int n0 = (tile / args.m_tiles) * BN;
             int64_t wrow, wblk;
             if (!DGRAD) {
@@ -267,64 +302,129 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red] bf1
                 wrow = static_cast<int64_t>(it) * kBK + r_loc;
                 wblk = n0 / 64 + kb;
             }
-            if (wrow >= args.Nw || wblk >= args.kblocks) return rs;
-            const int64_t b = wrow * args.kblocks + wblk;
-            rs.valid = true;
-            if (args.dq) {
-                rs.q8 = __ldg(args.q8 + b);
-                rs.v = __ldg(args.cg + (b >> 8));
-            } else {
-                rs.v = __ldg(args.absmax + b);
-            }
+            if (wrow >= args.Nw || wblk >= args.kblocks) return -1;
+            return wrow * args.kblocks + wblk;
+        };
+        struct RawScale { int64_t b; uint32_t q8; float v; };
+        auto load_scale = [&](int64_t b) -> RawScale {
+            RawScale rs{b, 0u, 0.0f};
+            if (b < 0) return rs;
+            if (args.dq) rs.q8 = __ldg(args.q8 + b);
+            else rs.v = __ldg(args.absmax + b);
             return rs;
         };
+        int64_t kg_group = -1;      // cached fl32(c_g / 127) of the last group seen
+        float kg = 0.0f;
 
-        int st = 0;
-        uint32_t ph = 0;
+        // walk every (tile, stage) in order; this group acts on every other one
         int tile = blockIdx.x, it = 0;
-        RawScale nxt = load_scale(tile, it);
+        int64_t gstep = 0;          // global stage counter (weight-tile ring)
+        int64_t mstep = 0;          // global main-stage counter (code ring)
+        // the next stage of this group, and its prefetched scale
+        auto advance = [&](int &tl, int &st_, int64_t &g, int64_t &m) {
+            if (st_ < args.main_steps) ++m;
+            ++g;
+            if (++st_ == nsteps) { st_ = 0; tl += gridDim.x; }
+        };
+        if (grp == 1 && tile < total_tiles) advance(tile, it, gstep, mstep);
+        RawScale nxt = load_scale(block_of(tile, it));
         while (tile < total_tiles) {
             const RawScale cur = nxt;
             const bool main = it < args.main_steps;
-            // advance to the next (tile, step) and start its scale load now
-            int ntile = tile, nit = it + 1;
-            if (nit == nsteps) { nit = 0; ntile += gridDim.x; }
-            nxt = load_scale(ntile, nit);
-            if (!mbar_wait(&full[st], ph, abort_flag)) goto done;
-            if (main && active) {
-                const uint8_t *cp = slot_c + st * Cfg::kCBytes + code_off;
-                const uint4 c0 = *reinterpret_cast<const uint4 *>(cp + 16 * cswz);
-                const uint4 c1 = *reinterpret_cast<const uint4 *>(cp + 16 * (cswz ^ 1));
-                const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                uint8_t *brow = slot_b + st * Cfg::kBBytes + row_off;
-                if (cur.valid) {
-                    float s = cur.v;
-                    if (args.dq) s = __fmul_rn(static_cast<float>(cur.q8), __fdiv_rn(cur.v, 127.0f));
-                    const BlockLut L = make_block_lut(s);
+            const int n0 = (tile / args.m_tiles) * BN;
+            const int sb = static_cast<int>(gstep % SB);
+            const uint32_t pb = static_cast<uint32_t>((gstep / SB) & 1);
+            const int sc = static_cast<int>(mstep % SC);
+            const uint32_t pc = static_cast<uint32_t>((mstep / SC) & 1);
+            // this group's following stage: skip the other group's one
+            int ntile = tile, nit = it;
+            int64_t ng = gstep, nm = mstep;
+            advance(ntile, nit, ng, nm);
+            if (ntile < total_tiles) advance(ntile, nit, ng, nm);
+            nxt = load_scale(block_of(ntile, nit));
+
+            uint32_t out[32];
+            if (main) {
+                if (!mbar_wait(&c_full[sc], pc, abort_flag)) goto done;
+                const uint8_t *cp = slot_c + sc * Cfg::kCBytes + code_off;
+                const uint4 h0 = *reinterpret_cast<const uint4 *>(cp + 16 * cswz);
+                const uint4 h1 = *reinterpret_cast<const uint4 *>(cp + 16 * (cswz ^ 1));
+                float s = 0.0f;
+                if (cur.b >= 0) {
+                    if (args.dq) {
+                        const int64_t g = cur.b >> 8;
+                        if (g != kg_group) {
+                            kg_group = g;
+                            kg = __fdiv_rn(__ldg(args.cg + g), 127.0f);
+                        }
+                        s = __fmul_rn(static_cast<float>(cur.q8), kg);
+                    } else {
+                        s = cur.v;
+                    }
+                }
+                const BlockLut L = make_block_lut(s);
+                const uint32_t words[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
 #pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) {
-                        uint32_t o[4];
-                        dequant8(L, words[ch], o);
-                        *reinterpret_cast<uint4 *>(brow + ((ch ^ swz) << 4)) =
-                            make_uint4(o[0], o[1], o[2], o[3]);
+                for (int wd = 0; wd < 8; ++wd) {
+                    uint32_t o[4];
+                    dequant8(L, words[wd], o);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) out[4 * wd + e] = cur.b >= 0 ? o[e] : 0u;
+                }
+                // the codes are consumed (out depends on them): release the slot
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&c_empty[sc]);
+            } else {
+                // LoRA stage: the adapter tile comes straight from global memory
+                //   forward: B[n0 + i][64 ls .. +64)        (zero beyond r, N)
+                //   dgrad:   A[64 ls + r_loc][n0 + 64 kb .. +64)  (zero beyond r, K)
+                const int ls = it - args.main_steps;
+                const uint16_t *src = nullptr;
+                int nvalid = 0;   // valid 8-element chunks
+                if (!DGRAD) {
+                    const int64_t n = n0 + i;
+                    const int j0 = 64 * ls;
+                    if (n < args.Nw && j0 < args.r) {
+                        src = args.lora_b + n * args.r + j0;
+                        nvalid = (args.r - j0) / 8 >= 8 ? 8 : (args.r - j0) / 8;
                     }
                 } else {
-#pragma unroll
-                    for (int ch = 0; ch < 8; ++ch)
-                        *reinterpret_cast<uint4 *>(brow + (ch << 4)) = make_uint4(0, 0, 0, 0);
+                    const int j = 64 * ls + r_loc;
+                    const int64_t k0 = static_cast<int64_t>(n0) + 64 * kb;
+                    if (j < args.r && k0 < args.Kw) {
+                        src = args.lora_b + static_cast<int64_t>(j) * args.Kw + k0;
+                        nvalid = (args.Kw - k0) / 8 >= 8 ? 8 : static_cast<int>((args.Kw - k0) / 8);
+                    }
                 }
-                fence_proxy_async_smem();
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint4 v = make_uint4(0, 0, 0, 0);
+                    if (c < nvalid) v = __ldg(reinterpret_cast<const uint4 *>(src) + c);
+                    out[4 * c] = v.x;
+                    out[4 * c + 1] = v.y;
+                    out[4 * c + 2] = v.z;
+                    out[4 * c + 3] = v.w;
+                }
             }
+            if (!mbar_wait(&b_empty[sb], pb ^ 1, abort_flag)) goto done;
+            uint8_t *brow = slot_b + sb * Cfg::kBBytes + row_off;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4 *>(brow + ((c ^ swz) << 4)) =
+                    make_uint4(out[4 * c], out[4 * c + 1], out[4 * c + 2], out[4 * c + 3]);
+            fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bfull[st]);
-            if (++st == Cfg::kStages) { st = 0; ph ^= 1; }
+            if (lane == 0) mbar_arrive(&b_full[sb]);
             tile = ntile;
             it = nit;
+            gstep = ng;
+            mstep = nm;
         }
     }
 done:
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem_base, Cfg::kTmemCols);
     }

@@ -301,7 +301,7 @@ nf4_status launch_gemm(const nf4_weight *w, const uint16_t *act, int64_t M, int6
                        int64_t out, const uint16_t *la, int32_t r, const uint16_t *lb,
                        uint16_t *D, cudaStream_t stream) {
     using Cfg = GemmCfg<BN, DGRAD>;
-    CUtensorMap tm_act, tm_codes, tm_la, tm_lb;
+    CUtensorMap tm_act, tm_codes, tm_la;
     const int64_t N = w->n, K = w->k;
     bool ok = make_map(&tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, act, red, M, kBK, kBM,
                        CU_TENSOR_MAP_SWIZZLE_128B);
@@ -312,12 +312,6 @@ nf4_status launch_gemm(const nf4_weight *w, const uint16_t *act, int64_t M, int6
                         DGRAD ? kBK : BN, CU_TENSOR_MAP_SWIZZLE_32B);
     ok = ok && make_map(&tm_la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, la, r, M, kBK, kBM,
                         CU_TENSOR_MAP_SWIZZLE_128B);
-    if (!DGRAD)  // B [N, r]: rows n, K-major over j
-        ok = ok && make_map(&tm_lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, lb, r, N, kBK, BN,
-                            CU_TENSOR_MAP_SWIZZLE_128B);
-    else         // A [r, K]: rows j, 64 output columns per box (MN-major atoms)
-        ok = ok && make_map(&tm_lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, lb, K, r, 64, kBK,
-                            CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok) return NF4_ERR_CUDA;
 
     GemmArgs a;
@@ -328,12 +322,15 @@ nf4_status launch_gemm(const nf4_weight *w, const uint16_t *act, int64_t M, int6
     a.lora_steps = (r + kBK - 1) / kBK;
     a.m_tiles = static_cast<int>((M + kBM - 1) / kBM);
     a.n_tiles = static_cast<int>((out + BN - 1) / BN);
+    a.r = r;
     a.Nw = N;
+    a.Kw = K;
     a.kblocks = K / kBlock;
     a.absmax = w->absmax;
     a.q8 = w->absmax_q8;
     a.cg = w->absmax_c;
     a.dq = w->double_quant;
+    a.lora_b = lb;
     a.D = D;
 
     const int dev = current_device();
@@ -343,7 +340,7 @@ nf4_status launch_gemm(const nf4_weight *w, const uint16_t *act, int64_t M, int6
     NF4_TRY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       Cfg::kSmemBytes));
     LaunchTimer t(DGRAD ? KK_GEMM_DGRAD : KK_GEMM_FWD, stream);
-    kern<<<grid, kGemmThreads, Cfg::kSmemBytes, stream>>>(tm_act, tm_codes, tm_la, tm_lb, a);
+    kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tm_act, tm_codes, tm_la, a);
     t.stop();
     NF4_TRY_CUDA(cudaGetLastError());
     return NF4_OK;
