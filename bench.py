@@ -378,16 +378,22 @@ def decode_leg(q, dev, peaks):
             q.qlora_linear_fwd(copies[i], x, A, B, w.alpha, save_u=False, h=h, workspace=ws)
         torch.cuda.synchronize()
         iters = 64
-        q.profiling(True)
+        # whole calls, no per-kernel events in between (they would serialise
+        # the dependent launch inside the call)
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s.record()
         for i in range(iters):
             q.qlora_linear_fwd(copies[i % 8], x, A, B, w.alpha, save_u=False, h=h, workspace=ws)
         e.record()
         torch.cuda.synchronize()
+        call_us = 1e3 * s.elapsed_time(e) / iters
+        # per-kernel durations
+        q.profiling(True)
+        for i in range(iters):
+            q.qlora_linear_fwd(copies[i % 8], x, A, B, w.alpha, save_u=False, h=h, workspace=ws)
+        torch.cuda.synchronize()
         q.profiling(False)
         prof = q.profile_read()
-        call_us = 1e3 * s.elapsed_time(e) / iters
         kern = {k: 1e3 * t / max(n, 1) for k, (n, t) in prof.items()}
         main_us = kern.get("qlora_gemm_fwd") or kern.get("qlora_decode")
         out[f"M{M}"] = {"call_us": call_us, "gbs_call": code_bytes / (call_us * 1e-6) / 1e9,

@@ -16,6 +16,7 @@
 #include "codec.cuh"
 #include "gemm_tc.cuh"
 #include "skinny_tc.cuh"
+#include "decode.cuh"
 
 using namespace nf4;
 
@@ -33,11 +34,12 @@ constexpr int kMaxDevices = 64;
 // ---------------------------------------------------------------------------
 enum KernelKind {
     KK_QUANTIZE, KK_DEQUANTIZE, KK_LORA_U, KK_LORA_V, KK_LORA_DB, KK_LORA_DA, KK_LORA_REDUCE,
-    KK_SCALE, KK_ZERO, KK_GEMM_FWD, KK_GEMM_DGRAD, KK_COUNT
+    KK_SCALE, KK_ZERO, KK_GEMM_FWD, KK_GEMM_DGRAD, KK_DECODE, KK_DECODE_U, KK_COUNT
 };
 const char *const kKindNames[KK_COUNT] = {
     "nf4_quantize", "nf4_dequantize", "lora_u", "lora_v", "lora_dB", "lora_dA", "lora_reduce",
-    "lora_scale", "zero_fill", "qlora_gemm_fwd", "qlora_gemm_dgrad"};
+    "lora_scale", "zero_fill", "qlora_gemm_fwd", "qlora_gemm_dgrad", "qlora_decode",
+    "decode_lora_u"};
 
 struct ProfRecord {
     int kind;
@@ -346,6 +348,59 @@ nf4_status launch_gemm(const nf4_weight *w, const uint16_t *act, int64_t M, int6
     return NF4_OK;
 }
 
+// Forward for M <= 16 tokens: u = x A^T (and its scaled bf16 copy), then the
+// decode kernel, launched as a programmatic dependent of the first so that
+// it streams the weight while u is being computed.
+constexpr int64_t kDecodeMaxTokens = 16;
+
+// The decode kernel keeps B and u tiles of rank <= kDecMaxRank in shared memory.
+bool decode_shape(const nf4_weight *w, int64_t M, int32_t r) {
+    return M <= kDecodeMaxTokens && r <= kDecMaxRank;
+}
+
+nf4_status launch_decode(const nf4_weight *w, const uint16_t *x, int64_t M, const uint16_t *A,
+                         const uint16_t *B, int32_t r, float scale, uint16_t *h, float *u_out,
+                         uint16_t *u_s, cudaStream_t stream) {
+    {
+        LaunchTimer t(KK_DECODE_U, stream);
+        decode_lora_u_kernel<<<r, kDecUThreads, 0, stream>>>(x, A, static_cast<int>(M), w->k, r,
+                                                            scale, u_out, u_s);
+        t.stop();
+    }
+    NF4_TRY_CUDA(cudaGetLastError());
+    DecodeArgs a;
+    a.M = static_cast<int>(M);
+    a.N = w->n;
+    a.K = w->k;
+    a.r = r;
+    a.codes = w->codes;
+    a.absmax = w->absmax;
+    a.q8 = w->absmax_q8;
+    a.cg = w->absmax_c;
+    a.dq = w->double_quant;
+    a.x = x;
+    a.B = B;
+    a.u_s = u_s;
+    a.h = h;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>((w->n + kDecRows - 1) / kDecRows));
+    cfg.blockDim = dim3(kDecThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    LaunchTimer t(KK_DECODE, stream);
+    cudaError_t e = M <= 8 ? cudaLaunchKernelEx(&cfg, qlora_decode_kernel<1>, a)
+                           : cudaLaunchKernelEx(&cfg, qlora_decode_kernel<2>, a);
+    t.stop();
+    if (e != cudaSuccess) return NF4_ERR_CUDA;
+    NF4_TRY_CUDA(cudaGetLastError());
+    return NF4_OK;
+}
+
 // Output-column tile: the candidate with the smallest (rounds of tiles over
 // the SMs) x (tile width), i.e. the least per-SM time under even tiles.
 int pick_bn(int64_t M, int64_t out, int sms) {
@@ -511,6 +566,7 @@ nf4_status qlora_linear_fwd(const nf4_weight *w, const uint16_t *x, int64_t M, c
     uint16_t *u_s = reinterpret_cast<uint16_t *>(ws + L.us);
     float *part = reinterpret_cast<float *>(ws + L.part);
     const float scale = alpha / static_cast<float>(r);
+    if (decode_shape(w, M, r)) return launch_decode(w, x, M, A, B, r, scale, h, u_out, u_s, s);
     // u = x A^T (fp32, optional) and bf16((alpha/r) u) for the up-projection stage
     st = skinny_product(KK_LORA_U, x, M, w->k, Major::K, A, r, w->k, Major::K, r, part, u_out, u_s,
                         scale, 0, s);
@@ -539,6 +595,8 @@ nf4_status qlora_linear_fwd_noalloc(const nf4_weight *w, const uint16_t *x, int6
     uint16_t *u_s = reinterpret_cast<uint16_t *>(ws);
     float *part = reinterpret_cast<float *>(ws + us_bytes);
     const float scale = alpha / static_cast<float>(r);
+    // same dispatch as qlora_linear_fwd: a few tokens take the decode kernel
+    if (decode_shape(w, M, r)) return launch_decode(w, x, M, A, B, r, scale, h, u_out, u_s, s);
     st = skinny_product(KK_LORA_U, x, M, w->k, Major::K, A, r, w->k, Major::K, r, part, u_out, u_s,
                         scale, 0, s, max_splits);
     if (st != NF4_OK) return st;
