@@ -192,6 +192,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--skip-extras", action="store_true",
                     help="only the main fwd+bwd line (no decode/quantize/oracle/e2e legs)")
+    ap.add_argument("--leg", default="all", choices=["all", "decode", "quantize"],
+                    help="run one secondary leg alone and print its JSON (for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -208,6 +210,11 @@ def main():
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
+    if args.leg != "all":
+        if rank == 0:
+            leg = decode_leg if args.leg == "decode" else quantize_leg
+            print(json.dumps({"leg": args.leg, **leg(q, dev, load_peaks())}), flush=True)
+        return
     if world > 1:
         import datetime
         import torch.distributed as dist
