@@ -1,0 +1,415 @@
+// gemm_pair_tc.cuh -- fused NF4-dequantise + GEMM on CTA pairs
+// (tcgen05.mma.cta_group::2: one 256 x BN MMA spans the two CTAs of a cluster).
+//
+// Same products as gemm_tc.cuh,
+//   forward: D = x W~^T + bf16((alpha/r) x A^T) B^T
+//   dgrad:   D = dY W~  + bf16((alpha/r) dY B) A
+// ("QLoRA explained", section "The LoRA adapter path", and the chain rule
+// through the frozen dequantised weight), but each output tile is 256 tokens
+// x BN columns computed by a pair of CTAs on two SMs:
+//   CTA v of the pair loads tokens [128v, 128v+128) of the tile (A operand),
+//   dequantises only half of the weight tile -- columns [v BN/2, v BN/2 + BN/2)
+//   of the MMA's B operand -- into its own shared memory, and keeps rows
+//   [128v, 128v+128) of the fp32 accumulator in its own tensor memory.
+// The tensor core of the even CTA reads both halves of A and B directly, so
+// every dequantised element is produced once per 256 tokens instead of once
+// per 128, and each SM writes and the tensor core reads only half of the
+// weight tile: the dequantisation ALU work and the shared-memory traffic per
+// SM are both halved relative to a one-CTA tile of the same width.
+//
+// Synchronisation across the pair:
+//   a_full  (even CTA)   both CTAs' activation loads credit their bytes here
+//   b_full  (even CTA)   the dequant warps of both CTAs arrive here
+//   acc_empty (even CTA) the epilogue warps of both CTAs arrive here
+//   a_empty, b_empty, acc_full (both CTAs)  one multicast tcgen05.commit
+// The code-tile ring is private to each CTA.
+//
+// Warp roles per CTA: 0..3 epilogue, 4 TMA activations, 5 TMEM owner and (even
+// CTA) MMA issuer, 6 TMA codes, 7.. dequantisation (G groups of BN/2 threads
+// taking every G-th stage).
+#pragma once
+
+#include "gemm_tc.cuh"
+
+namespace nf4 {
+
+
+template <int BN, bool DGRAD, int G>
+struct PairCfg {
+    static constexpr int kBH = BN / 2;                    // B columns held by one CTA
+    static constexpr int kABytes = kBM * kBK * 2;         // 16 KB
+    static constexpr int kBBytes = kBH * kBK * 2;         // this CTA's half of the B tile
+    static constexpr int kCBytes = kBH * kBK / 2;         // its 4-bit codes
+    static constexpr int kSB = G >= 4 ? G : 2 * G;       // weight-tile stages
+    static constexpr int kSC = 8;                         // code-tile stages
+    static constexpr int kSAFit = (220 * 1024 - kSB * kBBytes - kSC * kCBytes) / kABytes;
+    static constexpr int kSA = kSAFit > 8 ? 8 : kSAFit;
+    static constexpr int kGroupWarps = kBH / 32;
+    static constexpr int kThreads = 32 * (kDequantWarp0 + G * kGroupWarps);
+    static constexpr int kTmemCols = (2 * BN <= 256) ? 256 : 512;
+    static constexpr int kSmemBytes =
+        kSA * kABytes + kSB * kBBytes + kSC * kCBytes + 1024 /*align*/ + 512 /*barriers*/;
+    static constexpr uint32_t kIdesc = idesc_bf16_f32(2 * kBM, BN, 0, DGRAD ? 1 : 0);
+    static_assert(BN % 16 == 0 && BN >= 64 && BN <= 256, "pair MMA N");
+    static_assert(kBH % 32 == 0, "whole dequant warps");
+    static_assert(!DGRAD || kBH % 64 == 0, "MN-major halves are whole 64-column swizzle atoms");
+    static_assert(kBBytes % 1024 == 0 && kCBytes % 1024 == 0, "stage alignment");
+    static_assert(kSC % G == 0 && kSB % G == 0, "each dequant group owns every G-th slot");
+    static_assert(kSA >= 3, "pipeline depth");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+};
+
+template <int BN, bool DGRAD, int G>
+__global__ void __launch_bounds__(PairCfg<BN, DGRAD, G>::kThreads, 1)
+qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red] bf16, box {64,128}
+                       const __grid_constant__ CUtensorMap tm_codes,  // [Nw, K/2] u8, box {32, rows}
+                       const __grid_constant__ CUtensorMap tm_la,     // [M, r] bf16, box {64,128}
+                       const GemmArgs args) {
+    using Cfg = PairCfg<BN, DGRAD, G>;
+    constexpr int SA = Cfg::kSA, SB = Cfg::kSB, SC = Cfg::kSC, BH = Cfg::kBH;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    uint8_t *slot_a = smem;                              // [SA][kABytes]
+    uint8_t *slot_b = slot_a + SA * Cfg::kABytes;        // [SB][kBBytes]
+    uint8_t *slot_c = slot_b + SB * Cfg::kBBytes;        // [SC][kCBytes]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(slot_c + SC * Cfg::kCBytes);
+    uint64_t *a_full = bars;                 // even CTA: both loads landed (1 + tx)
+    uint64_t *a_empty = a_full + SA;         // MMA done (pair commit)
+    uint64_t *c_full = a_empty + SA;         // code TMA landed (1 + tx) or LoRA stage (1)
+    uint64_t *c_empty = c_full + SC;         // codes read (one dequant group of this CTA)
+    uint64_t *b_full = c_empty + SC;         // even CTA: halves written (groups of both CTAs)
+    uint64_t *b_empty = b_full + SB;         // MMA done (pair commit)
+    uint64_t *acc_full = b_empty + SB;       // [2] accumulator complete (pair commit)
+    uint64_t *acc_empty = acc_full + 2;      // [2] even CTA: drained (epilogue warps of both)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();             // 0 or 1 within the pair
+    const int pair = static_cast<int>(cluster_id_x());
+    const int npairs = static_cast<int>(cluster_count_x());
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < SA; ++s) {
+            mbar_init(&a_full[s], 1);
+            mbar_init(&a_empty[s], 1);
+        }
+        for (int s = 0; s < SC; ++s) {
+            mbar_init(&c_full[s], 1);
+            mbar_init(&c_empty[s], Cfg::kGroupWarps);
+        }
+        for (int s = 0; s < SB; ++s) {
+            mbar_init(&b_full[s], 2 * Cfg::kGroupWarps);
+            mbar_init(&b_empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 8);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_act);
+        tma_prefetch_desc(&tm_codes);
+        tma_prefetch_desc(&tm_la);
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc_pair(tmem_slot, Cfg::kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();            // barriers of both CTAs initialised before any remote use
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int m_pairs = (args.M + 2 * kBM - 1) / (2 * kBM);
+    const int total_tiles = m_pairs * args.n_tiles;
+    const int nsteps = args.main_steps + args.lora_steps;
+
+    if (warp == kTmaAWarp) {
+        // ------------------------------------------------ TMA: activations
+        if (lane == 0) {
+            const uint32_t full0 = mapa_shared(smem_u32(a_full), 0);
+            int sa = 0;
+            uint32_t pa = 0;
+            for (int tile = pair; tile < total_tiles; tile += npairs) {
+                const int m0 = (tile % m_pairs) * (2 * kBM) + static_cast<int>(rank) * kBM;
+                for (int it = 0; it < nsteps; ++it) {
+                    if (!mbar_wait_cluster(&a_empty[sa], pa ^ 1, abort_flag)) goto done;
+                    if (rank == 0) mbar_arrive_expect_tx(&a_full[sa], 2 * Cfg::kABytes);
+                    if (it < args.main_steps)
+                        tma_load_2d_pair(slot_a + sa * Cfg::kABytes, &tm_act, full0 + 8u * sa,
+                                         it * kBK, m0);
+                    else
+                        tma_load_2d_pair(slot_a + sa * Cfg::kABytes, &tm_la, full0 + 8u * sa,
+                                         (it - args.main_steps) * kBK, m0);
+                    if (++sa == SA) { sa = 0; pa ^= 1; }
+                }
+            }
+        }
+    } else if (warp == kTmaCWarp) {
+        // ------------------------------------------------ TMA: 4-bit codes
+        if (lane == 0) {
+            int sc = 0;
+            uint32_t pc = 0;
+            for (int tile = pair; tile < total_tiles; tile += npairs) {
+                const int nh = (tile / m_pairs) * BN + static_cast<int>(rank) * BH;
+                for (int it = 0; it < nsteps; ++it) {
+                    if (!mbar_wait(&c_empty[sc], pc ^ 1, abort_flag)) goto done;
+                    uint8_t *c = slot_c + sc * Cfg::kCBytes;
+                    if (it < args.main_steps) {
+                        mbar_arrive_expect_tx(&c_full[sc], Cfg::kCBytes);
+                        if (!DGRAD) {
+                            tma_load_2d(c, &tm_codes, &c_full[sc], it * (kBK / 2), nh);
+                        } else {
+#pragma unroll
+                            for (int kb = 0; kb < BH / 64; ++kb)
+                                tma_load_2d(c + kb * 2048, &tm_codes, &c_full[sc], nh / 2 + kb * 32,
+                                            it * kBK);
+                        }
+                    } else {
+                        mbar_arrive(&c_full[sc]);      // LoRA stage: no codes
+                    }
+                    if (++sc == SC) { sc = 0; pc ^= 1; }
+                }
+            }
+        }
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA
+        if (lane == 0 && rank == 0) {
+            int sa = 0, sb = 0, ab = 0;
+            uint32_t pa = 0, pb = 0, aph = 0;
+            const uint32_t a_base = smem_u32(slot_a), b_base = smem_u32(slot_b);
+            for (int tile = pair; tile < total_tiles; tile += npairs) {
+                if (!mbar_wait_cluster(&acc_empty[ab], aph ^ 1, abort_flag)) goto done;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + ab * BN;
+                for (int it = 0; it < nsteps; ++it) {
+                    if (!mbar_wait_cluster(&a_full[sa], pa, abort_flag)) goto done;
+                    if (!mbar_wait_cluster(&b_full[sb], pb, abort_flag)) goto done;
+                    tc_fence_after();
+                    const uint32_t a_addr = a_base + sa * Cfg::kABytes;
+                    const uint32_t b_addr = b_base + sb * Cfg::kBBytes;
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                        const uint64_t ad = smem_desc_sw128(a_addr + kk * 32, 16, 1024);
+                        const uint64_t bd = DGRAD ? smem_desc_sw128(b_addr + kk * 2048, 8192, 1024)
+                                                  : smem_desc_sw128(b_addr + kk * 32, 16, 1024);
+                        umma_bf16_ss_pair(d_tmem, ad, bd, Cfg::kIdesc, (it > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit_pair(&a_empty[sa], 0x3);
+                    umma_commit_pair(&b_empty[sb], 0x3);
+                    if (++sa == SA) { sa = 0; pa ^= 1; }
+                    if (++sb == SB) { sb = 0; pb ^= 1; }
+                }
+                umma_commit_pair(&acc_full[ab], 0x3);
+                if (++ab == 2) { ab = 0; aph ^= 1; }
+            }
+        }
+    } else if (warp < kEpiWarp0 + 4) {
+        // ------------------------------------------------------- epilogue
+        const int q = warp - kEpiWarp0;                   // TMEM lane quadrant (== warp % 4)
+        const uint32_t empty0 = mapa_shared(smem_u32(acc_empty), 0);
+        int ab = 0;
+        uint32_t aph = 0;
+        for (int tile = pair; tile < total_tiles; tile += npairs) {
+            const int m0 = (tile % m_pairs) * (2 * kBM) + static_cast<int>(rank) * kBM;
+            const int n0 = (tile / m_pairs) * BN;
+            if (!mbar_wait_cluster(&acc_full[ab], aph, abort_flag)) goto done;
+            tc_fence_after();
+            const int row = m0 + q * 32 + lane;
+            uint16_t *drow = args.D + static_cast<int64_t>(row) * args.out;
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem_base + ((q * 32) << 16) + ab * BN + c * 32, v);
+                tmem_ld_wait();
+                if (row < args.M) {
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        const int col = n0 + c * 32 + g * 8;
+                        if (col < args.out) {
+                            uint32_t p[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                __nv_bfloat162 h2 = __floats2bfloat162_rn(
+                                    __uint_as_float(v[g * 8 + 2 * e]),
+                                    __uint_as_float(v[g * 8 + 2 * e + 1]));
+                                p[e] = *reinterpret_cast<uint32_t *>(&h2);
+                            }
+                            *reinterpret_cast<uint4 *>(drow + col) = make_uint4(p[0], p[1], p[2], p[3]);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(empty0 + 8u * ab);
+            if (++ab == 2) { ab = 0; aph ^= 1; }
+        }
+    } else {
+        // -------------------------------------------------- dequantisation
+        // G groups of BH threads; group g takes the stages whose global index
+        // is g mod G. Thread i of a group owns one work item per stage:
+        //   forward: W row nh + i, block `it`
+        //   dgrad:   W row 64 it + r_loc, block nh/64 + kb
+        // where nh is the first B column this CTA holds. Eight consecutive
+        // lanes take eight consecutive rows of one 8-row swizzle atom, so each
+        // 8-lane phase of a 16-byte shared access hits distinct banks.
+        const int t = threadIdx.x - kDequantWarp0 * 32;
+        const int grp = t / BH;
+        const int i = t % BH;
+        constexpr int kBPR = BH / 64;
+        const int kb = DGRAD ? (i / 8) % kBPR : 0;
+        const int r_loc = DGRAD ? (i / (8 * kBPR)) * 8 + (i & 7) : i;
+        const uint32_t row_off = DGRAD ? static_cast<uint32_t>(kb * 8192 + r_loc * 128)
+                                       : static_cast<uint32_t>(i * 128);
+        // code tiles carry the 32-byte TMA swizzle: 16-byte chunk hh of row j
+        // sits at chunk hh ^ ((j >> 2) & 1)
+        const uint32_t code_off = DGRAD ? static_cast<uint32_t>(kb * 2048 + r_loc * 32)
+                                        : static_cast<uint32_t>(i * 32);
+        const uint32_t cswz = static_cast<uint32_t>((r_loc >> 2) & 1);
+        const uint32_t swz = static_cast<uint32_t>(r_loc & 7);
+        const uint32_t full0 = mapa_shared(smem_u32(b_full), 0);
+
+        // a position in this group's walk over (tile, stage)
+        struct Pos {
+            int tile, it;
+            int64_t item;      // W row (forward) or W block column (dgrad); -1 outside W
+        };
+        auto set_tile = [&](Pos &p) {
+            p.item = -1;
+            if (p.tile >= total_tiles) return;
+            const int64_t nh = static_cast<int64_t>(p.tile / m_pairs) * BN + rank * BH;
+            if (!DGRAD) {
+                if (nh + i < args.Nw) p.item = nh + i;
+            } else {
+                if (nh / 64 + kb < args.kblocks) p.item = nh / 64 + kb;
+            }
+        };
+        auto step = [&](Pos &p, int n) {
+            p.it += n;
+            bool moved = false;
+            while (p.it >= nsteps && p.tile < total_tiles) {
+                p.it -= nsteps;
+                p.tile += npairs;
+                moved = true;
+            }
+            if (moved) set_tile(p);
+        };
+        auto block_of = [&](const Pos &p) -> int64_t {
+            if (p.tile >= total_tiles || p.it >= args.main_steps || p.item < 0) return -1;
+            if (!DGRAD) return p.item * args.kblocks + p.it;
+            const int64_t wrow = static_cast<int64_t>(p.it) * kBK + r_loc;
+            return wrow < args.Nw ? wrow * args.kblocks + p.item : -1;
+        };
+        // raw scale of a block: q8 and c_g under double quantisation, else absmax
+        struct RawScale { int64_t b; uint32_t q8; float v; };
+        auto load_scale = [&](int64_t b) -> RawScale {
+            RawScale rs{b, 0u, 0.0f};
+            if (b < 0) return rs;
+            if (args.dq) {
+                rs.q8 = __ldg(args.q8 + b);
+                rs.v = __ldg(args.cg + (b >> 8));
+            } else {
+                rs.v = __ldg(args.absmax + b);
+            }
+            return rs;
+        };
+
+        Pos cur{pair, 0, -1};
+        set_tile(cur);
+        step(cur, grp);
+        // The scale of the next item is loaded after this item's last fence,
+        // so that no load is outstanding across a proxy fence.
+        RawScale cs = load_scale(block_of(cur));
+        int sb = grp, sc = grp;
+        uint32_t pb = 0, pc = 0;
+        while (cur.tile < total_tiles) {
+            const bool main = cur.it < args.main_steps;
+
+            if (!mbar_wait(&c_full[sc], pc, abort_flag)) goto done;
+            uint32_t out[32];
+            if (main) {
+                const uint8_t *cp = slot_c + sc * Cfg::kCBytes + code_off;
+                const uint4 h0 = *reinterpret_cast<const uint4 *>(cp + 16 * cswz);
+                const uint4 h1 = *reinterpret_cast<const uint4 *>(cp + 16 * (cswz ^ 1));
+                // blocks outside W get scale 0: every level maps to +-0
+                float s = 0.0f;
+                if (cs.b >= 0)
+                    s = args.dq ? __fmul_rn(static_cast<float>(cs.q8), __fdiv_rn(cs.v, 127.0f))
+                                : cs.v;
+                const BlockLut L = make_block_lut(s);
+                const uint32_t words[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+#pragma unroll
+                for (int wd = 0; wd < 8; ++wd) {
+                    uint32_t o[4];
+                    dequant8(L, words[wd], o);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) out[4 * wd + e] = o[e];
+                }
+            } else {
+                // LoRA stage: the adapter tile comes straight from global memory
+                //   forward: B[nh + i][64 ls .. +64)           (zero beyond r, N)
+                //   dgrad:   A[64 ls + r_loc][64 item .. +64)  (zero beyond r, K)
+                const int ls = cur.it - args.main_steps;
+                const uint16_t *src = nullptr;
+                int nvalid = 0;   // valid 8-element chunks
+                if (cur.item >= 0) {
+                    if (!DGRAD) {
+                        const int j0 = 64 * ls;
+                        if (j0 < args.r) {
+                            src = args.lora_b + cur.item * args.r + j0;
+                            nvalid = (args.r - j0) / 8 >= 8 ? 8 : (args.r - j0) / 8;
+                        }
+                    } else {
+                        const int j = 64 * ls + r_loc;
+                        const int64_t k0 = cur.item * 64;
+                        if (j < args.r) {
+                            src = args.lora_b + static_cast<int64_t>(j) * args.Kw + k0;
+                            nvalid = (args.Kw - k0) / 8 >= 8 ? 8 : static_cast<int>((args.Kw - k0) / 8);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint4 v = make_uint4(0, 0, 0, 0);
+                    if (c < nvalid) v = __ldg(reinterpret_cast<const uint4 *>(src) + c);
+                    out[4 * c] = v.x;
+                    out[4 * c + 1] = v.y;
+                    out[4 * c + 2] = v.z;
+                    out[4 * c + 3] = v.w;
+                }
+            }
+            // codes and scales are consumed (out depends on them): release the slot
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&c_empty[sc]);
+
+            if (!mbar_wait_cluster(&b_empty[sb], pb ^ 1, abort_flag)) goto done;
+            uint8_t *brow = slot_b + sb * Cfg::kBBytes + row_off;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4 *>(brow + ((c ^ swz) << 4)) =
+                    make_uint4(out[4 * c], out[4 * c + 1], out[4 * c + 2], out[4 * c + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(full0 + 8u * sb);
+
+            sb += G;
+            if (sb >= SB) { sb -= SB; pb ^= 1; }
+            sc += G;
+            if (sc >= SC) { sc -= SC; pc ^= 1; }
+            step(cur, G);
+            cs = load_scale(block_of(cur));
+        }
+    }
+done:
+    __syncthreads();
+    cluster_sync();            // neither CTA leaves while the other may still use its memory
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, Cfg::kTmemCols);
+    }
+}
+
+}  // namespace nf4

@@ -15,6 +15,7 @@
 
 #include "codec.cuh"
 #include "gemm_tc.cuh"
+#include "gemm_pair_tc.cuh"
 #include "skinny_tc.cuh"
 #include "decode.cuh"
 
@@ -348,6 +349,101 @@ nf4_status launch_gemm(const nf4_weight *w, const uint16_t *act, int64_t M, int6
     return NF4_OK;
 }
 
+// Clusters of two CTAs of one pair-kernel configuration that can be resident
+// at once on the device (0 if the query fails).
+template <int BN, bool DGRAD, int G>
+int pair_capacity(int dev) {
+    using Cfg = PairCfg<BN, DGRAD, G>;
+    static int cache[kMaxDevices] = {0};
+    if (dev < 0 || dev >= kMaxDevices) return 0;
+    if (cache[dev] == 0) {
+        auto kern = qlora_gemm_pair_kernel<BN, DGRAD, G>;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg::kSmemBytes) != cudaSuccess)
+            return 0;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * 74);
+        cfg.blockDim = dim3(Cfg::kThreads);
+        cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            return 0;
+        }
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+template <int BN, bool DGRAD, int G>
+nf4_status launch_gemm_pair(const nf4_weight *w, const uint16_t *act, int64_t M, int64_t red,
+                            int64_t out, const uint16_t *la, int32_t r, const uint16_t *lb,
+                            uint16_t *D, cudaStream_t stream) {
+    using Cfg = PairCfg<BN, DGRAD, G>;
+    CUtensorMap tm_act, tm_codes, tm_la;
+    const int64_t N = w->n, K = w->k;
+    bool ok = make_map(&tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, act, red, M, kBK, kBM,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+    // 4-bit codes of this CTA's half tile: one 32-byte block column per box
+    // (BN/2 rows forward, 64 rows dgrad), 32-byte swizzle
+    ok = ok && make_map(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, K / 2, N, kBK / 2,
+                        DGRAD ? kBK : Cfg::kBH, CU_TENSOR_MAP_SWIZZLE_32B);
+    ok = ok && make_map(&tm_la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, la, r, M, kBK, kBM,
+                        CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!ok) return NF4_ERR_CUDA;
+
+    GemmArgs a;
+    a.M = static_cast<int>(M);
+    a.red = static_cast<int>(red);
+    a.out = static_cast<int>(out);
+    a.main_steps = static_cast<int>((red + kBK - 1) / kBK);
+    a.lora_steps = (r + kBK - 1) / kBK;
+    a.m_tiles = static_cast<int>((M + kBM - 1) / kBM);
+    a.n_tiles = static_cast<int>((out + BN - 1) / BN);
+    a.r = r;
+    a.Nw = N;
+    a.Kw = K;
+    a.kblocks = K / kBlock;
+    a.absmax = w->absmax;
+    a.q8 = w->absmax_q8;
+    a.cg = w->absmax_c;
+    a.dq = w->double_quant;
+    a.lora_b = lb;
+    a.D = D;
+
+    const int dev = current_device();
+    const int cap = pair_capacity<BN, DGRAD, G>(dev);
+    if (cap <= 0) return NF4_ERR_CUDA;
+    const int64_t m_pairs = (M + 2 * kBM - 1) / (2 * kBM);
+    const int pairs = static_cast<int>(std::min<int64_t>(m_pairs * a.n_tiles, cap));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+    cfg.blockDim = dim3(Cfg::kThreads);
+    cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    LaunchTimer t(DGRAD ? KK_GEMM_DGRAD : KK_GEMM_FWD, stream);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, qlora_gemm_pair_kernel<BN, DGRAD, G>, tm_act,
+                                       tm_codes, tm_la, a);
+    t.stop();
+    if (e != cudaSuccess) return NF4_ERR_CUDA;
+    NF4_TRY_CUDA(cudaGetLastError());
+    return NF4_OK;
+}
+
 // Forward for M <= 16 tokens: u = x A^T (and its scaled bf16 copy), then the
 // decode kernel, launched as a programmatic dependent of the first so that
 // it streams the weight while u is being computed.
@@ -418,11 +514,52 @@ int pick_bn(int64_t M, int64_t out, int sms) {
     return best;
 }
 
+// Pair-tile width: the candidate with the smallest (rounds of 256-token
+// tiles over the resident pairs) x (time of one tile). A tile's time is
+// modelled as proportional to (width + 320): measured on B200, a stage costs
+// nearly as much at width 128 as at 256 (activation loads and pipeline
+// latency do not shrink with the width). Dgrad halves must be whole 64-column
+// swizzle atoms, so dgrad chooses between 256 and 128.
+int pick_pair_bn(int64_t M, int64_t out, int pairs, bool dgrad) {
+    const int64_t m_pairs = (M + 2 * kBM - 1) / (2 * kBM);
+    int best = 256;
+    int64_t best_cost = -1;
+    for (int bn : {256, 192, 128}) {
+        if (dgrad && bn == 192) continue;
+        const int64_t tiles = m_pairs * ((out + bn - 1) / bn);
+        const int64_t cost = ((tiles + pairs - 1) / pairs) * (bn + 320);
+        if (best_cost < 0 || cost < best_cost) {
+            best = bn;
+            best_cost = cost;
+        }
+    }
+    return best;
+}
+
+// Dequantisation groups per CTA of the pair kernel (each takes every
+// kPairGroups-th stage).
+constexpr int kPairGroups = 4;
+
 template <bool DGRAD>
 nf4_status launch_gemm_auto(const nf4_weight *w, const uint16_t *act, int64_t M, int64_t red,
                             int64_t out, const uint16_t *la, int32_t r, const uint16_t *lb,
                             uint16_t *D, cudaStream_t stream) {
-    if (pick_bn(M, out, num_sms(current_device())) == 192)
+    const int dev = current_device();
+    const int pairs = pair_capacity<256, DGRAD, kPairGroups>(dev);
+    if (pairs > 0) {
+        switch (pick_pair_bn(M, out, pairs, DGRAD)) {
+        case 128:
+            return launch_gemm_pair<128, DGRAD, kPairGroups>(w, act, M, red, out, la, r, lb, D, stream);
+        case 192:
+            if constexpr (!DGRAD)
+                return launch_gemm_pair<192, DGRAD, kPairGroups>(w, act, M, red, out, la, r, lb, D,
+                                                                 stream);
+            break;
+        default:
+            return launch_gemm_pair<256, DGRAD, kPairGroups>(w, act, M, red, out, la, r, lb, D, stream);
+        }
+    }
+    if (pick_bn(M, out, num_sms(dev)) == 192)
         return launch_gemm<192, DGRAD>(w, act, M, red, out, la, r, lb, D, stream);
     return launch_gemm<256, DGRAD>(w, act, M, red, out, la, r, lb, D, stream);
 }
