@@ -34,12 +34,10 @@ constexpr int kMaxDevices = 64;
 // Optional per-kernel event timing (nf4_profiling / nf4_profile_read)
 // ---------------------------------------------------------------------------
 enum KernelKind {
-    KK_QUANTIZE, KK_DEQUANTIZE, KK_LORA_U, KK_LORA_V, KK_LORA_DB, KK_LORA_DA, KK_LORA_REDUCE,
-    KK_SCALE, KK_ZERO, KK_GEMM_FWD, KK_GEMM_DGRAD, KK_DECODE, KK_DECODE_U, KK_COUNT
+    KK_QUANTIZE, KK_DEQUANTIZE, KK_LORA_U, KK_LORA_V, KK_LORA_DB, KK_LORA_DA, KK_SCALE, KK_ZERO, KK_GEMM_FWD, KK_GEMM_DGRAD, KK_DECODE, KK_DECODE_U, KK_COUNT
 };
 const char *const kKindNames[KK_COUNT] = {
-    "nf4_quantize", "nf4_dequantize", "lora_u", "lora_v", "lora_dB", "lora_dA", "lora_reduce",
-    "lora_scale", "zero_fill", "qlora_gemm_fwd", "qlora_gemm_dgrad", "qlora_decode",
+    "nf4_quantize", "nf4_dequantize", "lora_u", "lora_v", "lora_dB", "lora_dA", "lora_scale", "zero_fill", "qlora_gemm_fwd", "qlora_gemm_dgrad", "qlora_decode",
     "decode_lora_u"};
 
 struct ProfRecord {
@@ -187,73 +185,65 @@ nf4_status check_layer(const nf4_weight *w, const void *x, int64_t M, const void
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Split plan of one rank-r product: P output rows (tiles of 128), Q reduction
-// elements (steps of 64), split so that about two CTAs per SM stream the
-// large operand.
+// elements (steps of 64). The splits of one tile form a cluster of at most
+// kSkMaxSplits CTAs, and the grid is sized to about one CTA per SM. (At r <= 64
+// two CTAs fit on an SM, which lets the clusters pack into one wave; more
+// splits than one per SM measured slower on B200.)
 struct SkinnyPlan {
     int RN, p_tiles, steps, sps, splits;
-    size_t part_bytes;
 };
 
-SkinnyPlan plan_skinny(int64_t P, int64_t Q, int32_t r, int sms, int max_splits = 0) {
+SkinnyPlan plan_skinny(int64_t P, int64_t Q, int32_t r, int sms) {
     SkinnyPlan p{};
     p.RN = r <= 64 ? 64 : 128;
     p.p_tiles = static_cast<int>((P + 127) / 128);
     p.steps = static_cast<int>((Q + 63) / 64);
-    int want = std::max(1, (2 * sms + p.p_tiles - 1) / p.p_tiles);
-    if (max_splits > 0) want = std::min(want, max_splits);
-    int splits = std::max(1, std::min(want, p.steps));
+    int splits = std::max(1, sms / std::max(1, p.p_tiles));
+    splits = std::min({splits, kSkMaxSplits, p.steps});
     p.sps = (p.steps + splits - 1) / splits;
-    p.splits = std::max(1, (p.steps + p.sps - 1) / p.sps);
-    p.part_bytes = size_t(p.splits) * size_t(P) * p.RN * 4;
+    p.splits = (p.steps + p.sps - 1) / p.sps;   // every split has at least one step
     return p;
 }
 
 struct FwdLayout {
-    size_t us, part, total;
+    size_t us, total;
 };
 
-FwdLayout fwd_layout(int64_t M, int64_t n, int64_t k, int32_t r, int sms) {
-    (void)n;
+FwdLayout fwd_layout(int64_t M, int32_t r) {
     FwdLayout L{};
     size_t off = 0;
     L.us = off;   off = align256(off + size_t(M) * r * 2);
-    L.part = off; off = align256(off + plan_skinny(M, k, r, sms).part_bytes);
     L.total = off;
     return L;
 }
 
 struct BwdLayout {
-    size_t us, vs, part, total;
+    size_t us, vs, total;
 };
 
-BwdLayout bwd_layout(int64_t M, int64_t n, int64_t k, int32_t r, int sms) {
+BwdLayout bwd_layout(int64_t M, int32_t r) {
     BwdLayout L{};
     size_t off = 0;
     L.us = off;   off = align256(off + size_t(M) * r * 2);
     L.vs = off;   off = align256(off + size_t(M) * r * 2);
-    size_t part = std::max(std::max(plan_skinny(M, k, r, sms).part_bytes,   // u (recompute)
-                                    plan_skinny(M, n, r, sms).part_bytes),  // v
-                           std::max(plan_skinny(n, M, r, sms).part_bytes,   // dB
-                                    plan_skinny(k, M, r, sms).part_bytes)); // dA
-    L.part = off; off = align256(off + part);
     L.total = off;
     return L;
 }
 
 enum class Major { K, MN };
 
-// Rank-r product out[p][j] = sum_q P(p,q) Q(q,j) through the skinny tcgen05
-// kernel, then the ordered split reduction.
+// Rank-r product out[p][j] = sum_q P(p,q) Q(q,j) through the clustered
+// skinny tcgen05 kernel (split reduction included).
 //   a: row-major bf16 [a_rows, a_cols]; K-major: p = row, q = col; MN-major: q = row, p = col
 //   b: row-major bf16 [b_rows, b_cols]; K-major: j = row, q = col; MN-major: q = row, j = col
 nf4_status skinny_product(int kind, const void *a, int64_t a_rows, int64_t a_cols, Major am,
                           const void *b, int64_t b_rows, int64_t b_cols, Major bm, int32_t r,
-                          float *part, float *out_f32, uint16_t *out_bf16, float scale,
-                          int transposed, cudaStream_t stream, int max_splits = 0) {
+                          float *out_f32, uint16_t *out_bf16, float scale, int transposed,
+                          cudaStream_t stream) {
     const int sms = num_sms(current_device());
     const int64_t P = am == Major::K ? a_rows : a_cols;
     const int64_t Q = am == Major::K ? a_cols : a_rows;
-    const SkinnyPlan pl = plan_skinny(P, Q, r, sms, max_splits);
+    const SkinnyPlan pl = plan_skinny(P, Q, r, sms);
     CUtensorMap ta, tb;
     bool ok = am == Major::K
                   ? make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a, a_cols, a_rows, 64, 128,
@@ -266,16 +256,28 @@ nf4_status skinny_product(int kind, const void *a, int64_t a_rows, int64_t a_col
                     : make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, b, b_cols, b_rows, 64, 64,
                                CU_TENSOR_MAP_SWIZZLE_128B));
     if (!ok) return NF4_ERR_CUDA;
-    SkinnyArgs args{static_cast<int>(P), pl.steps, pl.sps, part};
-    dim3 grid(static_cast<unsigned>(pl.p_tiles), static_cast<unsigned>(pl.splits));
+    SkinnyArgs args{static_cast<int>(P), pl.steps, pl.sps, r, out_f32, out_bf16, scale, transposed};
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(pl.splits), static_cast<unsigned>(pl.p_tiles));
+    cfg.blockDim = dim3(kSkThreads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(pl.splits);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaErrorInvalidValue;
     {
         LaunchTimer t(kind, stream);
 #define NF4_SKINNY_CASE(RN_, AMN, BMN)                                                      \
     if (pl.RN == RN_ && (am == Major::MN) == AMN && (bm == Major::MN) == BMN) {             \
-        auto kern = skinny_gemm_kernel<RN_, AMN, BMN>;                                      \
+        auto kern = skinny_cluster_kernel<RN_, AMN, BMN>;                                   \
         NF4_TRY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                                           SkCfg<RN_, AMN, BMN>::kSmemBytes));               \
-        kern<<<grid, kSkThreads, SkCfg<RN_, AMN, BMN>::kSmemBytes, stream>>>(ta, tb, args); \
+        cfg.dynamicSmemBytes = SkCfg<RN_, AMN, BMN>::kSmemBytes;                            \
+        e = cudaLaunchKernelEx(&cfg, kern, ta, tb, args);                                   \
     }
         NF4_SKINNY_CASE(64, false, false)
         NF4_SKINNY_CASE(128, false, false)
@@ -286,15 +288,7 @@ nf4_status skinny_product(int kind, const void *a, int64_t a_rows, int64_t a_col
 #undef NF4_SKINNY_CASE
         t.stop();
     }
-    NF4_TRY_CUDA(cudaGetLastError());
-    const int64_t total = P * r;
-    const int rgrid = static_cast<int>(std::min<int64_t>((total + 255) / 256, int64_t(sms) * 8));
-    {
-        LaunchTimer t(KK_LORA_REDUCE, stream);
-        skinny_reduce_kernel<<<rgrid, 256, 0, stream>>>(part, pl.splits, static_cast<int>(P), pl.RN,
-                                                        r, out_f32, out_bf16, scale, transposed);
-        t.stop();
-    }
+    if (e != cudaSuccess) return NF4_ERR_CUDA;
     NF4_TRY_CUDA(cudaGetLastError());
     return NF4_OK;
 }
@@ -684,7 +678,7 @@ nf4_status nf4_dequantize(const nf4_weight *w, void *out, int32_t out_bf16, void
 
 size_t qlora_fwd_workspace_bytes(int64_t M, int64_t n, int64_t k, int32_t r) {
     if (M <= 0 || n <= 0 || k <= 0 || r <= 0) return 256;
-    return fwd_layout(M, n, k, r, num_sms(current_device())).total;
+    return fwd_layout(M, r).total;
 }
 
 nf4_status qlora_linear_fwd(const nf4_weight *w, const uint16_t *x, int64_t M, const uint16_t *A,
@@ -695,17 +689,16 @@ nf4_status qlora_linear_fwd(const nf4_weight *w, const uint16_t *x, int64_t M, c
     if (M == 0) return NF4_OK;
     if (!h) return NF4_ERR_INVALID_ARG;
     if (!aligned16(h) || !aligned16(u_out)) return NF4_ERR_ALIGNMENT;
-    const FwdLayout L = fwd_layout(M, w->n, w->k, r, num_sms(current_device()));
+    const FwdLayout L = fwd_layout(M, r);
     if (!workspace || ws_bytes < L.total) return NF4_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return NF4_ERR_ALIGNMENT;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     uint16_t *u_s = reinterpret_cast<uint16_t *>(ws + L.us);
-    float *part = reinterpret_cast<float *>(ws + L.part);
     const float scale = alpha / static_cast<float>(r);
     if (decode_shape(w, M, r)) return launch_decode(w, x, M, A, B, r, scale, h, u_out, u_s, s);
     // u = x A^T (fp32, optional) and bf16((alpha/r) u) for the up-projection stage
-    st = skinny_product(KK_LORA_U, x, M, w->k, Major::K, A, r, w->k, Major::K, r, part, u_out, u_s,
+    st = skinny_product(KK_LORA_U, x, M, w->k, Major::K, A, r, w->k, Major::K, r, u_out, u_s,
                         scale, 0, s);
     if (st != NF4_OK) return st;
     return launch_gemm_auto<false>(w, x, M, w->k, w->n, u_s, r, B, h, s);
@@ -719,31 +712,24 @@ nf4_status qlora_linear_fwd_noalloc(const nf4_weight *w, const uint16_t *x, int6
     if (M == 0) return NF4_OK;
     if (!h) return NF4_ERR_INVALID_ARG;
     if (!aligned16(h) || !aligned16(u_out)) return NF4_ERR_ALIGNMENT;
-    // scratch: bf16 (alpha/r) x A^T [M, r], then fp32 partial sums of x A^T
-    // [splits, M, RN] with as many splits as fit (at least one)
-    const size_t us_bytes = align256(size_t(M) * r * 2);
-    const size_t part_row = size_t(M) * (r <= 64 ? 64 : 128) * 4;
-    if (us_bytes >= kStaticScratchBytes || part_row > kStaticScratchBytes - us_bytes)
-        return NF4_ERR_UNSUPPORTED_SHAPE;
-    const int max_splits = static_cast<int>((kStaticScratchBytes - us_bytes) / part_row);
+    // scratch: bf16 (alpha/r) x A^T [M, r], the workspace of qlora_linear_fwd
+    if (fwd_layout(M, r).total > kStaticScratchBytes) return NF4_ERR_UNSUPPORTED_SHAPE;
     uint8_t *ws = static_cast<uint8_t *>(static_scratch_on_current_device());
     if (!ws) return NF4_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    uint16_t *u_s = reinterpret_cast<uint16_t *>(ws);
-    float *part = reinterpret_cast<float *>(ws + us_bytes);
+    uint16_t *u_s = reinterpret_cast<uint16_t *>(ws + fwd_layout(M, r).us);
     const float scale = alpha / static_cast<float>(r);
     // same dispatch as qlora_linear_fwd: a few tokens take the decode kernel
     if (decode_shape(w, M, r)) return launch_decode(w, x, M, A, B, r, scale, h, u_out, u_s, s);
-    st = skinny_product(KK_LORA_U, x, M, w->k, Major::K, A, r, w->k, Major::K, r, part, u_out, u_s,
-                        scale, 0, s, max_splits);
+    st = skinny_product(KK_LORA_U, x, M, w->k, Major::K, A, r, w->k, Major::K, r, u_out, u_s,
+                        scale, 0, s);
     if (st != NF4_OK) return st;
     return launch_gemm_auto<false>(w, x, M, w->k, w->n, u_s, r, B, h, s);
 }
 
 size_t qlora_bwd_workspace_bytes(int64_t M, int64_t n, int64_t k, int32_t r) {
     if (M < 0 || n <= 0 || k <= 0 || r <= 0) return 256;
-    const int sms = num_sms(current_device());
-    return bwd_layout(std::max<int64_t>(M, 1), n, k, r, sms).total;
+    return bwd_layout(std::max<int64_t>(M, 1), r).total;
 }
 
 nf4_status qlora_linear_bwd(const nf4_weight *w, const uint16_t *x, int64_t M, const uint16_t *A,
@@ -765,14 +751,12 @@ nf4_status qlora_linear_bwd(const nf4_weight *w, const uint16_t *x, int64_t M, c
         NF4_TRY_CUDA(cudaGetLastError());
         return NF4_OK;
     }
-    const int sms = num_sms(current_device());
-    const BwdLayout L = bwd_layout(M, N, K, r, sms);
+    const BwdLayout L = bwd_layout(M, r);
     if (!workspace || ws_bytes < L.total) return NF4_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return NF4_ERR_ALIGNMENT;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     uint16_t *u_s = reinterpret_cast<uint16_t *>(ws + L.us);
     uint16_t *v_s = reinterpret_cast<uint16_t *>(ws + L.vs);
-    float *part = reinterpret_cast<float *>(ws + L.part);
     const float scale = alpha / static_cast<float>(r);
 
     // bf16(s u), from the saved u or recomputed from x
@@ -783,20 +767,20 @@ nf4_status qlora_linear_bwd(const nf4_weight *w, const uint16_t *x, int64_t M, c
         t.stop();
         NF4_TRY_CUDA(cudaGetLastError());
     } else {
-        st = skinny_product(KK_LORA_U, x, M, K, Major::K, A, r, K, Major::K, r, part, nullptr, u_s,
+        st = skinny_product(KK_LORA_U, x, M, K, Major::K, A, r, K, Major::K, r, nullptr, u_s,
                             scale, 0, s);
         if (st != NF4_OK) return st;
     }
     // v = dY B  ->  bf16(s v)
-    st = skinny_product(KK_LORA_V, dY, M, N, Major::K, B, N, r, Major::MN, r, part, nullptr, v_s,
+    st = skinny_product(KK_LORA_V, dY, M, N, Major::K, B, N, r, Major::MN, r, nullptr, v_s,
                         scale, 0, s);
     if (st != NF4_OK) return st;
     // dB = dY^T bf16(s u)   ([N, r])
-    st = skinny_product(KK_LORA_DB, dY, M, N, Major::MN, u_s, M, r, Major::MN, r, part, nullptr, dB,
+    st = skinny_product(KK_LORA_DB, dY, M, N, Major::MN, u_s, M, r, Major::MN, r, nullptr, dB,
                         1.0f, 0, s);
     if (st != NF4_OK) return st;
     // dA = (x^T bf16(s v))^T   ([r, K])
-    st = skinny_product(KK_LORA_DA, x, M, K, Major::MN, v_s, M, r, Major::MN, r, part, nullptr, dA,
+    st = skinny_product(KK_LORA_DA, x, M, K, Major::MN, v_s, M, r, Major::MN, r, nullptr, dA,
                         1.0f, 1, s);
     if (st != NF4_OK) return st;
     // dX = dY W~ + bf16(s v) A

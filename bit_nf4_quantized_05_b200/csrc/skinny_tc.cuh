@@ -6,24 +6,33 @@
 //   dA^T = x^T (s v)    P = x^T:  x  [M, K] read MN-major, Q = bf16(s v) [M, r] (MN-major)
 // (forward down-projection, "QLoRA explained", section "The LoRA adapter
 // path"; the adapter gradients follow by the chain rule with W0 frozen).
-// They stream one large operand once, so they are HBM-bound: the reduction is
-// split across CTAs so that every SM streams, each CTA writes fp32 partial
-// sums, and a second kernel adds the splits in a fixed order (deterministic)
-// and applies the scale, rounding and layout of the destination.
+// They stream one large operand once, so they are HBM-bound. The reduction
+// is split across the CTAs of one thread-block cluster per 128-row output
+// tile (at most 8 splits, sized so that the whole grid is one wave): each CTA
+// streams its share into a tensor-memory accumulator, parks its fp32 partial
+// in its own shared memory, and after a cluster barrier the CTAs add the
+// partials of all splits in split order through distributed shared memory
+// (deterministic) and write the destination with its scale, rounding and
+// layout. No partial sums go to global memory.
 #pragma once
 
 #include "nf4_common.cuh"
 
 namespace nf4 {
 
-constexpr int kSkStages = 6;
+constexpr int kSkStages = 4;     // two CTAs fit on one SM
 constexpr int kSkThreads = 256;   // warp 0 TMA, warp 1 MMA, warps 4..7 epilogue
+constexpr int kSkMaxSplits = 8;   // portable cluster size
 
 struct SkinnyArgs {
     int P;               // output rows (MMA M, tiles of 128)
     int steps;           // reduction steps of 64
     int steps_per_split;
-    float *part;         // [splits][P][RN] fp32
+    int r;               // output columns actually written (<= RN)
+    float *out_f32;      // [P][r] sum, or null
+    uint16_t *out_bf16;  // bf16(scale * sum): [P][r], or [r][P] when transposed; or null
+    float scale;
+    int transposed;
 };
 
 template <int RN, bool A_MN, bool B_MN>
@@ -31,29 +40,40 @@ struct SkCfg {
     static constexpr int kABytes = 128 * 64 * 2;                 // 16 KB
     static constexpr int kBBytes = RN * 64 * 2;                  // RN x 64 bf16
     static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kPartStride = RN + 4;                   // floats per partial row
     static constexpr int kSmemBytes = kSkStages * kStageBytes + 1024 + 256;
     static constexpr uint32_t kIdesc = idesc_bf16_f32(128, RN, A_MN ? 1 : 0, B_MN ? 1 : 0);
     static_assert(RN == 64 || RN == 128, "RN");
+    static_assert(128 * kPartStride * 4 <= kSkStages * kStageBytes, "partial fits the stages");
 };
 
+__device__ __forceinline__ float ld_cluster_f32(uint32_t caddr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(caddr) : "memory");
+    return v;
+}
+
+// Grid (splits, p_tiles), cluster (splits, 1, 1): blockIdx.x is the split.
 template <int RN, bool A_MN, bool B_MN>
-__global__ void __launch_bounds__(kSkThreads, 1)
-skinny_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                   const SkinnyArgs args) {
+__global__ void __launch_bounds__(kSkThreads, 2)
+skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a,
+                      const __grid_constant__ CUtensorMap tm_b, const SkinnyArgs args) {
     using Cfg = SkCfg<RN, A_MN, B_MN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
     uint8_t *slot_a = smem;
     uint8_t *slot_b = smem + kSkStages * Cfg::kABytes;
+    float *part = reinterpret_cast<float *>(smem);   // [128][kPartStride], after the main loop
     uint64_t *bars = reinterpret_cast<uint64_t *>(slot_b + kSkStages * Cfg::kBBytes);
     uint64_t *full = bars, *empty = bars + kSkStages, *done_bar = bars + 2 * kSkStages;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done_bar + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int p0 = blockIdx.x * 128;
-    const int s0 = blockIdx.y * args.steps_per_split;
+    const int split = blockIdx.x, splits = gridDim.x;
+    const int p0 = blockIdx.y * 128;
+    const int s0 = split * args.steps_per_split;
     const int s1 = min(args.steps, s0 + args.steps_per_split);
     const int nsteps = s1 - s0;
 
@@ -121,58 +141,64 @@ skinny_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_consta
         }
         if (ok) umma_commit(done_bar);
     } else if (warp >= 4 && warp < 8) {
+        // accumulator -> this CTA's partial (the stage buffers are free once
+        // the last MMA has completed: every load it waited for has landed)
         const int q = warp - 4;
-        const int p = p0 + q * 32 + lane;
-        float *dst = args.part + (static_cast<int64_t>(blockIdx.y) * args.P + p) * RN;
+        float *prow = part + (q * 32 + lane) * Cfg::kPartStride;
         if (nsteps <= 0) {
-            if (p < args.P)
-                for (int j = 0; j < RN; j += 4)
-                    *reinterpret_cast<float4 *>(dst + j) = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int j = 0; j < RN; j += 4)
+                *reinterpret_cast<float4 *>(prow + j) = make_float4(0.f, 0.f, 0.f, 0.f);
         } else if (mbar_wait(done_bar, 0, abort_flag)) {
             tc_fence_after();
 #pragma unroll 1
             for (int c = 0; c < RN / 32; ++c) {
+                if (c * 32 >= args.r) break;
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(tmem_base + ((q * 32) << 16) + c * 32, v);
                 tmem_ld_wait();
-                if (p < args.P) {
 #pragma unroll
-                    for (int e = 0; e < 32; e += 4)
-                        *reinterpret_cast<float4 *>(dst + c * 32 + e) =
-                            make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
-                                        __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
-                }
+                for (int e = 0; e < 32; e += 4)
+                    *reinterpret_cast<float4 *>(prow + c * 32 + e) =
+                        make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                                    __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
             }
         }
     }
     tc_fence_before();
     __syncthreads();
+    cluster_sync();            // every split's partial is written and visible
+
+    // Ordered sum over the splits: CTA `split` takes its share of the tile's
+    // (row, column) elements, numbered column-major when the destination is
+    // transposed so that consecutive threads write consecutive addresses.
+    {
+        const int r = args.r;
+        const int E = 128 * r;
+        const int e0 = static_cast<int>((static_cast<int64_t>(E) * split) / splits);
+        const int e1 = static_cast<int>((static_cast<int64_t>(E) * (split + 1)) / splits);
+        const uint32_t part_addr = smem_u32(part);
+        for (int e = e0 + threadIdx.x; e < e1; e += kSkThreads) {
+            const int row = args.transposed ? e % 128 : e / r;
+            const int j = args.transposed ? e / 128 : e % r;
+            const int p = p0 + row;
+            if (p >= args.P) continue;
+            const uint32_t off = static_cast<uint32_t>((row * Cfg::kPartStride + j) * 4);
+            float acc = 0.0f;
+            for (int s = 0; s < splits; ++s)
+                acc += ld_cluster_f32(mapa_shared(part_addr + off, static_cast<uint32_t>(s)));
+            if (args.out_f32) args.out_f32[static_cast<int64_t>(p) * r + j] = acc;
+            if (args.out_bf16) {
+                __nv_bfloat16 b = __float2bfloat16_rn(args.scale * acc);
+                const int64_t o = args.transposed ? static_cast<int64_t>(j) * args.P + p
+                                                  : static_cast<int64_t>(p) * r + j;
+                args.out_bf16[o] = *reinterpret_cast<uint16_t *>(&b);
+            }
+        }
+    }
+    cluster_sync();            // no CTA leaves while another still reads its partial
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, RN);
-    }
-}
-
-// out = sum over splits of part[s][p][j] (j < r), in split order; then
-//   out_f32[p][j]  = sum                       (if out_f32)
-//   out_bf16[..]   = bf16(scale * sum)         (if out_bf16; [p][j], or [j][p] when transposed)
-__global__ void skinny_reduce_kernel(const float *__restrict__ part, int splits, int P, int RN, int r,
-                                     float *__restrict__ out_f32, uint16_t *__restrict__ out_bf16,
-                                     float scale, int transposed) {
-    const int64_t total = static_cast<int64_t>(P) * r;
-    const int64_t stride = static_cast<int64_t>(P) * RN;
-    for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
-         e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t p = e / r, j = e % r;
-        const float *src = part + p * RN + j;
-        float acc = 0.0f;
-        for (int s = 0; s < splits; ++s) acc += src[s * stride];
-        if (out_f32) out_f32[p * r + j] = acc;
-        if (out_bf16) {
-            __nv_bfloat16 b = __float2bfloat16_rn(scale * acc);
-            const int64_t o = transposed ? j * P + p : p * r + j;
-            out_bf16[o] = *reinterpret_cast<uint16_t *>(&b);
-        }
     }
 }
 

@@ -140,10 +140,9 @@ QLORA_API nf4_status qlora_linear_fwd(const nf4_weight *w, const uint16_t *x, in
  * entry point: it is an interface variant of this library, not part of the
  * method.
  *   - Same arguments and results as qlora_linear_fwd, minus the workspace.
- *   - Limit: M * (2 r + 4 RN) bytes must fit in 4 MiB, with RN = 64 for
- *     r <= 64 and 128 otherwise (about 14.5 K tokens at r = 16, 10.9 K at
- *     r = 64, 5.4 K at r = 128); larger M returns
- *     NF4_ERR_UNSUPPORTED_SHAPE and launches nothing.
+ *   - Limit: the scaled rank-r activations, M * 2 r bytes, must fit in
+ *     4 MiB (128 K tokens at r = 16, 32 K at r = 64, 16 K at r = 128);
+ *     larger M returns NF4_ERR_UNSUPPORTED_SHAPE and launches nothing.
  *   - The first call on a device looks up the scratch array's device address
  *     (once per device); make that first call before any stream capture.
  *   - Every call on a device shares the one scratch array, and a call only

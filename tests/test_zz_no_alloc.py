@@ -57,8 +57,8 @@ def test_noalloc_forward_matches_workspace_forward(q, name):
 
 
 def test_noalloc_rejects_batches_beyond_its_scratch(q):
-    # r = 64 needs M * (2*64 + 4*64) bytes <= 4 MiB, i.e. at most 10922 tokens
-    N, K, r, M = 64, 64, 64, 10923
+    # r = 64 needs M * 2 * 64 bytes <= 4 MiB, i.e. at most 32768 tokens
+    N, K, r, M = 64, 64, 64, 32769
     dev = torch.device("cuda")
     qw = q.nf4_quantize(torch.randn(N, K, device=dev) * 0.02, double_quant=False)
     x = torch.randn(M, K, device=dev).to(torch.bfloat16)
