@@ -255,7 +255,9 @@ def main():
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
-    q.profiling(True)
+    # Timed region: K steps with only the two step events each (per-launch
+    # events would sit between the kernels and stop each launch from
+    # overlapping the tail of the one before).
     with ClockSampler(local_rank) as clk:
         for i in range(args.steps):
             flush.zero_()                      # L2 flush between timed steps (untimed)
@@ -263,6 +265,14 @@ def main():
             step()
             ends[i].record()
         torch.cuda.synchronize()
+    barrier()
+    # Kernel durations: the same K steps again with the library's per-launch
+    # CUDA events (recorded on the stream each kernel is launched on).
+    q.profiling(True)
+    for i in range(args.steps):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
     barrier()
     q.profiling(False)
     prof = q.profile_read()

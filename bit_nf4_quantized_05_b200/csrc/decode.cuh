@@ -56,13 +56,6 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ void griddep_wait() {
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-__device__ __forceinline__ void griddep_launch_dependents() {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
 // Scale of block b, with the group constant fl32(c_g / 127) cached by the caller.
 __device__ __forceinline__ float decode_scale(const DecodeArgs &a, int64_t b, int64_t &kg_group,
                                               float &kg) {
@@ -221,6 +214,7 @@ qlora_decode_kernel(const DecodeArgs a) {
 
     // LoRA up-projection: needs bf16((alpha/r) x A^T) from the preceding kernel
     griddep_wait();
+    griddep_launch_dependents();
     {
         const int chunks = a.M * a.r / 8;
         for (int c = lane; c < chunks; c += 32)
@@ -264,6 +258,7 @@ __global__ void __launch_bounds__(kDecUThreads)
 decode_lora_u_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ A, int M,
                      int64_t K, int r, float scale, float *__restrict__ u_out,
                      uint16_t *__restrict__ u_s) {
+    griddep_wait();
     griddep_launch_dependents();
     __shared__ float red[kDecUThreads / 32][16];
     const int j = blockIdx.x;

@@ -121,6 +121,8 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
     cluster_sync();            // barriers of both CTAs initialised before any remote use
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    griddep_wait();
+    griddep_launch_dependents();
 
     const int m_pairs = (args.M + 2 * kBM - 1) / (2 * kBM);
     const int total_tiles = m_pairs * args.n_tiles;

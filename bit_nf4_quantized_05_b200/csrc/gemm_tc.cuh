@@ -147,6 +147,8 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red] bf1
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    griddep_wait();
+    griddep_launch_dependents();
 
     const int total_tiles = args.m_tiles * args.n_tiles;
     const int nsteps = args.main_steps + args.lora_steps;

@@ -127,6 +127,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch. Every kernel of this library that is launched
+// as a programmatic dependent first waits for the grid before it in the stream
+// (complete, memory visible), then lets the next grid launch; so a kernel may
+// run its set-up while its predecessor finishes, and any grid that starts early
+// finds every grid two places before it complete.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void griddep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // Thread-block clusters: ranks, cluster addresses, remote arrivals
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t cluster_ctarank() {

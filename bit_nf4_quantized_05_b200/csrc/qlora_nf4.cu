@@ -101,6 +101,34 @@ class LaunchTimer {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Launch as a programmatic dependent of the previous grid in the stream (the
+// kernel waits for it before touching memory), optionally as clusters of
+// cluster_x CTAs along x.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t stream, unsigned cluster_x, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    unsigned n = 0;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+    if (cluster_x > 0) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = cluster_x;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 int current_device() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return -1;
@@ -257,17 +285,7 @@ nf4_status skinny_product(int kind, const void *a, int64_t a_rows, int64_t a_col
                                CU_TENSOR_MAP_SWIZZLE_128B));
     if (!ok) return NF4_ERR_CUDA;
     SkinnyArgs args{static_cast<int>(P), pl.steps, pl.sps, r, out_f32, out_bf16, scale, transposed};
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(pl.splits), static_cast<unsigned>(pl.p_tiles));
-    cfg.blockDim = dim3(kSkThreads);
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = static_cast<unsigned>(pl.splits);
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    const dim3 grid(static_cast<unsigned>(pl.splits), static_cast<unsigned>(pl.p_tiles));
     cudaError_t e = cudaErrorInvalidValue;
     {
         LaunchTimer t(kind, stream);
@@ -276,8 +294,8 @@ nf4_status skinny_product(int kind, const void *a, int64_t a_rows, int64_t a_col
         auto kern = skinny_cluster_kernel<RN_, AMN, BMN>;                                   \
         NF4_TRY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                                           SkCfg<RN_, AMN, BMN>::kSmemBytes));               \
-        cfg.dynamicSmemBytes = SkCfg<RN_, AMN, BMN>::kSmemBytes;                            \
-        e = cudaLaunchKernelEx(&cfg, kern, ta, tb, args);                                   \
+        e = launch_ex(kern, grid, dim3(kSkThreads), SkCfg<RN_, AMN, BMN>::kSmemBytes, stream, \
+                      static_cast<unsigned>(pl.splits), ta, tb, args);                      \
     }
         NF4_SKINNY_CASE(64, false, false)
         NF4_SKINNY_CASE(128, false, false)
@@ -337,8 +355,10 @@ nf4_status launch_gemm(const nf4_weight *w, const uint16_t *act, int64_t M, int6
     NF4_TRY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       Cfg::kSmemBytes));
     LaunchTimer t(DGRAD ? KK_GEMM_DGRAD : KK_GEMM_FWD, stream);
-    kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(tm_act, tm_codes, tm_la, a);
+    const cudaError_t e = launch_ex(kern, dim3(grid), dim3(Cfg::kThreads), Cfg::kSmemBytes, stream,
+                                    0u, tm_act, tm_codes, tm_la, a);
     t.stop();
+    if (e != cudaSuccess) return NF4_ERR_CUDA;
     NF4_TRY_CUDA(cudaGetLastError());
     return NF4_OK;
 }
@@ -417,21 +437,10 @@ nf4_status launch_gemm_pair(const nf4_weight *w, const uint16_t *act, int64_t M,
     if (cap <= 0) return NF4_ERR_CUDA;
     const int64_t m_pairs = (M + 2 * kBM - 1) / (2 * kBM);
     const int pairs = static_cast<int>(std::min<int64_t>(m_pairs * a.n_tiles, cap));
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
-    cfg.blockDim = dim3(Cfg::kThreads);
-    cfg.dynamicSmemBytes = Cfg::kSmemBytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
     LaunchTimer t(DGRAD ? KK_GEMM_DGRAD : KK_GEMM_FWD, stream);
-    cudaError_t e = cudaLaunchKernelEx(&cfg, qlora_gemm_pair_kernel<BN, DGRAD, G>, tm_act,
-                                       tm_codes, tm_la, a);
+    const cudaError_t e =
+        launch_ex(qlora_gemm_pair_kernel<BN, DGRAD, G>, dim3(static_cast<unsigned>(2 * pairs)),
+                  dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, 2u, tm_act, tm_codes, tm_la, a);
     t.stop();
     if (e != cudaSuccess) return NF4_ERR_CUDA;
     NF4_TRY_CUDA(cudaGetLastError());
@@ -453,9 +462,10 @@ nf4_status launch_decode(const nf4_weight *w, const uint16_t *x, int64_t M, cons
                          uint16_t *u_s, cudaStream_t stream) {
     {
         LaunchTimer t(KK_DECODE_U, stream);
-        decode_lora_u_kernel<<<r, kDecUThreads, 0, stream>>>(x, A, static_cast<int>(M), w->k, r,
-                                                            scale, u_out, u_s);
+        const cudaError_t e = launch_ex(decode_lora_u_kernel, dim3(r), dim3(kDecUThreads), 0, stream,
+                                        0u, x, A, static_cast<int>(M), w->k, r, scale, u_out, u_s);
         t.stop();
+        if (e != cudaSuccess) return NF4_ERR_CUDA;
     }
     NF4_TRY_CUDA(cudaGetLastError());
     DecodeArgs a;
@@ -745,9 +755,11 @@ nf4_status qlora_linear_bwd(const nf4_weight *w, const uint16_t *x, int64_t M, c
     const int64_t N = w->n, K = w->k;
     if (M == 0) {
         LaunchTimer t(KK_ZERO, s);
-        zero_u16_kernel<<<64, 256, 0, s>>>(dA, int64_t(r) * K);
-        zero_u16_kernel<<<64, 256, 0, s>>>(dB, N * r);
+        const cudaError_t e1 = launch_ex(zero_u16_kernel, dim3(64), dim3(256), 0, s, 0u, dA,
+                                         int64_t(r) * K);
+        const cudaError_t e2 = launch_ex(zero_u16_kernel, dim3(64), dim3(256), 0, s, 0u, dB, N * r);
         t.stop();
+        if (e1 != cudaSuccess || e2 != cudaSuccess) return NF4_ERR_CUDA;
         NF4_TRY_CUDA(cudaGetLastError());
         return NF4_OK;
     }
@@ -762,9 +774,11 @@ nf4_status qlora_linear_bwd(const nf4_weight *w, const uint16_t *x, int64_t M, c
     // bf16(s u), from the saved u or recomputed from x
     if (u) {
         LaunchTimer t(KK_SCALE, s);
-        scale_to_bf16_kernel<<<static_cast<int>(std::min<int64_t>((M * r + 255) / 256, 4096)), 256,
-                               0, s>>>(u, M * r, scale, u_s);
+        const unsigned grid = static_cast<unsigned>(std::min<int64_t>((M * r + 255) / 256, 4096));
+        const cudaError_t e =
+            launch_ex(scale_to_bf16_kernel, dim3(grid), dim3(256), 0, s, 0u, u, M * r, scale, u_s);
         t.stop();
+        if (e != cudaSuccess) return NF4_ERR_CUDA;
         NF4_TRY_CUDA(cudaGetLastError());
     } else {
         st = skinny_product(KK_LORA_U, x, M, K, Major::K, A, r, K, Major::K, r, nullptr, u_s,

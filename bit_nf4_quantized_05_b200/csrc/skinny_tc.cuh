@@ -96,6 +96,8 @@ skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    griddep_wait();
+    griddep_launch_dependents();
 
     if (warp == 0 && lane == 0) {
         for (int it = 0; it < nsteps; ++it) {
@@ -205,6 +207,8 @@ skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a,
 // dst[i] = bf16(scale * src[i])
 __global__ void scale_to_bf16_kernel(const float *__restrict__ src, int64_t n, float scale,
                                      uint16_t *__restrict__ dst) {
+    griddep_wait();
+    griddep_launch_dependents();
     for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
          e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         __nv_bfloat16 b = __float2bfloat16_rn(scale * src[e]);
@@ -213,6 +217,8 @@ __global__ void scale_to_bf16_kernel(const float *__restrict__ src, int64_t n, f
 }
 
 __global__ void zero_u16_kernel(uint16_t *__restrict__ p, int64_t n) {
+    griddep_wait();
+    griddep_launch_dependents();
     for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
          e += static_cast<int64_t>(gridDim.x) * blockDim.x)
         p[e] = 0;
