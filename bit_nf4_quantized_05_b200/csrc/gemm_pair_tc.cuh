@@ -59,6 +59,73 @@ struct PairCfg {
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
+// The work of one pair: segments of stages [k0, k1) of a tile.
+//   Whole-tile schedule: tiles p, p + P, p + 2P, ... with every stage.
+//   Stream-K schedule: the units (tile, stage), numbered tile-major, are cut
+//   into P contiguous runs [W p / P, W (p + 1) / P) with W = T S; with T > P
+//   every run spans more than one tile, so a tile is split between at most
+//   two consecutive pairs: its head (stages [0, k)) is the last segment of
+//   pair p and its tail (stages [k, S)) the first segment of pair p + 1.
+struct PairSeg {
+    int tile, k0, k1;
+};
+
+struct PairSched {
+    int S, T, P, p, sk;
+    int64_t u0, u1;
+
+    __device__ __forceinline__ void init(int S_, int T_, int P_, int p_, int sk_) {
+        S = S_; T = T_; P = P_; p = p_; sk = sk_;
+        const int64_t W = static_cast<int64_t>(T) * S;
+        u0 = sk ? (W * p) / P : 0;
+        u1 = sk ? (W * (p + 1)) / P : 0;
+    }
+    __device__ __forceinline__ bool first(PairSeg &g) const {
+        if (!sk) {
+            g = {p, 0, S};
+            return p < T;
+        }
+        if (u0 >= u1) return false;
+        const int t = static_cast<int>(u0 / S);
+        const int k0 = static_cast<int>(u0 - static_cast<int64_t>(t) * S);
+        const int64_t rest = u1 - static_cast<int64_t>(t) * S;
+        g = {t, k0, rest < S ? static_cast<int>(rest) : S};
+        return true;
+    }
+    __device__ __forceinline__ bool next(PairSeg &g) const {
+        if (!sk) {
+            g = {g.tile + P, 0, S};
+            return g.tile < T;
+        }
+        const int t = g.tile + 1;
+        const int64_t rest = u1 - static_cast<int64_t>(t) * S;
+        if (g.k1 < S || rest <= 0) return false;
+        g = {t, 0, rest < S ? static_cast<int>(rest) : S};
+        return true;
+    }
+};
+
+// Bounded wait until a flag in global memory becomes non-zero (acquire, GPU
+// scope). On timeout the kernel's status is set and the caller gives up.
+__device__ __forceinline__ bool wait_flag_gpu(const int *flag, volatile int *abort_flag) {
+    const long long t0 = clock64();
+    while (true) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+        if (v != 0) return true;
+        if (*abort_flag) return false;
+        if (clock64() - t0 > kWaitLimitCycles) {
+            record_status(NF4_ERR_TIMEOUT);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void set_flag_gpu(int *flag) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(1) : "memory");
+}
+
 template <int BN, bool DGRAD, int G>
 __global__ void __launch_bounds__(PairCfg<BN, DGRAD, G>::kThreads, 1)
 qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red] bf16, box {64,128}
@@ -127,6 +194,9 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
     const int m_pairs = (args.M + 2 * kBM - 1) / (2 * kBM);
     const int total_tiles = m_pairs * args.n_tiles;
     const int nsteps = args.main_steps + args.lora_steps;
+    PairSched sched;
+    sched.init(nsteps, total_tiles, npairs, pair, args.sk);
+    PairSeg sg;
 
     if (warp == kTmaAWarp) {
         // ------------------------------------------------ TMA: activations
@@ -134,9 +204,9 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
             const uint32_t full0 = mapa_shared(smem_u32(a_full), 0);
             int sa = 0;
             uint32_t pa = 0;
-            for (int tile = pair; tile < total_tiles; tile += npairs) {
-                const int m0 = (tile % m_pairs) * (2 * kBM) + static_cast<int>(rank) * kBM;
-                for (int it = 0; it < nsteps; ++it) {
+            for (bool more = sched.first(sg); more; more = sched.next(sg)) {
+                const int m0 = (sg.tile % m_pairs) * (2 * kBM) + static_cast<int>(rank) * kBM;
+                for (int it = sg.k0; it < sg.k1; ++it) {
                     if (!mbar_wait_cluster(&a_empty[sa], pa ^ 1, abort_flag)) goto done;
                     if (rank == 0) mbar_arrive_expect_tx(&a_full[sa], 2 * Cfg::kABytes);
                     if (it < args.main_steps)
@@ -154,9 +224,9 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
         if (lane == 0) {
             int sc = 0;
             uint32_t pc = 0;
-            for (int tile = pair; tile < total_tiles; tile += npairs) {
-                const int nh = (tile / m_pairs) * BN + static_cast<int>(rank) * BH;
-                for (int it = 0; it < nsteps; ++it) {
+            for (bool more = sched.first(sg); more; more = sched.next(sg)) {
+                const int nh = (sg.tile / m_pairs) * BN + static_cast<int>(rank) * BH;
+                for (int it = sg.k0; it < sg.k1; ++it) {
                     if (!mbar_wait(&c_empty[sc], pc ^ 1, abort_flag)) goto done;
                     uint8_t *c = slot_c + sc * Cfg::kCBytes;
                     if (it < args.main_steps) {
@@ -182,11 +252,11 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
             int sa = 0, sb = 0, ab = 0;
             uint32_t pa = 0, pb = 0, aph = 0;
             const uint32_t a_base = smem_u32(slot_a), b_base = smem_u32(slot_b);
-            for (int tile = pair; tile < total_tiles; tile += npairs) {
+            for (bool more = sched.first(sg); more; more = sched.next(sg)) {
                 if (!mbar_wait_cluster(&acc_empty[ab], aph ^ 1, abort_flag)) goto done;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + ab * BN;
-                for (int it = 0; it < nsteps; ++it) {
+                for (int it = sg.k0; it < sg.k1; ++it) {
                     if (!mbar_wait_cluster(&a_full[sa], pa, abort_flag)) goto done;
                     if (!mbar_wait_cluster(&b_full[sb], pb, abort_flag)) goto done;
                     tc_fence_after();
@@ -197,7 +267,8 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
                         const uint64_t ad = smem_desc_sw128(a_addr + kk * 32, 16, 1024);
                         const uint64_t bd = DGRAD ? smem_desc_sw128(b_addr + kk * 2048, 8192, 1024)
                                                   : smem_desc_sw128(b_addr + kk * 32, 16, 1024);
-                        umma_bf16_ss_pair(d_tmem, ad, bd, Cfg::kIdesc, (it > 0 || kk > 0) ? 1u : 0u);
+                        umma_bf16_ss_pair(d_tmem, ad, bd, Cfg::kIdesc,
+                                          (it > sg.k0 || kk > 0) ? 1u : 0u);
                     }
                     umma_commit_pair(&a_empty[sa], 0x3);
                     umma_commit_pair(&b_empty[sb], 0x3);
@@ -210,43 +281,93 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
         }
     } else if (warp < kEpiWarp0 + 4) {
         // ------------------------------------------------------- epilogue
+        // Per segment: a whole tile is rounded to bf16 and stored; the tail
+        // of a split tile is stored as an fp32 partial (layout [BN/32][128
+        // rows][32], 128-byte rows per thread) and its flag set; the head of
+        // a split tile waits for the flag of the next pair's partial, adds it
+        // and stores the sum. Flags are per epilogue warp: warp q of the head
+        // reads exactly the rows warp q of the tail wrote.
         const int q = warp - kEpiWarp0;                   // TMEM lane quadrant (== warp % 4)
         const uint32_t empty0 = mapa_shared(smem_u32(acc_empty), 0);
+        constexpr int kChunks = BN / 32;
         int ab = 0;
         uint32_t aph = 0;
-        for (int tile = pair; tile < total_tiles; tile += npairs) {
-            const int m0 = (tile % m_pairs) * (2 * kBM) + static_cast<int>(rank) * kBM;
-            const int n0 = (tile / m_pairs) * BN;
+        for (bool more = sched.first(sg); more; more = sched.next(sg)) {
+            const int m0 = (sg.tile % m_pairs) * (2 * kBM) + static_cast<int>(rank) * kBM;
+            const int n0 = (sg.tile / m_pairs) * BN;
+            const bool tail = sg.k0 > 0;
+            const bool head = !tail && sg.k1 < nsteps;
+            const int rloc = q * 32 + lane;               // row within this CTA's 128
             if (!mbar_wait_cluster(&acc_full[ab], aph, abort_flag)) goto done;
             tc_fence_after();
-            const int row = m0 + q * 32 + lane;
-            uint16_t *drow = args.D + static_cast<int64_t>(row) * args.out;
+            if (tail) {
+                float *pp = args.partial +
+                            (static_cast<int64_t>(pair) * 2 + rank) * kChunks * (128 * 32) + rloc * 32;
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem_base + ((q * 32) << 16) + ab * BN + c * 32, v);
-                tmem_ld_wait();
-                if (row < args.M) {
+                for (int c = 0; c < kChunks; ++c) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tmem_base + ((q * 32) << 16) + ab * BN + c * 32, v);
+                    tmem_ld_wait();
 #pragma unroll
-                    for (int g = 0; g < 4; ++g) {
-                        const int col = n0 + c * 32 + g * 8;
-                        if (col < args.out) {
-                            uint32_t p[4];
+                    for (int e = 0; e < 32; e += 4)
+                        *reinterpret_cast<float4 *>(pp + c * (128 * 32) + e) =
+                            make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                                        __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+                }
+                tc_fence_before();
+                __syncwarp();                 // this warp's 32 rows of the partial are written
+                if (lane == 0) {
+                    mbar_arrive_cluster(empty0 + 8u * ab);
+                    __threadfence();
+                    set_flag_gpu(args.flags + (pair * 2 + rank) * 4 + q);
+                }
+            } else {
+                const float *pp = nullptr;
+                if (head) {
+                    // rows rloc of the partial were written by warp q of the
+                    // same-rank CTA of the next pair
+                    const int src = (pair + 1) * 2 + static_cast<int>(rank);
+                    if (!wait_flag_gpu(args.flags + src * 4 + q, abort_flag)) goto done;
+                    pp = args.partial + static_cast<int64_t>(src) * kChunks * (128 * 32) + rloc * 32;
+                }
+                const int row = m0 + rloc;
+                uint16_t *drow = args.D + static_cast<int64_t>(row) * args.out;
+#pragma unroll 1
+                for (int c = 0; c < kChunks; ++c) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tmem_base + ((q * 32) << 16) + ab * BN + c * 32, v);
+                    tmem_ld_wait();
+                    if (row < args.M) {
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                __nv_bfloat162 h2 = __floats2bfloat162_rn(
-                                    __uint_as_float(v[g * 8 + 2 * e]),
-                                    __uint_as_float(v[g * 8 + 2 * e + 1]));
-                                p[e] = *reinterpret_cast<uint32_t *>(&h2);
+                        for (int g = 0; g < 4; ++g) {
+                            const int col = n0 + c * 32 + g * 8;
+                            if (col < args.out) {
+                                float f[8];
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[g * 8 + e]);
+                                if (head) {
+                                    const float4 *pv = reinterpret_cast<const float4 *>(
+                                        pp + c * (128 * 32) + g * 8);
+                                    const float4 p0 = pv[0], p1 = pv[1];
+                                    f[0] += p0.x; f[1] += p0.y; f[2] += p0.z; f[3] += p0.w;
+                                    f[4] += p1.x; f[5] += p1.y; f[6] += p1.z; f[7] += p1.w;
+                                }
+                                uint32_t p[4];
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    __nv_bfloat162 h2 = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
+                                    p[e] = *reinterpret_cast<uint32_t *>(&h2);
+                                }
+                                *reinterpret_cast<uint4 *>(drow + col) =
+                                    make_uint4(p[0], p[1], p[2], p[3]);
                             }
-                            *reinterpret_cast<uint4 *>(drow + col) = make_uint4(p[0], p[1], p[2], p[3]);
                         }
                     }
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(empty0 + 8u * ab);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(empty0 + 8u * ab);
             if (++ab == 2) { ab = 0; aph ^= 1; }
         }
     } else {
@@ -274,7 +395,8 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
         const uint32_t swz = static_cast<uint32_t>(r_loc & 7);
         const uint32_t full0 = mapa_shared(smem_u32(b_full), 0);
 
-        // a position in this group's walk over (tile, stage)
+        // a position in this group's walk over the pair's (tile, stage) units,
+        // in the order of the schedule's segments
         struct Pos {
             int tile, it;
             int64_t item;      // W row (forward) or W block column (dgrad); -1 outside W
@@ -289,15 +411,25 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
                 if (nh / 64 + kb < args.kblocks) p.item = nh / 64 + kb;
             }
         };
+        const int tile_step = args.sk ? 1 : npairs;
         auto step = [&](Pos &p, int n) {
             p.it += n;
             bool moved = false;
-            while (p.it >= nsteps && p.tile < total_tiles) {
+            while (p.it >= nsteps) {
                 p.it -= nsteps;
-                p.tile += npairs;
+                p.tile += tile_step;
                 moved = true;
             }
             if (moved) set_tile(p);
+        };
+        // the walk ends at unit (end_tile, end_it)
+        int end_tile = total_tiles, end_it = 0;
+        if (args.sk) {
+            end_tile = static_cast<int>(sched.u1 / nsteps);
+            end_it = static_cast<int>(sched.u1 - static_cast<int64_t>(end_tile) * nsteps);
+        }
+        auto alive = [&](const Pos &p) -> bool {
+            return p.tile < end_tile || (p.tile == end_tile && p.it < end_it);
         };
         auto block_of = [&](const Pos &p) -> int64_t {
             if (p.tile >= total_tiles || p.it >= args.main_steps || p.item < 0) return -1;
@@ -320,6 +452,10 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
         };
 
         Pos cur{pair, 0, -1};
+        if (args.sk) {
+            cur.tile = static_cast<int>(sched.u0 / nsteps);
+            cur.it = static_cast<int>(sched.u0 - static_cast<int64_t>(cur.tile) * nsteps);
+        }
         set_tile(cur);
         step(cur, grp);
         // The scale of the next item is loaded after this item's last fence,
@@ -327,7 +463,7 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
         RawScale cs = load_scale(block_of(cur));
         int sb = grp, sc = grp;
         uint32_t pb = 0, pc = 0;
-        while (cur.tile < total_tiles) {
+        while (alive(cur)) {
             const bool main = cur.it < args.main_steps;
 
             if (!mbar_wait(&c_full[sc], pc, abort_flag)) goto done;

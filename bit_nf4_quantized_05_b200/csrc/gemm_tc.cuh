@@ -62,6 +62,10 @@ struct GemmArgs {
     int dq;
     const uint16_t *lora_b;   // forward: B [N, r]; dgrad: A [r, K]
     uint16_t *D;        // [M, out] bf16
+    // stream-K schedule (CTA-pair kernel only): 0 = whole tiles round-robin
+    int sk;
+    float *partial;     // [pairs][2][BN/32][128][32] fp32 partial tiles
+    int *flags;         // [pairs][2][4 epilogue warps], zero at launch; 1 = rows written
 };
 
 template <int BN, bool DGRAD>

@@ -233,27 +233,48 @@ SkinnyPlan plan_skinny(int64_t P, int64_t Q, int32_t r, int sms) {
     return p;
 }
 
-struct FwdLayout {
-    size_t us, total;
+// Stream-K scratch of one fused GEMM launch: per CTA pair one fp32 partial
+// tile (2 CTAs x 128 rows x 256 columns) and 8 flags (2 CTAs x 4 epilogue
+// warps). Sized for sms / 2 pairs, the most that can be resident.
+constexpr int kSkFlagsPerPair = 8;
+int sk_pairs_max(int sms) { return std::max(1, sms / 2); }
+size_t sk_flag_bytes(int sms) { return size_t(sk_pairs_max(sms)) * kSkFlagsPerPair * 4; }
+size_t sk_partial_bytes(int sms) { return size_t(sk_pairs_max(sms)) * 2 * 128 * 256 * 4; }
+
+struct SkBuf {
+    float *partial;
+    int *flags;
+    int pairs_max;
 };
 
-FwdLayout fwd_layout(int64_t M, int32_t r) {
+struct FwdLayout {
+    size_t us, flags, partial, total;
+};
+
+// with_sk = false: only the bf16 rank-r activations (the whole-tile schedule)
+FwdLayout fwd_layout(int64_t M, int32_t r, int sms, bool with_sk = true) {
     FwdLayout L{};
     size_t off = 0;
     L.us = off;   off = align256(off + size_t(M) * r * 2);
+    if (with_sk) {
+        L.flags = off;   off = align256(off + sk_flag_bytes(sms));
+        L.partial = off; off = align256(off + sk_partial_bytes(sms));
+    }
     L.total = off;
     return L;
 }
 
 struct BwdLayout {
-    size_t us, vs, total;
+    size_t us, vs, flags, partial, total;
 };
 
-BwdLayout bwd_layout(int64_t M, int32_t r) {
+BwdLayout bwd_layout(int64_t M, int32_t r, int sms) {
     BwdLayout L{};
     size_t off = 0;
-    L.us = off;   off = align256(off + size_t(M) * r * 2);
-    L.vs = off;   off = align256(off + size_t(M) * r * 2);
+    L.us = off;      off = align256(off + size_t(M) * r * 2);
+    L.vs = off;      off = align256(off + size_t(M) * r * 2);
+    L.flags = off;   off = align256(off + sk_flag_bytes(sms));
+    L.partial = off; off = align256(off + sk_partial_bytes(sms));
     L.total = off;
     return L;
 }
@@ -267,7 +288,7 @@ enum class Major { K, MN };
 nf4_status skinny_product(int kind, const void *a, int64_t a_rows, int64_t a_cols, Major am,
                           const void *b, int64_t b_rows, int64_t b_cols, Major bm, int32_t r,
                           float *out_f32, uint16_t *out_bf16, float scale, int transposed,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, int *zero_ints = nullptr, int zero_count = 0) {
     const int sms = num_sms(current_device());
     const int64_t P = am == Major::K ? a_rows : a_cols;
     const int64_t Q = am == Major::K ? a_cols : a_rows;
@@ -284,7 +305,8 @@ nf4_status skinny_product(int kind, const void *a, int64_t a_rows, int64_t a_col
                     : make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, b, b_cols, b_rows, 64, 64,
                                CU_TENSOR_MAP_SWIZZLE_128B));
     if (!ok) return NF4_ERR_CUDA;
-    SkinnyArgs args{static_cast<int>(P), pl.steps, pl.sps, r, out_f32, out_bf16, scale, transposed};
+    SkinnyArgs args{static_cast<int>(P), pl.steps, pl.sps, r,          out_f32,
+                    out_bf16,            scale,    transposed, zero_ints, zero_count};
     const dim3 grid(static_cast<unsigned>(pl.splits), static_cast<unsigned>(pl.p_tiles));
     cudaError_t e = cudaErrorInvalidValue;
     {
@@ -329,7 +351,7 @@ nf4_status launch_gemm(const nf4_weight *w, const uint16_t *act, int64_t M, int6
                         CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok) return NF4_ERR_CUDA;
 
-    GemmArgs a;
+    GemmArgs a{};
     a.M = static_cast<int>(M);
     a.red = static_cast<int>(red);
     a.out = static_cast<int>(out);
@@ -396,10 +418,12 @@ int pair_capacity(int dev) {
     return cache[dev];
 }
 
+// sk: stream-K scratch, or null for the whole-tile schedule. Stream-K runs
+// when there are more tiles than resident pairs and they do not divide evenly.
 template <int BN, bool DGRAD, int G>
 nf4_status launch_gemm_pair(const nf4_weight *w, const uint16_t *act, int64_t M, int64_t red,
                             int64_t out, const uint16_t *la, int32_t r, const uint16_t *lb,
-                            uint16_t *D, cudaStream_t stream) {
+                            uint16_t *D, cudaStream_t stream, const SkBuf *sk = nullptr) {
     using Cfg = PairCfg<BN, DGRAD, G>;
     CUtensorMap tm_act, tm_codes, tm_la;
     const int64_t N = w->n, K = w->k;
@@ -413,7 +437,7 @@ nf4_status launch_gemm_pair(const nf4_weight *w, const uint16_t *act, int64_t M,
                         CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok) return NF4_ERR_CUDA;
 
-    GemmArgs a;
+    GemmArgs a{};
     a.M = static_cast<int>(M);
     a.red = static_cast<int>(red);
     a.out = static_cast<int>(out);
@@ -436,7 +460,15 @@ nf4_status launch_gemm_pair(const nf4_weight *w, const uint16_t *act, int64_t M,
     const int cap = pair_capacity<BN, DGRAD, G>(dev);
     if (cap <= 0) return NF4_ERR_CUDA;
     const int64_t m_pairs = (M + 2 * kBM - 1) / (2 * kBM);
-    const int pairs = static_cast<int>(std::min<int64_t>(m_pairs * a.n_tiles, cap));
+    const int64_t tiles = m_pairs * a.n_tiles;
+    const bool use_sk = BN == 256 && sk && sk->partial && sk->flags && cap <= sk->pairs_max &&
+                        tiles > cap && tiles % cap != 0;
+    const int pairs = use_sk ? cap : static_cast<int>(std::min<int64_t>(tiles, cap));
+    if (use_sk) {
+        a.sk = 1;
+        a.partial = sk->partial;
+        a.flags = sk->flags;
+    }
     LaunchTimer t(DGRAD ? KK_GEMM_DGRAD : KK_GEMM_FWD, stream);
     const cudaError_t e =
         launch_ex(qlora_gemm_pair_kernel<BN, DGRAD, G>, dim3(static_cast<unsigned>(2 * pairs)),
@@ -544,13 +576,20 @@ int pick_pair_bn(int64_t M, int64_t out, int pairs, bool dgrad) {
 // kPairGroups-th stage).
 constexpr int kPairGroups = 4;
 
+// sk: stream-K scratch (null: whole tiles only). With it, problems with more
+// 256-column tiles than resident pairs run 256-wide tiles under stream-K
+// (the tensor core takes as long for a 192-wide tile as for a 256-wide one).
 template <bool DGRAD>
 nf4_status launch_gemm_auto(const nf4_weight *w, const uint16_t *act, int64_t M, int64_t red,
                             int64_t out, const uint16_t *la, int32_t r, const uint16_t *lb,
-                            uint16_t *D, cudaStream_t stream) {
+                            uint16_t *D, cudaStream_t stream, const SkBuf *sk = nullptr) {
     const int dev = current_device();
     const int pairs = pair_capacity<256, DGRAD, kPairGroups>(dev);
     if (pairs > 0) {
+        const int64_t tiles256 = ((M + 2 * kBM - 1) / (2 * kBM)) * ((out + 255) / 256);
+        if (sk && tiles256 > pairs)
+            return launch_gemm_pair<256, DGRAD, kPairGroups>(w, act, M, red, out, la, r, lb, D,
+                                                             stream, sk);
         switch (pick_pair_bn(M, out, pairs, DGRAD)) {
         case 128:
             return launch_gemm_pair<128, DGRAD, kPairGroups>(w, act, M, red, out, la, r, lb, D, stream);
@@ -688,7 +727,7 @@ nf4_status nf4_dequantize(const nf4_weight *w, void *out, int32_t out_bf16, void
 
 size_t qlora_fwd_workspace_bytes(int64_t M, int64_t n, int64_t k, int32_t r) {
     if (M <= 0 || n <= 0 || k <= 0 || r <= 0) return 256;
-    return fwd_layout(M, r).total;
+    return fwd_layout(M, r, num_sms(current_device())).total;
 }
 
 nf4_status qlora_linear_fwd(const nf4_weight *w, const uint16_t *x, int64_t M, const uint16_t *A,
@@ -699,19 +738,23 @@ nf4_status qlora_linear_fwd(const nf4_weight *w, const uint16_t *x, int64_t M, c
     if (M == 0) return NF4_OK;
     if (!h) return NF4_ERR_INVALID_ARG;
     if (!aligned16(h) || !aligned16(u_out)) return NF4_ERR_ALIGNMENT;
-    const FwdLayout L = fwd_layout(M, r);
+    const int sms = num_sms(current_device());
+    const FwdLayout L = fwd_layout(M, r, sms);
     if (!workspace || ws_bytes < L.total) return NF4_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return NF4_ERR_ALIGNMENT;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     uint16_t *u_s = reinterpret_cast<uint16_t *>(ws + L.us);
+    const SkBuf sk{reinterpret_cast<float *>(ws + L.partial), reinterpret_cast<int *>(ws + L.flags),
+                   sk_pairs_max(sms)};
     const float scale = alpha / static_cast<float>(r);
     if (decode_shape(w, M, r)) return launch_decode(w, x, M, A, B, r, scale, h, u_out, u_s, s);
-    // u = x A^T (fp32, optional) and bf16((alpha/r) u) for the up-projection stage
+    // u = x A^T (fp32, optional) and bf16((alpha/r) u) for the up-projection
+    // stage; this kernel also clears the GEMM's stream-K flags
     st = skinny_product(KK_LORA_U, x, M, w->k, Major::K, A, r, w->k, Major::K, r, u_out, u_s,
-                        scale, 0, s);
+                        scale, 0, s, sk.flags, sk.pairs_max * kSkFlagsPerPair);
     if (st != NF4_OK) return st;
-    return launch_gemm_auto<false>(w, x, M, w->k, w->n, u_s, r, B, h, s);
+    return launch_gemm_auto<false>(w, x, M, w->k, w->n, u_s, r, B, h, s, &sk);
 }
 
 nf4_status qlora_linear_fwd_noalloc(const nf4_weight *w, const uint16_t *x, int64_t M,
@@ -723,11 +766,12 @@ nf4_status qlora_linear_fwd_noalloc(const nf4_weight *w, const uint16_t *x, int6
     if (!h) return NF4_ERR_INVALID_ARG;
     if (!aligned16(h) || !aligned16(u_out)) return NF4_ERR_ALIGNMENT;
     // scratch: bf16 (alpha/r) x A^T [M, r], the workspace of qlora_linear_fwd
-    if (fwd_layout(M, r).total > kStaticScratchBytes) return NF4_ERR_UNSUPPORTED_SHAPE;
+    const FwdLayout L = fwd_layout(M, r, 0, false);   // whole-tile schedule: no stream-K scratch
+    if (L.total > kStaticScratchBytes) return NF4_ERR_UNSUPPORTED_SHAPE;
     uint8_t *ws = static_cast<uint8_t *>(static_scratch_on_current_device());
     if (!ws) return NF4_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    uint16_t *u_s = reinterpret_cast<uint16_t *>(ws + fwd_layout(M, r).us);
+    uint16_t *u_s = reinterpret_cast<uint16_t *>(ws + L.us);
     const float scale = alpha / static_cast<float>(r);
     // same dispatch as qlora_linear_fwd: a few tokens take the decode kernel
     if (decode_shape(w, M, r)) return launch_decode(w, x, M, A, B, r, scale, h, u_out, u_s, s);
@@ -739,7 +783,7 @@ nf4_status qlora_linear_fwd_noalloc(const nf4_weight *w, const uint16_t *x, int6
 
 size_t qlora_bwd_workspace_bytes(int64_t M, int64_t n, int64_t k, int32_t r) {
     if (M < 0 || n <= 0 || k <= 0 || r <= 0) return 256;
-    return bwd_layout(std::max<int64_t>(M, 1), r).total;
+    return bwd_layout(std::max<int64_t>(M, 1), r, num_sms(current_device())).total;
 }
 
 nf4_status qlora_linear_bwd(const nf4_weight *w, const uint16_t *x, int64_t M, const uint16_t *A,
@@ -763,12 +807,15 @@ nf4_status qlora_linear_bwd(const nf4_weight *w, const uint16_t *x, int64_t M, c
         NF4_TRY_CUDA(cudaGetLastError());
         return NF4_OK;
     }
-    const BwdLayout L = bwd_layout(M, r);
+    const int sms = num_sms(current_device());
+    const BwdLayout L = bwd_layout(M, r, sms);
     if (!workspace || ws_bytes < L.total) return NF4_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return NF4_ERR_ALIGNMENT;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     uint16_t *u_s = reinterpret_cast<uint16_t *>(ws + L.us);
     uint16_t *v_s = reinterpret_cast<uint16_t *>(ws + L.vs);
+    const SkBuf sk{reinterpret_cast<float *>(ws + L.partial), reinterpret_cast<int *>(ws + L.flags),
+                   sk_pairs_max(sms)};
     const float scale = alpha / static_cast<float>(r);
 
     // bf16(s u), from the saved u or recomputed from x
@@ -793,12 +840,12 @@ nf4_status qlora_linear_bwd(const nf4_weight *w, const uint16_t *x, int64_t M, c
     st = skinny_product(KK_LORA_DB, dY, M, N, Major::MN, u_s, M, r, Major::MN, r, nullptr, dB,
                         1.0f, 0, s);
     if (st != NF4_OK) return st;
-    // dA = (x^T bf16(s v))^T   ([r, K])
+    // dA = (x^T bf16(s v))^T   ([r, K]); also clears the dgrad GEMM's stream-K flags
     st = skinny_product(KK_LORA_DA, x, M, K, Major::MN, v_s, M, r, Major::MN, r, nullptr, dA,
-                        1.0f, 1, s);
+                        1.0f, 1, s, sk.flags, sk.pairs_max * kSkFlagsPerPair);
     if (st != NF4_OK) return st;
     // dX = dY W~ + bf16(s v) A
-    if (dX) return launch_gemm_auto<true>(w, dY, M, N, K, v_s, r, A, dX, s);
+    if (dX) return launch_gemm_auto<true>(w, dY, M, N, K, v_s, r, A, dX, s, &sk);
     return NF4_OK;
 }
 

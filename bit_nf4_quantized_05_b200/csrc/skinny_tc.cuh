@@ -33,6 +33,8 @@ struct SkinnyArgs {
     uint16_t *out_bf16;  // bf16(scale * sum): [P][r], or [r][P] when transposed; or null
     float scale;
     int transposed;
+    int *zero_ints;      // optional: zeroed by the first CTA (flags for a later kernel)
+    int zero_count;
 };
 
 template <int RN, bool A_MN, bool B_MN>
@@ -98,6 +100,8 @@ skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a,
     const uint32_t tmem_base = *tmem_slot;
     griddep_wait();
     griddep_launch_dependents();
+    if (args.zero_ints && blockIdx.x == 0 && blockIdx.y == 0)
+        for (int z = threadIdx.x; z < args.zero_count; z += kSkThreads) args.zero_ints[z] = 0;
 
     if (warp == 0 && lane == 0) {
         for (int it = 0; it < nsteps; ++it) {

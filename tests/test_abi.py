@@ -64,7 +64,7 @@ def weight(q, n=64, k=64, block=64, dq=0, codes=FAKE, absmax=FAKE, q8=FAKE, cg=F
 
 
 def call_fwd(q, w, M=4, r=8, alpha=16.0, x=FAKE, A=FAKE, B=FAKE, h=FAKE, u=None, ws=FAKE,
-             wsb=1 << 20):
+             wsb=1 << 30):
     return q.lib.qlora_linear_fwd(ctypes.byref(w), x, M, A, B, r, alpha, h, u, ws, wsb, None)
 
 

@@ -8,8 +8,12 @@ takes no workspace and uses a fixed 4 MiB scratch array inside the library
 instead. These tests call it through the C ABI, twice in a row on the same
 inputs (the second call finds the first call's leftovers in the shared
 scratch), and compare both results with the workspace forward, within the
-tolerance the other layer tests use. This file is named so that pytest
-collects it last."""
+tolerance the other layer tests use. The workspace forward may split a
+tile's reduction between two CTA pairs (stream-K), so the two forwards add
+the same fp32 terms in a different grouping and each rounds its own sum to
+bf16: h may differ by one bf16 unit in the last place (at most 2^-7 of the
+value) on top of that tolerance. This file is named so that pytest collects
+it last."""
 import numpy as np
 import pytest
 import torch
@@ -28,10 +32,15 @@ def q():
     return mod
 
 
-def rel_err(got: torch.Tensor, ref: torch.Tensor) -> float:
+def rel_err(got: torch.Tensor, ref: torch.Tensor, bf16_ulp: bool = False) -> float:
+    """max |got - ref| / rms(ref); with bf16_ulp, one bf16 ulp of ref (2^-7 |ref|)
+    is allowed per element first."""
     g = got.double().cpu().numpy()
     r = ref.double().cpu().numpy()
-    return float(np.max(np.abs(g - r)) / max(np.sqrt(np.mean(r ** 2)), 1e-300))
+    d = np.abs(g - r)
+    if bf16_ulp:
+        d = d - 2.0 ** -7 * np.abs(r)
+    return float(np.max(d) / max(np.sqrt(np.mean(r ** 2)), 1e-300))
 
 
 @pytest.mark.parametrize("name", ["single_1024", "llama13b_attn_5120"])
@@ -52,7 +61,7 @@ def test_noalloc_forward_matches_workspace_forward(q, name):
         torch.cuda.synchronize()
         assert q.device_status() == q.NF4_OK
         assert torch.isfinite(h).all() and torch.isfinite(u).all()
-        eh, eu = rel_err(h, h_ref), rel_err(u, u_ref)
+        eh, eu = rel_err(h, h_ref, bf16_ulp=True), rel_err(u, u_ref)
         assert eh <= TOL and eu <= TOL, f"call {call}: h {eh:.3g}, u {eu:.3g} x rms"
 
 
