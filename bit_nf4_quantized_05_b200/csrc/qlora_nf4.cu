@@ -17,7 +17,7 @@
 #include "gemm_tc.cuh"
 #include "gemm_pair_tc.cuh"
 #include "skinny_tc.cuh"
-#include "decode.cuh"
+#include "decode2.cuh"
 
 using namespace nf4;
 
@@ -484,9 +484,10 @@ nf4_status launch_gemm_pair(const nf4_weight *w, const uint16_t *act, int64_t M,
 // it streams the weight while u is being computed.
 constexpr int64_t kDecodeMaxTokens = 16;
 
-// The decode kernel keeps B and u tiles of rank <= kDecMaxRank in shared memory.
+// The decode kernel keeps u tiles of rank <= kDc2MaxRank in shared memory.
 bool decode_shape(const nf4_weight *w, int64_t M, int32_t r) {
-    return M <= kDecodeMaxTokens && r <= kDecMaxRank;
+    return M <= kDecodeMaxTokens && r <= kDc2MaxRank &&
+           w->n * (w->k / kBlock) < (int64_t(1) << 31);   // 32-bit block indices
 }
 
 nf4_status launch_decode(const nf4_weight *w, const uint16_t *x, int64_t M, const uint16_t *A,
@@ -500,7 +501,7 @@ nf4_status launch_decode(const nf4_weight *w, const uint16_t *x, int64_t M, cons
         if (e != cudaSuccess) return NF4_ERR_CUDA;
     }
     NF4_TRY_CUDA(cudaGetLastError());
-    DecodeArgs a;
+    Decode2Args a;
     a.M = static_cast<int>(M);
     a.N = w->n;
     a.K = w->k;
@@ -514,19 +515,15 @@ nf4_status launch_decode(const nf4_weight *w, const uint16_t *x, int64_t M, cons
     a.B = B;
     a.u_s = u_s;
     a.h = h;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>((w->n + kDecRows - 1) / kDecRows));
-    cfg.blockDim = dim3(kDecThreads);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    const int64_t tiles = (w->n + kDc2Rows - 1) / kDc2Rows;
+    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, num_sms(current_device())));
+    auto k1 = qlora_decode2_kernel<1>;
+    auto k2 = qlora_decode2_kernel<2>;
+    NF4_TRY_CUDA(cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, kDc2DynBytes));
+    NF4_TRY_CUDA(cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, kDc2DynBytes));
     LaunchTimer t(KK_DECODE, stream);
-    cudaError_t e = M <= 8 ? cudaLaunchKernelEx(&cfg, qlora_decode_kernel<1>, a)
-                           : cudaLaunchKernelEx(&cfg, qlora_decode_kernel<2>, a);
+    const cudaError_t e = M <= 8 ? launch_ex(k1, dim3(grid), dim3(kDc2Threads), kDc2DynBytes, stream, 0u, a)
+                                 : launch_ex(k2, dim3(grid), dim3(kDc2Threads), kDc2DynBytes, stream, 0u, a);
     t.stop();
     if (e != cudaSuccess) return NF4_ERR_CUDA;
     NF4_TRY_CUDA(cudaGetLastError());
