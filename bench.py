@@ -34,6 +34,10 @@ import torch  # noqa: E402
 import workloads  # noqa: E402
 
 METRIC = "QLoRA linear fwd+bwd TFLOP/s (large M) & NF4 weight GB/s (decode) vs roofline"
+# DRAM bytes (read + write) per launch of the fused GEMM on this workload, mean of the forward and
+# dgrad launches, from one ncu capture of the kernels as they are now (summary and command under
+# profiles/). None whenever the kernel has changed since that capture.
+GEMM_TRAFFIC_BYTES = 46.7e6
 MAIN = "llama13b_attn_5120"
 DECODE = "decode_mlp_up_13824x5120"
 QUANT = "llama2_70b_mlp_28672x8192"
@@ -292,7 +296,8 @@ def main():
     g_tflops = g_flops / (g_ms * 1e-3) / 1e12 if g_ms > 0 else None
     roofline = {"bound": "tensor", "achieved": g_tflops, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": (g_tflops / peaks["bf16_tflops"]) if g_tflops else None,
-                "traffic": None, "kernel": "qlora_gemm (forward + dgrad launches)",
+                "traffic": GEMM_TRAFFIC_BYTES, "traffic_unit": "bytes per launch (ncu dram read + write)",
+                "kernel": "qlora_gemm (forward + dgrad launches)",
                 "peak_source": peaks["source"] + " bf16 burst",
                 "avg_launch_us": 1e3 * g_ms / max(g_launch, 1)}
     kernels = {k: {"launches": n, "avg_us": 1e3 * t / max(n, 1), "share": t / max(
