@@ -697,8 +697,10 @@ nf4_status nf4_quantize(const float *W0, const nf4_weight *w, void *stream) {
     const int64_t nb = w->n * w->k / kBlock;
     const int64_t groups = (nb + kGroup - 1) / kGroup;
     if (groups > 0x7fffffff) return NF4_ERR_UNSUPPORTED_SHAPE;
+    // persistent: kQuantCtasPerSm CTAs per SM walk the groups
+    const int64_t grid = std::min<int64_t>(groups, int64_t(kQuantCtasPerSm) * num_sms(current_device()));
     LaunchTimer t(KK_QUANTIZE, static_cast<cudaStream_t>(stream));
-    nf4_quantize_kernel<<<static_cast<unsigned>(groups), kQuantThreads, 0,
+    nf4_quantize_kernel<<<static_cast<unsigned>(grid), kQuantThreads, 0,
                           static_cast<cudaStream_t>(stream)>>>(
         W0, nb, w->double_quant, w->codes, w->absmax, w->absmax_q8, w->absmax_c);
     t.stop();
