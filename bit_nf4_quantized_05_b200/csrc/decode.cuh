@@ -1,8 +1,8 @@
 // decode.cuh -- pieces shared by the decode-shaped forward (M <= 16 tokens):
 // the m16n8k16 bf16 tensor-core product used on register fragments, and the
-// small kernel that forms u = x A^T and bf16((alpha/r) u) ("QLoRA explained",
+// small kernel that forms partial sums of u = x A^T ("QLoRA explained",
 // section "The LoRA adapter path") ahead of the weight-streaming kernel in
-// decode2.cuh.
+// decode3.cuh.
 #pragma once
 
 #include "nf4_common.cuh"
@@ -18,24 +18,27 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// u = x A^T for a few tokens (M <= 16): one CTA per rank column j, threads
-// split k, fixed-order reduction; writes u (fp32, optional) and
-// bf16(scale * u). Lets the decode kernel that follows start right away.
-constexpr int kDecUThreads = 256;
+// Partial sums of u = x A^T for a few tokens (M <= 16): CTA (j, s) reduces
+// the s-th of kDecUSplits k-slices for rank column j and all tokens, in a
+// fixed order, and writes upart[s][m][j]. The decode kernel that follows adds
+// the kDecUSplits partials of each u[m][j] in order of s. Splitting k spreads
+// the reads of x over r * kDecUSplits CTAs.
+constexpr int kDecUThreads = 128;
+constexpr int kDecUSplits = 8;
 
 __global__ void __launch_bounds__(kDecUThreads)
 decode_lora_u_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ A, int M,
-                     int64_t K, int r, float scale, float *__restrict__ u_out,
-                     uint16_t *__restrict__ u_s) {
+                     int64_t K, int r, float *__restrict__ upart) {
     griddep_wait();
     griddep_launch_dependents();
     __shared__ float red[kDecUThreads / 32][16];
-    const int j = blockIdx.x;
+    const int j = blockIdx.x, sl = blockIdx.y;
+    const int64_t k0 = K * sl / kDecUSplits / 8 * 8, k1 = K * (sl + 1) / kDecUSplits / 8 * 8;
     float acc[16];
 #pragma unroll
     for (int m = 0; m < 16; ++m) acc[m] = 0.0f;
     const uint16_t *ar = A + static_cast<int64_t>(j) * K;
-    for (int64_t k = 8 * threadIdx.x; k < K; k += 8 * kDecUThreads) {
+    for (int64_t k = k0 + 8 * threadIdx.x; k < k1; k += 8 * kDecUThreads) {
         const uint4 av = __ldg(reinterpret_cast<const uint4 *>(ar + k));
         const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
 #pragma unroll
@@ -63,9 +66,7 @@ decode_lora_u_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
         const int m = threadIdx.x;
         float v = 0.0f;
         for (int w = 0; w < kDecUThreads / 32; ++w) v += red[w][m];
-        if (u_out) u_out[static_cast<int64_t>(m) * r + j] = v;
-        __nv_bfloat16 b = __float2bfloat16_rn(scale * v);
-        u_s[static_cast<int64_t>(m) * r + j] = *reinterpret_cast<uint16_t *>(&b);
+        upart[(static_cast<int64_t>(sl) * M + m) * r + j] = v;
     }
 }
 

@@ -17,7 +17,7 @@
 #include "gemm_tc.cuh"
 #include "gemm_pair_tc.cuh"
 #include "skinny_tc.cuh"
-#include "decode2.cuh"
+#include "decode3.cuh"
 
 using namespace nf4;
 
@@ -248,14 +248,18 @@ struct SkBuf {
 };
 
 struct FwdLayout {
-    size_t us, flags, partial, total;
+    size_t us, upart, flags, partial, total;
 };
 
-// with_sk = false: only the bf16 rank-r activations (the whole-tile schedule)
+// us: bf16 rank-r activations; upart: the decode path's partial sums of x A^T
+// (M <= 16 tokens only); flags/partial: stream-K scratch (with_sk = false: the
+// whole-tile schedule, none)
 FwdLayout fwd_layout(int64_t M, int32_t r, int sms, bool with_sk = true) {
     FwdLayout L{};
     size_t off = 0;
     L.us = off;   off = align256(off + size_t(M) * r * 2);
+    L.upart = off;
+    if (M <= 16) off = align256(off + size_t(kDecUSplits) * size_t(M) * r * 4);
     if (with_sk) {
         L.flags = off;   off = align256(off + sk_flag_bytes(sms));
         L.partial = off; off = align256(off + sk_partial_bytes(sms));
@@ -479,51 +483,71 @@ nf4_status launch_gemm_pair(const nf4_weight *w, const uint16_t *act, int64_t M,
     return NF4_OK;
 }
 
-// Forward for M <= 16 tokens: u = x A^T (and its scaled bf16 copy), then the
-// decode kernel, launched as a programmatic dependent of the first so that
-// it streams the weight while u is being computed.
+// Forward for M <= 16 tokens: partial sums of u = x A^T over k slices, then
+// the decode kernel, launched as a programmatic dependent of the first so
+// that it streams the weight while u is being computed (it adds the partials
+// once it needs u).
 constexpr int64_t kDecodeMaxTokens = 16;
 
-// The decode kernel keeps u tiles of rank <= kDc2MaxRank in shared memory.
+// The decode kernel keeps u tiles of rank <= kDc3MaxRank in shared memory.
 bool decode_shape(const nf4_weight *w, int64_t M, int32_t r) {
-    return M <= kDecodeMaxTokens && r <= kDc2MaxRank &&
+    return M <= kDecodeMaxTokens && r <= kDc3MaxRank &&
            w->n * (w->k / kBlock) < (int64_t(1) << 31);   // 32-bit block indices
 }
 
 nf4_status launch_decode(const nf4_weight *w, const uint16_t *x, int64_t M, const uint16_t *A,
                          const uint16_t *B, int32_t r, float scale, uint16_t *h, float *u_out,
-                         uint16_t *u_s, cudaStream_t stream) {
+                         float *upart, cudaStream_t stream) {
     {
         LaunchTimer t(KK_DECODE_U, stream);
-        const cudaError_t e = launch_ex(decode_lora_u_kernel, dim3(r), dim3(kDecUThreads), 0, stream,
-                                        0u, x, A, static_cast<int>(M), w->k, r, scale, u_out, u_s);
+        const cudaError_t e = launch_ex(decode_lora_u_kernel, dim3(r, kDecUSplits), dim3(kDecUThreads), 0,
+                                        stream, 0u, x, A, static_cast<int>(M), w->k, r, upart);
         t.stop();
         if (e != cudaSuccess) return NF4_ERR_CUDA;
     }
     NF4_TRY_CUDA(cudaGetLastError());
-    Decode2Args a;
+    // each of the 16 warps takes rb blocks of every 32-row tile, fetched in
+    // chunks of cb blocks (the largest divisor of rb that is at most 5)
+    const int64_t kblocks = w->k / kBlock;
+    const int rb = static_cast<int>((kblocks + kDc3Warps - 1) / kDc3Warps);
+    int cb = 1;
+    for (int d = kDc3MaxChunk; d >= 1; --d)
+        if (rb % d == 0) {
+            cb = d;
+            break;
+        }
+    Decode3Args a;
     a.M = static_cast<int>(M);
     a.N = w->n;
     a.K = w->k;
     a.r = r;
-    a.codes = w->codes;
+    a.rb = rb;
+    a.cb = cb;
+    a.slot_bytes = std::max(32 * 32 * cb, 2048);
     a.absmax = w->absmax;
     a.q8 = w->absmax_q8;
     a.cg = w->absmax_c;
     a.dq = w->double_quant;
     a.x = x;
     a.B = B;
-    a.u_s = u_s;
+    a.upart = upart;
+    a.scale = scale;
+    a.u_out = u_out;
     a.h = h;
-    const int64_t tiles = (w->n + kDc2Rows - 1) / kDc2Rows;
+    CUtensorMap tm_codes;
+    if (!make_map(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, w->k / 2, w->n,
+                  static_cast<uint32_t>(32 * cb), kDc3Rows, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return NF4_ERR_CUDA;
+    const int64_t tiles = (w->n + kDc3Rows - 1) / kDc3Rows;
     const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, num_sms(current_device())));
-    auto k1 = qlora_decode2_kernel<1>;
-    auto k2 = qlora_decode2_kernel<2>;
-    NF4_TRY_CUDA(cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, kDc2DynBytes));
-    NF4_TRY_CUDA(cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, kDc2DynBytes));
+    auto k1 = qlora_decode3_kernel<1>;
+    auto k2 = qlora_decode3_kernel<2>;
+    NF4_TRY_CUDA(cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, kDc3DynBytes));
+    NF4_TRY_CUDA(cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, kDc3DynBytes));
     LaunchTimer t(KK_DECODE, stream);
-    const cudaError_t e = M <= 8 ? launch_ex(k1, dim3(grid), dim3(kDc2Threads), kDc2DynBytes, stream, 0u, a)
-                                 : launch_ex(k2, dim3(grid), dim3(kDc2Threads), kDc2DynBytes, stream, 0u, a);
+    const cudaError_t e =
+        M <= 8 ? launch_ex(k1, dim3(grid), dim3(kDc3Threads), kDc3DynBytes, stream, 0u, tm_codes, a)
+               : launch_ex(k2, dim3(grid), dim3(kDc3Threads), kDc3DynBytes, stream, 0u, tm_codes, a);
     t.stop();
     if (e != cudaSuccess) return NF4_ERR_CUDA;
     NF4_TRY_CUDA(cudaGetLastError());
@@ -747,7 +771,8 @@ nf4_status qlora_linear_fwd(const nf4_weight *w, const uint16_t *x, int64_t M, c
     const SkBuf sk{reinterpret_cast<float *>(ws + L.partial), reinterpret_cast<int *>(ws + L.flags),
                    sk_pairs_max(sms)};
     const float scale = alpha / static_cast<float>(r);
-    if (decode_shape(w, M, r)) return launch_decode(w, x, M, A, B, r, scale, h, u_out, u_s, s);
+    if (decode_shape(w, M, r))
+        return launch_decode(w, x, M, A, B, r, scale, h, u_out, reinterpret_cast<float *>(ws + L.upart), s);
     // u = x A^T (fp32, optional) and bf16((alpha/r) u) for the up-projection
     // stage; this kernel also clears the GEMM's stream-K flags
     st = skinny_product(KK_LORA_U, x, M, w->k, Major::K, A, r, w->k, Major::K, r, u_out, u_s,
@@ -773,7 +798,8 @@ nf4_status qlora_linear_fwd_noalloc(const nf4_weight *w, const uint16_t *x, int6
     uint16_t *u_s = reinterpret_cast<uint16_t *>(ws + L.us);
     const float scale = alpha / static_cast<float>(r);
     // same dispatch as qlora_linear_fwd: a few tokens take the decode kernel
-    if (decode_shape(w, M, r)) return launch_decode(w, x, M, A, B, r, scale, h, u_out, u_s, s);
+    if (decode_shape(w, M, r))
+        return launch_decode(w, x, M, A, B, r, scale, h, u_out, reinterpret_cast<float *>(ws + L.upart), s);
     st = skinny_product(KK_LORA_U, x, M, w->k, Major::K, A, r, w->k, Major::K, r, u_out, u_s,
                         scale, 0, s);
     if (st != NF4_OK) return st;
