@@ -17,7 +17,7 @@
 #include "gemm_tc.cuh"
 #include "gemm_pair_tc.cuh"
 #include "skinny_tc.cuh"
-#include "decode3.cuh"
+#include "decode_stream.cuh"
 
 using namespace nf4;
 
@@ -251,15 +251,15 @@ struct FwdLayout {
     size_t us, upart, flags, partial, total;
 };
 
-// us: bf16 rank-r activations; upart: the decode path's partial sums of x A^T
-// (M <= 16 tokens only); flags/partial: stream-K scratch (with_sk = false: the
-// whole-tile schedule, none)
+// us: bf16 rank-r activations; upart: the decode path's partial sums of
+// x A^T (M <= 16 tokens only); flags/partial: stream-K scratch (with_sk =
+// false: the whole-tile schedule, none)
 FwdLayout fwd_layout(int64_t M, int32_t r, int sms, bool with_sk = true) {
     FwdLayout L{};
     size_t off = 0;
     L.us = off;   off = align256(off + size_t(M) * r * 2);
     L.upart = off;
-    if (M <= 16) off = align256(off + size_t(kDecUSplits) * size_t(M) * r * 4);
+    if (M <= 16) off = align256(off + size_t(kDsUCtas) * size_t(M) * r * 4);
     if (with_sk) {
         L.flags = off;   off = align256(off + sk_flag_bytes(sms));
         L.partial = off; off = align256(off + sk_partial_bytes(sms));
@@ -483,71 +483,97 @@ nf4_status launch_gemm_pair(const nf4_weight *w, const uint16_t *act, int64_t M,
     return NF4_OK;
 }
 
-// Forward for M <= 16 tokens: partial sums of u = x A^T over k slices, then
-// the decode kernel, launched as a programmatic dependent of the first so
-// that it streams the weight while u is being computed (it adds the partials
-// once it needs u).
+// One instantiation of the decode kernel per (token groups, chunk blocks).
+template <int TG, int CB>
+cudaError_t launch_decode_stream_t(unsigned grid, cudaStream_t stream, const CUtensorMap &tm,
+                                   const DecodeArgs &a) {
+    auto k = qlora_decode_stream_kernel<TG, CB>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kDsDynBytes);
+    if (e != cudaSuccess) return e;
+    return launch_ex(k, dim3(grid), dim3(kDsThreads), kDsDynBytes, stream, 0u, tm, a);
+}
+
+template <int TG>
+cudaError_t launch_decode_stream_cb(int cb, unsigned grid, cudaStream_t stream, const CUtensorMap &tm,
+                                    const DecodeArgs &a) {
+    switch (cb) {
+        case 1: return launch_decode_stream_t<TG, 1>(grid, stream, tm, a);
+        case 2: return launch_decode_stream_t<TG, 2>(grid, stream, tm, a);
+        case 3: return launch_decode_stream_t<TG, 3>(grid, stream, tm, a);
+        case 4: return launch_decode_stream_t<TG, 4>(grid, stream, tm, a);
+        case 5: return launch_decode_stream_t<TG, 5>(grid, stream, tm, a);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_decode_stream(int tg, int cb, unsigned grid, cudaStream_t stream, const CUtensorMap &tm,
+                                 const DecodeArgs &a) {
+    return tg == 1 ? launch_decode_stream_cb<1>(cb, grid, stream, tm, a)
+                   : launch_decode_stream_cb<2>(cb, grid, stream, tm, a);
+}
+
+// Forward for M <= 16 tokens: partial sums of u = x A^T on a few SMs, then
+// the decode kernel on the rest, launched as a programmatic dependent of the
+// first so that it streams the weight while u is being formed (it adds the
+// partials once it needs u).
 constexpr int64_t kDecodeMaxTokens = 16;
 
-// The decode kernel keeps u tiles of rank <= kDc3MaxRank in shared memory.
+// The decode kernel keeps u tiles of rank <= kDsMaxRank in shared memory.
 bool decode_shape(const nf4_weight *w, int64_t M, int32_t r) {
-    return M <= kDecodeMaxTokens && r <= kDc3MaxRank &&
+    return M <= kDecodeMaxTokens && r <= kDsMaxRank &&
            w->n * (w->k / kBlock) < (int64_t(1) << 31);   // 32-bit block indices
 }
 
 nf4_status launch_decode(const nf4_weight *w, const uint16_t *x, int64_t M, const uint16_t *A,
                          const uint16_t *B, int32_t r, float scale, uint16_t *h, float *u_out,
                          float *upart, cudaStream_t stream) {
-    {
-        LaunchTimer t(KK_DECODE_U, stream);
-        const cudaError_t e = launch_ex(decode_lora_u_kernel, dim3(r, kDecUSplits), dim3(kDecUThreads), 0,
-                                        stream, 0u, x, A, static_cast<int>(M), w->k, r, upart);
-        t.stop();
-        if (e != cudaSuccess) return NF4_ERR_CUDA;
-    }
-    NF4_TRY_CUDA(cudaGetLastError());
     // each of the 16 warps takes rb blocks of every 32-row tile, fetched in
     // chunks of cb blocks (the largest divisor of rb that is at most 5)
     const int64_t kblocks = w->k / kBlock;
-    const int rb = static_cast<int>((kblocks + kDc3Warps - 1) / kDc3Warps);
+    const int rb = static_cast<int>((kblocks + kDsWarps - 1) / kDsWarps);
     int cb = 1;
-    for (int d = kDc3MaxChunk; d >= 1; --d)
+    for (int d = kDsMaxChunk; d >= 1; --d)
         if (rb % d == 0) {
             cb = d;
             break;
         }
-    Decode3Args a;
+    DecodeArgs a;
     a.M = static_cast<int>(M);
     a.N = w->n;
     a.K = w->k;
     a.r = r;
     a.rb = rb;
-    a.cb = cb;
-    a.slot_bytes = std::max(32 * 32 * cb, 2048);
     a.absmax = w->absmax;
     a.q8 = w->absmax_q8;
     a.cg = w->absmax_c;
     a.dq = w->double_quant;
     a.x = x;
     a.B = B;
+    a.A = A;
     a.upart = upart;
     a.scale = scale;
     a.u_out = u_out;
     a.h = h;
     CUtensorMap tm_codes;
     if (!make_map(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, w->k / 2, w->n,
-                  static_cast<uint32_t>(32 * cb), kDc3Rows, CU_TENSOR_MAP_SWIZZLE_NONE))
+                  static_cast<uint32_t>(32 * cb), kDsRows, CU_TENSOR_MAP_SWIZZLE_NONE))
         return NF4_ERR_CUDA;
-    const int64_t tiles = (w->n + kDc3Rows - 1) / kDc3Rows;
-    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, num_sms(current_device())));
-    auto k1 = qlora_decode3_kernel<1>;
-    auto k2 = qlora_decode3_kernel<2>;
-    NF4_TRY_CUDA(cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, kDc3DynBytes));
-    NF4_TRY_CUDA(cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, kDc3DynBytes));
+    const int64_t tiles = (w->n + kDsRows - 1) / kDsRows;
+    // the decode grid leaves kDsUCtas SMs to the u kernel
+    const int sms = num_sms(current_device());
+    const unsigned grid = static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(tiles, sms - kDsUCtas)));
+    const int tg = M <= 8 ? 1 : 2;
+    {
+        // u = x A^T on kDsUCtas CTAs, beside the decode grid
+        LaunchTimer t(KK_DECODE_U, stream);
+        auto ku = tg == 1 ? qlora_decode_u_kernel<1> : qlora_decode_u_kernel<2>;
+        NF4_TRY_CUDA(cudaFuncSetAttribute(ku, cudaFuncAttributeMaxDynamicSharedMemorySize, kDsUParkBytes));
+        const cudaError_t e = launch_ex(ku, dim3(kDsUCtas), dim3(kDsThreads), kDsUParkBytes, stream, 0u, a);
+        t.stop();
+        if (e != cudaSuccess) return NF4_ERR_CUDA;
+    }
     LaunchTimer t(KK_DECODE, stream);
-    const cudaError_t e =
-        M <= 8 ? launch_ex(k1, dim3(grid), dim3(kDc3Threads), kDc3DynBytes, stream, 0u, tm_codes, a)
-               : launch_ex(k2, dim3(grid), dim3(kDc3Threads), kDc3DynBytes, stream, 0u, tm_codes, a);
+    const cudaError_t e = launch_decode_stream(tg, cb, grid, stream, tm_codes, a);
     t.stop();
     if (e != cudaSuccess) return NF4_ERR_CUDA;
     NF4_TRY_CUDA(cudaGetLastError());
