@@ -7,7 +7,7 @@ import re
 
 import pytest
 
-from conftest import ROOT
+from conftest import ROOT, build_library
 
 HEADER = os.path.join(ROOT, "include", "qlora_nf4.h")
 
@@ -19,8 +19,7 @@ def declared_functions():
 
 @pytest.fixture(scope="module")
 def q():
-    from bit_nf4_quantized_05_b200 import build
-    build.build()
+    build_library()
     import bit_nf4_quantized_05_b200 as mod
     return mod
 
