@@ -41,6 +41,7 @@ GEMM_TRAFFIC_BYTES = 46.7e6
 MAIN = "llama13b_attn_5120"
 DECODE = "decode_mlp_up_13824x5120"
 QUANT = "llama2_70b_mlp_28672x8192"
+STACK = "llama13b_stack_40x4"
 L2_FLUSH_BYTES = 512 << 20
 
 
@@ -71,7 +72,7 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x100: "display_clock_setting"}
 
-    def __init__(self, device_index, period_s=0.01):
+    def __init__(self, device_index, period_s=0.002):
         self.samples, self.reasons = [], 0
         self.period = period_s
         self.ok = False
@@ -191,12 +192,12 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--skip-extras", action="store_true",
                     help="only the main fwd+bwd line (no decode/quantize/oracle/e2e legs)")
-    ap.add_argument("--leg", default="all", choices=["all", "decode", "quantize"],
+    ap.add_argument("--leg", default="all", choices=["all", "decode", "quantize", "stack", "mlp70b"],
                     help="run one secondary leg alone and print its JSON (for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -216,7 +217,8 @@ def main():
     dev = torch.device("cuda", local_rank)
     if args.leg != "all":
         if rank == 0:
-            leg = decode_leg if args.leg == "decode" else quantize_leg
+            leg = {"decode": decode_leg, "quantize": quantize_leg, "stack": stack_leg,
+                   "mlp70b": mlp70b_leg}[args.leg]
             print(json.dumps({"leg": args.leg, **leg(q, dev, load_peaks())}), flush=True)
         return
     if world > 1:
@@ -323,6 +325,8 @@ def main():
         line["e2e"] = e2e_leg(q, dp, qw, inp, w, args, dev, world)
         line["decode"] = decode_leg(q, dev, peaks)
         line["quantize"] = quantize_leg(q, dev, peaks)
+        line["mlp70b"] = mlp70b_leg(q, dev, peaks)
+        line["stack"] = stack_leg(q, dev, peaks)
         line["cpu_baseline"] = cpu_baseline_leg(w, inp)
     elif not args.skip_extras:
         e2e_leg(q, dp, qw, inp, w, args, dev, world)  # same collectives on every rank
@@ -466,6 +470,115 @@ def quantize_leg(q, dev, peaks):
     return {"workload": f"{QUANT}: W0 {w.N}x{w.K} fp32 -> NF4 + double quant",
             "bytes_moved": moved, "kernel_us": us, "gbs": gbs, "frac": gbs / peaks["hbm_gbs"],
             "peak_gbs": peaks["hbm_gbs"]}
+
+
+def _time_steps(step, warmup, steps):
+    """Mean device time (ms) of `steps` calls of step() after `warmup` untimed ones."""
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        step()
+    e.record()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / steps
+
+
+def mlp70b_leg(q, dev, peaks, warmup=3, steps=5):
+    """Forward + backward of the Llama-2-70B-like MLP projection (W0 28672x8192 NF4 with
+    double quant, 8192 tokens, r = 64, alpha = 16). Every operand is larger than L2."""
+    from bit_nf4_quantized_05_b200 import dp
+    w = workloads.WORKLOADS[QUANT]
+    M, N, K, r, alpha = w.M, w.N, w.K, w.r, w.alpha
+    inp = workloads.make_inputs(w)
+    qw = q.nf4_quantize(inp["W0"].to(dev), double_quant=True)
+    x, A, B, dY = (inp[k].to(dev) for k in ("x", "A", "B", "dY"))
+    del inp
+    h = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    u = torch.empty(M, r, dtype=torch.float32, device=dev)
+    dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    flat, dA, dB = dp.grad_buffer(r, K, N, device=dev)
+    ws_f = torch.empty(q.fwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(q.bwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
+
+    def step():
+        q.qlora_linear_fwd(qw, x, A, B, alpha, h=h, u=u, workspace=ws_f)
+        q.qlora_linear_bwd(qw, x, A, B, alpha, dY, u=u, workspace=ws_b, outs=(dX, dA, dB))
+
+    ms = _time_steps(step, warmup, steps)
+    q.profiling(True)
+    for _ in range(steps):
+        step()
+    torch.cuda.synchronize()
+    q.profiling(False)
+    prof = q.profile_read()
+    f, b = layer_flops(M, N, K, r)
+    g_ms = sum(prof.get(k, (0, 0.0))[1] for k in ("qlora_gemm_fwd", "qlora_gemm_dgrad")) / steps
+    g_flops = (2 * M * N * K + 2 * M * N * r) + (2 * M * N * K + 2 * M * K * r)
+    del qw, x, A, B, dY, h, u, dX, flat, ws_f, ws_b
+    torch.cuda.empty_cache()
+    tflops = (f + b) / (ms * 1e-3) / 1e12
+    gemm_tflops = g_flops / (g_ms * 1e-3) / 1e12 if g_ms > 0 else None
+    return {"workload": f"{QUANT}: W0 {N}x{K} NF4 double quant, x {M}x{K} bf16, r={r}, "
+                        f"alpha={alpha:g}, forward+backward",
+            "ms_per_step": ms, "tflops": tflops, "frac": tflops / peaks["bf16_tflops"],
+            "gemm_tflops": gemm_tflops,
+            "gemm_frac": gemm_tflops / peaks["bf16_tflops"] if gemm_tflops else None,
+            "peak_tflops": peaks["bf16_tflops"], "steps": steps,
+            "kernel_avg_us": {k: 1e3 * t / max(n, 1) for k, (n, t) in prof.items()}}
+
+
+def stack_leg(q, dev, peaks, warmup=2, steps=3):
+    """The LLaMA-13B-like adapter stack: 40 layers x {Q, K, V, O}, each a 5120x5120 NF4
+    weight with double quant and its own r = 16 adapters (weights and adapters drawn from the
+    per-projection seeds), forward + backward of every projection at 4096 tokens. One batch
+    of tokens and output gradients (drawn from the first projection's seed) serves every
+    projection. The 160 weights (2.2 GB of codes and scales) far exceed L2."""
+    from concurrent.futures import ThreadPoolExecutor
+    from bit_nf4_quantized_05_b200 import dp
+    w = workloads.WORKLOADS[STACK]
+    M, N, K, r, alpha = w.M, w.N, w.K, w.r, w.alpha
+    seeds = [workloads.stack_seed(l, p) for l in range(w.layers // 4) for p in range(4)]
+    base = workloads.make_inputs(w, seed=seeds[0])
+    x, dY = base["x"].to(dev), base["dY"].to(dev)
+    del base
+    t0 = time.perf_counter()
+    projs = []
+
+    def draw(seed):
+        return workloads.make_inputs(w, M=0, seed=seed, with_dy=False)
+
+    with ThreadPoolExecutor(max_workers=min(16, max(1, cpu_cores()))) as ex:
+        for i in range(0, len(seeds), 16):
+            for inp in ex.map(draw, seeds[i:i + 16]):
+                qw = q.nf4_quantize(inp["W0"].to(dev), double_quant=True)
+                projs.append((qw, inp["A"].to(dev), inp["B"].to(dev)))
+    gen_s = time.perf_counter() - t0
+    h = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    u = torch.empty(M, r, dtype=torch.float32, device=dev)
+    dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    grads = [dp.grad_buffer(r, K, N, device=dev) for _ in projs]
+    ws_f = torch.empty(q.fwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(q.bwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
+
+    def step():
+        for (qw, A, B), (_, dA, dB) in zip(projs, grads):
+            q.qlora_linear_fwd(qw, x, A, B, alpha, h=h, u=u, workspace=ws_f)
+            q.qlora_linear_bwd(qw, x, A, B, alpha, dY, u=u, workspace=ws_b, outs=(dX, dA, dB))
+
+    ms = _time_steps(step, warmup, steps)
+    f, b = layer_flops(M, N, K, r)
+    total = len(projs) * (f + b)
+    del projs, grads, x, dY, h, u, dX, ws_f, ws_b
+    torch.cuda.empty_cache()
+    tflops = total / (ms * 1e-3) / 1e12
+    return {"workload": f"{STACK}: {w.layers} projections x (W0 {N}x{K} NF4 double quant, "
+                        f"x {M}x{K} bf16, r={r}, alpha={alpha:g}), forward+backward each",
+            "ms_per_step": ms, "tflops": tflops, "frac": tflops / peaks["bf16_tflops"],
+            "peak_tflops": peaks["bf16_tflops"], "algorithmic_tflop": total / 1e12,
+            "steps": steps, "input_generation_s": gen_s}
 
 
 def cpu_baseline_leg(w, inp):

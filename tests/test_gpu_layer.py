@@ -156,6 +156,17 @@ def test_llama13b_attention_full_size(q):
                          rows=sampled_rows(w.M, 48, 1), tag=w.name)
 
 
+@pytest.mark.parametrize("layer,proj", [(0, 0), (17, 2), (39, 3)])
+def test_llama13b_stack_projection_full_size(q, layer, proj):
+    """Projections of the 40-layer x {Q,K,V,O} adapter stack, each with its own seed, at the
+    stack's 4096 tokens: every row of dA and dB, sampled rows of h and dX."""
+    w = workloads.WORKLOADS["llama13b_stack_40x4"]
+    inp = workloads.make_inputs(w, seed=workloads.stack_seed(layer, proj))
+    res = run_layer(q, inp["W0"], inp["A"], inp["B"], inp["x"], inp["dY"], w.alpha, w.double_quant)
+    check_against_oracle(q, res, inp["A"], inp["B"], inp["x"], inp["dY"], w.alpha,
+                         rows=sampled_rows(w.M, 32, 100 + layer), tag=f"{w.name} {layer}/{proj}")
+
+
 @pytest.mark.parametrize("M", [1, 4, 16])
 def test_decode_workload_full_size(q, M):
     w = workloads.WORKLOADS["decode_mlp_up_13824x5120"]
