@@ -37,7 +37,7 @@ METRIC = "QLoRA linear fwd+bwd TFLOP/s (large M) & NF4 weight GB/s (decode) vs r
 # DRAM bytes (read + write) per launch of the fused GEMM on this workload, mean of the forward and
 # dgrad launches, from one ncu capture of the kernels as they are now (summary and command under
 # profiles/). None whenever the kernel has changed since that capture.
-GEMM_TRAFFIC_BYTES = 46.7e6
+GEMM_TRAFFIC_BYTES = 44.6e6
 MAIN = "llama13b_attn_5120"
 DECODE = "decode_mlp_up_13824x5120"
 QUANT = "llama2_70b_mlp_28672x8192"

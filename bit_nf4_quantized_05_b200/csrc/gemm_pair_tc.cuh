@@ -41,7 +41,7 @@ struct PairCfg {
     static constexpr int kBBytes = kBH * kBK * 2;         // this CTA's half of the B tile
     static constexpr int kCBytes = kBH * kBK / 2;         // its 4-bit codes
     static constexpr int kSB = G >= 4 ? G : 2 * G;       // weight-tile stages
-    static constexpr int kSC = 8;                         // code-tile stages
+    static constexpr int kSC = G >= 4 ? G : 2 * G;       // code-tile stages
     static constexpr int kSAFit = (220 * 1024 - kSB * kBBytes - kSC * kCBytes) / kABytes;
     static constexpr int kSA = kSAFit > 8 ? 8 : kSAFit;
     static constexpr int kGroupWarps = kBH / 32;
