@@ -20,171 +20,270 @@ __device__ __forceinline__ float dq_block_scale(const float *absmax, const uint8
     return __fmul_rn(static_cast<float>(__ldg(q8 + b)), kg);
 }
 
-// Quantisation. Persistent CTAs walk the groups of 256 blocks (16384
-// weights); each half-warp owns one block at a time: 16 lanes x 4 consecutive
-// fp32 = 64 elements, loaded as float4. Blocks are taken four at a time, and
-// the next four are loaded (across group boundaries) while the current four
-// are coded.
+// Quantisation. Persistent CTAs (two per SM) walk the groups of 256 blocks
+// (16384 weights, 64 KB of fp32). A producer lane streams each group into
+// shared memory by TMA, a quarter group (64 blocks, 16 KB) per stage through
+// a ring of kQzStages stages, with the 128-byte swizzle. Eight consumer warps
+// code a stage: four lanes per block, each lane 16 consecutive elements
+// (elements [16q, 16q + 16) of its block, two 128-byte rows per block), read
+// as four 16-byte pieces whose swizzled addresses fall on eight distinct bank
+// groups in every quarter warp. The absmax is an integer max over |w|'s bit
+// patterns (NaN above +inf, so one compare flags any non-finite block), then
+// two shuffles across the block's four lanes.
 //
 // The code of w is #{i : fl32(w / s) > t_i}, where the 15 decision thresholds
 // t_i are the level midpoints rounded toward -inf in fp32, so that a value on
 // a midpoint falls to the lower level. Instead of dividing and comparing with
-// every threshold, each element forms p = fl32(w * fl32(1/s)), which differs
-// from fl32(w / s) by at most 2.5 units in the last place (two roundings of
-// relative size 2^-24 each, plus the half unit of the exact quotient), and
-// looks up p's bucket in a table of 32 equal buckets over [-1, 1]: the table
-// gives the number of thresholds below the bucket and the one threshold
-// inside it (no bucket holds two, and no threshold lies within 1/1024 of a
-// bucket boundary, so a bucket misplaced by rounding gives the same count).
-// The table is held in 32 copies, one per lane, so the data-dependent lookups
-// of a warp never collide on a shared-memory bank.
-// When p is within kQuantGuard of that threshold the element falls back to
-// the exact quotient and the full comparison.
-constexpr int kQuantThreads = 256;
-constexpr int kQuantBuckets = 32;
-constexpr float kQuantGuard = 4.76837158203125e-07f;   // 2^-21 > 2.5 ulp of any |p| <= 1
+// every threshold, each element forms p = fl32(w * rcp(s)) with the hardware
+// reciprocal (at most 1 ulp from 1/s), so that |p - fl32(w / s)| <= 2.4e-7 for
+// |w| <= s, and looks up p's bucket in a table of 32 equal buckets over
+// [-1, 1] plus one on either side: the table gives the number of thresholds
+// below the bucket and the one threshold inside it (no bucket holds two, and
+// no threshold lies within 1/1024 of a bucket boundary, so a bucket misplaced
+// by the rounding of p + 3 gives the same count). The bucket is read from bits
+// 18..23 of fl32(p + 3) (masked, so every bit pattern addresses the table);
+// the table is held in 32 copies, one per lane, so data-dependent lookups
+// never collide on a bank.
+// When p is within kQuantGuard (2^-21) of that threshold, or s is so small or
+// large that its reciprocal loses precision, the lane recomputes its 16 codes
+// from the exact quotient and the full comparison.
+constexpr int kQzConsumerWarps = 8;
+constexpr int kQzThreads = 32 * (kQzConsumerWarps + 1);   // the last warp issues the TMA copies
+constexpr int kQzStages = 5;
+constexpr int kQzStageBlocks = 64;
+constexpr int kQzStageBytes = kQzStageBlocks * kBlock * 4;  // 16 KB of fp32
+constexpr int kQzTabRows = 64;                              // bits 18..23 of fl32(p + 3)
+constexpr int kQzCtasPerSm = 2;
+constexpr int kQzTabOff = kQzStages * kQzStageBytes;                // float2 [34][32]
+constexpr int kQzAbsOff = kQzTabOff + kQzTabRows * 32 * 8;          // float [2][256]
+constexpr int kQzBarOff = kQzAbsOff + 2 * kGroup * 4;               // full, empty, group
+constexpr int kQzSmemBytes = kQzBarOff + (2 * kQzStages + 2) * 8 + 16 + 1024;
+constexpr float kQuantGuard = 4.76837158203125e-07f;   // 2^-21 > 2.4e-7 bound on |p - fl32(w/s)|
+static_assert(kQzConsumerWarps * 32 == kGroup, "one consumer thread per block of a group");
+static_assert(kQzStageBlocks == 8 * kQzConsumerWarps, "eight blocks per consumer warp and stage");
 
-constexpr int kQuantCtasPerSm = 3;
+__device__ __forceinline__ float2 lds_f2(uint32_t addr) {
+    float2 v;
+    asm("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+    return v;
+}
 
-__global__ void __launch_bounds__(kQuantThreads, kQuantCtasPerSm)
-nf4_quantize_kernel(const float *__restrict__ W, int64_t nb, int dq, uint8_t *__restrict__ codes,
-                    float *__restrict__ absmax, uint8_t *__restrict__ q8, float *__restrict__ cg) {
-    __shared__ float s_abs[kGroup];
-    __shared__ float s_red[kQuantThreads / 32];
-    __shared__ float s_t[16];
-    __shared__ float2 s_tab[kQuantBuckets * 32];   // [bucket][lane copy]: {threshold inside or +inf, count below}
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
 
-    if (threadIdx.x < 15)
-        s_t[threadIdx.x] = __double2float_rd((static_cast<double>(c_levels[threadIdx.x]) +
-                                              static_cast<double>(c_levels[threadIdx.x + 1])) * 0.5);
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < kQuantBuckets * 32; idx += kQuantThreads) {
-        const int bkt = idx >> 5;
-        const float lo = -1.0f + static_cast<float>(bkt) * (2.0f / kQuantBuckets);   // exact
-        const float hi = -1.0f + static_cast<float>(bkt + 1) * (2.0f / kQuantBuckets);
-        int below = 0;
-        float inside = __int_as_float(0x7f800000);   // +inf: no threshold in this bucket
+// Exact code of one element: the quotient rounded once, compared with every
+// threshold.
+__device__ __forceinline__ uint32_t nf4_code_exact(float w, float s, const float (&t)[15]) {
+    const float wn = __fdiv_rn(w, s);
+    uint32_t c = 0;
 #pragma unroll
-        for (int i = 0; i < 15; ++i) {
-            if (s_t[i] < lo) ++below;
-            else if (s_t[i] < hi) inside = s_t[i];
-        }
-        s_tab[idx] = make_float2(inside, __int_as_float(below));
-    }
-    float t[15];
-#pragma unroll
-    for (int i = 0; i < 15; ++i) t[i] = s_t[i];
-    __syncthreads();
+    for (int i = 0; i < 15; ++i) c += (wn > t[i]) ? 1u : 0u;
+    return c;
+}
+
+// Bounded wait that ignores the abort flag: used only to let copies already
+// issued land before the CTA exits.
+__device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity))
+        if (clock64() - t0 > kWaitLimitCycles) return;
+}
+
+__global__ void __launch_bounds__(kQzThreads, kQzCtasPerSm)
+nf4_quantize_kernel(const __grid_constant__ CUtensorMap tm_w,   // W0 as [2 nb, 32] fp32, box {32, 128}
+                    int64_t nb, int dq, uint8_t *__restrict__ codes, float *__restrict__ absmax,
+                    uint8_t *__restrict__ q8, float *__restrict__ cg) {
+    extern __shared__ uint8_t qsm_raw[];
+    uint8_t *qsm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(qsm_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    float2 *tab = reinterpret_cast<float2 *>(qsm + kQzTabOff);
+    float *s_abs = reinterpret_cast<float *>(qsm + kQzAbsOff);
+    uint64_t *full = reinterpret_cast<uint64_t *>(qsm + kQzBarOff);
+    uint64_t *empty = full + kQzStages;
+    uint64_t *grp = empty + kQzStages;                 // [2] all consumer warps done with a group
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(grp + 2);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int half = lane >> 4, hl = lane & 15;
-    const int hw = warp * 2 + half;                 // half-warp 0..15
-    // the two half-warps may take different branches below (ragged last group)
-    const unsigned hmask = half ? 0xffff0000u : 0x0000ffffu;
-    const int64_t ngroups = (nb + kGroup - 1) / kGroup;
-    bool bad = false;
-
-    static_assert(kQuantBuckets == 32, "bucket = top 5 mantissa bits of p + 3");
-    auto code_of = [&](float e, float s, float inv) -> uint32_t {
-        const float p = __fmul_rn(e, inv);
-        // p + 3 lies in [2, 4) (clamped), where the exponent is fixed and the
-        // top five mantissa bits are floor(16 (p + 1)); its rounding (2^-22)
-        // is far below the distance of any threshold from a bucket boundary
-        const float p3 = fminf(fmaxf(p + 3.0f, 2.0f), 3.99999976f);
-        const uint32_t bkt = (__float_as_uint(p3) >> 18) & 31u;
-        const float2 tb = s_tab[bkt * 32 + lane];
-        if (fabsf(p - tb.x) > kQuantGuard)
-            return static_cast<uint32_t>(__float_as_int(tb.y)) + (p > tb.x ? 1u : 0u);
-        // within the guard of a threshold: the exact quotient decides
-        const float wn = __fdiv_rn(e, s);
-        uint32_t c = 0;
+    // thresholds: the exact (fp64) midpoints of adjacent levels, rounded toward -inf
+    float t[15];
 #pragma unroll
-        for (int l = 0; l < 15; ++l) c += (wn > t[l]) ? 1u : 0u;
-        return c;
-    };
-
-    // the half-warp's quads of blocks in order: (group g, first block j0 = hw + 64 k), k = 0..3
-    auto load_quad = [&](int64_t g, int j0, float4 (&v)[4]) {
-        const int64_t b0 = g * kGroup;
-        const int nblk = g < ngroups ? ((nb - b0 < kGroup) ? static_cast<int>(nb - b0) : kGroup) : 0;
+    for (int i = 0; i < 15; ++i)
+        t[i] = __double2float_rd((static_cast<double>(c_levels[i]) + static_cast<double>(c_levels[i + 1])) * 0.5);
+    for (int idx = threadIdx.x; idx < kQzTabRows * 32; idx += kQzThreads) {
+        // Row i holds bucket k = min((i + 1) mod 64, 33) of p. For |p| <= 1 + 2^-22,
+        // fl32(p + 3) lies in [2 - 2^-22, 4]; its bits 18..23 are 63 below 2
+        // (bucket 0: everything below -1), 0..31 on [2, 4) (bucket k = 1..32:
+        // p in [-1 + (k - 1) / 16, -1 + k / 16)) and 32 at 4 (bucket 33:
+        // everything from 1 up). Rows 33..62 are never addressed.
+        const int k = min(((idx >> 5) + 1) & 63, 33);
+        const float inf = __int_as_float(0x7f800000);
+        const float lo = k == 0 ? -inf : -1.0f + static_cast<float>(k - 1) * 0.0625f;
+        const float hi = k == 33 ? inf : -1.0f + static_cast<float>(k) * 0.0625f;
+        int below = 0;
+        float inside = inf;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int j = j0 + 16 * u;
-            v[u] = j < nblk ? __ldg(reinterpret_cast<const float4 *>(W + (b0 + j) * kBlock) + hl)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i = 0; i < 15; ++i) {
+            if (t[i] < lo) ++below;
+            else if (t[i] < hi) inside = t[i];
         }
-    };
-    float4 nxt[4];
-    load_quad(blockIdx.x, hw, nxt);
-    for (int64_t g = blockIdx.x; g < ngroups; g += gridDim.x) {
-        const int64_t b0 = g * kGroup;
-        const int nblk = (nb - b0 < kGroup) ? static_cast<int>(nb - b0) : kGroup;
-#pragma unroll 1
-        for (int j0 = hw; j0 < kGroup; j0 += 4 * 16) {
-            float4 v[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) v[u] = nxt[u];
-            if (j0 + 64 < kGroup) load_quad(g, j0 + 64, nxt);
-            else load_quad(g + gridDim.x, hw, nxt);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int j = j0 + 16 * u;
-                if (j >= nblk) {
-                    if (hl == 0) s_abs[j] = 0.0f;
-                    continue;
-                }
-                const int64_t b = b0 + j;
-                // absmax as the integer max of |w|'s bit patterns: the order of
-                // non-negative floats, with NaN above +inf, so one compare per
-                // block flags any non-finite element
-                uint32_t sb = max(max(__float_as_uint(v[u].x) & 0x7fffffffu, __float_as_uint(v[u].y) & 0x7fffffffu),
-                                  max(__float_as_uint(v[u].z) & 0x7fffffffu, __float_as_uint(v[u].w) & 0x7fffffffu));
-#pragma unroll
-                for (int o = 8; o >= 1; o >>= 1) sb = max(sb, __shfl_xor_sync(hmask, sb, o));
-                bad |= sb >= 0x7f800000u;
-                const float s = __uint_as_float(sb);
-                uint32_t q[4] = {7u, 7u, 7u, 7u};
-                if (s != 0.0f) {
-                    const float inv = __frcp_rn(s);
-                    q[0] = code_of(v[u].x, s, inv);
-                    q[1] = code_of(v[u].y, s, inv);
-                    q[2] = code_of(v[u].z, s, inv);
-                    q[3] = code_of(v[u].w, s, inv);
-                }
-                const uint16_t packed = static_cast<uint16_t>(((q[0] << 4) | q[1]) |
-                                                              (((q[2] << 4) | q[3]) << 8));
-                reinterpret_cast<uint16_t *>(codes + b * (kBlock / 2))[hl] = packed;
-                if (hl == 0) {
-                    absmax[b] = s;
-                    s_abs[j] = s;
+        tab[idx] = make_float2(inside, __int_as_float(below));
+    }
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kQzStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kQzConsumerWarps);
+        }
+        mbar_init(&grp[0], kQzConsumerWarps);
+        mbar_init(&grp[1], kQzConsumerWarps);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_w);
+    }
+    __syncthreads();
+
+    const int64_t ngroups = (nb + kGroup - 1) / kGroup;
+    if (warp == kQzConsumerWarps) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            int n = 0;
+            for (int64_t g = blockIdx.x; g < ngroups; g += gridDim.x) {
+                for (int qq = 0; qq < kGroup / kQzStageBlocks; ++qq) {
+                    const int64_t b0 = g * kGroup + qq * kQzStageBlocks;
+                    if (b0 >= nb) break;
+                    const int s = n % kQzStages;
+                    const uint32_t ph = static_cast<uint32_t>(n / kQzStages) & 1u;
+                    if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) goto drain;
+                    mbar_arrive_expect_tx(&full[s], kQzStageBytes);
+                    tma_load_2d(qsm + s * kQzStageBytes, &tm_w, &full[s], 0, static_cast<int32_t>(2 * b0));
+                    ++n;
                 }
             }
+        drain:
+            // every copy issued has landed before the CTA's memory is released
+            for (int m = n - kQzStages > 0 ? n - kQzStages : 0; m < n; ++m)
+                mbar_drain(&full[m % kQzStages], static_cast<uint32_t>(m / kQzStages) & 1u);
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------- consumers
+    const int bq = lane >> 2;                    // block of this lane among the warp's eight
+    const int q = lane & 3;                      // elements [16q, 16q + 16) of that block
+    const int lb = warp * 8 + bq;                // block within a stage
+    const int row = 2 * lb + (q >> 1);           // 128-byte row within the stage
+    uint32_t off[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        off[j] = static_cast<uint32_t>(row * 128 + (((4 * (q & 1) + j) ^ (row & 7)) << 4));
+    const uint32_t mytab = smem_u32(tab) + 8u * lane;
+    bool bad = false;
+    int n = 0, gi = 0;
+    for (int64_t g = blockIdx.x; g < ngroups; g += gridDim.x, ++gi) {
+        float *sa = s_abs + (gi & 1) * kGroup;
+        for (int qq = 0; qq < kGroup / kQzStageBlocks; ++qq) {
+            const int64_t b0 = g * kGroup + qq * kQzStageBlocks;
+            if (b0 >= nb) break;
+            const int s = n % kQzStages;
+            const uint32_t ph = static_cast<uint32_t>(n / kQzStages) & 1u;
+            ++n;
+            if (!mbar_wait(&full[s], ph, abort_flag)) goto done;
+            const uint8_t *st = qsm + s * kQzStageBytes;
+            float x[16];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float4 v = *reinterpret_cast<const float4 *>(st + off[j]);
+                x[4 * j] = v.x;
+                x[4 * j + 1] = v.y;
+                x[4 * j + 2] = v.z;
+                x[4 * j + 3] = v.w;
+            }
+            // |w| bit patterns, reduced as a tree
+            uint32_t mm[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                mm[e] = max(__float_as_uint(x[e]) & 0x7fffffffu, __float_as_uint(x[e + 8]) & 0x7fffffffu);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) mm[e] = max(mm[e], mm[e + 4]);
+            uint32_t m = max(max(mm[0], mm[1]), max(mm[2], mm[3]));
+            m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+            m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+            const float sc = __uint_as_float(m);
+            uint32_t c[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) c[e] = 7u;          // all-zero block: the exact zero level
+            if (m >= 0x7f800000u) {
+                bad = true;                                  // non-finite input: codes unspecified
+            } else if (m != 0u) {
+                // a reciprocal of s this small or large loses precision: exact path
+                bool near = !(sc >= 0x1p-125f && sc <= 0x1p125f);
+                if (!near) {
+                    const float inv = rcp_approx(sc);
+                    float dmin = 1.0f;           // smallest distance of p to its bucket's threshold
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float p = x[e] * inv;
+                        const uint32_t row = (__float_as_uint(p + 3.0f) >> 10) & 0x3F00u;   // 256 bytes per row
+                        const float2 te = lds_f2(mytab + row);
+                        const float d = p - te.x;
+                        c[e] = static_cast<uint32_t>(__float_as_int(te.y)) + (d > 0.0f ? 1u : 0u);
+                        dmin = fminf(dmin, fabsf(d));
+                    }
+                    near = dmin <= kQuantGuard;
+                }
+                if (near) {
+                    // some element lies within the guard of its threshold: the
+                    // exact quotient decides all sixteen (rare)
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) c[e] = nf4_code_exact(x[e], sc, t);
+                }
+            }
+            // byte j of the lane's 8: element 2j in the high nibble, 2j + 1 in the low
+            uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                w0 |= ((c[2 * j] << 4) | c[2 * j + 1]) << (8 * j);
+                w1 |= ((c[8 + 2 * j] << 4) | c[8 + 2 * j + 1]) << (8 * j);
+            }
+            const int64_t b = b0 + lb;
+            if (b < nb) {
+                *reinterpret_cast<uint2 *>(codes + b * (kBlock / 2) + 8 * q) = make_uint2(w0, w1);
+                if (q == 0) absmax[b] = sc;
+            }
+            if (q == 0) sa[qq * kQzStageBlocks + lb] = sc;
+            // the stage's values are consumed (the stores above depend on all of them)
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
         }
         if (dq) {
-            __syncthreads();
-            // group constant c_g = max of the block scales of this group
-            float m = s_abs[threadIdx.x];
+            // double quantisation of this group's 256 scales: every consumer
+            // warp has written its scales before the group barrier completes
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&grp[gi & 1]);
+            if (!mbar_wait(&grp[gi & 1], static_cast<uint32_t>(gi >> 1) & 1u, abort_flag)) goto done;
+            const int64_t gb = g * kGroup;
+            float cmax = 0.0f;
 #pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-            if (lane == 0) s_red[warp] = m;
-            __syncthreads();
-            float c = s_red[0];
+            for (int k = 0; k < kGroup / 32; ++k)
+                if (gb + lane + 32 * k < nb) cmax = fmaxf(cmax, sa[lane + 32 * k]);
 #pragma unroll
-            for (int i = 1; i < kQuantThreads / 32; ++i) c = fmaxf(c, s_red[i]);
-            const int j = threadIdx.x;
-            if (j < nblk) {
+            for (int o = 16; o >= 1; o >>= 1) cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
+            const int j = warp * 32 + lane;
+            if (gb + j < nb) {
                 uint8_t code = 0;
-                if (c > 0.0f) {
+                if (cmax > 0.0f) {
                     // fl32(fl32(s / c) * 127), rounded half to even
-                    const float ratio = __fdiv_rn(s_abs[j], c);
+                    const float ratio = __fdiv_rn(sa[j], cmax);
                     code = static_cast<uint8_t>(__float2int_rn(__fmul_rn(ratio, 127.0f)));
                 }
-                q8[b0 + j] = code;
+                q8[gb + j] = code;
             }
-            if (threadIdx.x == 0) cg[g] = c;
+            if (warp == 0 && lane == 0) cg[g] = cmax;
         }
-        __syncthreads();      // s_abs is reused by the next group
     }
+done:
     if (__any_sync(0xffffffffu, bad) && lane == 0) record_status(NF4_ERR_NONFINITE);
 }
 

@@ -12,7 +12,8 @@
 //     groups of the tile, so one token-fragment load serves 32 weight rows;
 //   * each warp fetches its k range of a tile in chunks of CB blocks -- 32
 //     rows x CB * 32 contiguous bytes -- with one 2-D TMA copy into a
-//     two-slot ring; a slot is refilled as soon as its chunk is consumed;
+//     two-slot ring; chunk c + 1 is requested as soon as chunk c has landed
+//     (its slot held chunk c - 1, already consumed);
 //   * a byte of codes becomes a pair of bf16 levels through a 256-entry table
 //     in shared memory whose entry b, copy l sits at address
 //     65536 + 256 b + 4 l: a single byte permute turns (code byte, lane) into
@@ -141,7 +142,7 @@ struct DsScales {
 //
 // Warp w takes blocks [w rb, w rb + rb) of every tile, in chunks of CB
 // blocks. Its chunks are numbered c = 0, 1, ... over all of the CTA's tiles;
-// chunk c goes to ring slot c % 2, and the slot takes chunk c + 2 as soon as
+// chunk c goes to ring slot c % 2, and the other slot takes chunk c + 1 as soon as
 // every lane has read chunk c.
 template <int TG, int CB>
 __global__ void __launch_bounds__(kDsThreads, 1)
@@ -167,12 +168,6 @@ qlora_decode_stream_kernel(const __grid_constant__ CUtensorMap tm_codes,   // [N
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
 
-    // level pairs: byte b -> (bf16(level[b >> 4]) low half, bf16(level[b & 15]) high half)
-    for (int idx = threadIdx.x; idx < 256 * 32; idx += kDsThreads) {
-        const int b = idx >> 5, l = idx & 31;
-        __nv_bfloat162 p = __floats2bfloat162_rn(c_levels[b >> 4], c_levels[b & 15]);
-        *reinterpret_cast<uint32_t *>(lut_g + b * 256 + 4 * l) = *reinterpret_cast<uint32_t *>(&p);
-    }
     if (threadIdx.x == 0) {
         for (int i = 0; i < kDsWarps * 2; ++i) mbar_init(&bars[i], 1);
         *abort_flag = 0;
@@ -275,12 +270,20 @@ qlora_decode_stream_kernel(const __grid_constant__ CUtensorMap tm_codes,   // [N
     // triggers this launch only after its own wait on the kernel before.
     griddep_launch_dependents();
 
-    // the first two chunks and the first chunk's scales
+    // the first chunk and its scales
     issue(0);
-    issue(1);
     DsScales<CB> sc = load_scales(0);
 
     // the first two blocks' tokens
+    // The lookup table is filled while the first chunks are in flight.
+    // level pairs: byte b -> (bf16(level[b >> 4]) low half, bf16(level[b & 15]) high half)
+    for (int idx = threadIdx.x; idx < 256 * 32; idx += kDsThreads) {
+        const int b = idx >> 5, l = idx & 31;
+        __nv_bfloat162 p = __floats2bfloat162_rn(c_levels[b >> 4], c_levels[b & 15]);
+        *reinterpret_cast<uint32_t *>(lut_g + b * 256 + 4 * l) = *reinterpret_cast<uint32_t *>(&p);
+    }
+    __syncthreads();
+
     uint4 xa0[TG], xb0[TG], xa1[TG], xb1[TG];
     load_x(xa0, xb0);
     load_x(xa1, xb1);
@@ -333,6 +336,11 @@ qlora_decode_stream_kernel(const __grid_constant__ CUtensorMap tm_codes,   // [N
             sc = load_scales(c + 1);
             if (!mbar_wait(&bars[warp * 2 + (c & 1)], static_cast<uint32_t>(c >> 1) & 1u, abort_flag))
                 goto done;
+            // the next chunk goes out as soon as this one has landed, into the
+            // slot of the chunk before, which every lane has finished reading:
+            // at start-up each SM first fetches one chunk per warp, so the
+            // first tile's data arrives before the rest of the burst
+            issue(c + 1);
             const uint32_t cbase = ((c & 1) ? slot1 : slot0) + static_cast<uint32_t>(g) * kRowStride + 8u * t +
                                    after_wait_zero();
             const int nbc = min(CB, nkb - ch * CB);
@@ -411,7 +419,6 @@ qlora_decode_stream_kernel(const __grid_constant__ CUtensorMap tm_codes,   // [N
                 for (int i = 0; i < nbc; ++i) block(i);
             }
             __syncwarp();        // every lane has read the chunk
-            issue(c + 2);
         }
 
         // ---- the tile's k-split partials -> one ordered sum with the LoRA

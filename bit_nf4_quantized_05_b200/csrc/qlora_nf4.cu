@@ -748,13 +748,20 @@ nf4_status nf4_quantize(const float *W0, const nf4_weight *w, void *stream) {
     if (!aligned16(W0)) return NF4_ERR_ALIGNMENT;
     const int64_t nb = w->n * w->k / kBlock;
     const int64_t groups = (nb + kGroup - 1) / kGroup;
-    if (groups > 0x7fffffff) return NF4_ERR_UNSUPPORTED_SHAPE;
-    // persistent: kQuantCtasPerSm CTAs per SM walk the groups
-    const int64_t grid = std::min<int64_t>(groups, int64_t(kQuantCtasPerSm) * num_sms(current_device()));
+    // TMA row coordinates (two 128-byte rows per block) are 32-bit
+    if (2 * nb > 0x7fffffffLL) return NF4_ERR_UNSUPPORTED_SHAPE;
+    CUtensorMap tm_w;
+    if (!make_map(&tm_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, W0, 32, static_cast<uint64_t>(2 * nb), 32,
+                  2 * kQzStageBlocks, CU_TENSOR_MAP_SWIZZLE_128B))
+        return NF4_ERR_CUDA;
+    // persistent: kQzCtasPerSm CTAs per SM walk the groups
+    const int64_t grid = std::min<int64_t>(groups, int64_t(kQzCtasPerSm) * num_sms(current_device()));
+    NF4_TRY_CUDA(cudaFuncSetAttribute(nf4_quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      kQzSmemBytes));
     LaunchTimer t(KK_QUANTIZE, static_cast<cudaStream_t>(stream));
-    nf4_quantize_kernel<<<static_cast<unsigned>(grid), kQuantThreads, 0,
+    nf4_quantize_kernel<<<static_cast<unsigned>(grid), kQzThreads, kQzSmemBytes,
                           static_cast<cudaStream_t>(stream)>>>(
-        W0, nb, w->double_quant, w->codes, w->absmax, w->absmax_q8, w->absmax_c);
+        tm_w, nb, w->double_quant, w->codes, w->absmax, w->absmax_q8, w->absmax_c);
     t.stop();
     NF4_TRY_CUDA(cudaGetLastError());
     return NF4_OK;
