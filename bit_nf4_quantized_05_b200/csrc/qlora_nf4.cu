@@ -34,10 +34,10 @@ constexpr int kMaxDevices = 64;
 // Optional per-kernel event timing (nf4_profiling / nf4_profile_read)
 // ---------------------------------------------------------------------------
 enum KernelKind {
-    KK_QUANTIZE, KK_DEQUANTIZE, KK_LORA_U, KK_LORA_V, KK_LORA_DB, KK_LORA_DA, KK_SCALE, KK_ZERO, KK_GEMM_FWD, KK_GEMM_DGRAD, KK_DECODE, KK_DECODE_U, KK_COUNT
+    KK_QUANTIZE, KK_DEQUANTIZE, KK_LORA_U, KK_LORA_V, KK_LORA_DBDA, KK_ZERO, KK_GEMM_FWD, KK_GEMM_DGRAD, KK_DECODE, KK_DECODE_U, KK_COUNT
 };
 const char *const kKindNames[KK_COUNT] = {
-    "nf4_quantize", "nf4_dequantize", "lora_u", "lora_v", "lora_dB", "lora_dA", "lora_scale", "zero_fill", "qlora_gemm_fwd", "qlora_gemm_dgrad", "qlora_decode",
+    "nf4_quantize", "nf4_dequantize", "lora_u", "lora_v", "lora_dB_dA", "zero_fill", "qlora_gemm_fwd", "qlora_gemm_dgrad", "qlora_decode",
     "decode_lora_u"};
 
 struct ProfRecord {
@@ -217,22 +217,6 @@ size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 // kSkMaxSplits CTAs, and the grid is sized to about one CTA per SM. (At r <= 64
 // two CTAs fit on an SM, which lets the clusters pack into one wave; more
 // splits than one per SM measured slower on B200.)
-struct SkinnyPlan {
-    int RN, p_tiles, steps, sps, splits;
-};
-
-SkinnyPlan plan_skinny(int64_t P, int64_t Q, int32_t r, int sms) {
-    SkinnyPlan p{};
-    p.RN = r <= 64 ? 64 : 128;
-    p.p_tiles = static_cast<int>((P + 127) / 128);
-    p.steps = static_cast<int>((Q + 63) / 64);
-    int splits = std::max(1, sms / std::max(1, p.p_tiles));
-    splits = std::min({splits, kSkMaxSplits, p.steps});
-    p.sps = (p.steps + splits - 1) / splits;
-    p.splits = (p.steps + p.sps - 1) / p.sps;   // every split has at least one step
-    return p;
-}
-
 // Stream-K scratch of one fused GEMM launch: per CTA pair one fp32 partial
 // tile (2 CTAs x 128 rows x 256 columns) and 8 flags (2 CTAs x 4 epilogue
 // warps). Sized for sms / 2 pairs, the most that can be resident.
@@ -289,39 +273,95 @@ enum class Major { K, MN };
 // skinny tcgen05 kernel (split reduction included).
 //   a: row-major bf16 [a_rows, a_cols]; K-major: p = row, q = col; MN-major: q = row, p = col
 //   b: row-major bf16 [b_rows, b_cols]; K-major: j = row, q = col; MN-major: q = row, j = col
-nf4_status skinny_product(int kind, const void *a, int64_t a_rows, int64_t a_cols, Major am,
-                          const void *b, int64_t b_rows, int64_t b_cols, Major bm, int32_t r,
-                          float *out_f32, uint16_t *out_bf16, float scale, int transposed,
-                          cudaStream_t stream, int *zero_ints = nullptr, int zero_count = 0) {
-    const int sms = num_sms(current_device());
-    const int64_t P = am == Major::K ? a_rows : a_cols;
-    const int64_t Q = am == Major::K ? a_cols : a_rows;
-    const SkinnyPlan pl = plan_skinny(P, Q, r, sms);
-    CUtensorMap ta, tb;
-    bool ok = am == Major::K
-                  ? make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a, a_cols, a_rows, 64, 128,
+struct SkinnySpec {
+    const void *a;
+    int64_t a_rows, a_cols;
+    Major am;
+    const void *b;
+    int64_t b_rows, b_cols;
+    Major bm;
+    int32_t r;
+    float *out_f32;
+    uint16_t *out_bf16;
+    float scale;
+    int transposed;
+};
+
+// Tensor maps and job fields of one product; splits is the launch's split count.
+bool skinny_job(const SkinnySpec &sp, int RN, int splits, CUtensorMap *ta, CUtensorMap *tb,
+                SkinnyJob *job) {
+    const int64_t P = sp.am == Major::K ? sp.a_rows : sp.a_cols;
+    const int64_t Q = sp.am == Major::K ? sp.a_cols : sp.a_rows;
+    bool ok = sp.am == Major::K
+                  ? make_map(ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, sp.a, sp.a_cols, sp.a_rows, 64, 128,
                              CU_TENSOR_MAP_SWIZZLE_128B)
-                  : make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a, a_cols, a_rows, 64, 64,
+                  : make_map(ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, sp.a, sp.a_cols, sp.a_rows, 64, 64,
                              CU_TENSOR_MAP_SWIZZLE_128B);
-    ok = ok && (bm == Major::K
-                    ? make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, b, b_cols, b_rows, 64,
-                               static_cast<uint32_t>(pl.RN), CU_TENSOR_MAP_SWIZZLE_128B)
-                    : make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, b, b_cols, b_rows, 64, 64,
+    ok = ok && (sp.bm == Major::K
+                    ? make_map(tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, sp.b, sp.b_cols, sp.b_rows, 64,
+                               static_cast<uint32_t>(RN), CU_TENSOR_MAP_SWIZZLE_128B)
+                    : make_map(tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, sp.b, sp.b_cols, sp.b_rows, 64, 64,
                                CU_TENSOR_MAP_SWIZZLE_128B));
-    if (!ok) return NF4_ERR_CUDA;
-    SkinnyArgs args{static_cast<int>(P), pl.steps, pl.sps, r,          out_f32,
-                    out_bf16,            scale,    transposed, zero_ints, zero_count};
-    const dim3 grid(static_cast<unsigned>(pl.splits), static_cast<unsigned>(pl.p_tiles));
+    job->P = static_cast<int>(P);
+    job->p_tiles = static_cast<int>((P + 127) / 128);
+    job->steps = static_cast<int>((Q + 63) / 64);
+    job->steps_per_split = (job->steps + splits - 1) / splits;
+    job->r = sp.r;
+    job->out_f32 = sp.out_f32;
+    job->out_bf16 = sp.out_bf16;
+    job->scale = sp.scale;
+    job->transposed = sp.transposed;
+    return ok;
+}
+
+// One launch of one or two products (n = 1, 2) with the same operand layouts
+// and rank, plus optional flag zeroing and an element-wise side task.
+nf4_status skinny_launch(int kind, const SkinnySpec *sp, int n, cudaStream_t stream,
+                         int *zero_ints = nullptr, int zero_count = 0, const float *conv_src = nullptr,
+                         uint16_t *conv_dst = nullptr, int64_t conv_n = 0, float conv_scale = 0.f) {
+    const int sms = num_sms(current_device());
+    const int RN = sp[0].r <= 64 ? 64 : 128;
+    int p_tiles = 0, steps = 1;
+    for (int i = 0; i < n; ++i) {
+        if (sp[i].am != sp[0].am || sp[i].bm != sp[0].bm || sp[i].r != sp[0].r) return NF4_ERR_INVALID_ARG;
+        const int64_t P = sp[i].am == Major::K ? sp[i].a_rows : sp[i].a_cols;
+        const int64_t Q = sp[i].am == Major::K ? sp[i].a_cols : sp[i].a_rows;
+        p_tiles += static_cast<int>((P + 127) / 128);
+        steps = std::max(steps, static_cast<int>((Q + 63) / 64));
+    }
+    // one wave: the splits of all tiles fill the SMs once (clusters of at most 8)
+    int splits = std::max(1, sms / std::max(1, p_tiles));
+    splits = std::min({splits, kSkMaxSplits, steps});
+    const int sps = (steps + splits - 1) / splits;
+    splits = (steps + sps - 1) / sps;            // every split has at least one step
+    SkinnyArgs args{};
+    CUtensorMap ta[2], tb[2];
+    for (int i = 0; i < n; ++i)
+        if (!skinny_job(sp[i], RN, splits, &ta[i], &tb[i], &args.job[i])) return NF4_ERR_CUDA;
+    if (n == 1) {
+        ta[1] = ta[0];
+        tb[1] = tb[0];
+        args.job[1] = args.job[0];
+    }
+    args.njobs = n;
+    args.zero_ints = zero_ints;
+    args.zero_count = zero_count;
+    args.conv_src = conv_src;
+    args.conv_dst = conv_dst;
+    args.conv_n = conv_n;
+    args.conv_scale = conv_scale;
+    const dim3 grid(static_cast<unsigned>(splits), static_cast<unsigned>(p_tiles));
+    const Major am = sp[0].am, bm = sp[0].bm;
     cudaError_t e = cudaErrorInvalidValue;
     {
         LaunchTimer t(kind, stream);
 #define NF4_SKINNY_CASE(RN_, AMN, BMN)                                                      \
-    if (pl.RN == RN_ && (am == Major::MN) == AMN && (bm == Major::MN) == BMN) {             \
+    if (RN == RN_ && (am == Major::MN) == AMN && (bm == Major::MN) == BMN) {                \
         auto kern = skinny_cluster_kernel<RN_, AMN, BMN>;                                   \
         NF4_TRY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                                           SkCfg<RN_, AMN, BMN>::kSmemBytes));               \
         e = launch_ex(kern, grid, dim3(kSkThreads), SkCfg<RN_, AMN, BMN>::kSmemBytes, stream, \
-                      static_cast<unsigned>(pl.splits), ta, tb, args);                      \
+                      static_cast<unsigned>(splits), ta[0], tb[0], ta[1], tb[1], args);     \
     }
         NF4_SKINNY_CASE(64, false, false)
         NF4_SKINNY_CASE(128, false, false)
@@ -335,6 +375,14 @@ nf4_status skinny_product(int kind, const void *a, int64_t a_rows, int64_t a_col
     if (e != cudaSuccess) return NF4_ERR_CUDA;
     NF4_TRY_CUDA(cudaGetLastError());
     return NF4_OK;
+}
+
+nf4_status skinny_product(int kind, const void *a, int64_t a_rows, int64_t a_cols, Major am,
+                          const void *b, int64_t b_rows, int64_t b_cols, Major bm, int32_t r,
+                          float *out_f32, uint16_t *out_bf16, float scale, int transposed,
+                          cudaStream_t stream, int *zero_ints = nullptr, int zero_count = 0) {
+    const SkinnySpec sp{a, a_rows, a_cols, am, b, b_rows, b_cols, bm, r, out_f32, out_bf16, scale, transposed};
+    return skinny_launch(kind, &sp, 1, stream, zero_ints, zero_count);
 }
 
 template <int BN, bool DGRAD>
@@ -878,32 +926,26 @@ nf4_status qlora_linear_bwd(const nf4_weight *w, const uint16_t *x, int64_t M, c
                    sk_pairs_max(sms)};
     const float scale = alpha / static_cast<float>(r);
 
-    // bf16(s u), from the saved u or recomputed from x
-    if (u) {
-        LaunchTimer t(KK_SCALE, s);
-        const unsigned grid = static_cast<unsigned>(std::min<int64_t>((M * r + 255) / 256, 4096));
-        const cudaError_t e =
-            launch_ex(scale_to_bf16_kernel, dim3(grid), dim3(256), 0, s, 0u, u, M * r, scale, u_s);
-        t.stop();
-        if (e != cudaSuccess) return NF4_ERR_CUDA;
-        NF4_TRY_CUDA(cudaGetLastError());
-    } else {
+    // bf16(s u): recomputed from x here, or converted from the saved u by the v launch
+    if (!u) {
         st = skinny_product(KK_LORA_U, x, M, K, Major::K, A, r, K, Major::K, r, nullptr, u_s,
                             scale, 0, s);
         if (st != NF4_OK) return st;
     }
     // v = dY B  ->  bf16(s v)
-    st = skinny_product(KK_LORA_V, dY, M, N, Major::K, B, N, r, Major::MN, r, nullptr, v_s,
-                        scale, 0, s);
-    if (st != NF4_OK) return st;
-    // dB = dY^T bf16(s u)   ([N, r])
-    st = skinny_product(KK_LORA_DB, dY, M, N, Major::MN, u_s, M, r, Major::MN, r, nullptr, dB,
-                        1.0f, 0, s);
-    if (st != NF4_OK) return st;
-    // dA = (x^T bf16(s v))^T   ([r, K]); also clears the dgrad GEMM's stream-K flags
-    st = skinny_product(KK_LORA_DA, x, M, K, Major::MN, v_s, M, r, Major::MN, r, nullptr, dA,
-                        1.0f, 1, s, sk.flags, sk.pairs_max * kSkFlagsPerPair);
-    if (st != NF4_OK) return st;
+    {
+        const SkinnySpec sv{dY, M, N, Major::K, B, N, r, Major::MN, r, nullptr, v_s, scale, 0};
+        st = skinny_launch(KK_LORA_V, &sv, 1, s, nullptr, 0, u, u ? u_s : nullptr, u ? M * r : 0, scale);
+        if (st != NF4_OK) return st;
+    }
+    // dB = dY^T bf16(s u) ([N, r]) and dA = (x^T bf16(s v))^T ([r, K]) in one launch,
+    // which also clears the dgrad GEMM's stream-K flags
+    {
+        const SkinnySpec j[2] = {{dY, M, N, Major::MN, u_s, M, r, Major::MN, r, nullptr, dB, 1.0f, 0},
+                                 {x, M, K, Major::MN, v_s, M, r, Major::MN, r, nullptr, dA, 1.0f, 1}};
+        st = skinny_launch(KK_LORA_DBDA, j, 2, s, sk.flags, sk.pairs_max * kSkFlagsPerPair);
+        if (st != NF4_OK) return st;
+    }
     // dX = dY W~ + bf16(s v) A
     if (dX) return launch_gemm_auto<true>(w, dY, M, N, K, v_s, r, A, dX, s, &sk);
     return NF4_OK;

@@ -13,7 +13,10 @@
 // in its own shared memory, and after a cluster barrier the CTAs add the
 // partials of all splits in split order through distributed shared memory
 // (deterministic) and write the destination with its scale, rounding and
-// layout. No partial sums go to global memory.
+// layout. No partial sums go to global memory. One launch may carry two
+// products of the same operand layouts (the backward's dB and dA, which are
+// independent) and an element-wise side task (bf16(s u) from the saved u),
+// so that each launch's ramp and drain are paid once.
 #pragma once
 
 #include "nf4_common.cuh"
@@ -24,8 +27,11 @@ constexpr int kSkStages = 4;     // two CTAs fit on one SM
 constexpr int kSkThreads = 256;   // warp 0 TMA, warp 1 MMA, warps 4..7 epilogue
 constexpr int kSkMaxSplits = 8;   // portable cluster size
 
-struct SkinnyArgs {
+// One product of a launch. A launch carries one or two products of the same
+// operand layouts; grid rows [0, p_tiles of job 0) take job 0, the rest job 1.
+struct SkinnyJob {
     int P;               // output rows (MMA M, tiles of 128)
+    int p_tiles;
     int steps;           // reduction steps of 64
     int steps_per_split;
     int r;               // output columns actually written (<= RN)
@@ -33,8 +39,18 @@ struct SkinnyArgs {
     uint16_t *out_bf16;  // bf16(scale * sum): [P][r], or [r][P] when transposed; or null
     float scale;
     int transposed;
+};
+
+struct SkinnyArgs {
+    SkinnyJob job[2];
+    int njobs;
     int *zero_ints;      // optional: zeroed by the first CTA (flags for a later kernel)
     int zero_count;
+    // optional element-wise side task over all CTAs: conv_dst[i] = bf16(conv_scale * conv_src[i])
+    const float *conv_src;
+    uint16_t *conv_dst;
+    int64_t conv_n;
+    float conv_scale;
 };
 
 template <int RN, bool A_MN, bool B_MN>
@@ -58,8 +74,10 @@ __device__ __forceinline__ float ld_cluster_f32(uint32_t caddr) {
 // Grid (splits, p_tiles), cluster (splits, 1, 1): blockIdx.x is the split.
 template <int RN, bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(kSkThreads, 2)
-skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a,
-                      const __grid_constant__ CUtensorMap tm_b, const SkinnyArgs args) {
+skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a0,
+                      const __grid_constant__ CUtensorMap tm_b0,
+                      const __grid_constant__ CUtensorMap tm_a1,
+                      const __grid_constant__ CUtensorMap tm_b1, const SkinnyArgs args) {
     using Cfg = SkCfg<RN, A_MN, B_MN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -74,9 +92,13 @@ skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a,
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int split = blockIdx.x, splits = gridDim.x;
-    const int p0 = blockIdx.y * 128;
-    const int s0 = split * args.steps_per_split;
-    const int s1 = min(args.steps, s0 + args.steps_per_split);
+    const int jb = (args.njobs > 1 && static_cast<int>(blockIdx.y) >= args.job[0].p_tiles) ? 1 : 0;
+    const SkinnyJob &J = args.job[jb];
+    const CUtensorMap *tm_a = jb ? &tm_a1 : &tm_a0;
+    const CUtensorMap *tm_b = jb ? &tm_b1 : &tm_b0;
+    const int p0 = (static_cast<int>(blockIdx.y) - (jb ? args.job[0].p_tiles : 0)) * 128;
+    const int s0 = split * J.steps_per_split;
+    const int s1 = min(J.steps, s0 + J.steps_per_split);
     const int nsteps = s1 - s0;
 
     if (threadIdx.x == 0) {
@@ -87,8 +109,8 @@ skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a,
         mbar_init(done_bar, 1);
         *abort_flag = 0;
         fence_mbar_init();
-        tma_prefetch_desc(&tm_a);
-        tma_prefetch_desc(&tm_b);
+        tma_prefetch_desc(tm_a);
+        tma_prefetch_desc(tm_b);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, RN);
@@ -102,6 +124,14 @@ skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a,
     griddep_launch_dependents();
     if (args.zero_ints && blockIdx.x == 0 && blockIdx.y == 0)
         for (int z = threadIdx.x; z < args.zero_count; z += kSkThreads) args.zero_ints[z] = 0;
+    if (args.conv_n > 0) {
+        const int64_t ctas = static_cast<int64_t>(gridDim.x) * gridDim.y;
+        const int64_t cta = static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x;
+        for (int64_t e = cta * kSkThreads + threadIdx.x; e < args.conv_n; e += ctas * kSkThreads) {
+            __nv_bfloat16 b = __float2bfloat16_rn(args.conv_scale * args.conv_src[e]);
+            args.conv_dst[e] = *reinterpret_cast<uint16_t *>(&b);
+        }
+    }
 
     if (warp == 0 && lane == 0) {
         for (int it = 0; it < nsteps; ++it) {
@@ -113,17 +143,17 @@ skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a,
             const int q0 = (s0 + it) * 64;
             mbar_arrive_expect_tx(&full[st], Cfg::kStageBytes);
             if (!A_MN) {
-                tma_load_2d(a, &tm_a, &full[st], q0, p0);
+                tma_load_2d(a, tm_a, &full[st], q0, p0);
             } else {
-                tma_load_2d(a, &tm_a, &full[st], p0, q0);
-                tma_load_2d(a + 8192, &tm_a, &full[st], p0 + 64, q0);
+                tma_load_2d(a, tm_a, &full[st], p0, q0);
+                tma_load_2d(a + 8192, tm_a, &full[st], p0 + 64, q0);
             }
             if (!B_MN) {
-                tma_load_2d(b, &tm_b, &full[st], q0, 0);
+                tma_load_2d(b, tm_b, &full[st], q0, 0);
             } else {
 #pragma unroll
                 for (int ja = 0; ja < RN / 64; ++ja)
-                    tma_load_2d(b + ja * 8192, &tm_b, &full[st], ja * 64, q0);
+                    tma_load_2d(b + ja * 8192, tm_b, &full[st], ja * 64, q0);
             }
         }
     } else if (warp == 1 && lane == 0) {
@@ -158,7 +188,7 @@ skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a,
             tc_fence_after();
 #pragma unroll 1
             for (int c = 0; c < RN / 32; ++c) {
-                if (c * 32 >= args.r) break;
+                if (c * 32 >= J.r) break;
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(tmem_base + ((q * 32) << 16) + c * 32, v);
                 tmem_ld_wait();
@@ -178,26 +208,26 @@ skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a,
     // (row, column) elements, numbered column-major when the destination is
     // transposed so that consecutive threads write consecutive addresses.
     {
-        const int r = args.r;
+        const int r = J.r;
         const int E = 128 * r;
         const int e0 = static_cast<int>((static_cast<int64_t>(E) * split) / splits);
         const int e1 = static_cast<int>((static_cast<int64_t>(E) * (split + 1)) / splits);
         const uint32_t part_addr = smem_u32(part);
         for (int e = e0 + threadIdx.x; e < e1; e += kSkThreads) {
-            const int row = args.transposed ? e % 128 : e / r;
-            const int j = args.transposed ? e / 128 : e % r;
+            const int row = J.transposed ? e % 128 : e / r;
+            const int j = J.transposed ? e / 128 : e % r;
             const int p = p0 + row;
-            if (p >= args.P) continue;
+            if (p >= J.P) continue;
             const uint32_t off = static_cast<uint32_t>((row * Cfg::kPartStride + j) * 4);
             float acc = 0.0f;
             for (int s = 0; s < splits; ++s)
                 acc += ld_cluster_f32(mapa_shared(part_addr + off, static_cast<uint32_t>(s)));
-            if (args.out_f32) args.out_f32[static_cast<int64_t>(p) * r + j] = acc;
-            if (args.out_bf16) {
-                __nv_bfloat16 b = __float2bfloat16_rn(args.scale * acc);
-                const int64_t o = args.transposed ? static_cast<int64_t>(j) * args.P + p
-                                                  : static_cast<int64_t>(p) * r + j;
-                args.out_bf16[o] = *reinterpret_cast<uint16_t *>(&b);
+            if (J.out_f32) J.out_f32[static_cast<int64_t>(p) * r + j] = acc;
+            if (J.out_bf16) {
+                __nv_bfloat16 b = __float2bfloat16_rn(J.scale * acc);
+                const int64_t o = J.transposed ? static_cast<int64_t>(j) * J.P + p
+                                               : static_cast<int64_t>(p) * r + j;
+                J.out_bf16[o] = *reinterpret_cast<uint16_t *>(&b);
             }
         }
     }
@@ -205,18 +235,6 @@ skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a,
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, RN);
-    }
-}
-
-// dst[i] = bf16(scale * src[i])
-__global__ void scale_to_bf16_kernel(const float *__restrict__ src, int64_t n, float scale,
-                                     uint16_t *__restrict__ dst) {
-    griddep_wait();
-    griddep_launch_dependents();
-    for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
-         e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        __nv_bfloat16 b = __float2bfloat16_rn(scale * src[e]);
-        dst[e] = *reinterpret_cast<uint16_t *>(&b);
     }
 }
 

@@ -58,6 +58,8 @@ def lib() -> ctypes.CDLL:
         L.oracle_qlora_bwd.argtypes = [vp, vp, vp, vp, i32, i64, i64, vp, i64, vp, vp, i32,
                                        f64, vp, vp, i64, vp, vp, vp]
         L.oracle_qlora_bwd.restype = ctypes.c_int
+        L.oracle_qlora_merge.argtypes = [vp, vp, vp, vp, i32, i64, i64, vp, vp, i32, f64, vp]
+        L.oracle_qlora_merge.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -243,3 +245,21 @@ def qlora_bwd(qw: Quantized, N: int, K: int, x: np.ndarray, A: np.ndarray, B: np
     if rc != 0:
         raise OracleError(f"oracle_qlora_bwd failed ({rc})")
     return dX, dA, dB
+
+
+def qlora_merge(qw: Quantized, N: int, K: int, A: np.ndarray, B: np.ndarray, r: int,
+                alpha: float) -> np.ndarray:
+    """W~ + (alpha/r) B A in fp64, [N, K]: the adapters folded into the dequantised
+    (fp32) base weight, as for inference without adapters.
+
+    A: uint16 [r, K] bf16 bits; B: uint16 [N, r]."""
+    _check_layer(qw, N, K)
+    A = np.ascontiguousarray(A, dtype=np.uint16)
+    B = np.ascontiguousarray(B, dtype=np.uint16)
+    assert A.shape == (r, K) and B.shape == (N, r)
+    out = np.zeros((N, K), dtype=np.float64)
+    rc = lib().oracle_qlora_merge(_ptr(qw.codes), _ptr(qw.absmax), _ptr(qw.q8), _ptr(qw.cg),
+                                  int(qw.dq), N, K, _ptr(A), _ptr(B), r, float(alpha), _ptr(out))
+    if rc != 0:
+        raise OracleError(f"oracle_qlora_merge failed ({rc})")
+    return out

@@ -445,3 +445,38 @@ int oracle_qlora_bwd(const uint8_t *codes, const float *absmax, const uint8_t *q
     free(Ad); free(Bd); free(v); free(u);
     return err ? ORACLE_ERR_ARG : ORACLE_OK;
 }
+
+/* Adapter merge ([P3] "Merging and deploying": the adapters are folded into
+ * the base weight for inference; [P4] FAQ on merging: W_new = W + (alpha/r) B A):
+ *   out[n][k] = W~[n][k] + (alpha/r) sum_j B[n][j] A[j][k]
+ * where W~ is the dequantised base weight in fp32 (fl32(scale * NF4[q]), the
+ * value before any rounding to a 16-bit compute type), and B, A are the bf16
+ * adapters. Computed in fp64; out is N x K. Returns 0 or ORACLE_ERR_ARG. */
+int oracle_qlora_merge(const uint8_t *codes, const float *absmax, const uint8_t *q8,
+                       const float *cg, int32_t dq, int64_t N, int64_t K,
+                       const uint16_t *A, const uint16_t *B, int32_t r, double alpha,
+                       double *out)
+{
+    if (N <= 0 || K <= 0 || K % 64 != 0 || r <= 0)
+        return ORACLE_ERR_ARG;
+    float *W = (float *)malloc(sizeof(float) * (size_t)(N * K));
+    double *Ad = widen_bf16(A, (int64_t)r * K);
+    double *Bd = widen_bf16(B, N * r);
+    if (!W || !Ad || !Bd) {
+        free(W); free(Ad); free(Bd);
+        return ORACLE_ERR_ARG;
+    }
+    oracle_nf4_dequantize(codes, absmax, q8, cg, N * K, 64, dq, 256, W);
+    const double s = alpha / (double)r;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            double ba = 0.0;
+            for (int32_t j = 0; j < r; ++j)
+                ba += Bd[n * r + j] * Ad[(int64_t)j * K + k];
+            out[n * K + k] = (double)W[n * K + k] + s * ba;
+        }
+    }
+    free(W); free(Ad); free(Bd);
+    return ORACLE_OK;
+}

@@ -146,3 +146,43 @@ def test_adapter_gradient_sizes_match_parameter_count():
     assert dA.size + dB.size == int(g["per_matrix"])
     assert 4 * (dA.size + dB.size) == int(g["per_layer"])
     assert round(int(g["layers"]) * 4 * (dA.size + dB.size) / 1e6, 1) == float(g["total_millions"])
+
+
+# ------------------------------------------------------------------ merge --
+def test_merge_with_b_zero_is_the_dequantised_weight():
+    rng = np.random.default_rng(31)
+    N, K, r = 24, 192, 8
+    qw, _, A, B, _ = random_layer(rng, N, K, 1, r, dq=True)
+    out = oracle.qlora_merge(qw, N, K, A, np.zeros_like(B), r, 16.0)
+    assert np.array_equal(out, oracle.dequantize(qw).astype(np.float64).reshape(N, K))
+
+
+def test_merge_of_zero_weight_is_the_scaled_adapter_product():
+    """W0 = 0 quantises to the zero level everywhere, so the merge is (alpha/r) B A alone,
+    here checked against a library matrix product of the widened adapters."""
+    rng = np.random.default_rng(32)
+    N, K, r, alpha = 40, 128, 16, 32.0
+    qw = oracle.quantize(np.zeros(N * K, dtype=np.float32), dq=False)
+    A = oracle.f32_to_bf16(rng.uniform(-0.1, 0.1, size=(r, K)).astype(np.float32))
+    B = oracle.f32_to_bf16(rng.normal(0, 0.01, size=(N, r)).astype(np.float32))
+    out = oracle.qlora_merge(qw, N, K, A, B, r, alpha)
+    ref = (alpha / r) * (f64(B) @ f64(A))
+    assert np.allclose(out, ref, rtol=1e-13, atol=1e-16)
+    # orientation: a transposed or unscaled product is far off
+    assert not np.allclose(out, f64(B) @ f64(A), rtol=1e-3)
+
+
+@pytest.mark.parametrize("dq", [False, True])
+def test_merged_weight_reproduces_the_layer_forward(dq):
+    """x W_merged^T equals the layer's forward up to the bf16 rounding of the base
+    operand (the forward multiplies RNE_bf16(w~); the merge keeps w~ in fp32)."""
+    rng = np.random.default_rng(33 + dq)
+    N, K, M, r, alpha = 48, 256, 6, 16, 32.0
+    qw, x, A, B, _ = random_layer(rng, N, K, M, r, dq)
+    merged = oracle.qlora_merge(qw, N, K, A, B, r, alpha)
+    h, _ = oracle.qlora_fwd_rows(qw, N, K, x, A, B, r, alpha)
+    w32 = oracle.dequantize(qw).astype(np.float64).reshape(N, K)
+    bound = np.abs(f64(x)) @ np.abs(operand(qw, N, K) - w32).T + 1e-12
+    assert np.all(np.abs(f64(x) @ merged.T - h) <= bound)
+    # without the adapter term the gap is far larger than the bound
+    assert np.max(np.abs(f64(x) @ w32.T - h) - bound) > 0
