@@ -197,7 +197,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--skip-extras", action="store_true",
                     help="only the main fwd+bwd line (no decode/quantize/oracle/e2e legs)")
-    ap.add_argument("--leg", default="all", choices=["all", "decode", "quantize", "stack", "mlp70b"],
+    ap.add_argument("--leg", default="all", choices=["all", "decode", "quantize", "stack", "mlp70b",
+                                                     "merge"],
                     help="run one secondary leg alone and print its JSON (for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -218,7 +219,7 @@ def main():
     if args.leg != "all":
         if rank == 0:
             leg = {"decode": decode_leg, "quantize": quantize_leg, "stack": stack_leg,
-                   "mlp70b": mlp70b_leg}[args.leg]
+                   "mlp70b": mlp70b_leg, "merge": merge_leg}[args.leg]
             print(json.dumps({"leg": args.leg, **leg(q, dev, load_peaks())}), flush=True)
         return
     if world > 1:
@@ -327,6 +328,7 @@ def main():
         line["quantize"] = quantize_leg(q, dev, peaks)
         line["mlp70b"] = mlp70b_leg(q, dev, peaks)
         line["stack"] = stack_leg(q, dev, peaks)
+        line["merge"] = merge_leg(q, dev, peaks)
         line["cpu_baseline"] = cpu_baseline_leg(w, inp)
     elif not args.skip_extras:
         e2e_leg(q, dp, qw, inp, w, args, dev, world)  # same collectives on every rank
@@ -470,6 +472,42 @@ def quantize_leg(q, dev, peaks):
     return {"workload": f"{QUANT}: W0 {w.N}x{w.K} fp32 -> NF4 + double quant",
             "bytes_moved": moved, "kernel_us": us, "gbs": gbs, "frac": gbs / peaks["hbm_gbs"],
             "peak_gbs": peaks["hbm_gbs"]}
+
+
+def merge_leg(q, dev, peaks):
+    """Adapter merge W~ + (alpha/r) B A of the 5120x5120 attention projection (r = 16), to a
+    bf16 and to an fp32 weight. GB/s counts the bytes a merge must move: codes, 8-bit scale
+    codes and group constants in, the merged weight out (the adapters are 0.3 MB). Four
+    weight copies and outputs are rotated so that no launch finds its operands in L2."""
+    w = workloads.WORKLOADS[MAIN]
+    inp = workloads.make_inputs(w, M=0, with_dy=False)
+    W0 = inp["W0"].to(dev)
+    copies = [q.nf4_quantize(W0, double_quant=True) for _ in range(4)]
+    del W0
+    A, B = inp["A"].to(dev), inp["B"].to(dev)
+    nb = w.N * w.K // 64
+    out = {"workload": f"{MAIN}: W0 {w.N}x{w.K} NF4 double quant, r={w.r}, alpha={w.alpha:g}",
+           "peak_gbs": peaks["hbm_gbs"]}
+    for name, bf16 in (("bf16", True), ("fp32", False)):
+        outs = [torch.empty(w.N, w.K, dtype=torch.bfloat16 if bf16 else torch.float32, device=dev)
+                for _ in range(4)]
+        moved = w.N * w.K // 2 + nb + ((nb + 255) // 256) * 4 + w.N * w.K * (2 if bf16 else 4)
+        for i in range(4):
+            q.qlora_merge(copies[i], A, B, w.alpha, bf16=bf16, out=outs[i])
+        torch.cuda.synchronize()
+        q.profiling(True)
+        for i in range(20):
+            q.qlora_merge(copies[i % 4], A, B, w.alpha, bf16=bf16, out=outs[i % 4])
+        torch.cuda.synchronize()
+        q.profiling(False)
+        n, t = q.profile_read()["qlora_merge"]
+        us = 1e3 * t / n
+        gbs = moved / (us * 1e-6) / 1e9
+        out[name] = {"bytes_moved": moved, "kernel_us": us, "gbs": gbs, "frac": gbs / peaks["hbm_gbs"]}
+        del outs
+    del copies
+    torch.cuda.empty_cache()
+    return out
 
 
 def _time_steps(step, warmup, steps):

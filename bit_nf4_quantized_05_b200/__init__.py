@@ -76,6 +76,7 @@ def _load() -> ctypes.CDLL:
         "qlora_bwd_workspace_bytes": ([i64, i64, i64, i32], sz),
         "qlora_linear_bwd": ([W, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, vp, vp, sz, vp],
                              ctypes.c_int),
+        "qlora_merge": ([W, vp, vp, i32, f32, vp, i32, vp], ctypes.c_int),
         "nf4_device_status": ([vp], ctypes.c_int),
         "nf4_status_string": ([ctypes.c_int], ctypes.c_char_p),
         "nf4_profiling": ([i32], ctypes.c_int),
@@ -246,6 +247,21 @@ def qlora_linear_bwd(qw: QuantizedWeight, x: torch.Tensor, A: torch.Tensor, B: t
                                 ws.numel(), _stream(x.device)),
            "qlora_linear_bwd")
     return dX, dA, dB
+
+
+def qlora_merge(qw: QuantizedWeight, A: torch.Tensor, B: torch.Tensor, alpha: float,
+                bf16: bool = True, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """W~ + (alpha/r) B A as a [n, k] tensor (bf16, or fp32 for re-quantisation):
+    the adapters folded into the dequantised frozen weight."""
+    _need_cuda(A, B)
+    r = A.shape[0]
+    if out is None:
+        out = torch.empty(qw.n, qw.k, dtype=torch.bfloat16 if bf16 else torch.float32,
+                          device=qw.device)
+    s = qw.struct()
+    _check(lib.qlora_merge(ctypes.byref(s), _ptr(A), _ptr(B), r, float(alpha), _ptr(out),
+                           int(bf16), _stream(qw.device)), "qlora_merge")
+    return out
 
 
 def device_status(device=None) -> int:

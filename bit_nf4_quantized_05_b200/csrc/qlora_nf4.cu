@@ -18,6 +18,7 @@
 #include "gemm_pair_tc.cuh"
 #include "skinny_tc.cuh"
 #include "decode_stream.cuh"
+#include "merge.cuh"
 
 using namespace nf4;
 
@@ -34,11 +35,11 @@ constexpr int kMaxDevices = 64;
 // Optional per-kernel event timing (nf4_profiling / nf4_profile_read)
 // ---------------------------------------------------------------------------
 enum KernelKind {
-    KK_QUANTIZE, KK_DEQUANTIZE, KK_LORA_U, KK_LORA_V, KK_LORA_DBDA, KK_ZERO, KK_GEMM_FWD, KK_GEMM_DGRAD, KK_DECODE, KK_DECODE_U, KK_COUNT
+    KK_QUANTIZE, KK_DEQUANTIZE, KK_LORA_U, KK_LORA_V, KK_LORA_DBDA, KK_ZERO, KK_GEMM_FWD, KK_GEMM_DGRAD, KK_DECODE, KK_DECODE_U, KK_MERGE, KK_COUNT
 };
 const char *const kKindNames[KK_COUNT] = {
     "nf4_quantize", "nf4_dequantize", "lora_u", "lora_v", "lora_dB_dA", "zero_fill", "qlora_gemm_fwd", "qlora_gemm_dgrad", "qlora_decode",
-    "decode_lora_u"};
+    "decode_lora_u", "qlora_merge"};
 
 struct ProfRecord {
     int kind;
@@ -827,6 +828,53 @@ nf4_status nf4_dequantize(const nf4_weight *w, void *out, int32_t out_bf16, void
     nf4_dequantize_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
         w->codes, w->absmax, w->absmax_q8, w->absmax_c, w->double_quant, nb, out_bf16, out);
     t.stop();
+    NF4_TRY_CUDA(cudaGetLastError());
+    return NF4_OK;
+}
+
+nf4_status qlora_merge(const nf4_weight *w, const uint16_t *A, const uint16_t *B, int32_t r,
+                       float alpha, void *out, int32_t out_is_bf16, void *stream) {
+    nf4_status st = check_weight(w, true);
+    if (st != NF4_OK) return st;
+    if (r < 1 || r > kMgMaxRank || (r % 8) != 0) return NF4_ERR_UNSUPPORTED_SHAPE;
+    if (!std::isfinite(alpha)) return NF4_ERR_INVALID_ARG;
+    if (!A || !B || !out || (out_is_bf16 != 0 && out_is_bf16 != 1)) return NF4_ERR_INVALID_ARG;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(out)) return NF4_ERR_ALIGNMENT;
+    if ((w->n + kMgRows - 1) / kMgRows > 65535) return NF4_ERR_UNSUPPORTED_SHAPE;
+    MergeArgs a{};
+    a.N = w->n;
+    a.K = w->k;
+    a.r = r;
+    a.rp = (r + 15) / 16 * 16;
+    a.codes = w->codes;
+    a.absmax = w->absmax;
+    a.q8 = w->absmax_q8;
+    a.cg = w->absmax_c;
+    a.dq = w->double_quant;
+    a.A = A;
+    a.B = B;
+    a.scale = alpha / static_cast<float>(r);
+    a.out = out;
+    const dim3 grid(static_cast<unsigned>((w->k + kMgCols - 1) / kMgCols),
+                    static_cast<unsigned>((w->n + kMgRows - 1) / kMgRows));
+    const int smem = merge_smem_bytes(a.rp, out_is_bf16 != 0);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    void (*kern)(const MergeArgs) = nullptr;
+#define NF4_MERGE_CASE(RQ_)                                                                    \
+    case RQ_:                                                                                  \
+        kern = out_is_bf16 ? qlora_merge_kernel<true, RQ_> : qlora_merge_kernel<false, RQ_>; \
+        break;
+    switch (a.rp / 16) {
+        NF4_MERGE_CASE(1) NF4_MERGE_CASE(2) NF4_MERGE_CASE(3) NF4_MERGE_CASE(4)
+        NF4_MERGE_CASE(5) NF4_MERGE_CASE(6) NF4_MERGE_CASE(7) NF4_MERGE_CASE(8)
+        default: return NF4_ERR_UNSUPPORTED_SHAPE;
+    }
+#undef NF4_MERGE_CASE
+    NF4_TRY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    LaunchTimer t(KK_MERGE, s);
+    const cudaError_t e = launch_ex(kern, grid, dim3(kMgThreads), static_cast<size_t>(smem), s, 0u, a);
+    t.stop();
+    if (e != cudaSuccess) return NF4_ERR_CUDA;
     NF4_TRY_CUDA(cudaGetLastError());
     return NF4_OK;
 }

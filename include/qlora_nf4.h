@@ -172,6 +172,20 @@ QLORA_API nf4_status qlora_linear_bwd(const nf4_weight *w, const uint16_t *x, in
                             const uint16_t *dY, const float *u, uint16_t *dX, uint16_t *dA,
                             uint16_t *dB, void *workspace, size_t ws_bytes, void *stream);
 
+/* Adapter merge for inference without adapters ("QLoRA explained", section
+ * "Merging and deploying"; "How Fine-Tuning LLMs with LoRA and QLoRA Works",
+ * FAQ on merging: W_new = W + (alpha/r) B A):
+ *     out[n][k] = w~[n][k] + s * sum_j B[n][j] A[j][k],   s = fl32(alpha / r)
+ * with w~ = fl32(scale * NF4[q]) the dequantised weight in fp32. The rank-r
+ * sum is accumulated in fp32, added to w~ with one fused multiply-add and
+ * rounded once to the output type: out is [n, k] row-major, bf16 when
+ * out_is_bf16 == 1 (the 16-bit merged weight), fp32 when 0 (for example to
+ * re-quantise it with nf4_quantize). A is [r, k], B is [n, r] (bf16), with
+ * the same requirements on r and alpha as the layer. */
+QLORA_API nf4_status qlora_merge(const nf4_weight *w, const uint16_t *A, const uint16_t *B,
+                                 int32_t r, float alpha, void *out, int32_t out_is_bf16,
+                                 void *stream);
+
 /* Synchronises `stream`, then returns and clears the status word that the
  * kernels of the current device set (NF4_OK if nothing was recorded). */
 QLORA_API nf4_status nf4_device_status(void *stream);

@@ -184,3 +184,62 @@ def test_llama2_70b_mlp_full_size(q):
     res = run_layer(q, inp["W0"], inp["A"], inp["B"], inp["x"], inp["dY"], w.alpha, w.double_quant)
     check_against_oracle(q, res, inp["A"], inp["B"], inp["x"], inp["dY"], w.alpha,
                          rows=sampled_rows(w.M, 12, 2), tag=w.name)
+
+
+# ------------------------------------------------------------------ merge --
+def merge_bound(qw, A, B, r, alpha, oracle_out, out_bf16):
+    """Element-wise bar for the merge: the fp32 rank-r sum (r + 2 roundings of
+    relative size 2^-24 on the sum of |terms|) plus, for bf16 output, the final
+    rounding (2^-8 of the value, one bf16 unit in the last place)."""
+    K = qw.k
+    absBA = np.abs(oracle.bf16_to_f64(B)) @ np.abs(oracle.bf16_to_f64(A))
+    w32 = np.abs(oracle.dequantize(oracle_weight(qw)).astype(np.float64).reshape(qw.n, K))
+    acc = (r + 2) * 2.0 ** -24 * (w32 + (alpha / r) * absBA)
+    return acc + (2.0 ** -8 * np.abs(oracle_out) if out_bf16 else 0.0)
+
+
+MERGE_SHAPES = [
+    # (N, K, r, alpha, dq)   ragged tiles in both dimensions; every supported rank class
+    (200, 320, 16, 32.0, True),
+    (64, 128, 8, 16.0, False),
+    (136, 576, 64, 16.0, True),
+    (72, 192, 128, 32.0, False),
+]
+
+
+@pytest.mark.parametrize("N,K,r,alpha,dq", MERGE_SHAPES)
+@pytest.mark.parametrize("out_bf16", [True, False])
+def test_merge_matches_oracle(q, N, K, r, alpha, dq, out_bf16):
+    w = workloads.LayerWorkload("t", N, K, 1, r, alpha, 0.02, dq, 777 + N + r)
+    inp = workloads.make_inputs(w)
+    qw = q.nf4_quantize(inp["W0"].to("cuda"), double_quant=dq)
+    out = q.qlora_merge(qw, inp["A"].cuda(), inp["B"].cuda(), alpha, bf16=out_bf16)
+    torch.cuda.synchronize()
+    assert q.device_status() == q.NF4_OK
+    ref = oracle.qlora_merge(oracle_weight(qw), N, K, bits(inp["A"]), bits(inp["B"]), r, alpha)
+    got = to_f64(out)
+    bound = merge_bound(qw, bits(inp["A"]), bits(inp["B"]), r, alpha, ref, out_bf16)
+    assert np.all(np.abs(got - ref) <= bound), float(np.max(np.abs(got - ref) - bound))
+    assert np.max(np.abs(got - ref)) <= TOL * np.sqrt(np.mean(ref ** 2))
+
+
+def test_merge_b_zero_is_dequantize(q):
+    w = workloads.LayerWorkload("t", 128, 256, 1, 16, 32.0, 0.02, True, 4321)
+    inp = workloads.make_inputs(w)
+    qw = q.nf4_quantize(inp["W0"].to("cuda"), double_quant=True)
+    B0 = torch.zeros_like(inp["B"]).cuda()
+    for bf16 in (True, False):
+        out = q.qlora_merge(qw, inp["A"].cuda(), B0, 32.0, bf16=bf16)
+        assert torch.equal(out, q.nf4_dequantize(qw, bf16=bf16))
+
+
+def test_merge_full_size_attention_projection(q):
+    """The LLaMA-13B-like attention projection: every element against the oracle."""
+    w = workloads.WORKLOADS["llama13b_attn_5120"]
+    inp = workloads.make_inputs(w, M=0, with_dy=False)
+    qw = q.nf4_quantize(inp["W0"].to("cuda"), double_quant=True)
+    out = q.qlora_merge(qw, inp["A"].cuda(), inp["B"].cuda(), w.alpha, bf16=True)
+    torch.cuda.synchronize()
+    ref = oracle.qlora_merge(oracle_weight(qw), w.N, w.K, bits(inp["A"]), bits(inp["B"]), w.r, w.alpha)
+    bound = merge_bound(qw, bits(inp["A"]), bits(inp["B"]), w.r, w.alpha, ref, True)
+    assert np.all(np.abs(to_f64(out) - ref) <= bound)
