@@ -198,7 +198,7 @@ def main():
     ap.add_argument("--skip-extras", action="store_true",
                     help="only the main fwd+bwd line (no decode/quantize/oracle/e2e legs)")
     ap.add_argument("--leg", default="all", choices=["all", "decode", "quantize", "stack", "mlp70b",
-                                                     "merge"],
+                                                     "merge", "multi"],
                     help="run one secondary leg alone and print its JSON (for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -219,7 +219,7 @@ def main():
     if args.leg != "all":
         if rank == 0:
             leg = {"decode": decode_leg, "quantize": quantize_leg, "stack": stack_leg,
-                   "mlp70b": mlp70b_leg, "merge": merge_leg}[args.leg]
+                   "mlp70b": mlp70b_leg, "merge": merge_leg, "multi": multi_leg}[args.leg]
             print(json.dumps({"leg": args.leg, **leg(q, dev, load_peaks())}), flush=True)
         return
     if world > 1:
@@ -329,6 +329,7 @@ def main():
         line["mlp70b"] = mlp70b_leg(q, dev, peaks)
         line["stack"] = stack_leg(q, dev, peaks)
         line["merge"] = merge_leg(q, dev, peaks)
+        line["multi_adapter"] = multi_leg(q, dev, peaks)
         line["cpu_baseline"] = cpu_baseline_leg(w, inp)
     elif not args.skip_extras:
         e2e_leg(q, dp, qw, inp, w, args, dev, world)  # same collectives on every rank
@@ -472,6 +473,49 @@ def quantize_leg(q, dev, peaks):
     return {"workload": f"{QUANT}: W0 {w.N}x{w.K} fp32 -> NF4 + double quant",
             "bytes_moved": moved, "kernel_us": us, "gbs": gbs, "frac": gbs / peaks["hbm_gbs"],
             "peak_gbs": peaks["hbm_gbs"]}
+
+
+def multi_leg(q, dev, peaks):
+    """Decode-shaped forward with per-token adapters over one NF4 base: the 13824x5120 weight
+    (double quant), 16 tokens spread over 8 adapters of rank 8 (alpha 16), as one batch of a
+    multi-adapter server. Device time per call from a CUDA-graph replay of 64 calls over 8
+    rotated weight copies; GB/s on the 4-bit code bytes, as the decode leg."""
+    w = workloads.WORKLOADS[DECODE]
+    n_ad, r, M = 8, 8, 16
+    W0 = workloads.make_weight(w).to(dev)
+    copies = [q.nf4_quantize(W0, double_quant=True) for _ in range(8)]
+    del W0
+    wl = w.with_(r=n_ad * r)
+    inp = workloads.make_inputs(wl, M=M, with_dy=False)
+    x, A_all, B_all = (inp[k].to(dev) for k in ("x", "A", "B"))
+    idx = (torch.arange(M, dtype=torch.int32) % n_ad).to(dev)
+    alphas = [16.0] * n_ad
+    h = torch.empty(M, w.N, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(q.fwd_workspace_bytes(M, w.N, w.K, n_ad * r), dtype=torch.uint8, device=dev)
+    for i in range(8):
+        q.qlora_multi_lora_fwd(copies[i], x, A_all, B_all, r, alphas, idx, h=h, workspace=ws)
+    torch.cuda.synchronize()
+    gs = torch.cuda.Stream()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=gs):
+        for i in range(64):
+            q.qlora_multi_lora_fwd(copies[i % 8], x, A_all, B_all, r, alphas, idx, h=h, workspace=ws)
+    graph.replay()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(4):
+        graph.replay()
+    e.record()
+    torch.cuda.synchronize()
+    us = 1e3 * s.elapsed_time(e) / (4 * 64)
+    del graph, copies
+    torch.cuda.empty_cache()
+    code_bytes = w.N * w.K // 2
+    gbs = code_bytes / (us * 1e-6) / 1e9
+    return {"workload": f"{DECODE}: W0 {w.N}x{w.K} NF4 double quant; {M} tokens over {n_ad} "
+                        f"adapters of r={r} (alpha 16), forward", "graph_call_us": us,
+            "gbs_graph_call": gbs, "frac_graph_call": gbs / peaks["hbm_gbs"], "code_bytes": code_bytes}
 
 
 def merge_leg(q, dev, peaks):

@@ -77,6 +77,8 @@ def _load() -> ctypes.CDLL:
         "qlora_linear_bwd": ([W, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, vp, vp, sz, vp],
                              ctypes.c_int),
         "qlora_merge": ([W, vp, vp, i32, f32, vp, i32, vp], ctypes.c_int),
+        "qlora_multi_lora_fwd": ([W, vp, i64, vp, vp, i32, i32, ctypes.POINTER(f32), vp, vp, vp, sz,
+                                  vp], ctypes.c_int),
         "nf4_device_status": ([vp], ctypes.c_int),
         "nf4_status_string": ([ctypes.c_int], ctypes.c_char_p),
         "nf4_profiling": ([i32], ctypes.c_int),
@@ -247,6 +249,30 @@ def qlora_linear_bwd(qw: QuantizedWeight, x: torch.Tensor, A: torch.Tensor, B: t
                                 ws.numel(), _stream(x.device)),
            "qlora_linear_bwd")
     return dX, dA, dB
+
+
+def qlora_multi_lora_fwd(qw: QuantizedWeight, x: torch.Tensor, A_all: torch.Tensor,
+                         B_all: torch.Tensor, r: int, alphas, adapter_of_token: torch.Tensor,
+                         h: Optional[torch.Tensor] = None,
+                         workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """h[m] = x[m] W~^T + (alphas[a]/r)(x[m] A_a^T) B_a^T with a = adapter_of_token[m]
+    (int32 CUDA tensor; values outside [0, len(alphas)) mean no adapter). A_all stacks
+    the adapters' A as [n_adapters * r, k], B_all their B as [n, n_adapters * r]."""
+    _need_cuda(x, A_all, B_all, adapter_of_token)
+    if adapter_of_token.dtype != torch.int32:
+        raise ValueError("adapter_of_token must be int32")
+    M = x.shape[0]
+    n_ad = len(alphas)
+    if h is None:
+        h = torch.empty(M, qw.n, dtype=torch.bfloat16, device=x.device)
+    nbytes = fwd_workspace_bytes(M, qw.n, qw.k, n_ad * r)
+    ws = workspace if workspace is not None else _workspace(nbytes, x.device)
+    al = (ctypes.c_float * n_ad)(*[float(a) for a in alphas])
+    s = qw.struct()
+    _check(lib.qlora_multi_lora_fwd(ctypes.byref(s), _ptr(x), M, _ptr(A_all), _ptr(B_all), int(r),
+                                    n_ad, al, _ptr(adapter_of_token), _ptr(h), _ptr(ws), ws.numel(),
+                                    _stream(x.device)), "qlora_multi_lora_fwd")
+    return h
 
 
 def qlora_merge(qw: QuantizedWeight, A: torch.Tensor, B: torch.Tensor, alpha: float,

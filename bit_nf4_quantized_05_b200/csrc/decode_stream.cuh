@@ -72,6 +72,18 @@ struct DecodeArgs {
     uint16_t *h;           // [M, N]
 };
 
+// Per-token adapter selection over stacked adapters (multi-adapter forward):
+// token m keeps the group_width rank columns of adapter row_group[m], scaled
+// by gscale of that adapter (no adapter term when row_group[m] is outside
+// [0, ngroups)). The single-adapter instantiations take the empty type.
+struct DsNoGroups {};
+struct DsGroups {
+    const int32_t *row_group;
+    int group_width;
+    int ngroups;
+    float gscale[16];
+};
+
 // Table lookup by shared address. The table is written once before a
 // barrier and never again, and every lookup address is derived from code
 // words read after that barrier, so the load needs no ordering of its own.
@@ -144,10 +156,12 @@ struct DsScales {
 // blocks. Its chunks are numbered c = 0, 1, ... over all of the CTA's tiles;
 // chunk c goes to ring slot c % 2, and the other slot takes chunk c + 1 as soon as
 // every lane has read chunk c.
-template <int TG, int CB>
+// GT: DsNoGroups, or DsGroups for per-token adapter selection.
+template <int TG, int CB, class GT>
 __global__ void __launch_bounds__(kDsThreads, 1)
 qlora_decode_stream_kernel(const __grid_constant__ CUtensorMap tm_codes,   // [N, K/2] u8, box {32 CB, 32}
-                           const DecodeArgs a) {
+                           const DecodeArgs a, const GT grp) {
+    constexpr bool GROUPS = sizeof(GT) > 1;
     extern __shared__ __align__(1024) uint8_t dsm[];
     constexpr uint32_t kSlot = 1024u * CB;           // bytes of one chunk (32 rows x 32 CB)
     constexpr uint32_t kRowStride = 32u * CB;        // bytes per row in a slot
@@ -446,7 +460,13 @@ qlora_decode_stream_kernel(const __grid_constant__ CUtensorMap tm_codes,   // [N
 #pragma unroll
                 for (int j = 0; j < kDsUCtas; ++j) u += a.upart[j * a.M * a.r + cc];
                 if (a.u_out && blockIdx.x == 0) a.u_out[cc] = u;
-                __nv_bfloat16 ub = __float2bfloat16_rn(__fmul_rn(a.scale, u));
+                float sc = a.scale;
+                if constexpr (GROUPS) {
+                    const int gp = grp.row_group[cc / a.r];
+                    const bool keep = gp >= 0 && gp < grp.ngroups && (cc % a.r) / grp.group_width == gp;
+                    sc = keep ? grp.gscale[gp] : 0.0f;
+                }
+                __nv_bfloat16 ub = __float2bfloat16_rn(__fmul_rn(sc, u));
                 u_tile[cc] = *reinterpret_cast<uint16_t *>(&ub);
             }
         }

@@ -25,6 +25,7 @@ using namespace nf4;
 namespace {
 
 constexpr int kMaxDevices = 64;
+constexpr int kMaxAdapters = 16;   // stacked adapters of one multi-adapter forward
 
 #define NF4_TRY_CUDA(expr)                          \
     do {                                            \
@@ -317,9 +318,18 @@ bool skinny_job(const SkinnySpec &sp, int RN, int splits, CUtensorMap *ta, CUten
 
 // One launch of one or two products (n = 1, 2) with the same operand layouts
 // and rank, plus optional flag zeroing and an element-wise side task.
+// Per-row adapter selection for the bf16 output of a one-product launch.
+struct RowGroups {
+    const int32_t *row_group = nullptr;
+    int group_width = 0;
+    int ngroups = 0;
+    const float *gscale = nullptr;   // host array [ngroups]
+};
+
 nf4_status skinny_launch(int kind, const SkinnySpec *sp, int n, cudaStream_t stream,
                          int *zero_ints = nullptr, int zero_count = 0, const float *conv_src = nullptr,
-                         uint16_t *conv_dst = nullptr, int64_t conv_n = 0, float conv_scale = 0.f) {
+                         uint16_t *conv_dst = nullptr, int64_t conv_n = 0, float conv_scale = 0.f,
+                         const RowGroups *groups = nullptr) {
     const int sms = num_sms(current_device());
     const int RN = sp[0].r <= 64 ? 64 : 128;
     int p_tiles = 0, steps = 1;
@@ -351,6 +361,12 @@ nf4_status skinny_launch(int kind, const SkinnySpec *sp, int n, cudaStream_t str
     args.conv_dst = conv_dst;
     args.conv_n = conv_n;
     args.conv_scale = conv_scale;
+    if (groups && groups->row_group) {
+        args.row_group = groups->row_group;
+        args.group_width = groups->group_width;
+        args.ngroups = groups->ngroups;
+        for (int i = 0; i < groups->ngroups && i < 16; ++i) args.gscale[i] = groups->gscale[i];
+    }
     const dim3 grid(static_cast<unsigned>(splits), static_cast<unsigned>(p_tiles));
     const Major am = sp[0].am, bm = sp[0].bm;
     cudaError_t e = cudaErrorInvalidValue;
@@ -532,33 +548,35 @@ nf4_status launch_gemm_pair(const nf4_weight *w, const uint16_t *act, int64_t M,
     return NF4_OK;
 }
 
-// One instantiation of the decode kernel per (token groups, chunk blocks).
-template <int TG, int CB>
+// One instantiation of the decode kernel per (token groups, chunk blocks,
+// per-token adapter selection).
+template <int TG, int CB, class GT>
 cudaError_t launch_decode_stream_t(unsigned grid, cudaStream_t stream, const CUtensorMap &tm,
-                                   const DecodeArgs &a) {
-    auto k = qlora_decode_stream_kernel<TG, CB>;
+                                   const DecodeArgs &a, const GT &grp) {
+    auto k = qlora_decode_stream_kernel<TG, CB, GT>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kDsDynBytes);
     if (e != cudaSuccess) return e;
-    return launch_ex(k, dim3(grid), dim3(kDsThreads), kDsDynBytes, stream, 0u, tm, a);
+    return launch_ex(k, dim3(grid), dim3(kDsThreads), kDsDynBytes, stream, 0u, tm, a, grp);
 }
 
-template <int TG>
+template <int TG, class GT>
 cudaError_t launch_decode_stream_cb(int cb, unsigned grid, cudaStream_t stream, const CUtensorMap &tm,
-                                    const DecodeArgs &a) {
+                                    const DecodeArgs &a, const GT &grp) {
     switch (cb) {
-        case 1: return launch_decode_stream_t<TG, 1>(grid, stream, tm, a);
-        case 2: return launch_decode_stream_t<TG, 2>(grid, stream, tm, a);
-        case 3: return launch_decode_stream_t<TG, 3>(grid, stream, tm, a);
-        case 4: return launch_decode_stream_t<TG, 4>(grid, stream, tm, a);
-        case 5: return launch_decode_stream_t<TG, 5>(grid, stream, tm, a);
+        case 1: return launch_decode_stream_t<TG, 1>(grid, stream, tm, a, grp);
+        case 2: return launch_decode_stream_t<TG, 2>(grid, stream, tm, a, grp);
+        case 3: return launch_decode_stream_t<TG, 3>(grid, stream, tm, a, grp);
+        case 4: return launch_decode_stream_t<TG, 4>(grid, stream, tm, a, grp);
+        case 5: return launch_decode_stream_t<TG, 5>(grid, stream, tm, a, grp);
         default: return cudaErrorInvalidValue;
     }
 }
 
+template <class GT>
 cudaError_t launch_decode_stream(int tg, int cb, unsigned grid, cudaStream_t stream, const CUtensorMap &tm,
-                                 const DecodeArgs &a) {
-    return tg == 1 ? launch_decode_stream_cb<1>(cb, grid, stream, tm, a)
-                   : launch_decode_stream_cb<2>(cb, grid, stream, tm, a);
+                                 const DecodeArgs &a, const GT &grp) {
+    return tg == 1 ? launch_decode_stream_cb<1>(cb, grid, stream, tm, a, grp)
+                   : launch_decode_stream_cb<2>(cb, grid, stream, tm, a, grp);
 }
 
 // Forward for M <= 16 tokens: partial sums of u = x A^T on a few SMs, then
@@ -575,7 +593,7 @@ bool decode_shape(const nf4_weight *w, int64_t M, int32_t r) {
 
 nf4_status launch_decode(const nf4_weight *w, const uint16_t *x, int64_t M, const uint16_t *A,
                          const uint16_t *B, int32_t r, float scale, uint16_t *h, float *u_out,
-                         float *upart, cudaStream_t stream) {
+                         float *upart, cudaStream_t stream, const RowGroups *groups = nullptr) {
     // each of the 16 warps takes rb blocks of every 32-row tile, fetched in
     // chunks of cb blocks (the largest divisor of rb that is at most 5)
     const int64_t kblocks = w->k / kBlock;
@@ -622,7 +640,17 @@ nf4_status launch_decode(const nf4_weight *w, const uint16_t *x, int64_t M, cons
         if (e != cudaSuccess) return NF4_ERR_CUDA;
     }
     LaunchTimer t(KK_DECODE, stream);
-    const cudaError_t e = launch_decode_stream(tg, cb, grid, stream, tm_codes, a);
+    cudaError_t e;
+    if (groups && groups->row_group) {
+        DsGroups gr{};
+        gr.row_group = groups->row_group;
+        gr.group_width = groups->group_width;
+        gr.ngroups = groups->ngroups;
+        for (int i = 0; i < groups->ngroups && i < 16; ++i) gr.gscale[i] = groups->gscale[i];
+        e = launch_decode_stream(tg, cb, grid, stream, tm_codes, a, gr);
+    } else {
+        e = launch_decode_stream(tg, cb, grid, stream, tm_codes, a, DsNoGroups{});
+    }
     t.stop();
     if (e != cudaSuccess) return NF4_ERR_CUDA;
     NF4_TRY_CUDA(cudaGetLastError());
@@ -910,6 +938,50 @@ nf4_status qlora_linear_fwd(const nf4_weight *w, const uint16_t *x, int64_t M, c
                         scale, 0, s, sk.flags, sk.pairs_max * kSkFlagsPerPair);
     if (st != NF4_OK) return st;
     return launch_gemm_auto<false>(w, x, M, w->k, w->n, u_s, r, B, h, s, &sk);
+}
+
+nf4_status qlora_multi_lora_fwd(const nf4_weight *w, const uint16_t *x, int64_t M,
+                                const uint16_t *A_all, const uint16_t *B_all, int32_t r,
+                                int32_t n_adapters, const float *alphas,
+                                const int32_t *adapter_of_token, uint16_t *h, void *workspace,
+                                size_t ws_bytes, void *stream) {
+    if (n_adapters < 1 || n_adapters > kMaxAdapters || !alphas) return NF4_ERR_INVALID_ARG;
+    const int32_t R = r * n_adapters;
+    if (r < 8 || (r % 8) != 0 || R > 128) return NF4_ERR_UNSUPPORTED_SHAPE;
+    float gscale[kMaxAdapters];
+    for (int i = 0; i < n_adapters; ++i) {
+        if (!std::isfinite(alphas[i])) return NF4_ERR_INVALID_ARG;
+        gscale[i] = alphas[i] / static_cast<float>(r);
+    }
+    nf4_status st = check_layer(w, x, M, A_all, B_all, R, 1.0f);
+    if (st != NF4_OK) return st;
+    if (M == 0) return NF4_OK;
+    if (!h || !adapter_of_token) return NF4_ERR_INVALID_ARG;
+    if (!aligned16(h) || !aligned16(adapter_of_token)) return NF4_ERR_ALIGNMENT;
+    const int sms = num_sms(current_device());
+    const FwdLayout L = fwd_layout(M, R, sms);
+    if (!workspace || ws_bytes < L.total) return NF4_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return NF4_ERR_ALIGNMENT;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint16_t *u_s = reinterpret_cast<uint16_t *>(ws + L.us);
+    const SkBuf sk{reinterpret_cast<float *>(ws + L.partial), reinterpret_cast<int *>(ws + L.flags),
+                   sk_pairs_max(sms)};
+    RowGroups groups;
+    groups.row_group = adapter_of_token;
+    groups.group_width = r;
+    groups.ngroups = n_adapters;
+    groups.gscale = gscale;
+    if (decode_shape(w, M, R))
+        return launch_decode(w, x, M, A_all, B_all, R, 1.0f, h, nullptr,
+                             reinterpret_cast<float *>(ws + L.upart), s, &groups);
+    // u = x A_all^T for every stacked adapter; each token keeps its own adapter's
+    // columns, scaled by that adapter's alpha / r; the launch also clears the GEMM's flags
+    const SkinnySpec su{x, M, w->k, Major::K, A_all, R, w->k, Major::K, R, nullptr, u_s, 1.0f, 0};
+    st = skinny_launch(KK_LORA_U, &su, 1, s, sk.flags, sk.pairs_max * kSkFlagsPerPair, nullptr, nullptr,
+                       0, 0.f, &groups);
+    if (st != NF4_OK) return st;
+    return launch_gemm_auto<false>(w, x, M, w->k, w->n, u_s, R, B_all, h, s, &sk);
 }
 
 nf4_status qlora_linear_fwd_noalloc(const nf4_weight *w, const uint16_t *x, int64_t M,

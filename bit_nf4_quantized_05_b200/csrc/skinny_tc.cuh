@@ -51,6 +51,14 @@ struct SkinnyArgs {
     uint16_t *conv_dst;
     int64_t conv_n;
     float conv_scale;
+    // optional per-row adapter selection (several stacked adapters, one per
+    // output row): row p keeps only the group_width columns of adapter
+    // row_group[p], scaled by gscale of that adapter; other columns, and rows
+    // whose adapter is outside [0, ngroups), get zero in out_bf16
+    const int32_t *row_group;
+    int group_width;
+    int ngroups;
+    float gscale[16];
 };
 
 template <int RN, bool A_MN, bool B_MN>
@@ -224,7 +232,13 @@ skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a0,
                 acc += ld_cluster_f32(mapa_shared(part_addr + off, static_cast<uint32_t>(s)));
             if (J.out_f32) J.out_f32[static_cast<int64_t>(p) * r + j] = acc;
             if (J.out_bf16) {
-                __nv_bfloat16 b = __float2bfloat16_rn(J.scale * acc);
+                float sc = J.scale;
+                if (args.row_group) {
+                    const int gp = args.row_group[p];
+                    const bool keep = gp >= 0 && gp < args.ngroups && j / args.group_width == gp;
+                    sc = keep ? args.gscale[gp] : 0.0f;
+                }
+                __nv_bfloat16 b = __float2bfloat16_rn(sc * acc);
                 const int64_t o = J.transposed ? static_cast<int64_t>(j) * J.P + p
                                                : static_cast<int64_t>(p) * r + j;
                 J.out_bf16[o] = *reinterpret_cast<uint16_t *>(&b);

@@ -155,6 +155,27 @@ QLORA_API nf4_status qlora_linear_fwd_noalloc(const nf4_weight *w, const uint16_
                                               float alpha, uint16_t *h, float *u_out,
                                               void *stream);
 
+/* Forward of one NF4 base with several adapters, one chosen per token, as a
+ * server keeps one quantised base resident and applies each request's own
+ * adapter ("Parameter-Efficient Fine-Tuning: From LoRA to QLoRA", "The PEFT
+ * Strategy (LoRA + QLoRA + Multi-Adapter Serving)"):
+ *     h[m] = x[m] W~^T + (alphas[a] / r) (x[m] A_a^T) B_a^T,   a = adapter_of_token[m]
+ * The n_adapters adapters of rank r are stacked: A_all is [n_adapters * r, k]
+ * (rows a*r .. a*r + r - 1 are A_a), B_all is [n, n_adapters * r] (columns
+ * a*r .. a*r + r - 1 are B_a), bf16. alphas is a HOST array of n_adapters
+ * floats; adapter_of_token is a DEVICE array of M int32 values, and a value
+ * outside [0, n_adapters) means no adapter term for that token.
+ * Requirements: 1 <= n_adapters <= 16, r % 8 == 0, n_adapters * r <= 128;
+ * the other requirements of qlora_linear_fwd. workspace: at least
+ * qlora_fwd_workspace_bytes(M, n, k, n_adapters * r) bytes, 256-byte aligned.
+ * Rounding as qlora_linear_fwd: each token's (alphas[a] / r)(x A_a^T) is
+ * rounded to bf16 before the up-projection. */
+QLORA_API nf4_status qlora_multi_lora_fwd(const nf4_weight *w, const uint16_t *x, int64_t M,
+                                          const uint16_t *A_all, const uint16_t *B_all, int32_t r,
+                                          int32_t n_adapters, const float *alphas,
+                                          const int32_t *adapter_of_token, uint16_t *h,
+                                          void *workspace, size_t ws_bytes, void *stream);
+
 /* Workspace needed by qlora_linear_bwd for M tokens at rank r. */
 QLORA_API size_t qlora_bwd_workspace_bytes(int64_t M, int64_t n, int64_t k, int32_t r);
 

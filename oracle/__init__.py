@@ -60,6 +60,9 @@ def lib() -> ctypes.CDLL:
         L.oracle_qlora_bwd.restype = ctypes.c_int
         L.oracle_qlora_merge.argtypes = [vp, vp, vp, vp, i32, i64, i64, vp, vp, i32, f64, vp]
         L.oracle_qlora_merge.restype = ctypes.c_int
+        L.oracle_qlora_multi_fwd_rows.argtypes = [vp, vp, vp, vp, i32, i64, i64, vp, i64, vp, vp,
+                                                  i32, i32, vp, vp, vp, i64, vp]
+        L.oracle_qlora_multi_fwd_rows.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -263,3 +266,32 @@ def qlora_merge(qw: Quantized, N: int, K: int, A: np.ndarray, B: np.ndarray, r: 
     if rc != 0:
         raise OracleError(f"oracle_qlora_merge failed ({rc})")
     return out
+
+
+def qlora_multi_fwd_rows(qw: Quantized, N: int, K: int, x: np.ndarray, A_all: np.ndarray,
+                         B_all: np.ndarray, r: int, alphas: Sequence[float], adapter: np.ndarray,
+                         rows: Optional[Sequence[int]] = None) -> np.ndarray:
+    """h rows (fp64) of one NF4 base with per-token adapters:
+    h[m] = x[m] W~^T + (alpha_a / r)(x[m] A_a^T) B_a^T for a = adapter[m] (none when < 0).
+
+    A_all: uint16 [n_ad * r, K] (stacked A_a); B_all: uint16 [N, n_ad * r] (stacked B_a);
+    adapter: int32 [M]."""
+    _check_layer(qw, N, K)
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    A_all = np.ascontiguousarray(A_all, dtype=np.uint16)
+    B_all = np.ascontiguousarray(B_all, dtype=np.uint16)
+    n_ad = len(alphas)
+    M = x.shape[0]
+    assert A_all.shape == (n_ad * r, K) and B_all.shape == (N, n_ad * r)
+    adapter = np.ascontiguousarray(adapter, dtype=np.int32)
+    assert adapter.shape == (M,)
+    al = np.ascontiguousarray(alphas, dtype=np.float64)
+    rows = np.arange(M, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    h = np.zeros((rows.size, N), dtype=np.float64)
+    rc = lib().oracle_qlora_multi_fwd_rows(_ptr(qw.codes), _ptr(qw.absmax), _ptr(qw.q8),
+                                           _ptr(qw.cg), int(qw.dq), N, K, _ptr(x), M, _ptr(A_all),
+                                           _ptr(B_all), r, n_ad, _ptr(al), _ptr(adapter),
+                                           _ptr(rows), rows.size, _ptr(h))
+    if rc != 0:
+        raise OracleError(f"oracle_qlora_multi_fwd_rows failed ({rc})")
+    return h

@@ -480,3 +480,71 @@ int oracle_qlora_merge(const uint8_t *codes, const float *absmax, const uint8_t 
     free(W); free(Ad); free(Bd);
     return ORACLE_OK;
 }
+
+/* Forward of one NF4 base with several adapters, one per token ([P5] "The
+ * PEFT Strategy (LoRA + QLoRA + Multi-Adapter Serving)": one quantised base
+ * resident, the adapter chosen per request; [P4] "Merging and Deployment
+ * Strategies": adapters swapped over one quantised base):
+ *   h[m] = x[m] W~^T + (alpha_a / r) (x[m] A_a^T) B_a^T,   a = adapter[m]
+ * and no adapter term when adapter[m] < 0. The n_ad adapters are stacked:
+ * A_all is [n_ad * r, K] (rows a*r .. a*r + r - 1 are A_a), B_all is
+ * [N, n_ad * r] (columns a*r .. a*r + r - 1 are B_a). fp64 from the bf16
+ * inputs and the bf16 dequantised operand, as the single-adapter forward.
+ *   rows[i]   token index of output row i;  h_out nrows x N. */
+int oracle_qlora_multi_fwd_rows(const uint8_t *codes, const float *absmax, const uint8_t *q8,
+                                const float *cg, int32_t dq, int64_t N, int64_t K,
+                                const uint16_t *x, int64_t M, const uint16_t *A_all,
+                                const uint16_t *B_all, int32_t r, int32_t n_ad,
+                                const double *alphas, const int32_t *adapter,
+                                const int64_t *rows, int64_t nrows, double *h_out)
+{
+    if (N <= 0 || K <= 0 || K % 64 != 0 || r <= 0 || n_ad <= 0 || M < 0)
+        return ORACLE_ERR_ARG;
+    const int64_t R = (int64_t)n_ad * r;
+    float *Wt = dequant_operand(codes, absmax, q8, cg, N, K, dq);
+    double *Ad = widen_bf16(A_all, R * K);
+    double *Bd = widen_bf16(B_all, N * R);
+    if (!Wt || !Ad || !Bd) {
+        free(Wt); free(Ad); free(Bd);
+        return ORACLE_ERR_ARG;
+    }
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < nrows; ++i) {
+        int64_t m = rows[i];
+        if (m < 0 || m >= M || adapter[m] >= n_ad) {
+            err = 1;
+            continue;
+        }
+        const int32_t a = adapter[m];
+        double *xr = widen_bf16(x + m * K, K);
+        double *u = (double *)malloc(sizeof(double) * (size_t)r);
+        if (!xr || !u) {
+            free(xr); free(u);
+            err = 1;
+            continue;
+        }
+        if (a >= 0)
+            for (int32_t j = 0; j < r; ++j) {        /* u = x A_a^T */
+                double acc = 0.0;
+                for (int64_t k = 0; k < K; ++k)
+                    acc += xr[k] * Ad[((int64_t)a * r + j) * K + k];
+                u[j] = acc;
+            }
+        const double s = a >= 0 ? alphas[a] / (double)r : 0.0;
+        for (int64_t n = 0; n < N; ++n) {
+            double base = 0.0;                       /* x W~^T */
+            for (int64_t k = 0; k < K; ++k)
+                base += xr[k] * (double)Wt[n * K + k];
+            double lora = 0.0;                       /* (x A_a^T) B_a^T */
+            if (a >= 0)
+                for (int32_t j = 0; j < r; ++j)
+                    lora += u[j] * Bd[n * R + (int64_t)a * r + j];
+            h_out[i * N + n] = base + s * lora;
+        }
+        free(xr);
+        free(u);
+    }
+    free(Wt); free(Ad); free(Bd);
+    return err ? ORACLE_ERR_ARG : ORACLE_OK;
+}

@@ -186,3 +186,28 @@ def test_merged_weight_reproduces_the_layer_forward(dq):
     assert np.all(np.abs(f64(x) @ merged.T - h) <= bound)
     # without the adapter term the gap is far larger than the bound
     assert np.max(np.abs(f64(x) @ w32.T - h) - bound) > 0
+
+
+# ---------------------------------------------------------- multi-adapter --
+def test_multi_adapter_rows_equal_single_adapter_forwards():
+    """Each token's row is the single-adapter forward with its own adapter (a
+    separately pinned oracle); tokens without an adapter get the base output."""
+    rng = np.random.default_rng(41)
+    N, K, M, r, n_ad = 40, 192, 9, 8, 3
+    alphas = [16.0, 8.0, 32.0]
+    qw, x, _, _, _ = random_layer(rng, N, K, M, r, dq=True)
+    As = [oracle.f32_to_bf16(rng.uniform(-0.1, 0.1, size=(r, K)).astype(np.float32)) for _ in range(n_ad)]
+    Bs = [oracle.f32_to_bf16(rng.normal(0, 0.05, size=(N, r)).astype(np.float32)) for _ in range(n_ad)]
+    A_all = np.concatenate(As, axis=0)
+    B_all = np.concatenate(Bs, axis=1)
+    adapter = np.array([0, 1, 2, -1, 2, 1, 0, -1, 1], dtype=np.int32)
+    h = oracle.qlora_multi_fwd_rows(qw, N, K, x, A_all, B_all, r, alphas, adapter)
+    for m in range(M):
+        a = adapter[m]
+        A1 = As[a] if a >= 0 else As[0]
+        B1 = Bs[a] if a >= 0 else np.zeros_like(Bs[0])
+        ref, _ = oracle.qlora_fwd_rows(qw, N, K, x, A1, B1, r, alphas[a] if a >= 0 else 1.0, rows=[m])
+        assert np.array_equal(h[m], ref[0])
+    # a wrong adapter for any token changes its row
+    h_wrong = oracle.qlora_multi_fwd_rows(qw, N, K, x, A_all, B_all, r, alphas, (adapter + 1) % n_ad)
+    assert not np.allclose(h_wrong, h, rtol=1e-3)
