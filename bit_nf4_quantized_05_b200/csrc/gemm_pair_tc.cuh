@@ -188,7 +188,12 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
     cluster_sync();            // barriers of both CTAs initialised before any remote use
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    griddep_wait();
+    // This grid is launched only after the kernel before it (the rank-r
+    // product of the same call) has passed its own wait on everything earlier
+    // in the stream, so the activations, codes, scales and adapters are final
+    // now. Only what that kernel writes -- the bf16 rank-r activations read by
+    // the last (LoRA) stage and the zeroed stream-K flags -- is waited for,
+    // by the roles that read it, so the main loop starts while it finishes.
     griddep_launch_dependents();
 
     const int m_pairs = (args.M + 2 * kBM - 1) / (2 * kBM);
@@ -204,6 +209,7 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
             const uint32_t full0 = mapa_shared(smem_u32(a_full), 0);
             int sa = 0;
             uint32_t pa = 0;
+            bool la_ready = false;     // the rank-r activations are written by the kernel before
             for (bool more = sched.first(sg); more; more = sched.next(sg)) {
                 const int m0 = (sg.tile % m_pairs) * (2 * kBM) + static_cast<int>(rank) * kBM;
                 for (int it = sg.k0; it < sg.k1; ++it) {
@@ -212,9 +218,14 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
                     if (it < args.main_steps)
                         tma_load_2d_pair(slot_a + sa * Cfg::kABytes, &tm_act, full0 + 8u * sa,
                                          it * kBK, m0);
-                    else
+                    else {
+                        if (!la_ready) {
+                            griddep_wait();
+                            la_ready = true;
+                        }
                         tma_load_2d_pair(slot_a + sa * Cfg::kABytes, &tm_la, full0 + 8u * sa,
                                          (it - args.main_steps) * kBK, m0);
+                    }
                     if (++sa == SA) { sa = 0; pa ^= 1; }
                 }
             }
@@ -289,6 +300,7 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
         // reads exactly the rows warp q of the tail wrote.
         const int q = warp - kEpiWarp0;                   // TMEM lane quadrant (== warp % 4)
         const uint32_t empty0 = mapa_shared(smem_u32(acc_empty), 0);
+        griddep_wait();            // the stream-K flags are zeroed by the kernel before
         constexpr int kChunks = BN / 32;
         int ab = 0;
         uint32_t aph = 0;
