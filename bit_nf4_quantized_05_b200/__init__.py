@@ -69,6 +69,7 @@ def _load() -> ctypes.CDLL:
     W = ctypes.POINTER(NF4WeightStruct)
     sig = {
         "nf4_quantize": ([vp, W, vp], ctypes.c_int),
+        "nf4_quantize_typed": ([vp, i32, W, vp], ctypes.c_int),
         "nf4_dequantize": ([W, vp, i32, vp], ctypes.c_int),
         "qlora_fwd_workspace_bytes": ([i64, i64, i64, i32], sz),
         "qlora_linear_fwd": ([W, vp, i64, vp, vp, i32, f32, vp, vp, vp, sz, vp], ctypes.c_int),
@@ -151,16 +152,23 @@ class QuantizedWeight:
             torch.empty(max(ng, 1), dtype=torch.float32, device=dev) if double_quant else None)
 
 
+_DTYPES = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}   # nf4_dtype
+
+
 def nf4_quantize(W0: torch.Tensor, double_quant: bool = True,
                  out: Optional[QuantizedWeight] = None) -> QuantizedWeight:
-    """Blockwise NF4 quantisation of a [n, k] fp32 CUDA tensor."""
+    """Blockwise NF4 quantisation of a [n, k] fp32, bf16 or fp16 CUDA tensor."""
     _need_cuda(W0)
-    if W0.dtype != torch.float32 or W0.dim() != 2 or not W0.is_contiguous():
-        raise ValueError("W0 must be a contiguous 2-D float32 tensor")
+    if W0.dtype not in _DTYPES or W0.dim() != 2 or not W0.is_contiguous():
+        raise ValueError("W0 must be a contiguous 2-D float32, bfloat16 or float16 tensor")
     n, k = W0.shape
     qw = out if out is not None else QuantizedWeight.empty(n, k, double_quant, W0.device)
     s = qw.struct()
-    _check(lib.nf4_quantize(_ptr(W0), ctypes.byref(s), _stream(W0.device)), "nf4_quantize")
+    if W0.dtype == torch.float32:
+        _check(lib.nf4_quantize(_ptr(W0), ctypes.byref(s), _stream(W0.device)), "nf4_quantize")
+    else:
+        _check(lib.nf4_quantize_typed(_ptr(W0), _DTYPES[W0.dtype], ctypes.byref(s), _stream(W0.device)),
+               "nf4_quantize_typed")
     return qw
 
 

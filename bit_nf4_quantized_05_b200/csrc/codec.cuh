@@ -8,6 +8,8 @@
 // the scales in groups of 256 blocks, one fp32 constant per group).
 #pragma once
 
+#include <cuda_fp16.h>
+
 #include "nf4_common.cuh"
 
 namespace nf4 {
@@ -51,7 +53,12 @@ constexpr int kQzConsumerWarps = 8;
 constexpr int kQzThreads = 32 * (kQzConsumerWarps + 1);   // the last warp issues the TMA copies
 constexpr int kQzStages = 5;
 constexpr int kQzStageBlocks = 64;
-constexpr int kQzStageBytes = kQzStageBlocks * kBlock * 4;  // 16 KB of fp32
+constexpr int kQzStageBytes = kQzStageBlocks * kBlock * 4;  // 16 KB: one stage slot (fp32 fills it)
+
+// Element type of W0: fp32, or a 16-bit type converted exactly to fp32 on
+// load ("QLoRA explained", section "The quantization backbone": weights are
+// quantised from 16-bit FP16/BF16). A 16-bit block is one 128-byte row.
+enum QzKind { kQzF32 = 0, kQzBF16 = 1, kQzF16 = 2 };
 constexpr int kQzTabRows = 64;                              // bits 18..23 of fl32(p + 3)
 constexpr int kQzCtasPerSm = 2;
 constexpr int kQzTabOff = kQzStages * kQzStageBytes;                // float2 [34][32]
@@ -92,8 +99,11 @@ __device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity) {
         if (clock64() - t0 > kWaitLimitCycles) return;
 }
 
+// tm_w views W0 as 128-byte rows: fp32 [2 nb, 32] with box {32, 128}, or
+// 16-bit [nb, 64] with box {64, 64}; either way a stage is 64 blocks.
+template <int KIND>
 __global__ void __launch_bounds__(kQzThreads, kQzCtasPerSm)
-nf4_quantize_kernel(const __grid_constant__ CUtensorMap tm_w,   // W0 as [2 nb, 32] fp32, box {32, 128}
+nf4_quantize_kernel(const __grid_constant__ CUtensorMap tm_w,
                     int64_t nb, int dq, uint8_t *__restrict__ codes, float *__restrict__ absmax,
                     uint8_t *__restrict__ q8, float *__restrict__ cg) {
     extern __shared__ uint8_t qsm_raw[];
@@ -156,8 +166,9 @@ nf4_quantize_kernel(const __grid_constant__ CUtensorMap tm_w,   // W0 as [2 nb, 
                     const int s = n % kQzStages;
                     const uint32_t ph = static_cast<uint32_t>(n / kQzStages) & 1u;
                     if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) goto drain;
-                    mbar_arrive_expect_tx(&full[s], kQzStageBytes);
-                    tma_load_2d(qsm + s * kQzStageBytes, &tm_w, &full[s], 0, static_cast<int32_t>(2 * b0));
+                    mbar_arrive_expect_tx(&full[s], KIND == kQzF32 ? kQzStageBytes : kQzStageBytes / 2);
+                    tma_load_2d(qsm + s * kQzStageBytes, &tm_w, &full[s], 0,
+                                static_cast<int32_t>(KIND == kQzF32 ? 2 * b0 : b0));
                     ++n;
                 }
             }
@@ -173,11 +184,16 @@ nf4_quantize_kernel(const __grid_constant__ CUtensorMap tm_w,   // W0 as [2 nb, 
     const int bq = lane >> 2;                    // block of this lane among the warp's eight
     const int q = lane & 3;                      // elements [16q, 16q + 16) of that block
     const int lb = warp * 8 + bq;                // block within a stage
-    const int row = 2 * lb + (q >> 1);           // 128-byte row within the stage
-    uint32_t off[4];
+    // 128-byte row within the stage, and the 16-byte pieces of the lane's
+    // elements: fp32 rows hold half a block, 16-bit rows a whole one
+    const int row = KIND == kQzF32 ? 2 * lb + (q >> 1) : lb;
+    constexpr int kPieces = KIND == kQzF32 ? 4 : 2;
+    uint32_t off[kPieces];
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
-        off[j] = static_cast<uint32_t>(row * 128 + (((4 * (q & 1) + j) ^ (row & 7)) << 4));
+    for (int j = 0; j < kPieces; ++j) {
+        const int piece = KIND == kQzF32 ? 4 * (q & 1) + j : 2 * q + j;
+        off[j] = static_cast<uint32_t>(row * 128 + ((piece ^ (row & 7)) << 4));
+    }
     const uint32_t mytab = smem_u32(tab) + 8u * lane;
     bool bad = false;
     int n = 0, gi = 0;
@@ -192,13 +208,32 @@ nf4_quantize_kernel(const __grid_constant__ CUtensorMap tm_w,   // W0 as [2 nb, 
             if (!mbar_wait(&full[s], ph, abort_flag)) goto done;
             const uint8_t *st = qsm + s * kQzStageBytes;
             float x[16];
+            if constexpr (KIND == kQzF32) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float4 v = *reinterpret_cast<const float4 *>(st + off[j]);
-                x[4 * j] = v.x;
-                x[4 * j + 1] = v.y;
-                x[4 * j + 2] = v.z;
-                x[4 * j + 3] = v.w;
+                for (int j = 0; j < 4; ++j) {
+                    const float4 v = *reinterpret_cast<const float4 *>(st + off[j]);
+                    x[4 * j] = v.x;
+                    x[4 * j + 1] = v.y;
+                    x[4 * j + 2] = v.z;
+                    x[4 * j + 3] = v.w;
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(st + off[j]);
+                    const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        if constexpr (KIND == kQzBF16) {
+                            // a bf16 value is the upper half of its fp32 value
+                            x[8 * j + 2 * e] = __uint_as_float(wd[e] << 16);
+                            x[8 * j + 2 * e + 1] = __uint_as_float(wd[e] & 0xffff0000u);
+                        } else {
+                            x[8 * j + 2 * e] = __half2float(__ushort_as_half(static_cast<unsigned short>(wd[e] & 0xffffu)));
+                            x[8 * j + 2 * e + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(wd[e] >> 16)));
+                        }
+                    }
+                }
             }
             // |w| bit patterns, reduced as a tree
             uint32_t mm[8];

@@ -818,30 +818,41 @@ nf4_status nf4_device_status(void *stream) {
     return static_cast<nf4_status>(v);
 }
 
-nf4_status nf4_quantize(const float *W0, const nf4_weight *w, void *stream) {
+nf4_status nf4_quantize_typed(const void *W0, int32_t dtype, const nf4_weight *w, void *stream) {
     nf4_status st = check_weight(w, false);
     if (st != NF4_OK) return st;
     if (!W0 || !w->absmax) return NF4_ERR_INVALID_ARG;
+    if (dtype != NF4_DTYPE_F32 && dtype != NF4_DTYPE_BF16 && dtype != NF4_DTYPE_F16) return NF4_ERR_INVALID_ARG;
     if (!aligned16(W0)) return NF4_ERR_ALIGNMENT;
     const int64_t nb = w->n * w->k / kBlock;
     const int64_t groups = (nb + kGroup - 1) / kGroup;
-    // TMA row coordinates (two 128-byte rows per block) are 32-bit
+    // TMA row coordinates (128-byte rows: two per fp32 block, one per 16-bit block) are 32-bit
     if (2 * nb > 0x7fffffffLL) return NF4_ERR_UNSUPPORTED_SHAPE;
     CUtensorMap tm_w;
-    if (!make_map(&tm_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, W0, 32, static_cast<uint64_t>(2 * nb), 32,
-                  2 * kQzStageBlocks, CU_TENSOR_MAP_SWIZZLE_128B))
-        return NF4_ERR_CUDA;
+    bool ok;
+    if (dtype == NF4_DTYPE_F32)
+        ok = make_map(&tm_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, W0, 32, static_cast<uint64_t>(2 * nb), 32,
+                      2 * kQzStageBlocks, CU_TENSOR_MAP_SWIZZLE_128B);
+    else
+        ok = make_map(&tm_w,
+                      dtype == NF4_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                      2, W0, 64, static_cast<uint64_t>(nb), 64, kQzStageBlocks, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!ok) return NF4_ERR_CUDA;
     // persistent: kQzCtasPerSm CTAs per SM walk the groups
     const int64_t grid = std::min<int64_t>(groups, int64_t(kQzCtasPerSm) * num_sms(current_device()));
-    NF4_TRY_CUDA(cudaFuncSetAttribute(nf4_quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      kQzSmemBytes));
+    auto kern = dtype == NF4_DTYPE_F32 ? nf4_quantize_kernel<kQzF32>
+                : dtype == NF4_DTYPE_BF16 ? nf4_quantize_kernel<kQzBF16> : nf4_quantize_kernel<kQzF16>;
+    NF4_TRY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kQzSmemBytes));
     LaunchTimer t(KK_QUANTIZE, static_cast<cudaStream_t>(stream));
-    nf4_quantize_kernel<<<static_cast<unsigned>(grid), kQzThreads, kQzSmemBytes,
-                          static_cast<cudaStream_t>(stream)>>>(
+    kern<<<static_cast<unsigned>(grid), kQzThreads, kQzSmemBytes, static_cast<cudaStream_t>(stream)>>>(
         tm_w, nb, w->double_quant, w->codes, w->absmax, w->absmax_q8, w->absmax_c);
     t.stop();
     NF4_TRY_CUDA(cudaGetLastError());
     return NF4_OK;
+}
+
+nf4_status nf4_quantize(const float *W0, const nf4_weight *w, void *stream) {
+    return nf4_quantize_typed(W0, NF4_DTYPE_F32, w, stream);
 }
 
 nf4_status nf4_dequantize(const nf4_weight *w, void *out, int32_t out_bf16, void *stream) {

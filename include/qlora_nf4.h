@@ -108,6 +108,17 @@ typedef struct {
  * absmax_q8 and absmax_c. */
 QLORA_API nf4_status nf4_quantize(const float *W0, const nf4_weight *w, void *stream);
 
+/* Element types of W0 accepted by nf4_quantize_typed. */
+typedef enum { NF4_DTYPE_F32 = 0, NF4_DTYPE_BF16 = 1, NF4_DTYPE_F16 = 2 } nf4_dtype;
+
+/* nf4_quantize for a W0 stored as fp32, bf16 or fp16 ([n, k] row-major, device
+ * memory): pretrained weights usually come as 16-bit floats ("QLoRA
+ * explained", section "The quantization backbone"). A 16-bit value converts
+ * to fp32 exactly, so the result equals nf4_quantize of the fp32 image of W0,
+ * bit for bit. Same outputs, requirements and device status as nf4_quantize;
+ * an unknown dtype returns NF4_ERR_INVALID_ARG. */
+QLORA_API nf4_status nf4_quantize_typed(const void *W0, int32_t dtype, const nf4_weight *w, void *stream);
+
 /* Dequantisation w~ = fl32(scale_i * NF4[q]) for every element ("QLoRA
  * Finetuner", section 2, on-the-fly dequantization). out is n*k elements:
  * fp32 when out_bf16 == 0, else bf16 (round to nearest even of the fp32

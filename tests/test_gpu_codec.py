@@ -128,3 +128,50 @@ def test_nonfinite_weight_sets_status(q):
     W[3, 17] = float("inf")
     q.nf4_quantize(W, double_quant=False)
     assert q.device_status() == q.NF4_ERR_NONFINITE
+
+
+# ------------------------------------------------------------ 16-bit input --
+def quant_16(q, W16: torch.Tensor, dq: bool):
+    """GPU quantisation of a 16-bit weight and the oracle's of its exact fp32 image."""
+    ref = oracle.quantize(W16.float().numpy().reshape(-1), dq=dq)
+    qw = q.nf4_quantize(W16.contiguous().cuda(), double_quant=dq)
+    torch.cuda.synchronize()
+    assert q.device_status() == q.NF4_OK
+    return ref, qw
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("shape,dq", [((64, 64), False), ((24, 832), True), ((136, 1280), True),
+                                      ((1000, 640), False)])
+def test_quantize_16bit_input(q, dtype, shape, dq):
+    rng = np.random.default_rng(shape[0] * 7 + shape[1])
+    W = rng.normal(0, 0.02, size=shape).astype(np.float32)
+    W *= rng.uniform(0.2, 5.0, size=(shape[0], 1)).astype(np.float32)
+    ref, qw = quant_16(q, torch.from_numpy(W).to(dtype), dq)
+    assert_quant_equal(ref, qw)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_quantize_16bit_special_blocks(q, dtype):
+    """Zero blocks, subnormals and the largest finite values of the type."""
+    info = torch.finfo(dtype)
+    rows = []
+    rows.append(torch.zeros(64))
+    rows.append(torch.full((64,), float(info.tiny)))                     # smallest normal
+    rows.append(torch.full((64,), float(info.tiny) / 4))                 # subnormal
+    # the largest finite value and smaller multiples of it (every one finite in the type)
+    rows.append(torch.tensor([(-1.0) ** j * float(info.max) * (1.0 - j / 64.0) for j in range(64)]))
+    rows.append(torch.tensor([(-1.0) ** i * 0.5 ** (i % 20) for i in range(64)]))
+    while len(rows) % 8:
+        rows.append(torch.from_numpy(np.random.default_rng(len(rows)).normal(size=64).astype(np.float32)))
+    W = torch.stack(rows).reshape(8, -1).to(dtype)
+    for dq in (False, True):
+        ref, qw = quant_16(q, W, dq)
+        assert_quant_equal(ref, qw)
+
+
+def test_quantize_bf16_outlier_workload_full_size(q):
+    w = workloads.WORKLOADS["decode_mlp_up_13824x5120"]
+    W = workloads.make_weight(w).to(torch.bfloat16)
+    ref, qw = quant_16(q, W, True)
+    assert_quant_equal(ref, qw)
