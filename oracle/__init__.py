@@ -63,6 +63,12 @@ def lib() -> ctypes.CDLL:
         L.oracle_qlora_multi_fwd_rows.argtypes = [vp, vp, vp, vp, i32, i64, i64, vp, i64, vp, vp,
                                                   i32, i32, vp, vp, vp, i64, vp]
         L.oracle_qlora_multi_fwd_rows.restype = ctypes.c_int
+        L.oracle_qlora_fwd_rows_dropout.argtypes = [vp, vp, vp, vp, i32, i64, i64, vp, i64, vp, vp,
+                                                    i32, f64, f64, vp, vp, i64, vp, vp]
+        L.oracle_qlora_fwd_rows_dropout.restype = ctypes.c_int
+        L.oracle_qlora_bwd_dropout.argtypes = [vp, vp, vp, vp, i32, i64, i64, vp, i64, vp, vp, i32,
+                                               f64, f64, vp, vp, vp, i64, vp, vp, vp]
+        L.oracle_qlora_bwd_dropout.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -295,3 +301,59 @@ def qlora_multi_fwd_rows(qw: Quantized, N: int, K: int, x: np.ndarray, A_all: np
     if rc != 0:
         raise OracleError(f"oracle_qlora_multi_fwd_rows failed ({rc})")
     return h
+
+
+def qlora_fwd_rows_dropout(qw: Quantized, N: int, K: int, x: np.ndarray, A: np.ndarray,
+                           B: np.ndarray, r: int, alpha: float, p: float, keep: np.ndarray,
+                           rows: Optional[Sequence[int]] = None):
+    """(h rows, u rows) in fp64 with dropout on the LoRA input:
+    u = (keep . x) A^T, h = x W~^T + (alpha/r)/(1-p) u B^T.
+
+    keep: uint8 bit mask over x, bit (e & 7) of byte e >> 3 for e = m K + k (1 = kept)."""
+    _check_layer(qw, N, K)
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    A = np.ascontiguousarray(A, dtype=np.uint16)
+    B = np.ascontiguousarray(B, dtype=np.uint16)
+    keep = np.ascontiguousarray(keep, dtype=np.uint8)
+    M = x.shape[0]
+    assert keep.size == M * K // 8
+    rows = np.arange(M, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    h = np.zeros((rows.size, N), dtype=np.float64)
+    u = np.zeros((rows.size, r), dtype=np.float64)
+    rc = lib().oracle_qlora_fwd_rows_dropout(_ptr(qw.codes), _ptr(qw.absmax), _ptr(qw.q8),
+                                             _ptr(qw.cg), int(qw.dq), N, K, _ptr(x), M, _ptr(A),
+                                             _ptr(B), r, float(alpha), float(p), _ptr(keep),
+                                             _ptr(rows), rows.size, _ptr(h), _ptr(u))
+    if rc != 0:
+        raise OracleError(f"oracle_qlora_fwd_rows_dropout failed ({rc})")
+    return h, u
+
+
+def qlora_bwd_dropout(qw: Quantized, N: int, K: int, x: np.ndarray, A: np.ndarray, B: np.ndarray,
+                      r: int, alpha: float, p: float, keep: np.ndarray, dY: np.ndarray,
+                      dx_rows: Optional[Sequence[int]] = None):
+    """(dX rows, dA, dB) in fp64 with dropout on the LoRA input (same mask convention)."""
+    _check_layer(qw, N, K)
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    A = np.ascontiguousarray(A, dtype=np.uint16)
+    B = np.ascontiguousarray(B, dtype=np.uint16)
+    dY = np.ascontiguousarray(dY, dtype=np.uint16)
+    keep = np.ascontiguousarray(keep, dtype=np.uint8)
+    M = x.shape[0]
+    assert keep.size == M * K // 8 and dY.shape == (M, N)
+    rows = np.arange(M, dtype=np.int64) if dx_rows is None else np.ascontiguousarray(dx_rows, dtype=np.int64)
+    dX = np.zeros((rows.size, K), dtype=np.float64)
+    dA = np.zeros((r, K), dtype=np.float64)
+    dB = np.zeros((N, r), dtype=np.float64)
+    rc = lib().oracle_qlora_bwd_dropout(_ptr(qw.codes), _ptr(qw.absmax), _ptr(qw.q8), _ptr(qw.cg),
+                                        int(qw.dq), N, K, _ptr(x), M, _ptr(A), _ptr(B), r,
+                                        float(alpha), float(p), _ptr(keep), _ptr(dY), _ptr(rows),
+                                        rows.size, _ptr(dX) if rows.size else None, _ptr(dA), _ptr(dB))
+    if rc != 0:
+        raise OracleError(f"oracle_qlora_bwd_dropout failed ({rc})")
+    return dX, dA, dB
+
+
+def pack_keep(keep_bool: np.ndarray) -> np.ndarray:
+    """Bit mask (uint8, bit e & 7 of byte e >> 3) of a boolean keep array, row-major."""
+    return np.packbits(np.ascontiguousarray(keep_bool, dtype=bool).reshape(-1), bitorder="little")

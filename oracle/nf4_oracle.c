@@ -548,3 +548,176 @@ int oracle_qlora_multi_fwd_rows(const uint8_t *codes, const float *absmax, const
     free(Wt); free(Ad); free(Bd);
     return err ? ORACLE_ERR_ARG : ORACLE_OK;
 }
+
+/* ------------------------------------------------------------------------ */
+/* LoRA dropout ([P1] section 1: h = W0 x + (alpha/r) B(A(dropout x)); the    */
+/* recipe in [P3] uses lora_dropout = 0.05). The random draw is an input:     */
+/* keep is a bit mask over x, bit (e & 7) of byte e >> 3 for element          */
+/* e = m K + k, 1 = kept. Inverted dropout: a kept element is scaled by       */
+/* 1 / (1 - p), a dropped one is zero; the scale is applied to the LoRA       */
+/* branch as a whole, (alpha/r)/(1-p), so the masked x is exact.              */
+/* ------------------------------------------------------------------------ */
+static int keep_bit(const uint8_t *keep, int64_t e) { return (keep[e >> 3] >> (e & 7)) & 1; }
+
+/* Forward rows with dropout on the LoRA input:
+ *   u[m] = (keep . x[m]) A^T,   h[m] = x[m] W~^T + (alpha / r) / (1 - p) u[m] B^T
+ * u_out (may be NULL) receives u without the 1/(1-p) factor. */
+int oracle_qlora_fwd_rows_dropout(const uint8_t *codes, const float *absmax, const uint8_t *q8,
+                                  const float *cg, int32_t dq, int64_t N, int64_t K,
+                                  const uint16_t *x, int64_t M, const uint16_t *A,
+                                  const uint16_t *B, int32_t r, double alpha, double p,
+                                  const uint8_t *keep, const int64_t *rows, int64_t nrows,
+                                  double *h_out, double *u_out)
+{
+    if (N <= 0 || K <= 0 || K % 64 != 0 || r <= 0 || M < 0 || !(p >= 0.0 && p < 1.0) || !keep)
+        return ORACLE_ERR_ARG;
+    float *Wt = dequant_operand(codes, absmax, q8, cg, N, K, dq);
+    double *Ad = widen_bf16(A, (int64_t)r * K);
+    double *Bd = widen_bf16(B, N * r);
+    if (!Wt || !Ad || !Bd) {
+        free(Wt); free(Ad); free(Bd);
+        return ORACLE_ERR_ARG;
+    }
+    const double s = alpha / (double)r / (1.0 - p);
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < nrows; ++i) {
+        int64_t m = rows[i];
+        if (m < 0 || m >= M) {
+            err = 1;
+            continue;
+        }
+        double *xr = widen_bf16(x + m * K, K);
+        double *u = (double *)malloc(sizeof(double) * (size_t)r);
+        if (!xr || !u) {
+            free(xr); free(u);
+            err = 1;
+            continue;
+        }
+        for (int32_t j = 0; j < r; ++j) {           /* u = (keep . x) A^T */
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                if (keep_bit(keep, m * K + k))
+                    acc += xr[k] * Ad[(int64_t)j * K + k];
+            u[j] = acc;
+            if (u_out)
+                u_out[i * r + j] = acc;
+        }
+        for (int64_t n = 0; n < N; ++n) {
+            double base = 0.0;                       /* x W~^T, without dropout */
+            for (int64_t k = 0; k < K; ++k)
+                base += xr[k] * (double)Wt[n * K + k];
+            double lora = 0.0;
+            for (int32_t j = 0; j < r; ++j)
+                lora += u[j] * Bd[n * r + j];
+            h_out[i * N + n] = base + s * lora;
+        }
+        free(xr);
+        free(u);
+    }
+    free(Wt); free(Ad); free(Bd);
+    return err ? ORACLE_ERR_ARG : ORACLE_OK;
+}
+
+/* Backward with dropout on the LoRA input (chain rule through the mask):
+ *   v  = dY B,  u = (keep . x) A^T,  s' = (alpha / r) / (1 - p)
+ *   dX = dY W~ + s' keep . (v A)       (rows in dx_rows)
+ *   dA = s' v^T (keep . x)
+ *   dB = s' dY^T u */
+int oracle_qlora_bwd_dropout(const uint8_t *codes, const float *absmax, const uint8_t *q8,
+                             const float *cg, int32_t dq, int64_t N, int64_t K,
+                             const uint16_t *x, int64_t M, const uint16_t *A,
+                             const uint16_t *B, int32_t r, double alpha, double p,
+                             const uint8_t *keep, const uint16_t *dY,
+                             const int64_t *dx_rows, int64_t ndx, double *dx_out,
+                             double *dA_out, double *dB_out)
+{
+    if (N <= 0 || K <= 0 || K % 64 != 0 || r <= 0 || M < 0 || !(p >= 0.0 && p < 1.0) || !keep)
+        return ORACLE_ERR_ARG;
+    const double s = alpha / (double)r / (1.0 - p);
+    double *Ad = widen_bf16(A, (int64_t)r * K);
+    double *Bd = widen_bf16(B, N * r);
+    double *v = (double *)calloc((size_t)(M * r + 1), sizeof(double));
+    double *u = (double *)calloc((size_t)(M * r + 1), sizeof(double));
+    if (!Ad || !Bd || !v || !u) {
+        free(Ad); free(Bd); free(v); free(u);
+        return ORACLE_ERR_ARG;
+    }
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            double g = oracle_bf16_to_f64(dY[m * N + n]);
+            for (int32_t j = 0; j < r; ++j)
+                v[m * r + j] += g * Bd[n * r + j];
+        }
+        for (int32_t j = 0; j < r; ++j) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                if (keep_bit(keep, m * K + k))
+                    acc += oracle_bf16_to_f64(x[m * K + k]) * Ad[(int64_t)j * K + k];
+            u[m * r + j] = acc;
+        }
+    }
+    int err = 0;
+    if (dx_out && ndx > 0) {
+        float *Wt = dequant_operand(codes, absmax, q8, cg, N, K, dq);
+        if (!Wt) {
+            err = 1;
+        } else {
+#pragma omp parallel for schedule(dynamic, 1)
+            for (int64_t i = 0; i < ndx; ++i) {
+                int64_t m = dx_rows[i];
+                if (m < 0 || m >= M) {
+                    err = 1;
+                    continue;
+                }
+                double *row = dx_out + i * K;
+                for (int64_t k = 0; k < K; ++k)
+                    row[k] = 0.0;
+                for (int64_t n = 0; n < N; ++n) {
+                    double g = oracle_bf16_to_f64(dY[m * N + n]);
+                    for (int64_t k = 0; k < K; ++k)
+                        row[k] += g * (double)Wt[n * K + k];
+                }
+                for (int64_t k = 0; k < K; ++k) {
+                    if (!keep_bit(keep, m * K + k))
+                        continue;
+                    double acc = 0.0;
+                    for (int32_t j = 0; j < r; ++j)
+                        acc += v[m * r + j] * Ad[(int64_t)j * K + k];
+                    row[k] += s * acc;
+                }
+            }
+            free(Wt);
+        }
+    }
+    if (dA_out) {
+#pragma omp parallel for schedule(static)
+        for (int64_t k = 0; k < K; ++k) {
+            for (int32_t j = 0; j < r; ++j) {
+                double acc = 0.0;
+                for (int64_t m = 0; m < M; ++m)
+                    if (keep_bit(keep, m * K + k))
+                        acc += v[m * r + j] * oracle_bf16_to_f64(x[m * K + k]);
+                dA_out[(int64_t)j * K + k] = s * acc;
+            }
+        }
+    }
+    if (dB_out) {
+        for (int64_t i = 0; i < N * r; ++i)
+            dB_out[i] = 0.0;
+#pragma omp parallel for schedule(static)
+        for (int64_t n = 0; n < N; ++n) {
+            double *acc = dB_out + n * r;
+            for (int64_t m = 0; m < M; ++m) {
+                double g = oracle_bf16_to_f64(dY[m * N + n]);
+                for (int32_t j = 0; j < r; ++j)
+                    acc[j] += g * u[m * r + j];
+            }
+            for (int32_t j = 0; j < r; ++j)
+                acc[j] *= s;
+        }
+    }
+    free(Ad); free(Bd); free(v); free(u);
+    return err ? ORACLE_ERR_ARG : ORACLE_OK;
+}

@@ -211,3 +211,50 @@ def test_multi_adapter_rows_equal_single_adapter_forwards():
     # a wrong adapter for any token changes its row
     h_wrong = oracle.qlora_multi_fwd_rows(qw, N, K, x, A_all, B_all, r, alphas, (adapter + 1) % n_ad)
     assert not np.allclose(h_wrong, h, rtol=1e-3)
+
+
+# ---------------------------------------------------------------- dropout --
+def dropout_case(seed, N=32, K=192, M=7, r=8, p=0.25):
+    rng = np.random.default_rng(seed)
+    qw, x, A, B, dY = random_layer(rng, N, K, M, r, dq=True)
+    keep_bool = rng.random((M, K)) >= p
+    return qw, x, A, B, dY, keep_bool, oracle.pack_keep(keep_bool)
+
+
+def test_dropout_with_nothing_dropped_is_the_plain_layer():
+    qw, x, A, B, dY, _, _ = dropout_case(51)
+    N, K, M, r = 32, 192, 7, 8
+    allkeep = oracle.pack_keep(np.ones((M, K), dtype=bool))
+    h, u = oracle.qlora_fwd_rows_dropout(qw, N, K, x, A, B, r, 16.0, 0.0, allkeep)
+    h0, u0 = oracle.qlora_fwd_rows(qw, N, K, x, A, B, r, 16.0)
+    assert np.array_equal(h, h0) and np.array_equal(u, u0)
+    g = oracle.qlora_bwd_dropout(qw, N, K, x, A, B, r, 16.0, 0.0, allkeep, dY)
+    g0 = oracle.qlora_bwd(qw, N, K, x, A, B, r, 16.0, dY)
+    for a, b in zip(g, g0):
+        assert np.array_equal(a, b)
+
+
+def test_dropout_is_the_masked_input_with_rescaled_alpha():
+    """Inverted dropout on the LoRA input equals the plain layer's adapter branch fed
+    the masked tokens with alpha / (1 - p), plus the base of the unmasked tokens;
+    the gradients follow the same composition, with the mask applied to the
+    adapter part of dX."""
+    N, K, M, r, alpha, p = 32, 192, 7, 8, 16.0, 0.25
+    qw, x, A, B, dY, keep_bool, keep = dropout_case(52, N, K, M, r, p)
+    xm = np.where(keep_bool, x, 0).astype(np.uint16)       # masked tokens (exact in bf16)
+    a2 = alpha / (1.0 - p)
+    zB = np.zeros_like(B)
+    h, u = oracle.qlora_fwd_rows_dropout(qw, N, K, x, A, B, r, alpha, p, keep)
+    base, _ = oracle.qlora_fwd_rows(qw, N, K, x, A, zB, r, alpha)
+    hm, um = oracle.qlora_fwd_rows(qw, N, K, xm, A, B, r, a2)
+    hm0, _ = oracle.qlora_fwd_rows(qw, N, K, xm, A, zB, r, a2)
+    assert np.allclose(h, base + (hm - hm0), rtol=1e-12, atol=1e-14)
+    assert np.array_equal(u, um)
+    dX, dA, dB = oracle.qlora_bwd_dropout(qw, N, K, x, A, B, r, alpha, p, keep, dY)
+    dXm, dAm, dBm = oracle.qlora_bwd(qw, N, K, xm, A, B, r, a2, dY)
+    dX0, _, _ = oracle.qlora_bwd(qw, N, K, xm, A, zB, r, a2, dY)
+    assert np.allclose(dA, dAm, rtol=1e-12, atol=1e-14)
+    assert np.allclose(dB, dBm, rtol=1e-12, atol=1e-14)
+    assert np.allclose(dX, dX0 + np.where(keep_bool, dXm - dX0, 0.0), rtol=1e-12, atol=1e-14)
+    # the mask matters: without it every output moves
+    assert not np.allclose(dA, oracle.qlora_bwd(qw, N, K, x, A, B, r, a2, dY)[1], rtol=1e-3)
