@@ -77,6 +77,11 @@ def _load() -> ctypes.CDLL:
         "qlora_bwd_workspace_bytes": ([i64, i64, i64, i32], sz),
         "qlora_linear_bwd": ([W, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, vp, vp, sz, vp],
                              ctypes.c_int),
+        "qlora_linear_fwd_dropout": ([W, vp, i64, vp, vp, i32, f32, f32, vp, vp, vp, vp, sz, vp],
+                                     ctypes.c_int),
+        "qlora_bwd_dropout_workspace_bytes": ([i64, i64, i64, i32], sz),
+        "qlora_linear_bwd_dropout": ([W, vp, i64, vp, vp, i32, f32, f32, vp, vp, vp, vp, vp, vp, vp,
+                                      sz, vp], ctypes.c_int),
         "qlora_merge": ([W, vp, vp, i32, f32, vp, i32, vp], ctypes.c_int),
         "qlora_multi_lora_fwd": ([W, vp, i64, vp, vp, i32, i32, ctypes.POINTER(f32), vp, vp, vp, sz,
                                   vp], ctypes.c_int),
@@ -296,6 +301,53 @@ def qlora_merge(qw: QuantizedWeight, A: torch.Tensor, B: torch.Tensor, alpha: fl
     _check(lib.qlora_merge(ctypes.byref(s), _ptr(A), _ptr(B), r, float(alpha), _ptr(out),
                            int(bf16), _stream(qw.device)), "qlora_merge")
     return out
+
+
+def pack_keep(keep: torch.Tensor) -> torch.Tensor:
+    """Device bit mask (uint8, bit e & 7 of byte e >> 3, e = m * k + kk) of a boolean
+    [M, k] CUDA tensor of kept elements."""
+    b = keep.reshape(-1, 8).to(torch.uint8)
+    w = torch.tensor([1, 2, 4, 8, 16, 32, 64, 128], dtype=torch.uint8, device=keep.device)
+    return (b * w).sum(dim=1, dtype=torch.int32).to(torch.uint8).contiguous()
+
+
+def qlora_linear_fwd_dropout(qw: QuantizedWeight, x: torch.Tensor, A: torch.Tensor,
+                             B: torch.Tensor, alpha: float, p: float, keep: torch.Tensor,
+                             save_u: bool = True, h: Optional[torch.Tensor] = None,
+                             workspace: Optional[torch.Tensor] = None):
+    """Forward with LoRA dropout; keep is the packed bit mask over x (see pack_keep).
+    Returns (h, u) with u = (keep . x) A^T."""
+    _need_cuda(x, A, B, keep)
+    M, r = x.shape[0], A.shape[0]
+    if h is None:
+        h = torch.empty(M, qw.n, dtype=torch.bfloat16, device=x.device)
+    u = torch.empty(M, r, dtype=torch.float32, device=x.device) if save_u else None
+    ws = workspace if workspace is not None else _workspace(fwd_workspace_bytes(M, qw.n, qw.k, r), x.device)
+    s = qw.struct()
+    _check(lib.qlora_linear_fwd_dropout(ctypes.byref(s), _ptr(x), M, _ptr(A), _ptr(B), r, float(alpha),
+                                        float(p), _ptr(keep), _ptr(h), _ptr(u), _ptr(ws), ws.numel(),
+                                        _stream(x.device)), "qlora_linear_fwd_dropout")
+    return h, u
+
+
+def qlora_linear_bwd_dropout(qw: QuantizedWeight, x: torch.Tensor, A: torch.Tensor,
+                             B: torch.Tensor, alpha: float, p: float, keep: torch.Tensor,
+                             dY: torch.Tensor, u: Optional[torch.Tensor] = None,
+                             need_dX: bool = True, workspace: Optional[torch.Tensor] = None):
+    """(dX, dA, dB) with LoRA dropout (the mask of the forward)."""
+    _need_cuda(x, A, B, dY, keep)
+    M, r = x.shape[0], A.shape[0]
+    dX = torch.empty(M, qw.k, dtype=torch.bfloat16, device=x.device) if need_dX else None
+    dA = torch.empty(r, qw.k, dtype=torch.bfloat16, device=x.device)
+    dB = torch.empty(qw.n, r, dtype=torch.bfloat16, device=x.device)
+    nbytes = int(lib.qlora_bwd_dropout_workspace_bytes(M, qw.n, qw.k, r))
+    ws = workspace if workspace is not None else _workspace(nbytes, x.device)
+    s = qw.struct()
+    _check(lib.qlora_linear_bwd_dropout(ctypes.byref(s), _ptr(x), M, _ptr(A), _ptr(B), r, float(alpha),
+                                        float(p), _ptr(keep), _ptr(dY), _ptr(u), _ptr(dX), _ptr(dA),
+                                        _ptr(dB), _ptr(ws), ws.numel(), _stream(x.device)),
+           "qlora_linear_bwd_dropout")
+    return dX, dA, dB
 
 
 def device_status(device=None) -> int:

@@ -533,7 +533,7 @@ constexpr int kDsUParkBytes = 256 * 32 * 4;
 
 template <int TG>
 __global__ void __launch_bounds__(kDsThreads, 1)
-qlora_decode_u_kernel(const DecodeArgs a) {
+qlora_decode_u_kernel(const DecodeArgs a, const uint8_t *__restrict__ keep) {
     extern __shared__ __align__(16) float upark[];     // [256][32]
     // x may come from the kernel before this one
     griddep_wait();
@@ -572,6 +572,20 @@ qlora_decode_u_kernel(const DecodeArgs a) {
                     const uint4 *px = reinterpret_cast<const uint4 *>(xrow[tg] + kb * 64);
                     xa[tg] = __ldg(px);
                     xb[tg] = __ldg(px + 1);
+                    if (keep) {
+                        // LoRA dropout: zero the dropped tokens' elements (16 k, two keep bytes)
+                        const int m = tg * 8 + g;
+                        const int64_t e = static_cast<int64_t>(m) * a.K + kb * 64 + 16 * t;
+                        const uint32_t kbits = keep[e >> 3] | (static_cast<uint32_t>(keep[(e >> 3) + 1]) << 8);
+                        uint32_t w[8] = {xa[tg].x, xa[tg].y, xa[tg].z, xa[tg].w,
+                                         xb[tg].x, xb[tg].y, xb[tg].z, xb[tg].w};
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            w[i] &= ((kbits >> (2 * i)) & 1u ? 0x0000ffffu : 0u) |
+                                    ((kbits >> (2 * i + 1)) & 1u ? 0xffff0000u : 0u);
+                        xa[tg] = make_uint4(w[0], w[1], w[2], w[3]);
+                        xb[tg] = make_uint4(w[4], w[5], w[6], w[7]);
+                    }
                 } else {
                     xa[tg] = make_uint4(0, 0, 0, 0);
                     xb[tg] = xa[tg];

@@ -126,7 +126,9 @@ __device__ __forceinline__ void set_flag_gpu(int *flag) {
     asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(1) : "memory");
 }
 
-template <int BN, bool DGRAD, int G>
+// OUT32: the result is written in fp32 to args.D32 (for a later kernel that
+// adds to it and rounds once) instead of bf16 to args.D.
+template <int BN, bool DGRAD, int G, bool OUT32>
 __global__ void __launch_bounds__(PairCfg<BN, DGRAD, G>::kThreads, 1)
 qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red] bf16, box {64,128}
                        const __grid_constant__ CUtensorMap tm_codes,  // [Nw, K/2] u8, box {32, rows}
@@ -363,6 +365,13 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
                                     const float4 p0 = pv[0], p1 = pv[1];
                                     f[0] += p0.x; f[1] += p0.y; f[2] += p0.z; f[3] += p0.w;
                                     f[4] += p1.x; f[5] += p1.y; f[6] += p1.z; f[7] += p1.w;
+                                }
+                                if constexpr (OUT32) {
+                                    // fp32 result (a later kernel adds to it and rounds once)
+                                    float4 *f4 = reinterpret_cast<float4 *>(args.D32 + static_cast<int64_t>(row) * args.out + col);
+                                    f4[0] = make_float4(f[0], f[1], f[2], f[3]);
+                                    f4[1] = make_float4(f[4], f[5], f[6], f[7]);
+                                    continue;
                                 }
                                 uint32_t p[4];
 #pragma unroll

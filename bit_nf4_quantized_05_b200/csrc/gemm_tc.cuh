@@ -66,6 +66,7 @@ struct GemmArgs {
     int sk;
     float *partial;     // [pairs][2][BN/32][128][32] fp32 partial tiles
     int *flags;         // [pairs][2][4 epilogue warps], zero at launch; 1 = rows written
+    float *D32;         // when non-null: the fp32 result goes here instead of D
 };
 
 template <int BN, bool DGRAD>
@@ -253,6 +254,14 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red] bf1
                     for (int g = 0; g < 4; ++g) {
                         const int col = n0 + c * 32 + g * 8;
                         if (col < args.out) {
+                            if (args.D32) {
+                                float4 *f4 = reinterpret_cast<float4 *>(args.D32 + static_cast<int64_t>(row) * args.out + col);
+                                f4[0] = make_float4(__uint_as_float(v[g * 8]), __uint_as_float(v[g * 8 + 1]),
+                                                    __uint_as_float(v[g * 8 + 2]), __uint_as_float(v[g * 8 + 3]));
+                                f4[1] = make_float4(__uint_as_float(v[g * 8 + 4]), __uint_as_float(v[g * 8 + 5]),
+                                                    __uint_as_float(v[g * 8 + 6]), __uint_as_float(v[g * 8 + 7]));
+                                continue;
+                            }
                             uint32_t p[4];
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {

@@ -182,3 +182,117 @@ __global__ void __launch_bounds__(kMgThreads, 4) qlora_merge_kernel(const MergeA
 }
 
 }  // namespace nf4
+
+namespace nf4 {
+
+// ---------------------------------------------------------------------------
+// The adapter part of dX under LoRA dropout: with dropout on the adapter input,
+// the gradient that reaches x through the adapters is masked element-wise,
+//     dX[m][k] += keep[m][k] * sum_j Vs[m][j] A[j][k],   Vs = bf16((alpha/r)/(1-p) v)
+// (the chain rule through inverted dropout; "QLoRA Finetuner", section 1,
+// h = W0 x + (alpha/r) B(A(dropout x))). base holds dY W~ in fp32 (written by
+// the dgrad GEMM); the sum is accumulated in fp32 on mma.sync fragments and
+// one rounding of base + kept sum gives dX in bf16. Same tiling as the merge kernel: 64 rows (tokens) x 128 columns
+// per CTA, warp w on rows [16 (w % 4), +16) and columns [64 (w / 4), +64).
+// ---------------------------------------------------------------------------
+struct LoraAddArgs {
+    int64_t M, K;
+    int r, rp;
+    const uint16_t *Vs;        // [M, r]
+    const uint16_t *A;         // [r, K]
+    const uint8_t *keep;       // bit mask over [M, K]
+    const float *base;         // [M, K] fp32: dY W~
+    uint16_t *dX;              // [M, K] bf16 result
+};
+
+__host__ __device__ inline int lora_add_smem_bytes(int rp) {
+    return kMgRows * merge_bs_stride(rp) * 2 + kMgCols * merge_bs_stride(rp) * 2 + 8 * 16 * (64 + 4) * 4;
+}
+
+template <int RQ>
+__global__ void __launch_bounds__(kMgThreads, 4) qlora_lora_add_kernel(const LoraAddArgs a) {
+    extern __shared__ __align__(16) uint8_t msm[];
+    constexpr int rs = merge_bs_stride(16 * RQ);
+    uint16_t *Vsm = reinterpret_cast<uint16_t *>(msm);                      // [64][rs]
+    uint16_t *Ats = Vsm + kMgRows * rs;                                     // [128][rs]
+    uint8_t *stage = reinterpret_cast<uint8_t *>(Ats + kMgCols * rs);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kMgRows;
+    const int64_t k0 = static_cast<int64_t>(blockIdx.x) * kMgCols;
+
+    griddep_wait();
+    griddep_launch_dependents();
+
+    for (int idx = tid; idx < kMgRows * (a.rp / 8); idx += kMgThreads) {
+        const int row = idx / (a.rp / 8), ch = idx % (a.rp / 8);
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (m0 + row < a.M && ch * 8 < a.r)
+            v = __ldg(reinterpret_cast<const uint4 *>(a.Vs + (m0 + row) * a.r) + ch);
+        *reinterpret_cast<uint4 *>(Vsm + row * rs + ch * 8) = v;
+    }
+    for (int idx = tid; idx < a.rp * (kMgCols / 8); idx += kMgThreads) {
+        const int j = idx % a.rp, ch = idx / a.rp;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (j < a.r && k0 + ch * 8 < a.K)
+            v = __ldg(reinterpret_cast<const uint4 *>(a.A + static_cast<int64_t>(j) * a.K + k0) + ch);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            Ats[(ch * 8 + e) * rs + j] = static_cast<uint16_t>(w[e >> 1] >> (16 * (e & 1)));
+    }
+    __syncthreads();
+
+    const int rw = 16 * (warp & 3), cw = 64 * (warp >> 2);
+    if (k0 + cw >= a.K) return;            // K is a multiple of 64: a warp's columns are all in or out
+    uint32_t af[RQ][4];
+#pragma unroll
+    for (int q = 0; q < RQ; ++q) {
+        const int ks = 16 * q;
+        af[q][0] = *reinterpret_cast<const uint32_t *>(Vsm + (rw + g) * rs + ks + 2 * t);
+        af[q][1] = *reinterpret_cast<const uint32_t *>(Vsm + (rw + g + 8) * rs + ks + 2 * t);
+        af[q][2] = *reinterpret_cast<const uint32_t *>(Vsm + (rw + g) * rs + ks + 2 * t + 8);
+        af[q][3] = *reinterpret_cast<const uint32_t *>(Vsm + (rw + g + 8) * rs + ks + 2 * t + 8);
+    }
+    float *st = reinterpret_cast<float *>(stage + warp * 16 * (64 + 4) * 4);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        const uint16_t *bc = Ats + (cw + 8 * i + g) * rs + 2 * t;
+#pragma unroll
+        for (int q = 0; q < RQ; ++q)
+            mma_bf16_16816(acc, af[q], *reinterpret_cast<const uint32_t *>(bc + 16 * q),
+                           *reinterpret_cast<const uint32_t *>(bc + 16 * q + 8));
+        *reinterpret_cast<float2 *>(st + g * (64 + 4) + 8 * i + 2 * t) = make_float2(acc[0], acc[1]);
+        *reinterpret_cast<float2 *>(st + (g + 8) * (64 + 4) + 8 * i + 2 * t) = make_float2(acc[2], acc[3]);
+    }
+    __syncwarp();
+    // 16 rows x 8 pieces of 8 columns: fp32 base plus the kept adapter terms, one rounding
+#pragma unroll
+    for (int c = lane; c < 16 * 8; c += 32) {
+        const int rl = c >> 3, ch = c & 7;
+        const int64_t m = m0 + rw + rl;
+        if (m >= a.M) continue;
+        const int64_t k = k0 + cw + 8 * ch;
+        const uint32_t kb = a.keep[(m * a.K + k) >> 3];
+        uint4 *px = reinterpret_cast<uint4 *>(a.dX + m * a.K + k);
+        const float4 b0 = *reinterpret_cast<const float4 *>(a.base + m * a.K + k);
+        const float4 b1 = *reinterpret_cast<const float4 *>(a.base + m * a.K + k + 4);
+        const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        const float4 l0 = *reinterpret_cast<const float4 *>(st + rl * (64 + 4) + 8 * ch);
+        const float4 l1 = *reinterpret_cast<const float4 *>(st + rl * (64 + 4) + 8 * ch + 4);
+        const float lv[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float x0 = bv[2 * e] + ((kb >> (2 * e)) & 1u ? lv[2 * e] : 0.0f);
+            const float x1 = bv[2 * e + 1] + ((kb >> (2 * e + 1)) & 1u ? lv[2 * e + 1] : 0.0f);
+            __nv_bfloat162 p = __floats2bfloat162_rn(x0, x1);
+            o[e] = *reinterpret_cast<uint32_t *>(&p);
+        }
+        *px = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+}  // namespace nf4

@@ -36,11 +36,11 @@ constexpr int kMaxAdapters = 16;   // stacked adapters of one multi-adapter forw
 // Optional per-kernel event timing (nf4_profiling / nf4_profile_read)
 // ---------------------------------------------------------------------------
 enum KernelKind {
-    KK_QUANTIZE, KK_DEQUANTIZE, KK_LORA_U, KK_LORA_V, KK_LORA_DBDA, KK_ZERO, KK_GEMM_FWD, KK_GEMM_DGRAD, KK_DECODE, KK_DECODE_U, KK_MERGE, KK_COUNT
+    KK_QUANTIZE, KK_DEQUANTIZE, KK_LORA_U, KK_LORA_V, KK_LORA_DBDA, KK_ZERO, KK_GEMM_FWD, KK_GEMM_DGRAD, KK_DECODE, KK_DECODE_U, KK_MERGE, KK_LORA_ADD, KK_COUNT
 };
 const char *const kKindNames[KK_COUNT] = {
     "nf4_quantize", "nf4_dequantize", "lora_u", "lora_v", "lora_dB_dA", "zero_fill", "qlora_gemm_fwd", "qlora_gemm_dgrad", "qlora_decode",
-    "decode_lora_u", "qlora_merge"};
+    "decode_lora_u", "qlora_merge", "lora_dX_add"};
 
 struct ProfRecord {
     int kind;
@@ -287,6 +287,9 @@ struct SkinnySpec {
     uint16_t *out_bf16;
     float scale;
     int transposed;
+    int mask_mode = 0;                 // dropout on x as the A operand (see SkinnyJob)
+    const uint8_t *keep = nullptr;
+    int64_t mx = 0, kx = 0;
 };
 
 // Tensor maps and job fields of one product; splits is the launch's split count.
@@ -313,6 +316,10 @@ bool skinny_job(const SkinnySpec &sp, int RN, int splits, CUtensorMap *ta, CUten
     job->out_bf16 = sp.out_bf16;
     job->scale = sp.scale;
     job->transposed = sp.transposed;
+    job->mask_mode = sp.mask_mode;
+    job->keep = sp.keep;
+    job->mx = sp.mx;
+    job->kx = sp.kx;
     return ok;
 }
 
@@ -340,8 +347,9 @@ nf4_status skinny_launch(int kind, const SkinnySpec *sp, int n, cudaStream_t str
         p_tiles += static_cast<int>((P + 127) / 128);
         steps = std::max(steps, static_cast<int>((Q + 63) / 64));
     }
-    // one wave: the splits of all tiles fill the SMs once (clusters of at most 8)
-    int splits = std::max(1, sms / std::max(1, p_tiles));
+    // one wave: the splits of all tiles fill the CTA slots once (two CTAs fit
+    // on an SM; clusters of at most 8)
+    int splits = std::max(1, 2 * sms / std::max(1, p_tiles));
     splits = std::min({splits, kSkMaxSplits, steps});
     const int sps = (steps + splits - 1) / splits;
     splits = (steps + sps - 1) / sps;            // every split has at least one step
@@ -405,7 +413,7 @@ nf4_status skinny_product(int kind, const void *a, int64_t a_rows, int64_t a_col
 template <int BN, bool DGRAD>
 nf4_status launch_gemm(const nf4_weight *w, const uint16_t *act, int64_t M, int64_t red,
                        int64_t out, const uint16_t *la, int32_t r, const uint16_t *lb,
-                       uint16_t *D, cudaStream_t stream) {
+                       uint16_t *D, cudaStream_t stream, float *D32 = nullptr) {
     using Cfg = GemmCfg<BN, DGRAD>;
     CUtensorMap tm_act, tm_codes, tm_la;
     const int64_t N = w->n, K = w->k;
@@ -416,8 +424,12 @@ nf4_status launch_gemm(const nf4_weight *w, const uint16_t *act, int64_t M, int6
     // distinct banks
     ok = ok && make_map(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, K / 2, N, kBK / 2,
                         DGRAD ? kBK : BN, CU_TENSOR_MAP_SWIZZLE_32B);
-    ok = ok && make_map(&tm_la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, la, r, M, kBK, kBM,
-                        CU_TENSOR_MAP_SWIZZLE_128B);
+    // no LoRA stage when la is null (the adapter term is added by another kernel)
+    if (la)
+        ok = ok && make_map(&tm_la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, la, r, M, kBK, kBM,
+                            CU_TENSOR_MAP_SWIZZLE_128B);
+    else
+        tm_la = tm_act;
     if (!ok) return NF4_ERR_CUDA;
 
     GemmArgs a{};
@@ -425,7 +437,7 @@ nf4_status launch_gemm(const nf4_weight *w, const uint16_t *act, int64_t M, int6
     a.red = static_cast<int>(red);
     a.out = static_cast<int>(out);
     a.main_steps = static_cast<int>((red + kBK - 1) / kBK);
-    a.lora_steps = (r + kBK - 1) / kBK;
+    a.lora_steps = la ? (r + kBK - 1) / kBK : 0;
     a.m_tiles = static_cast<int>((M + kBM - 1) / kBM);
     a.n_tiles = static_cast<int>((out + BN - 1) / BN);
     a.r = r;
@@ -438,6 +450,7 @@ nf4_status launch_gemm(const nf4_weight *w, const uint16_t *act, int64_t M, int6
     a.dq = w->double_quant;
     a.lora_b = lb;
     a.D = D;
+    a.D32 = D32;
 
     const int dev = current_device();
     const int tiles = a.m_tiles * a.n_tiles;
@@ -462,7 +475,7 @@ int pair_capacity(int dev) {
     static int cache[kMaxDevices] = {0};
     if (dev < 0 || dev >= kMaxDevices) return 0;
     if (cache[dev] == 0) {
-        auto kern = qlora_gemm_pair_kernel<BN, DGRAD, G>;
+        auto kern = qlora_gemm_pair_kernel<BN, DGRAD, G, false>;
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Cfg::kSmemBytes) != cudaSuccess)
             return 0;
@@ -492,7 +505,8 @@ int pair_capacity(int dev) {
 template <int BN, bool DGRAD, int G>
 nf4_status launch_gemm_pair(const nf4_weight *w, const uint16_t *act, int64_t M, int64_t red,
                             int64_t out, const uint16_t *la, int32_t r, const uint16_t *lb,
-                            uint16_t *D, cudaStream_t stream, const SkBuf *sk = nullptr) {
+                            uint16_t *D, cudaStream_t stream, const SkBuf *sk = nullptr,
+                            float *D32 = nullptr) {
     using Cfg = PairCfg<BN, DGRAD, G>;
     CUtensorMap tm_act, tm_codes, tm_la;
     const int64_t N = w->n, K = w->k;
@@ -502,8 +516,12 @@ nf4_status launch_gemm_pair(const nf4_weight *w, const uint16_t *act, int64_t M,
     // (BN/2 rows forward, 64 rows dgrad), 32-byte swizzle
     ok = ok && make_map(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, K / 2, N, kBK / 2,
                         DGRAD ? kBK : Cfg::kBH, CU_TENSOR_MAP_SWIZZLE_32B);
-    ok = ok && make_map(&tm_la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, la, r, M, kBK, kBM,
-                        CU_TENSOR_MAP_SWIZZLE_128B);
+    // no LoRA stage when la is null (the adapter term is added by another kernel)
+    if (la)
+        ok = ok && make_map(&tm_la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, la, r, M, kBK, kBM,
+                            CU_TENSOR_MAP_SWIZZLE_128B);
+    else
+        tm_la = tm_act;
     if (!ok) return NF4_ERR_CUDA;
 
     GemmArgs a{};
@@ -511,7 +529,7 @@ nf4_status launch_gemm_pair(const nf4_weight *w, const uint16_t *act, int64_t M,
     a.red = static_cast<int>(red);
     a.out = static_cast<int>(out);
     a.main_steps = static_cast<int>((red + kBK - 1) / kBK);
-    a.lora_steps = (r + kBK - 1) / kBK;
+    a.lora_steps = la ? (r + kBK - 1) / kBK : 0;
     a.m_tiles = static_cast<int>((M + kBM - 1) / kBM);
     a.n_tiles = static_cast<int>((out + BN - 1) / BN);
     a.r = r;
@@ -524,6 +542,7 @@ nf4_status launch_gemm_pair(const nf4_weight *w, const uint16_t *act, int64_t M,
     a.dq = w->double_quant;
     a.lora_b = lb;
     a.D = D;
+    a.D32 = D32;
 
     const int dev = current_device();
     const int cap = pair_capacity<BN, DGRAD, G>(dev);
@@ -540,8 +559,13 @@ nf4_status launch_gemm_pair(const nf4_weight *w, const uint16_t *act, int64_t M,
     }
     LaunchTimer t(DGRAD ? KK_GEMM_DGRAD : KK_GEMM_FWD, stream);
     const cudaError_t e =
-        launch_ex(qlora_gemm_pair_kernel<BN, DGRAD, G>, dim3(static_cast<unsigned>(2 * pairs)),
-                  dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, 2u, tm_act, tm_codes, tm_la, a);
+        D32 ? (cudaFuncSetAttribute(qlora_gemm_pair_kernel<BN, DGRAD, G, true>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes) != cudaSuccess
+                   ? cudaErrorInvalidValue
+                   : launch_ex(qlora_gemm_pair_kernel<BN, DGRAD, G, true>, dim3(static_cast<unsigned>(2 * pairs)),
+                        dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, 2u, tm_act, tm_codes, tm_la, a))
+            : launch_ex(qlora_gemm_pair_kernel<BN, DGRAD, G, false>, dim3(static_cast<unsigned>(2 * pairs)),
+                        dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, 2u, tm_act, tm_codes, tm_la, a);
     t.stop();
     if (e != cudaSuccess) return NF4_ERR_CUDA;
     NF4_TRY_CUDA(cudaGetLastError());
@@ -593,7 +617,8 @@ bool decode_shape(const nf4_weight *w, int64_t M, int32_t r) {
 
 nf4_status launch_decode(const nf4_weight *w, const uint16_t *x, int64_t M, const uint16_t *A,
                          const uint16_t *B, int32_t r, float scale, uint16_t *h, float *u_out,
-                         float *upart, cudaStream_t stream, const RowGroups *groups = nullptr) {
+                         float *upart, cudaStream_t stream, const RowGroups *groups = nullptr,
+                         const uint8_t *keep = nullptr) {
     // each of the 16 warps takes rb blocks of every 32-row tile, fetched in
     // chunks of cb blocks (the largest divisor of rb that is at most 5)
     const int64_t kblocks = w->k / kBlock;
@@ -635,7 +660,7 @@ nf4_status launch_decode(const nf4_weight *w, const uint16_t *x, int64_t M, cons
         LaunchTimer t(KK_DECODE_U, stream);
         auto ku = tg == 1 ? qlora_decode_u_kernel<1> : qlora_decode_u_kernel<2>;
         NF4_TRY_CUDA(cudaFuncSetAttribute(ku, cudaFuncAttributeMaxDynamicSharedMemorySize, kDsUParkBytes));
-        const cudaError_t e = launch_ex(ku, dim3(kDsUCtas), dim3(kDsThreads), kDsUParkBytes, stream, 0u, a);
+        const cudaError_t e = launch_ex(ku, dim3(kDsUCtas), dim3(kDsThreads), kDsUParkBytes, stream, 0u, a, keep);
         t.stop();
         if (e != cudaSuccess) return NF4_ERR_CUDA;
     }
@@ -708,29 +733,30 @@ constexpr int kPairGroups = 5;
 template <bool DGRAD>
 nf4_status launch_gemm_auto(const nf4_weight *w, const uint16_t *act, int64_t M, int64_t red,
                             int64_t out, const uint16_t *la, int32_t r, const uint16_t *lb,
-                            uint16_t *D, cudaStream_t stream, const SkBuf *sk = nullptr) {
+                            uint16_t *D, cudaStream_t stream, const SkBuf *sk = nullptr,
+                            float *D32 = nullptr) {
     const int dev = current_device();
     const int pairs = pair_capacity<256, DGRAD, kPairGroups>(dev);
     if (pairs > 0) {
         const int64_t tiles256 = ((M + 2 * kBM - 1) / (2 * kBM)) * ((out + 255) / 256);
         if (sk && tiles256 > pairs)
             return launch_gemm_pair<256, DGRAD, kPairGroups>(w, act, M, red, out, la, r, lb, D,
-                                                             stream, sk);
+                                                             stream, sk, D32);
         switch (pick_pair_bn(M, out, pairs, DGRAD)) {
         case 128:
-            return launch_gemm_pair<128, DGRAD, kPairGroups>(w, act, M, red, out, la, r, lb, D, stream);
+            return launch_gemm_pair<128, DGRAD, kPairGroups>(w, act, M, red, out, la, r, lb, D, stream, nullptr, D32);
         case 192:
             if constexpr (!DGRAD)
                 return launch_gemm_pair<192, DGRAD, kPairGroups>(w, act, M, red, out, la, r, lb, D,
-                                                                 stream);
+                                                                 stream, nullptr, D32);
             break;
         default:
-            return launch_gemm_pair<256, DGRAD, kPairGroups>(w, act, M, red, out, la, r, lb, D, stream);
+            return launch_gemm_pair<256, DGRAD, kPairGroups>(w, act, M, red, out, la, r, lb, D, stream, nullptr, D32);
         }
     }
     if (pick_bn(M, out, num_sms(dev)) == 192)
-        return launch_gemm<192, DGRAD>(w, act, M, red, out, la, r, lb, D, stream);
-    return launch_gemm<256, DGRAD>(w, act, M, red, out, la, r, lb, D, stream);
+        return launch_gemm<192, DGRAD>(w, act, M, red, out, la, r, lb, D, stream, D32);
+    return launch_gemm<256, DGRAD>(w, act, M, red, out, la, r, lb, D, stream, D32);
 }
 
 // ---------------------------------------------------------------------------
@@ -923,14 +949,18 @@ size_t qlora_fwd_workspace_bytes(int64_t M, int64_t n, int64_t k, int32_t r) {
     return fwd_layout(M, r, num_sms(current_device())).total;
 }
 
-nf4_status qlora_linear_fwd(const nf4_weight *w, const uint16_t *x, int64_t M, const uint16_t *A,
-                            const uint16_t *B, int32_t r, float alpha, uint16_t *h, float *u_out,
-                            void *workspace, size_t ws_bytes, void *stream) {
+// Forward, with LoRA dropout when keep is non-null (inverted dropout on the
+// adapter input with the keep mask given; the branch is scaled by
+// (alpha/r)/(1-p)).
+nf4_status fwd_impl(const nf4_weight *w, const uint16_t *x, int64_t M, const uint16_t *A,
+                    const uint16_t *B, int32_t r, float alpha, float p, const uint8_t *keep,
+                    uint16_t *h, float *u_out, void *workspace, size_t ws_bytes, void *stream) {
     nf4_status st = check_layer(w, x, M, A, B, r, alpha);
     if (st != NF4_OK) return st;
+    if (keep && !(p >= 0.0f && p < 1.0f)) return NF4_ERR_INVALID_ARG;
     if (M == 0) return NF4_OK;
     if (!h) return NF4_ERR_INVALID_ARG;
-    if (!aligned16(h) || !aligned16(u_out)) return NF4_ERR_ALIGNMENT;
+    if (!aligned16(h) || !aligned16(u_out) || !aligned16(keep)) return NF4_ERR_ALIGNMENT;
     const int sms = num_sms(current_device());
     const FwdLayout L = fwd_layout(M, r, sms);
     if (!workspace || ws_bytes < L.total) return NF4_ERR_WORKSPACE;
@@ -940,15 +970,38 @@ nf4_status qlora_linear_fwd(const nf4_weight *w, const uint16_t *x, int64_t M, c
     uint16_t *u_s = reinterpret_cast<uint16_t *>(ws + L.us);
     const SkBuf sk{reinterpret_cast<float *>(ws + L.partial), reinterpret_cast<int *>(ws + L.flags),
                    sk_pairs_max(sms)};
-    const float scale = alpha / static_cast<float>(r);
+    float scale = alpha / static_cast<float>(r);
+    if (keep) scale = scale / (1.0f - p);
     if (decode_shape(w, M, r))
-        return launch_decode(w, x, M, A, B, r, scale, h, u_out, reinterpret_cast<float *>(ws + L.upart), s);
-    // u = x A^T (fp32, optional) and bf16((alpha/r) u) for the up-projection
-    // stage; this kernel also clears the GEMM's stream-K flags
-    st = skinny_product(KK_LORA_U, x, M, w->k, Major::K, A, r, w->k, Major::K, r, u_out, u_s,
-                        scale, 0, s, sk.flags, sk.pairs_max * kSkFlagsPerPair);
+        return launch_decode(w, x, M, A, B, r, scale, h, u_out, reinterpret_cast<float *>(ws + L.upart), s,
+                             nullptr, keep);
+    // u = x A^T (fp32, optional; under dropout the dropped elements of x are
+    // zero) and bf16(scale u) for the up-projection stage; this kernel also
+    // clears the GEMM's stream-K flags
+    SkinnySpec su{x, M, w->k, Major::K, A, r, w->k, Major::K, r, u_out, u_s, scale, 0};
+    if (keep) {
+        su.mask_mode = 1;
+        su.keep = keep;
+        su.mx = M;
+        su.kx = w->k;
+    }
+    st = skinny_launch(KK_LORA_U, &su, 1, s, sk.flags, sk.pairs_max * kSkFlagsPerPair);
     if (st != NF4_OK) return st;
     return launch_gemm_auto<false>(w, x, M, w->k, w->n, u_s, r, B, h, s, &sk);
+}
+
+nf4_status qlora_linear_fwd(const nf4_weight *w, const uint16_t *x, int64_t M, const uint16_t *A,
+                            const uint16_t *B, int32_t r, float alpha, uint16_t *h, float *u_out,
+                            void *workspace, size_t ws_bytes, void *stream) {
+    return fwd_impl(w, x, M, A, B, r, alpha, 0.0f, nullptr, h, u_out, workspace, ws_bytes, stream);
+}
+
+nf4_status qlora_linear_fwd_dropout(const nf4_weight *w, const uint16_t *x, int64_t M,
+                                    const uint16_t *A, const uint16_t *B, int32_t r, float alpha,
+                                    float p, const uint8_t *keep, uint16_t *h, float *u_out,
+                                    void *workspace, size_t ws_bytes, void *stream) {
+    if (!keep) return NF4_ERR_INVALID_ARG;
+    return fwd_impl(w, x, M, A, B, r, alpha, p, keep, h, u_out, workspace, ws_bytes, stream);
 }
 
 nf4_status qlora_multi_lora_fwd(const nf4_weight *w, const uint16_t *x, int64_t M,
@@ -1025,14 +1078,55 @@ size_t qlora_bwd_workspace_bytes(int64_t M, int64_t n, int64_t k, int32_t r) {
     return bwd_layout(std::max<int64_t>(M, 1), r, num_sms(current_device())).total;
 }
 
-nf4_status qlora_linear_bwd(const nf4_weight *w, const uint16_t *x, int64_t M, const uint16_t *A,
-                            const uint16_t *B, int32_t r, float alpha, const uint16_t *dY,
-                            const float *u, uint16_t *dX, uint16_t *dA, uint16_t *dB,
-                            void *workspace, size_t ws_bytes, void *stream) {
+// dX += keep . (Vs A) on the tensor cores (the adapter part of dX under dropout).
+nf4_status lora_add(const float *base, const uint16_t *Vs, const uint16_t *A, const uint8_t *keep,
+                    int64_t M, int64_t K, int32_t r, uint16_t *dX, cudaStream_t s) {
+    LoraAddArgs a{};
+    a.base = base;
+    a.M = M;
+    a.K = K;
+    a.r = r;
+    a.rp = (r + 15) / 16 * 16;
+    a.Vs = Vs;
+    a.A = A;
+    a.keep = keep;
+    a.dX = dX;
+    if ((M + kMgRows - 1) / kMgRows > 65535) return NF4_ERR_UNSUPPORTED_SHAPE;
+    const dim3 grid(static_cast<unsigned>((K + kMgCols - 1) / kMgCols), static_cast<unsigned>((M + kMgRows - 1) / kMgRows));
+    const int smem = lora_add_smem_bytes(a.rp);
+    void (*kern)(const LoraAddArgs) = nullptr;
+    switch (a.rp / 16) {
+        case 1: kern = qlora_lora_add_kernel<1>; break;
+        case 2: kern = qlora_lora_add_kernel<2>; break;
+        case 3: kern = qlora_lora_add_kernel<3>; break;
+        case 4: kern = qlora_lora_add_kernel<4>; break;
+        case 5: kern = qlora_lora_add_kernel<5>; break;
+        case 6: kern = qlora_lora_add_kernel<6>; break;
+        case 7: kern = qlora_lora_add_kernel<7>; break;
+        case 8: kern = qlora_lora_add_kernel<8>; break;
+        default: return NF4_ERR_UNSUPPORTED_SHAPE;
+    }
+    NF4_TRY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    LaunchTimer t(KK_LORA_ADD, s);
+    const cudaError_t e = launch_ex(kern, grid, dim3(kMgThreads), static_cast<size_t>(smem), s, 0u, a);
+    t.stop();
+    if (e != cudaSuccess) return NF4_ERR_CUDA;
+    NF4_TRY_CUDA(cudaGetLastError());
+    return NF4_OK;
+}
+
+// Backward, with LoRA dropout when keep is non-null (u, when given, is the
+// forward's masked u = (keep . x) A^T).
+nf4_status bwd_impl(const nf4_weight *w, const uint16_t *x, int64_t M, const uint16_t *A,
+                    const uint16_t *B, int32_t r, float alpha, float p, const uint8_t *keep,
+                    const uint16_t *dY, const float *u, uint16_t *dX, uint16_t *dA, uint16_t *dB,
+                    void *workspace, size_t ws_bytes, void *stream) {
     nf4_status st = check_layer(w, x, M, A, B, r, alpha);
     if (st != NF4_OK) return st;
+    if (keep && !(p >= 0.0f && p < 1.0f)) return NF4_ERR_INVALID_ARG;
     if (!dA || !dB || (M > 0 && !dY)) return NF4_ERR_INVALID_ARG;
-    if (!aligned16(dY) || !aligned16(u) || !aligned16(dX) || !aligned16(dA) || !aligned16(dB))
+    if (!aligned16(dY) || !aligned16(u) || !aligned16(dX) || !aligned16(dA) || !aligned16(dB) ||
+        !aligned16(keep))
         return NF4_ERR_ALIGNMENT;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int64_t N = w->n, K = w->k;
@@ -1048,19 +1142,30 @@ nf4_status qlora_linear_bwd(const nf4_weight *w, const uint16_t *x, int64_t M, c
     }
     const int sms = num_sms(current_device());
     const BwdLayout L = bwd_layout(M, r, sms);
-    if (!workspace || ws_bytes < L.total) return NF4_ERR_WORKSPACE;
+    // under dropout the workspace also holds dY W~ in fp32 ([M, k]) for the masked add
+    const size_t need = keep ? L.total + align256(size_t(M) * size_t(K) * 4) : L.total;
+    if (!workspace || ws_bytes < need) return NF4_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return NF4_ERR_ALIGNMENT;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     uint16_t *u_s = reinterpret_cast<uint16_t *>(ws + L.us);
     uint16_t *v_s = reinterpret_cast<uint16_t *>(ws + L.vs);
+    float *base32 = reinterpret_cast<float *>(ws + L.total);
     const SkBuf sk{reinterpret_cast<float *>(ws + L.partial), reinterpret_cast<int *>(ws + L.flags),
                    sk_pairs_max(sms)};
-    const float scale = alpha / static_cast<float>(r);
+    float scale = alpha / static_cast<float>(r);
+    if (keep) scale = scale / (1.0f - p);
 
-    // bf16(s u): recomputed from x here, or converted from the saved u by the v launch
+    // bf16(s u): recomputed from x here (masked under dropout), or converted from
+    // the saved u by the v launch
     if (!u) {
-        st = skinny_product(KK_LORA_U, x, M, K, Major::K, A, r, K, Major::K, r, nullptr, u_s,
-                            scale, 0, s);
+        SkinnySpec su{x, M, K, Major::K, A, r, K, Major::K, r, nullptr, u_s, scale, 0};
+        if (keep) {
+            su.mask_mode = 1;
+            su.keep = keep;
+            su.mx = M;
+            su.kx = K;
+        }
+        st = skinny_launch(KK_LORA_U, &su, 1, s);
         if (st != NF4_OK) return st;
     }
     // v = dY B  ->  bf16(s v)
@@ -1069,17 +1174,50 @@ nf4_status qlora_linear_bwd(const nf4_weight *w, const uint16_t *x, int64_t M, c
         st = skinny_launch(KK_LORA_V, &sv, 1, s, nullptr, 0, u, u ? u_s : nullptr, u ? M * r : 0, scale);
         if (st != NF4_OK) return st;
     }
-    // dB = dY^T bf16(s u) ([N, r]) and dA = (x^T bf16(s v))^T ([r, K]) in one launch,
-    // which also clears the dgrad GEMM's stream-K flags
+    // dB = dY^T bf16(s u) ([N, r]) and dA = (x^T bf16(s v))^T ([r, K]) in one launch (under
+    // dropout dA takes the masked x), which also clears the dgrad GEMM's stream-K flags
     {
-        const SkinnySpec j[2] = {{dY, M, N, Major::MN, u_s, M, r, Major::MN, r, nullptr, dB, 1.0f, 0},
-                                 {x, M, K, Major::MN, v_s, M, r, Major::MN, r, nullptr, dA, 1.0f, 1}};
+        SkinnySpec j[2] = {{dY, M, N, Major::MN, u_s, M, r, Major::MN, r, nullptr, dB, 1.0f, 0},
+                           {x, M, K, Major::MN, v_s, M, r, Major::MN, r, nullptr, dA, 1.0f, 1}};
+        if (keep) {
+            j[1].mask_mode = 2;
+            j[1].keep = keep;
+            j[1].mx = M;
+            j[1].kx = K;
+        }
         st = skinny_launch(KK_LORA_DBDA, j, 2, s, sk.flags, sk.pairs_max * kSkFlagsPerPair);
         if (st != NF4_OK) return st;
     }
-    // dX = dY W~ + bf16(s v) A
-    if (dX) return launch_gemm_auto<true>(w, dY, M, N, K, v_s, r, A, dX, s, &sk);
-    return NF4_OK;
+    if (!dX) return NF4_OK;
+    // dX = dY W~ + bf16(s v) A; under dropout the adapter part is masked
+    // element-wise, so it is added by its own kernel after the GEMM
+    if (!keep) return launch_gemm_auto<true>(w, dY, M, N, K, v_s, r, A, dX, s, &sk);
+    st = launch_gemm_auto<true>(w, dY, M, N, K, nullptr, r, A, dX, s, &sk, base32);
+    if (st != NF4_OK) return st;
+    return lora_add(base32, v_s, A, keep, M, K, r, dX, s);
+}
+
+nf4_status qlora_linear_bwd(const nf4_weight *w, const uint16_t *x, int64_t M, const uint16_t *A,
+                            const uint16_t *B, int32_t r, float alpha, const uint16_t *dY,
+                            const float *u, uint16_t *dX, uint16_t *dA, uint16_t *dB,
+                            void *workspace, size_t ws_bytes, void *stream) {
+    return bwd_impl(w, x, M, A, B, r, alpha, 0.0f, nullptr, dY, u, dX, dA, dB, workspace, ws_bytes,
+                    stream);
+}
+
+size_t qlora_bwd_dropout_workspace_bytes(int64_t M, int64_t n, int64_t k, int32_t r) {
+    if (M < 0 || n <= 0 || k <= 0 || r <= 0) return 256;
+    return bwd_layout(std::max<int64_t>(M, 1), r, num_sms(current_device())).total +
+           align256(size_t(std::max<int64_t>(M, 1)) * size_t(k) * 4);
+}
+
+nf4_status qlora_linear_bwd_dropout(const nf4_weight *w, const uint16_t *x, int64_t M,
+                                    const uint16_t *A, const uint16_t *B, int32_t r, float alpha,
+                                    float p, const uint8_t *keep, const uint16_t *dY, const float *u,
+                                    uint16_t *dX, uint16_t *dA, uint16_t *dB, void *workspace,
+                                    size_t ws_bytes, void *stream) {
+    if (!keep) return NF4_ERR_INVALID_ARG;
+    return bwd_impl(w, x, M, A, B, r, alpha, p, keep, dY, u, dX, dA, dB, workspace, ws_bytes, stream);
 }
 
 }  // extern "C"

@@ -39,6 +39,13 @@ struct SkinnyJob {
     uint16_t *out_bf16;  // bf16(scale * sum): [P][r], or [r][P] when transposed; or null
     float scale;
     int transposed;
+    // dropout on x as the A operand (LoRA dropout: the keep mask is an input,
+    // bit (e & 7) of byte e >> 3 for element e = m * kx + k of x [mx, kx]):
+    // 0 = none, 1 = A is x K-major (tile rows are tokens), 2 = A is x
+    // MN-major (tile rows are tokens of two 64-column halves)
+    int mask_mode;
+    const uint8_t *keep;
+    int64_t mx, kx;
 };
 
 struct SkinnyArgs {
@@ -95,7 +102,8 @@ skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a0,
     float *part = reinterpret_cast<float *>(smem);   // [128][kPartStride], after the main loop
     uint64_t *bars = reinterpret_cast<uint64_t *>(slot_b + kSkStages * Cfg::kBBytes);
     uint64_t *full = bars, *empty = bars + kSkStages, *done_bar = bars + 2 * kSkStages;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done_bar + 1);
+    uint64_t *masked = done_bar + 1;            // [stages] dropout applied to the A tile
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(masked + kSkStages);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -113,6 +121,7 @@ skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a0,
         for (int s = 0; s < kSkStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
+            mbar_init(&masked[s], 2);
         }
         mbar_init(done_bar, 1);
         *abort_flag = 0;
@@ -170,7 +179,7 @@ skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a0,
         for (int it = 0; it < nsteps; ++it) {
             const int st = it % kSkStages;
             const uint32_t ph = (it / kSkStages) & 1;
-            if (!mbar_wait(&full[st], ph, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(J.mask_mode ? &masked[st] : &full[st], ph, abort_flag)) { ok = false; break; }
             tc_fence_after();
             const uint32_t aa = a_base + st * Cfg::kABytes, bb = b_base + st * Cfg::kBBytes;
 #pragma unroll
@@ -184,6 +193,39 @@ skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a0,
             umma_commit(&empty[st]);
         }
         if (ok) umma_commit(done_bar);
+    } else if ((warp == 2 || warp == 3) && J.mask_mode) {
+        // dropout: zero the dropped elements of each landed A tile in place.
+        // The tile is 128 rows of 128 bytes (64 consecutive k of one token,
+        // 128-byte swizzle); a 16-byte piece holds 8 k, i.e. one keep byte.
+        const int t64 = threadIdx.x - 64;
+        for (int it = 0; it < nsteps; ++it) {
+            const int st = it % kSkStages;
+            const uint32_t ph = (it / kSkStages) & 1;
+            if (!mbar_wait(&full[st], ph, abort_flag)) break;
+            uint8_t *a = slot_a + st * Cfg::kABytes;
+            const int q0 = (s0 + it) * 64;
+#pragma unroll 4
+            for (int pc = t64; pc < 128 * 8; pc += 64) {
+                const int row = pc >> 3, c = pc & 7;
+                const int64_t m = J.mask_mode == 1 ? p0 + row : q0 + (row & 63);
+                const int64_t k0 = (J.mask_mode == 1 ? q0 : p0 + 64 * (row >> 6)) + 8 * c;
+                uint4 *piece = reinterpret_cast<uint4 *>(a + row * 128 + ((c ^ (row & 7)) << 4));
+                if (m < J.mx && k0 < J.kx) {
+                    const uint32_t kb = J.keep[(m * J.kx + k0) >> 3];
+                    uint4 v = *piece;
+                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                    uint32_t o[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        o[e] = w[e] & (((kb >> (2 * e)) & 1u ? 0x0000ffffu : 0u) |
+                                       ((kb >> (2 * e + 1)) & 1u ? 0xffff0000u : 0u));
+                    *piece = make_uint4(o[0], o[1], o[2], o[3]);
+                }
+            }
+            fence_proxy_async_smem();     // generic writes before the tensor core reads the tile
+            __syncwarp();
+            if ((threadIdx.x & 31) == 0) mbar_arrive(&masked[st]);
+        }
     } else if (warp >= 4 && warp < 8) {
         // accumulator -> this CTA's partial (the stage buffers are free once
         // the last MMA has completed: every load it waited for has landed)

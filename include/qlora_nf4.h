@@ -166,6 +166,37 @@ QLORA_API nf4_status qlora_linear_fwd_noalloc(const nf4_weight *w, const uint16_
                                               float alpha, uint16_t *h, float *u_out,
                                               void *stream);
 
+/* Forward and backward with LoRA dropout on the adapter input ("QLoRA
+ * Finetuner", section 1: h = W0 x + (alpha/r) B(A(dropout x)); the recipe in
+ * "QLoRA explained" uses lora_dropout = 0.05). The random draw is an input:
+ * keep is a DEVICE bit mask over x, (M * k) / 8 bytes, where bit (e & 7) of
+ * byte e >> 3 keeps element e = m * k + kk of x (1 = kept, 0 = dropped).
+ * Inverted dropout with 0 <= p < 1: the kept elements are scaled by 1/(1-p),
+ * applied to the adapter branch as a whole, so
+ *     u  = (keep . x) A^T            (u_out receives this, without 1/(1-p))
+ *     h  = x W~^T + s' u B^T,        s' = (alpha/r)/(1-p), s' u rounded to bf16
+ *     dX = dY W~ + keep . (bf16(s' v) A),   v = dY B
+ *     dA = bf16(s' v)^T (keep . x),  dB = dY^T bf16(s' u)
+ * The base product uses x unmasked. In the backward, u (if given) must be the
+ * forward's u_out for the same mask; dY W~ is kept in fp32 in the workspace and
+ * the masked adapter part added to it before the one rounding to bf16, so the
+ * backward's workspace is qlora_bwd_dropout_workspace_bytes (M * k * 4 bytes
+ * more than qlora_bwd_workspace_bytes). Otherwise as qlora_linear_fwd /
+ * qlora_linear_bwd; a null keep or p outside [0, 1) returns
+ * NF4_ERR_INVALID_ARG. */
+QLORA_API nf4_status qlora_linear_fwd_dropout(const nf4_weight *w, const uint16_t *x, int64_t M,
+                                              const uint16_t *A, const uint16_t *B, int32_t r,
+                                              float alpha, float p, const uint8_t *keep,
+                                              uint16_t *h, float *u_out, void *workspace,
+                                              size_t ws_bytes, void *stream);
+QLORA_API size_t qlora_bwd_dropout_workspace_bytes(int64_t M, int64_t n, int64_t k, int32_t r);
+QLORA_API nf4_status qlora_linear_bwd_dropout(const nf4_weight *w, const uint16_t *x, int64_t M,
+                                              const uint16_t *A, const uint16_t *B, int32_t r,
+                                              float alpha, float p, const uint8_t *keep,
+                                              const uint16_t *dY, const float *u, uint16_t *dX,
+                                              uint16_t *dA, uint16_t *dB, void *workspace,
+                                              size_t ws_bytes, void *stream);
+
 /* Forward of one NF4 base with several adapters, one chosen per token, as a
  * server keeps one quantised base resident and applies each request's own
  * adapter ("Parameter-Efficient Fine-Tuning: From LoRA to QLoRA", "The PEFT

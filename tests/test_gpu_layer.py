@@ -296,3 +296,85 @@ def test_multi_adapter_single_adapter_equals_layer_forward(q):
     h1 = q.qlora_multi_lora_fwd(qw, x.cuda(), A.cuda(), B.cuda(), r, [16.0], idx)
     h2, _ = q.qlora_linear_fwd(qw, x.cuda(), A.cuda(), B.cuda(), 16.0)
     assert torch.equal(h1, h2)
+
+
+# ---------------------------------------------------------------- dropout --
+DROPOUT_SHAPES = [
+    # (N, K, M, r, p, dq)   GEMM path with ragged tiles, and the decode path (M <= 16)
+    (384, 512, 300, 16, 0.05, True),
+    (520, 640, 77, 64, 0.3, False),
+    (264, 512, 12, 16, 0.1, True),
+]
+
+
+def dropout_run(q, N, K, M, r, p, dq, seed, zero_w=False):
+    w = workloads.LayerWorkload("t", N, K, M, r, 32.0, 0.02, dq, seed)
+    inp = workloads.make_inputs(w)
+    W0 = torch.zeros(N, K) if zero_w else inp["W0"]
+    keep_bool = torch.from_numpy(np.random.default_rng(seed).random((M, K)) >= p)
+    keep = q.pack_keep(keep_bool.cuda())
+    qw = q.nf4_quantize(W0.cuda(), double_quant=dq)
+    x, A, B, dY = (inp[k].cuda() for k in ("x", "A", "B", "dY"))
+    h, u = q.qlora_linear_fwd_dropout(qw, x, A, B, w.alpha, p, keep)
+    dX, dA, dB = q.qlora_linear_bwd_dropout(qw, x, A, B, w.alpha, p, keep, dY, u=u)
+    torch.cuda.synchronize()
+    assert q.device_status() == q.NF4_OK
+    ow = oracle_weight(qw)
+    kb = oracle.pack_keep(keep_bool.numpy())
+    h_ref, u_ref = oracle.qlora_fwd_rows_dropout(ow, N, K, bits(inp["x"]), bits(inp["A"]), bits(inp["B"]),
+                                                 r, w.alpha, p, kb)
+    g_ref = oracle.qlora_bwd_dropout(ow, N, K, bits(inp["x"]), bits(inp["A"]), bits(inp["B"]), r,
+                                     w.alpha, p, kb, bits(inp["dY"]))
+    return (h, u, dX, dA, dB), (h_ref, u_ref) + tuple(g_ref)
+
+
+@pytest.mark.parametrize("N,K,M,r,p,dq", DROPOUT_SHAPES)
+@pytest.mark.parametrize("zero_w", [False, True])
+def test_dropout_forward_backward(q, N, K, M, r, p, dq, zero_w):
+    """With W0 = 0 the outputs are the masked adapter terms alone (h, dX), against their own rms."""
+    got, ref = dropout_run(q, N, K, M, r, p, dq, 321 + N + M, zero_w)
+    names = ("h", "u", "dX", "dA", "dB")
+    errs = {}
+    for name, g, rf in zip(names, got, ref):
+        gv = g.detach().float().cpu().numpy().astype(np.float64)
+        errs[name] = rel_err(gv, np.asarray(rf), M < 16 or zero_w)
+    bad = {k: v for k, v in errs.items() if not v <= TOL}
+    assert not bad, errs
+
+
+def test_dropout_keep_all_forward_is_the_plain_forward(q):
+    N, K, M, r = 384, 512, 200, 16
+    w = workloads.LayerWorkload("t", N, K, M, r, 32.0, 0.02, True, 999)
+    inp = workloads.make_inputs(w)
+    qw = q.nf4_quantize(inp["W0"].cuda(), double_quant=True)
+    x, A, B = (inp[k].cuda() for k in ("x", "A", "B"))
+    keep = q.pack_keep(torch.ones(M, K, dtype=torch.bool, device="cuda"))
+    h1, u1 = q.qlora_linear_fwd_dropout(qw, x, A, B, w.alpha, 0.0, keep)
+    h2, u2 = q.qlora_linear_fwd(qw, x, A, B, w.alpha)
+    assert torch.equal(h1, h2) and torch.equal(u1, u2)
+
+
+def test_dropout_full_size_attention_projection(q):
+    """The LLaMA-13B-like projection with p = 0.05 (the pages' recipe): sampled rows
+    of h and dX, all of dA and dB."""
+    wl = workloads.WORKLOADS["llama13b_attn_5120"]
+    N, K, M, r, p = wl.N, wl.K, wl.M, wl.r, 0.05
+    inp = workloads.make_inputs(wl)
+    keep_bool = torch.from_numpy(np.random.default_rng(5).random((M, K)) >= p)
+    keep = q.pack_keep(keep_bool.cuda())
+    qw = q.nf4_quantize(inp["W0"].cuda(), double_quant=True)
+    x, A, B, dY = (inp[k].cuda() for k in ("x", "A", "B", "dY"))
+    h, u = q.qlora_linear_fwd_dropout(qw, x, A, B, wl.alpha, p, keep)
+    dX, dA, dB = q.qlora_linear_bwd_dropout(qw, x, A, B, wl.alpha, p, keep, dY, u=u)
+    torch.cuda.synchronize()
+    rows = sampled_rows(M, 32, 11)
+    ow = oracle_weight(qw)
+    kb = oracle.pack_keep(keep_bool.numpy())
+    h_ref, _ = oracle.qlora_fwd_rows_dropout(ow, N, K, bits(inp["x"]), bits(inp["A"]), bits(inp["B"]),
+                                             r, wl.alpha, p, kb, rows=rows)
+    dX_ref, dA_ref, dB_ref = oracle.qlora_bwd_dropout(ow, N, K, bits(inp["x"]), bits(inp["A"]),
+                                                      bits(inp["B"]), r, wl.alpha, p, kb,
+                                                      bits(inp["dY"]), dx_rows=rows)
+    errs = {"h": rel_err(to_f64(h)[rows], h_ref), "dX": rel_err(to_f64(dX)[rows], dX_ref),
+            "dA": rel_err(to_f64(dA), dA_ref), "dB": rel_err(to_f64(dB), dB_ref)}
+    assert all(v <= TOL for v in errs.values()), errs
