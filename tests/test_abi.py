@@ -114,3 +114,66 @@ def test_python_binding_refuses_cpu_tensors(q):
     W = torch.zeros(64, 64)
     with pytest.raises(ValueError):
         q.nf4_quantize(W)
+
+
+def test_typed_quantize_and_merge_argument_checks(q):
+    L = q.lib
+    w = weight(q)
+    assert L.nf4_quantize_typed(FAKE, 3, ctypes.byref(w), None) == q.NF4_ERR_INVALID_ARG
+    assert L.nf4_quantize_typed(FAKE, -1, ctypes.byref(w), None) == q.NF4_ERR_INVALID_ARG
+    assert L.nf4_quantize_typed(FAKE + 2, 1, ctypes.byref(w), None) == q.NF4_ERR_ALIGNMENT
+    assert L.nf4_quantize_typed(None, 2, ctypes.byref(w), None) == q.NF4_ERR_INVALID_ARG
+    merge = lambda **kw: L.qlora_merge(ctypes.byref(kw.get("w", w)), kw.get("A", FAKE), kw.get("B", FAKE),
+                                       kw.get("r", 8), kw.get("alpha", 16.0), kw.get("out", FAKE),
+                                       kw.get("bf16", 1), None)
+    assert merge(r=12) == q.NF4_ERR_UNSUPPORTED_SHAPE
+    assert merge(r=136) == q.NF4_ERR_UNSUPPORTED_SHAPE
+    assert merge(alpha=float("nan")) == q.NF4_ERR_INVALID_ARG
+    assert merge(bf16=2) == q.NF4_ERR_INVALID_ARG
+    assert merge(out=None) == q.NF4_ERR_INVALID_ARG
+    assert merge(A=FAKE + 8) == q.NF4_ERR_ALIGNMENT
+    assert merge(w=weight(q, block=128)) == q.NF4_ERR_INVALID_ARG
+
+
+def test_multi_adapter_and_dropout_argument_checks(q):
+    L = q.lib
+    w = weight(q)
+    al = (ctypes.c_float * 16)(*([16.0] * 16))
+
+    def multi(**kw):
+        return L.qlora_multi_lora_fwd(ctypes.byref(w), FAKE, kw.get("M", 4), FAKE, FAKE, kw.get("r", 8),
+                                      kw.get("n", 2), kw.get("al", al), kw.get("idx", FAKE),
+                                      kw.get("h", FAKE), kw.get("ws", FAKE), kw.get("wsb", 1 << 30), None)
+    assert multi(n=0) == q.NF4_ERR_INVALID_ARG
+    assert multi(n=17) == q.NF4_ERR_INVALID_ARG
+    assert multi(al=None) == q.NF4_ERR_INVALID_ARG
+    assert multi(r=4) == q.NF4_ERR_UNSUPPORTED_SHAPE           # r % 8
+    assert multi(r=16, n=9) == q.NF4_ERR_UNSUPPORTED_SHAPE     # 144 stacked ranks > 128
+    bad = (ctypes.c_float * 2)(16.0, float("inf"))
+    assert multi(al=bad) == q.NF4_ERR_INVALID_ARG
+    assert multi(idx=None) == q.NF4_ERR_INVALID_ARG
+    assert multi(idx=FAKE + 4) == q.NF4_ERR_ALIGNMENT
+    assert multi(M=0) == q.NF4_OK
+    assert multi(wsb=16) == q.NF4_ERR_WORKSPACE
+
+    def fwd_do(**kw):
+        return L.qlora_linear_fwd_dropout(ctypes.byref(w), FAKE, kw.get("M", 4), FAKE, FAKE, 8, 16.0,
+                                          kw.get("p", 0.05), kw.get("keep", FAKE), FAKE, None,
+                                          FAKE, kw.get("wsb", 1 << 30), None)
+    assert fwd_do(keep=None) == q.NF4_ERR_INVALID_ARG
+    assert fwd_do(p=1.0) == q.NF4_ERR_INVALID_ARG
+    assert fwd_do(p=-0.1) == q.NF4_ERR_INVALID_ARG
+    assert fwd_do(p=float("nan")) == q.NF4_ERR_INVALID_ARG
+    assert fwd_do(keep=FAKE + 1) == q.NF4_ERR_ALIGNMENT
+    assert fwd_do(wsb=16) == q.NF4_ERR_WORKSPACE
+
+    def bwd_do(**kw):
+        return L.qlora_linear_bwd_dropout(ctypes.byref(w), FAKE, 4, FAKE, FAKE, 8, 16.0,
+                                          kw.get("p", 0.05), kw.get("keep", FAKE), FAKE, None, None,
+                                          FAKE, FAKE, FAKE, kw.get("wsb", 16), None)
+    assert bwd_do(keep=None) == q.NF4_ERR_INVALID_ARG
+    assert bwd_do(p=1.5) == q.NF4_ERR_INVALID_ARG
+    # the dropout backward needs M * k * 4 more workspace bytes than the plain one
+    plain = q.bwd_workspace_bytes(4, 64, 64, 8)
+    assert bwd_do(wsb=plain) == q.NF4_ERR_WORKSPACE
+    assert L.qlora_bwd_dropout_workspace_bytes(4, 64, 64, 8) >= plain + 4 * 64 * 4
