@@ -201,9 +201,19 @@ def bf16_to_f64(a: np.ndarray) -> np.ndarray:
 # --------------------------------------------------------------------------
 # layer
 # --------------------------------------------------------------------------
-def _check_layer(qw: Quantized, N: int, K: int):
-    if qw.block != 64 or qw.dq_group != 256 or qw.numel != N * K or K % 64:
-        raise OracleError("layer oracle expects block 64, groups of 256 and K % 64 == 0")
+def _check_layer(qw: Quantized, N: int, K: int) -> Quantized:
+    """The weight as the layer functions read it: 64-element blocks.
+
+    The C layer functions dequantise in 64-element blocks. A 128-element block
+    is handed to them as its two 64-element halves, each carrying the block's
+    dequantisation scale (s, or its double-quant image) as a plain fp32
+    absmax: every element then dequantises to the same fl32(scale * NF4[q])."""
+    if qw.block not in (64, 128) or qw.dq_group != 256 or qw.numel != N * K or K % qw.block:
+        raise OracleError("layer oracle expects blocks of 64 or 128, groups of 256 and K % block == 0")
+    if qw.block == 64:
+        return qw
+    halves = np.repeat(block_scales(qw), qw.block // 64).astype(np.float32)
+    return Quantized(qw.codes, halves, None, None, 64, False, 256, qw.numel)
 
 
 def qlora_fwd_rows(qw: Quantized, N: int, K: int, x: np.ndarray, A: np.ndarray, B: np.ndarray,
@@ -212,7 +222,7 @@ def qlora_fwd_rows(qw: Quantized, N: int, K: int, x: np.ndarray, A: np.ndarray, 
 
     x: uint16 [M, K] bf16 bits; A: uint16 [r, K]; B: uint16 [N, r].
     rows: token indices to compute (default: all)."""
-    _check_layer(qw, N, K)
+    qw = _check_layer(qw, N, K)
     x = np.ascontiguousarray(x, dtype=np.uint16)
     A = np.ascontiguousarray(A, dtype=np.uint16)
     B = np.ascontiguousarray(B, dtype=np.uint16)
@@ -236,7 +246,7 @@ def qlora_bwd(qw: Quantized, N: int, K: int, x: np.ndarray, A: np.ndarray, B: np
 
     dY: uint16 [M, N] bf16 bits. dx_rows: token rows of dX to compute
     (default: all; an empty list skips dX)."""
-    _check_layer(qw, N, K)
+    qw = _check_layer(qw, N, K)
     x = np.ascontiguousarray(x, dtype=np.uint16)
     A = np.ascontiguousarray(A, dtype=np.uint16)
     B = np.ascontiguousarray(B, dtype=np.uint16)
@@ -262,7 +272,7 @@ def qlora_merge(qw: Quantized, N: int, K: int, A: np.ndarray, B: np.ndarray, r: 
     (fp32) base weight, as for inference without adapters.
 
     A: uint16 [r, K] bf16 bits; B: uint16 [N, r]."""
-    _check_layer(qw, N, K)
+    qw = _check_layer(qw, N, K)
     A = np.ascontiguousarray(A, dtype=np.uint16)
     B = np.ascontiguousarray(B, dtype=np.uint16)
     assert A.shape == (r, K) and B.shape == (N, r)
@@ -282,7 +292,7 @@ def qlora_multi_fwd_rows(qw: Quantized, N: int, K: int, x: np.ndarray, A_all: np
 
     A_all: uint16 [n_ad * r, K] (stacked A_a); B_all: uint16 [N, n_ad * r] (stacked B_a);
     adapter: int32 [M]."""
-    _check_layer(qw, N, K)
+    qw = _check_layer(qw, N, K)
     x = np.ascontiguousarray(x, dtype=np.uint16)
     A_all = np.ascontiguousarray(A_all, dtype=np.uint16)
     B_all = np.ascontiguousarray(B_all, dtype=np.uint16)
@@ -310,7 +320,7 @@ def qlora_fwd_rows_dropout(qw: Quantized, N: int, K: int, x: np.ndarray, A: np.n
     u = (keep . x) A^T, h = x W~^T + (alpha/r)/(1-p) u B^T.
 
     keep: uint8 bit mask over x, bit (e & 7) of byte e >> 3 for e = m K + k (1 = kept)."""
-    _check_layer(qw, N, K)
+    qw = _check_layer(qw, N, K)
     x = np.ascontiguousarray(x, dtype=np.uint16)
     A = np.ascontiguousarray(A, dtype=np.uint16)
     B = np.ascontiguousarray(B, dtype=np.uint16)
@@ -333,7 +343,7 @@ def qlora_bwd_dropout(qw: Quantized, N: int, K: int, x: np.ndarray, A: np.ndarra
                       r: int, alpha: float, p: float, keep: np.ndarray, dY: np.ndarray,
                       dx_rows: Optional[Sequence[int]] = None):
     """(dX rows, dA, dB) in fp64 with dropout on the LoRA input (same mask convention)."""
-    _check_layer(qw, N, K)
+    qw = _check_layer(qw, N, K)
     x = np.ascontiguousarray(x, dtype=np.uint16)
     A = np.ascontiguousarray(A, dtype=np.uint16)
     B = np.ascontiguousarray(B, dtype=np.uint16)

@@ -143,7 +143,7 @@ def brute_quantize(W: np.ndarray, block: int):
     return np.array(packed, dtype=np.uint8), np.array(scales, dtype=np.float32)
 
 
-@pytest.mark.parametrize("block", [2, 4, 6, 64])
+@pytest.mark.parametrize("block", [2, 4, 6, 64, 128])
 def test_quantize_brute_force_tiny(block):
     rng = np.random.default_rng(block)
     W = rng.normal(0, 0.02, size=block * 12).astype(np.float32)
@@ -182,14 +182,15 @@ def test_rejects_nonfinite_and_bad_blocks():
         oracle.quantize(np.zeros(63, dtype=np.float32), block=63)
 
 
-def test_dequant_of_quant_is_exact_on_codebook_multiples():
+@pytest.mark.parametrize("block", [64, 128])
+def test_dequant_of_quant_is_exact_on_codebook_multiples(block):
     rng = np.random.default_rng(3)
     for _ in range(50):
         c = np.float32(rng.uniform(1e-3, 10.0))
-        js = rng.integers(0, 16, size=64)
-        js[rng.integers(0, 64)] = 15                    # absmax = c * 1 = c
+        js = rng.integers(0, 16, size=block)
+        js[rng.integers(0, block)] = 15                 # absmax = c * 1 = c
         W = (c * LEVELS[js]).astype(np.float32)         # fl32(c * c_j)
-        q = oracle.quantize(W)
+        q = oracle.quantize(W, block=block)
         assert q.absmax[0] == c
         got = []
         for b in q.codes:
@@ -198,13 +199,14 @@ def test_dequant_of_quant_is_exact_on_codebook_multiples():
         assert np.array_equal(oracle.dequantize(q), W)
 
 
-def test_roundtrip_error_bound():
+@pytest.mark.parametrize("block", [64, 128])
+def test_roundtrip_error_bound(block):
     rng = np.random.default_rng(11)
-    W = rng.normal(0, 0.02, size=64 * 500).astype(np.float32)
-    q = oracle.quantize(W)
+    W = rng.normal(0, 0.02, size=128 * 250).astype(np.float32)
+    q = oracle.quantize(W, block=block)
     wt = oracle.dequantize(q).astype(np.float64)
     half_gap = np.max(np.diff(LEVELS.astype(np.float64))) / 2     # 0.1519...
-    s = np.repeat(q.absmax.astype(np.float64), 64)
+    s = np.repeat(q.absmax.astype(np.float64), block)
     err = np.abs(W.astype(np.float64) - wt)
     assert np.all(err <= s * half_gap * (1 + 1e-6))
     # NF4 error is far below the half-gap bound on average for normal data

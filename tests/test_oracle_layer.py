@@ -16,9 +16,9 @@ def dyadic_bf16(rng, shape, scale_pow=2):
     return oracle.f32_to_bf16(vals)
 
 
-def random_layer(rng, N, K, M, r, dq, sigma=0.02):
+def random_layer(rng, N, K, M, r, dq, sigma=0.02, block=64):
     W = rng.normal(0, sigma, size=(N, K)).astype(np.float32)
-    qw = oracle.quantize(W.reshape(-1), dq=dq)
+    qw = oracle.quantize(W.reshape(-1), block=block, dq=dq)
     x = oracle.f32_to_bf16(rng.normal(size=(M, K)).astype(np.float32))
     A = oracle.f32_to_bf16(rng.uniform(-K ** -0.5, K ** -0.5, size=(r, K)).astype(np.float32))
     B = oracle.f32_to_bf16(rng.normal(0, 0.01, size=(N, r)).astype(np.float32))
@@ -35,11 +35,12 @@ def f64(a):
     return oracle.bf16_to_f64(a)
 
 
+@pytest.mark.parametrize("block", [64, 128])
 @pytest.mark.parametrize("dq", [False, True])
-def test_forward_equals_merged_weight(dq):
+def test_forward_equals_merged_weight(dq, block):
     rng = np.random.default_rng(21)
-    N, K, M, r, alpha = 96, 192, 7, 8, 16.0
-    qw, x, A, B, _ = random_layer(rng, N, K, M, r, dq)
+    N, K, M, r, alpha = 96, 256, 7, 8, 16.0
+    qw, x, A, B, _ = random_layer(rng, N, K, M, r, dq, block=block)
     h, u = oracle.qlora_fwd_rows(qw, N, K, x, A, B, r, alpha)
     s = alpha / r
     merged = operand(qw, N, K) + s * f64(B) @ f64(A)        # W~ + (alpha/r) B A
@@ -112,11 +113,12 @@ def test_backward_equals_exact_central_differences():
     assert np.abs(dX).max() > 0 and np.abs(dA).max() > 0 and np.abs(dB).max() > 0
 
 
+@pytest.mark.parametrize("block", [64, 128])
 @pytest.mark.parametrize("dq", [False, True])
-def test_backward_matches_fp64_autograd(dq):
+def test_backward_matches_fp64_autograd(dq, block):
     rng = np.random.default_rng(25)
     N, K, M, r, alpha = 48, 128, 9, 8, 16.0
-    qw, x, A, B, dY = random_layer(rng, N, K, M, r, dq)
+    qw, x, A, B, dY = random_layer(rng, N, K, M, r, dq, block=block)
     dX, dA, dB = oracle.qlora_bwd(qw, N, K, x, A, B, r, alpha, dY)
     Wt = torch.from_numpy(operand(qw, N, K))
     xt = torch.from_numpy(f64(x)).requires_grad_(True)
@@ -258,3 +260,27 @@ def test_dropout_is_the_masked_input_with_rescaled_alpha():
     assert np.allclose(dX, dX0 + np.where(keep_bool, dXm - dX0, 0.0), rtol=1e-12, atol=1e-14)
     # the mask matters: without it every output moves
     assert not np.allclose(dA, oracle.qlora_bwd(qw, N, K, x, A, B, r, a2, dY)[1], rtol=1e-3)
+
+
+def test_block128_with_equal_half_maxima_is_the_64_block_layer():
+    """A 128-element block whose two halves have the same absmax quantises to
+    the codes of two 64-element blocks with that scale; every layer result is
+    then that of the 64-block weight, bit for bit."""
+    rng = np.random.default_rng(41)
+    N, K, M, r, alpha = 40, 384, 6, 8, 16.0
+    W = np.clip(rng.normal(0, 0.02, size=(N, K)), -0.05, 0.05).astype(np.float32)
+    W[:, 0::128] = 0.08
+    W[:, 64::128] = -0.08
+    q128 = oracle.quantize(W.reshape(-1), block=128)
+    q64 = oracle.quantize(W.reshape(-1), block=64)
+    assert np.array_equal(q128.codes, q64.codes)
+    assert np.array_equal(np.repeat(q128.absmax, 2), q64.absmax)
+    _, x, A, B, dY = random_layer(rng, N, K, M, r, False)
+    h128, u128 = oracle.qlora_fwd_rows(q128, N, K, x, A, B, r, alpha)
+    h64, u64 = oracle.qlora_fwd_rows(q64, N, K, x, A, B, r, alpha)
+    assert np.array_equal(h128, h64) and np.array_equal(u128, u64)
+    for g128, g64 in zip(oracle.qlora_bwd(q128, N, K, x, A, B, r, alpha, dY),
+                         oracle.qlora_bwd(q64, N, K, x, A, B, r, alpha, dY)):
+        assert np.array_equal(g128, g64)
+    assert np.array_equal(oracle.qlora_merge(q128, N, K, A, B, r, alpha),
+                          oracle.qlora_merge(q64, N, K, A, B, r, alpha))
