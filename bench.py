@@ -37,7 +37,7 @@ METRIC = "QLoRA linear fwd+bwd TFLOP/s (large M) & NF4 weight GB/s (decode) vs r
 # DRAM bytes (read + write) per launch of the fused GEMM on this workload, mean of the forward and
 # dgrad launches, from one ncu capture of the kernels as they are now (summary and command under
 # profiles/). None whenever the kernel has changed since that capture.
-GEMM_TRAFFIC_BYTES = 44.6e6
+GEMM_TRAFFIC_BYTES = 42.3e6
 MAIN = "llama13b_attn_5120"
 DECODE = "decode_mlp_up_13824x5120"
 QUANT = "llama2_70b_mlp_28672x8192"
@@ -198,7 +198,7 @@ def main():
     ap.add_argument("--skip-extras", action="store_true",
                     help="only the main fwd+bwd line (no decode/quantize/oracle/e2e legs)")
     ap.add_argument("--leg", default="all", choices=["all", "decode", "quantize", "stack", "mlp70b",
-                                                     "merge", "multi"],
+                                                     "merge", "multi", "block128"],
                     help="run one secondary leg alone and print its JSON (for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -219,7 +219,8 @@ def main():
     if args.leg != "all":
         if rank == 0:
             leg = {"decode": decode_leg, "quantize": quantize_leg, "stack": stack_leg,
-                   "mlp70b": mlp70b_leg, "merge": merge_leg, "multi": multi_leg}[args.leg]
+                   "mlp70b": mlp70b_leg, "merge": merge_leg, "multi": multi_leg,
+                   "block128": block128_leg}[args.leg]
             print(json.dumps({"leg": args.leg, **leg(q, dev, load_peaks())}), flush=True)
         return
     if world > 1:
@@ -330,6 +331,7 @@ def main():
         line["stack"] = stack_leg(q, dev, peaks)
         line["merge"] = merge_leg(q, dev, peaks)
         line["multi_adapter"] = multi_leg(q, dev, peaks)
+        line["block128"] = block128_leg(q, dev, peaks)
         line["cpu_baseline"] = cpu_baseline_leg(w, inp)
     elif not args.skip_extras:
         e2e_leg(q, dp, qw, inp, w, args, dev, world)  # same collectives on every rank
@@ -387,20 +389,20 @@ def e2e_leg(q, dp, qw, inp, w, args, dev, world):
             "d2h_bytes_per_step": oh.nbytes + odX.nbytes + ograd.nbytes}
 
 
-def decode_leg(q, dev, peaks):
+def decode_leg(q, dev, peaks, block=64, tokens=(1, 4, 16)):
     """Decode-shaped forward, GB/s counted on the 4-bit code bytes; 8 weight
     copies are rotated so that no call finds its weight in L2. The headline
     per-call time is device time from a CUDA-graph replay of back-to-back
     calls (both kernels of a call, the u partials and the weight stream)."""
     w = workloads.WORKLOADS[DECODE]
     W0 = workloads.make_weight(w).to(dev)
-    copies = [q.nf4_quantize(W0, double_quant=True) for _ in range(8)]
+    copies = [q.nf4_quantize(W0, double_quant=True, block_size=block) for _ in range(8)]
     del W0
     code_bytes = w.N * w.K // 2
-    out = {"workload": f"{DECODE}: W0 {w.N}x{w.K} NF4 double quant (0.1% x20 outliers), "
-                       f"r={w.r}; forward only", "code_bytes": code_bytes,
+    out = {"workload": f"{DECODE}: W0 {w.N}x{w.K} NF4 (blocks of {block}) double quant "
+                       f"(0.1% x20 outliers), r={w.r}; forward only", "code_bytes": code_bytes,
            "peak_gbs": peaks["hbm_gbs"]}
-    for M in (1, 4, 16):
+    for M in tokens:
         inp = workloads.make_inputs(w, M=M, with_dy=False)
         x, A, B = (inp[k].to(dev) for k in ("x", "A", "B"))
         h = torch.empty(M, w.N, dtype=torch.bfloat16, device=dev)
@@ -451,13 +453,13 @@ def decode_leg(q, dev, peaks):
     return out
 
 
-def quantize_leg(q, dev, peaks):
+def quantize_leg(q, dev, peaks, block=64):
     """Full-weight nf4_quantize of the 28672x8192 fp32 weight (double quant)."""
     w = workloads.WORKLOADS[QUANT]
     W0 = workloads.make_weight(w).to(dev)
-    qw = q.nf4_quantize(W0, double_quant=True)
+    qw = q.nf4_quantize(W0, double_quant=True, block_size=block)
     torch.cuda.synchronize()
-    nb = w.N * w.K // 64
+    nb = w.N * w.K // block
     moved = w.N * w.K * 4 + w.N * w.K // 2 + nb * 4 + nb + ((nb + 255) // 256) * 4
     iters = 10
     q.profiling(True)
@@ -484,7 +486,7 @@ def quantize_leg(q, dev, peaks):
     gbs16 = moved16 / (us16 * 1e-6) / 1e9
     del W16, qw
     torch.cuda.empty_cache()
-    return {"workload": f"{QUANT}: W0 {w.N}x{w.K} fp32 -> NF4 + double quant",
+    return {"workload": f"{QUANT}: W0 {w.N}x{w.K} fp32 -> NF4 (blocks of {block}) + double quant",
             "bytes_moved": moved, "kernel_us": us, "gbs": gbs, "frac": gbs / peaks["hbm_gbs"],
             "peak_gbs": peaks["hbm_gbs"],
             "bf16_input": {"bytes_moved": moved16, "kernel_us": us16, "gbs": gbs16,
@@ -568,6 +570,49 @@ def merge_leg(q, dev, peaks):
     del copies
     torch.cuda.empty_cache()
     return out
+
+
+def block128_leg(q, dev, peaks, steps=50):
+    """The main workload's fused forward + backward, the decode forward and the
+    quantiser with 128-element blocks (the pages' other block size): the same
+    kernels with two 64-element steps per scale."""
+    from bit_nf4_quantized_05_b200 import dp
+    w = workloads.WORKLOADS[MAIN]
+    M, N, K, r, alpha = w.M, w.N, w.K, w.r, w.alpha
+    inp = workloads.make_inputs(w)
+    qw = q.nf4_quantize(inp["W0"].to(dev), double_quant=w.double_quant, block_size=128)
+    x, A, B, dY = (inp[k].to(dev) for k in ("x", "A", "B", "dY"))
+    h = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    u = torch.empty(M, r, dtype=torch.float32, device=dev)
+    dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    flat, dA, dB = dp.grad_buffer(r, K, N, device=dev)
+    ws_f = torch.empty(q.fwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(q.bwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        q.qlora_linear_fwd(qw, x, A, B, alpha, h=h, u=u, workspace=ws_f)
+        q.qlora_linear_bwd(qw, x, A, B, alpha, dY, u=u, workspace=ws_b, outs=(dX, dA, dB))
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for s, e in ev:
+        flush.zero_()
+        s.record()
+        step()
+        e.record()
+    torch.cuda.synchronize()
+    ms = statistics.mean(s.elapsed_time(e) for s, e in ev)
+    f_fwd, f_bwd = layer_flops(M, N, K, r)
+    del qw, x, A, B, dY, h, u, dX, ws_f, ws_b, flush, inp
+    torch.cuda.empty_cache()
+    return {"step": {"workload": f"{MAIN}: W0 {N}x{K} NF4 (blocks of 128, double quant), x {M}x{K}, "
+                                 f"r={r}, fwd+bwd", "ms_per_step": ms,
+                     "tflops": (f_fwd + f_bwd) / (ms * 1e-3) / 1e12},
+            "decode": decode_leg(q, dev, peaks, block=128, tokens=(1, 16)),
+            "quantize": quantize_leg(q, dev, peaks, block=128)}
 
 
 def _time_steps(step, warmup, steps):

@@ -130,12 +130,13 @@ class QuantizedWeight:
     k: int
     double_quant: bool
     codes: torch.Tensor                  # uint8 [n*k/2]
-    absmax: torch.Tensor                 # fp32 [n*k/64]
-    absmax_q8: Optional[torch.Tensor]    # uint8 [n*k/64]
-    absmax_c: Optional[torch.Tensor]     # fp32 [ceil(n*k/64/256)]
+    absmax: torch.Tensor                 # fp32 [n*k/block_size]
+    absmax_q8: Optional[torch.Tensor]    # uint8 [n*k/block_size]
+    absmax_c: Optional[torch.Tensor]     # fp32 [ceil(n*k/block_size/256)]
+    block_size: int = BLOCK_SIZE         # 64 or 128 elements per block
 
     def struct(self) -> NF4WeightStruct:
-        return NF4WeightStruct(self.n, self.k, BLOCK_SIZE, int(self.double_quant),
+        return NF4WeightStruct(self.n, self.k, self.block_size, int(self.double_quant),
                                self.codes.data_ptr(), self.absmax.data_ptr(),
                                self.absmax_q8.data_ptr() if self.absmax_q8 is not None else None,
                                self.absmax_c.data_ptr() if self.absmax_c is not None else None)
@@ -145,29 +146,33 @@ class QuantizedWeight:
         return self.codes.device
 
     @staticmethod
-    def empty(n: int, k: int, double_quant: bool, device) -> "QuantizedWeight":
-        nb = n * k // BLOCK_SIZE
+    def empty(n: int, k: int, double_quant: bool, device, block_size: int = BLOCK_SIZE) -> "QuantizedWeight":
+        if block_size not in (64, 128):
+            raise ValueError("block_size must be 64 or 128")
+        nb = n * k // block_size
         ng = (nb + DQ_GROUP - 1) // DQ_GROUP
         dev = torch.device(device)
         return QuantizedWeight(
             n, k, double_quant,
             torch.empty(n * k // 2, dtype=torch.uint8, device=dev),
-            torch.empty(nb, dtype=torch.float32, device=dev),
+            torch.empty(max(nb, 1), dtype=torch.float32, device=dev),
             torch.empty(max(nb, 1), dtype=torch.uint8, device=dev) if double_quant else None,
-            torch.empty(max(ng, 1), dtype=torch.float32, device=dev) if double_quant else None)
+            torch.empty(max(ng, 1), dtype=torch.float32, device=dev) if double_quant else None,
+            block_size)
 
 
 _DTYPES = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}   # nf4_dtype
 
 
 def nf4_quantize(W0: torch.Tensor, double_quant: bool = True,
-                 out: Optional[QuantizedWeight] = None) -> QuantizedWeight:
-    """Blockwise NF4 quantisation of a [n, k] fp32, bf16 or fp16 CUDA tensor."""
+                 out: Optional[QuantizedWeight] = None, block_size: int = BLOCK_SIZE) -> QuantizedWeight:
+    """Blockwise NF4 quantisation of a [n, k] fp32, bf16 or fp16 CUDA tensor in
+    blocks of 64 or 128 elements."""
     _need_cuda(W0)
     if W0.dtype not in _DTYPES or W0.dim() != 2 or not W0.is_contiguous():
         raise ValueError("W0 must be a contiguous 2-D float32, bfloat16 or float16 tensor")
     n, k = W0.shape
-    qw = out if out is not None else QuantizedWeight.empty(n, k, double_quant, W0.device)
+    qw = out if out is not None else QuantizedWeight.empty(n, k, double_quant, W0.device, block_size)
     s = qw.struct()
     if W0.dtype == torch.float32:
         _check(lib.nf4_quantize(_ptr(W0), ctypes.byref(s), _stream(W0.device)), "nf4_quantize")

@@ -26,12 +26,12 @@ __device__ __forceinline__ float dq_block_scale(const float *absmax, const uint8
 // (16384 weights, 64 KB of fp32). A producer lane streams each group into
 // shared memory by TMA, a quarter group (64 blocks, 16 KB) per stage through
 // a ring of kQzStages stages, with the 128-byte swizzle. Eight consumer warps
-// code a stage: four lanes per block, each lane 16 consecutive elements
-// (elements [16q, 16q + 16) of its block, two 128-byte rows per block), read
-// as four 16-byte pieces whose swizzled addresses fall on eight distinct bank
-// groups in every quarter warp. The absmax is an integer max over |w|'s bit
-// patterns (NaN above +inf, so one compare flags any non-finite block), then
-// two shuffles across the block's four lanes.
+// code a stage: four lanes per 64-element block (eight per 128-element
+// block), each lane 16 consecutive elements (elements [16q, 16q + 16) of its
+// block), read as 16-byte pieces whose swizzled addresses fall on eight
+// distinct bank groups in every quarter warp. The absmax is an integer max
+// over |w|'s bit patterns (NaN above +inf, so one compare flags any
+// non-finite block), then shuffles across the block's lanes.
 //
 // The code of w is #{i : fl32(w / s) > t_i}, where the 15 decision thresholds
 // t_i are the level midpoints rounded toward -inf in fp32, so that a value on
@@ -52,8 +52,8 @@ __device__ __forceinline__ float dq_block_scale(const float *absmax, const uint8
 constexpr int kQzConsumerWarps = 8;
 constexpr int kQzThreads = 32 * (kQzConsumerWarps + 1);   // the last warp issues the TMA copies
 constexpr int kQzStages = 5;
-constexpr int kQzStageBlocks = 64;
-constexpr int kQzStageBytes = kQzStageBlocks * kBlock * 4;  // 16 KB: one stage slot (fp32 fills it)
+constexpr int kQzStageElems = 4096;                        // a stage: 64 blocks of 64 or 32 of 128
+constexpr int kQzStageBytes = kQzStageElems * 4;            // 16 KB: one stage slot (fp32 fills it)
 
 // Element type of W0: fp32, or a 16-bit type converted exactly to fp32 on
 // load ("QLoRA explained", section "The quantization backbone": weights are
@@ -67,7 +67,7 @@ constexpr int kQzBarOff = kQzAbsOff + 2 * kGroup * 4;               // full, emp
 constexpr int kQzSmemBytes = kQzBarOff + (2 * kQzStages + 2) * 8 + 16 + 1024;
 constexpr float kQuantGuard = 4.76837158203125e-07f;   // 2^-21 > 2.4e-7 bound on |p - fl32(w/s)|
 static_assert(kQzConsumerWarps * 32 == kGroup, "one consumer thread per block of a group");
-static_assert(kQzStageBlocks == 8 * kQzConsumerWarps, "eight blocks per consumer warp and stage");
+static_assert(kQzStageElems == kQzConsumerWarps * 32 * 16, "16 elements per consumer lane and stage");
 
 __device__ __forceinline__ float2 lds_f2(uint32_t addr) {
     float2 v;
@@ -99,9 +99,10 @@ __device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity) {
         if (clock64() - t0 > kWaitLimitCycles) return;
 }
 
-// tm_w views W0 as 128-byte rows: fp32 [2 nb, 32] with box {32, 128}, or
-// 16-bit [nb, 64] with box {64, 64}; either way a stage is 64 blocks.
-template <int KIND>
+// tm_w views W0 as 128-byte rows: fp32 [numel / 32, 32] with box {32, 128},
+// or 16-bit [numel / 64, 64] with box {64, 64}; either way a stage is 4096
+// elements. BS (64 or 128) elements per block: BS / 16 lanes code a block.
+template <int KIND, int BS>
 __global__ void __launch_bounds__(kQzThreads, kQzCtasPerSm)
 nf4_quantize_kernel(const __grid_constant__ CUtensorMap tm_w,
                     int64_t nb, int dq, uint8_t *__restrict__ codes, float *__restrict__ absmax,
@@ -154,21 +155,24 @@ nf4_quantize_kernel(const __grid_constant__ CUtensorMap tm_w,
     }
     __syncthreads();
 
+    constexpr int kLanes = BS / 16;                  // lanes per block
+    constexpr int kStageBlocks = kQzStageElems / BS;
+    constexpr int kRowsPerBlock = KIND == kQzF32 ? BS / 32 : BS / 64;   // 128-byte rows
     const int64_t ngroups = (nb + kGroup - 1) / kGroup;
     if (warp == kQzConsumerWarps) {
         // ------------------------------------------------------ producer
         if (lane == 0) {
             int n = 0;
             for (int64_t g = blockIdx.x; g < ngroups; g += gridDim.x) {
-                for (int qq = 0; qq < kGroup / kQzStageBlocks; ++qq) {
-                    const int64_t b0 = g * kGroup + qq * kQzStageBlocks;
+                for (int qq = 0; qq < kGroup / kStageBlocks; ++qq) {
+                    const int64_t b0 = g * kGroup + qq * kStageBlocks;
                     if (b0 >= nb) break;
                     const int s = n % kQzStages;
                     const uint32_t ph = static_cast<uint32_t>(n / kQzStages) & 1u;
                     if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) goto drain;
                     mbar_arrive_expect_tx(&full[s], KIND == kQzF32 ? kQzStageBytes : kQzStageBytes / 2);
                     tma_load_2d(qsm + s * kQzStageBytes, &tm_w, &full[s], 0,
-                                static_cast<int32_t>(KIND == kQzF32 ? 2 * b0 : b0));
+                                static_cast<int32_t>(kRowsPerBlock * b0));
                     ++n;
                 }
             }
@@ -181,17 +185,19 @@ nf4_quantize_kernel(const __grid_constant__ CUtensorMap tm_w,
     }
 
     // ---------------------------------------------------------- consumers
-    const int bq = lane >> 2;                    // block of this lane among the warp's eight
-    const int q = lane & 3;                      // elements [16q, 16q + 16) of that block
-    const int lb = warp * 8 + bq;                // block within a stage
+    const int bq = lane / kLanes;                // block of this lane among the warp's 32 / kLanes
+    const int q = lane % kLanes;                 // elements [16q, 16q + 16) of that block
+    const int lb = warp * (32 / kLanes) + bq;    // block within a stage
     // 128-byte row within the stage, and the 16-byte pieces of the lane's
-    // elements: fp32 rows hold half a block, 16-bit rows a whole one
-    const int row = KIND == kQzF32 ? 2 * lb + (q >> 1) : lb;
+    // elements: an fp32 row holds 32 elements (two lanes), a 16-bit row 64
+    // (four lanes). In every quarter warp the eight lanes' pieces fall on
+    // eight distinct 16-byte bank groups after the swizzle.
+    const int row = KIND == kQzF32 ? kRowsPerBlock * lb + (q >> 1) : kRowsPerBlock * lb + (q >> 2);
     constexpr int kPieces = KIND == kQzF32 ? 4 : 2;
     uint32_t off[kPieces];
 #pragma unroll
     for (int j = 0; j < kPieces; ++j) {
-        const int piece = KIND == kQzF32 ? 4 * (q & 1) + j : 2 * q + j;
+        const int piece = KIND == kQzF32 ? 4 * (q & 1) + j : 2 * (q & 3) + j;
         off[j] = static_cast<uint32_t>(row * 128 + ((piece ^ (row & 7)) << 4));
     }
     const uint32_t mytab = smem_u32(tab) + 8u * lane;
@@ -199,8 +205,8 @@ nf4_quantize_kernel(const __grid_constant__ CUtensorMap tm_w,
     int n = 0, gi = 0;
     for (int64_t g = blockIdx.x; g < ngroups; g += gridDim.x, ++gi) {
         float *sa = s_abs + (gi & 1) * kGroup;
-        for (int qq = 0; qq < kGroup / kQzStageBlocks; ++qq) {
-            const int64_t b0 = g * kGroup + qq * kQzStageBlocks;
+        for (int qq = 0; qq < kGroup / kStageBlocks; ++qq) {
+            const int64_t b0 = g * kGroup + qq * kStageBlocks;
             if (b0 >= nb) break;
             const int s = n % kQzStages;
             const uint32_t ph = static_cast<uint32_t>(n / kQzStages) & 1u;
@@ -245,6 +251,7 @@ nf4_quantize_kernel(const __grid_constant__ CUtensorMap tm_w,
             uint32_t m = max(max(mm[0], mm[1]), max(mm[2], mm[3]));
             m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
             m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+            if constexpr (kLanes == 8) m = max(m, __shfl_xor_sync(0xffffffffu, m, 4));
             const float sc = __uint_as_float(m);
             uint32_t c[16];
 #pragma unroll
@@ -284,10 +291,10 @@ nf4_quantize_kernel(const __grid_constant__ CUtensorMap tm_w,
             }
             const int64_t b = b0 + lb;
             if (b < nb) {
-                *reinterpret_cast<uint2 *>(codes + b * (kBlock / 2) + 8 * q) = make_uint2(w0, w1);
+                *reinterpret_cast<uint2 *>(codes + b * (BS / 2) + 8 * q) = make_uint2(w0, w1);
                 if (q == 0) absmax[b] = sc;
             }
-            if (q == 0) sa[qq * kQzStageBlocks + lb] = sc;
+            if (q == 0) sa[qq * kStageBlocks + lb] = sc;
             // the stage's values are consumed (the stores above depend on all of them)
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
@@ -322,17 +329,18 @@ done:
     if (__any_sync(0xffffffffu, bad) && lane == 0) record_status(NF4_ERR_NONFINITE);
 }
 
-// Dequantisation, one thread per 64-element block.
+// Dequantisation, one thread per 64 elements (a block, or half of a
+// 128-element block: scale index b >> bshift).
 //   bf16 output: per-block register lookup table (the same routine that
 //   produces the tensor-core operand in the fused matmuls).
 //   fp32 output: fl32(scale * level) per element.
 __global__ void __launch_bounds__(256)
 nf4_dequantize_kernel(const uint8_t *__restrict__ codes, const float *__restrict__ absmax,
                       const uint8_t *__restrict__ q8, const float *__restrict__ cg, int dq,
-                      int64_t nb, int out_bf16, void *__restrict__ out) {
+                      int64_t nb, int bshift, int out_bf16, void *__restrict__ out) {
     for (int64_t b = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; b < nb;
          b += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const float s = dq_block_scale(absmax, q8, cg, dq, b);
+        const float s = dq_block_scale(absmax, q8, cg, dq, b >> bshift);
         const uint4 *src = reinterpret_cast<const uint4 *>(codes + b * (kBlock / 2));
         const uint4 c0 = __ldg(src), c1 = __ldg(src + 1);
         const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};

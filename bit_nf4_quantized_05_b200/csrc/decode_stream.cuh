@@ -70,6 +70,7 @@ struct DecodeArgs {
     float scale;           // fl32(alpha / r)
     float *u_out;          // [M, r] fp32 x A^T (optional; written by CTA 0)
     uint16_t *h;           // [M, N]
+    int bshift;            // log2(block size / 64): block of 64-element step j is j >> bshift
 };
 
 // Per-token adapter selection over stacked adapters (multi-adapter forward):
@@ -236,18 +237,21 @@ qlora_decode_stream_kernel(const __grid_constant__ CUtensorMap tm_codes,   // [N
         const int n = (static_cast<int>(blockIdx.x) + ti * static_cast<int>(gridDim.x)) * kDsRows + srow;
         if (n >= Nrows) return s;
         const int nb = min(CB, nkb - ch * CB);
-        const int b = n * kblocks + kb0 + ch * CB;
+        const int kbase = kb0 + ch * CB;                 // the chunk's first 64-element step
+        const int rowb = n * (kblocks >> a.bshift);      // first block of row n
+        const int b = rowb + (kbase >> a.bshift);
         if (a.dq) {
 #pragma unroll
             for (int i = 0; i < CB; ++i)
-                if (i < nb) s.raw[i] = __ldg(a.q8 + b + i);
+                if (i < nb) s.raw[i] = __ldg(a.q8 + rowb + ((kbase + i) >> a.bshift));
             s.c0 = __ldg(a.cg + (b >> 8));
-            s.c1 = __ldg(a.cg + ((b + nb - 1) >> 8));
-            s.split = 256 - (b & 255);
+            s.c1 = __ldg(a.cg + ((rowb + ((kbase + nb - 1) >> a.bshift)) >> 8));
+            // the first step of the chunk whose block is in the next group
+            s.split = (((kbase >> a.bshift) + 256 - (b & 255)) << a.bshift) - kbase;
         } else {
 #pragma unroll
             for (int i = 0; i < CB; ++i)
-                if (i < nb) s.raw[i] = __float_as_uint(__ldg(a.absmax + b + i));
+                if (i < nb) s.raw[i] = __float_as_uint(__ldg(a.absmax + rowb + ((kbase + i) >> a.bshift)));
         }
         return s;
     };

@@ -454,9 +454,10 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
         };
         auto block_of = [&](const Pos &p) -> int64_t {
             if (p.tile >= total_tiles || p.it >= args.main_steps || p.item < 0) return -1;
-            if (!DGRAD) return p.item * args.kblocks + p.it;
+            const int64_t bpr = args.kblocks >> args.bshift;      // blocks per W row
+            if (!DGRAD) return p.item * bpr + (p.it >> args.bshift);
             const int64_t wrow = static_cast<int64_t>(p.it) * kBK + r_loc;
-            return wrow < args.Nw ? wrow * args.kblocks + p.item : -1;
+            return wrow < args.Nw ? wrow * bpr + (p.item >> args.bshift) : -1;
         };
         // raw scale of a block: q8 and c_g under double quantisation, else absmax
         struct RawScale { int64_t b; uint32_t q8; float v; };

@@ -55,7 +55,7 @@ struct GemmArgs {
     // quantised weight (always the [N, K] weight)
     int64_t Nw;         // rows of W
     int64_t Kw;         // columns of W
-    int64_t kblocks;    // K / 64 (blocks per W row)
+    int64_t kblocks;    // K / 64 (64-element steps per W row)
     const float *absmax;
     const uint8_t *q8;
     const float *cg;
@@ -67,6 +67,7 @@ struct GemmArgs {
     float *partial;     // [pairs][2][BN/32][128][32] fp32 partial tiles
     int *flags;         // [pairs][2][4 epilogue warps], zero at launch; 1 = rows written
     float *D32;         // when non-null: the fp32 result goes here instead of D
+    int bshift;         // log2(block size / 64): block of step j is j >> bshift
 };
 
 template <int BN, bool DGRAD>
@@ -318,7 +319,7 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red] bf1
                 wblk = n0 / 64 + kb;
             }
             if (wrow >= args.Nw || wblk >= args.kblocks) return -1;
-            return wrow * args.kblocks + wblk;
+            return wrow * (args.kblocks >> args.bshift) + (wblk >> args.bshift);
         };
         struct RawScale { int64_t b; uint32_t q8; float v; };
         auto load_scale = [&](int64_t b) -> RawScale {

@@ -41,6 +41,7 @@ struct MergeArgs {
     const uint16_t *B;         // [N, r]
     float scale;               // fl32(alpha / r)
     void *out;                 // [N, K] bf16 or fp32
+    int block;                 // elements per NF4 block (64 or 128)
 };
 
 // Shared-memory layout of one CTA (bytes), for padded rank rp.
@@ -109,13 +110,13 @@ __global__ void __launch_bounds__(kMgThreads, 4) qlora_merge_kernel(const MergeA
     const int cw = 64 * (warp >> 2);         // first tile column of this warp
     const bool cols_ok = k0 + cw < a.K;      // K is a multiple of 64: a warp's block is all in or all out
 
-    // block scales of rows rw + g and rw + g + 8 (one 64-column block per warp)
+    // block scales of rows rw + g and rw + g + 8 (a warp's 64 columns lie in one block)
     float sc[2] = {0.0f, 0.0f};
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const int64_t n = n0 + rw + g + 8 * h;
         if (n < a.N && cols_ok) {
-            const int64_t b = n * (a.K / kBlock) + (k0 + cw) / kBlock;
+            const int64_t b = n * (a.K / a.block) + (k0 + cw) / a.block;
             sc[h] = a.dq ? __fmul_rn(static_cast<float>(__ldg(a.q8 + b)), __fdiv_rn(__ldg(a.cg + (b >> 8)), 127.0f))
                          : __ldg(a.absmax + b);
         }

@@ -26,7 +26,11 @@ namespace nf4 {
 
 __constant__ float c_levels[16] = {NF4_LEVEL_LIST};
 
-constexpr int kBlock = 64;       // elements per NF4 block
+// Elements per NF4 block: 64 or 128. The kernels walk K in 64-element steps
+// (kBlock); a 128-element block is two consecutive steps that share one
+// scale, block index = step >> block_shift.
+constexpr int kBlock = 64;
+__host__ __device__ constexpr int block_shift_of(int block_size) { return block_size == 128 ? 1 : 0; }
 constexpr int kGroup = 256;      // blocks per double-quant group
 
 // ---------------------------------------------------------------------------

@@ -186,9 +186,10 @@ bool make_map(CUtensorMap *map, CUtensorMapDataType dt, size_t elem, const void 
 
 nf4_status check_weight(const nf4_weight *w, bool need_scales) {
     if (!w) return NF4_ERR_INVALID_ARG;
-    if (w->block_size != kBlock || (w->double_quant != 0 && w->double_quant != 1))
+    if ((w->block_size != 64 && w->block_size != 128) || (w->double_quant != 0 && w->double_quant != 1))
         return NF4_ERR_INVALID_ARG;
-    if (w->n < 8 || w->k < 64 || (w->n % 8) != 0 || (w->k % 64) != 0) return NF4_ERR_UNSUPPORTED_SHAPE;
+    if (w->n < 8 || w->k < w->block_size || (w->n % 8) != 0 || (w->k % w->block_size) != 0)
+        return NF4_ERR_UNSUPPORTED_SHAPE;
     if (w->n > (int64_t(1) << 31) - 1 || w->k > (int64_t(1) << 31) - 1) return NF4_ERR_UNSUPPORTED_SHAPE;
     if (!w->codes || !w->absmax) {
         if (!w->codes || !(w->double_quant || !need_scales)) return NF4_ERR_INVALID_ARG;
@@ -444,6 +445,7 @@ nf4_status launch_gemm(const nf4_weight *w, const uint16_t *act, int64_t M, int6
     a.Nw = N;
     a.Kw = K;
     a.kblocks = K / kBlock;
+    a.bshift = block_shift_of(w->block_size);
     a.absmax = w->absmax;
     a.q8 = w->absmax_q8;
     a.cg = w->absmax_c;
@@ -536,6 +538,7 @@ nf4_status launch_gemm_pair(const nf4_weight *w, const uint16_t *act, int64_t M,
     a.Nw = N;
     a.Kw = K;
     a.kblocks = K / kBlock;
+    a.bshift = block_shift_of(w->block_size);
     a.absmax = w->absmax;
     a.q8 = w->absmax_q8;
     a.cg = w->absmax_c;
@@ -646,6 +649,7 @@ nf4_status launch_decode(const nf4_weight *w, const uint16_t *x, int64_t M, cons
     a.scale = scale;
     a.u_out = u_out;
     a.h = h;
+    a.bshift = block_shift_of(w->block_size);
     CUtensorMap tm_codes;
     if (!make_map(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, w->k / 2, w->n,
                   static_cast<uint32_t>(32 * cb), kDsRows, CU_TENSOR_MAP_SWIZZLE_NONE))
@@ -850,24 +854,31 @@ nf4_status nf4_quantize_typed(const void *W0, int32_t dtype, const nf4_weight *w
     if (!W0 || !w->absmax) return NF4_ERR_INVALID_ARG;
     if (dtype != NF4_DTYPE_F32 && dtype != NF4_DTYPE_BF16 && dtype != NF4_DTYPE_F16) return NF4_ERR_INVALID_ARG;
     if (!aligned16(W0)) return NF4_ERR_ALIGNMENT;
-    const int64_t nb = w->n * w->k / kBlock;
+    const int64_t numel = w->n * w->k;
+    const int64_t nb = numel / w->block_size;
     const int64_t groups = (nb + kGroup - 1) / kGroup;
-    // TMA row coordinates (128-byte rows: two per fp32 block, one per 16-bit block) are 32-bit
-    if (2 * nb > 0x7fffffffLL) return NF4_ERR_UNSUPPORTED_SHAPE;
+    // TMA row coordinates (128-byte rows: 32 fp32 or 64 16-bit elements) are 32-bit
+    if (numel / 32 > 0x7fffffffLL) return NF4_ERR_UNSUPPORTED_SHAPE;
     CUtensorMap tm_w;
     bool ok;
     if (dtype == NF4_DTYPE_F32)
-        ok = make_map(&tm_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, W0, 32, static_cast<uint64_t>(2 * nb), 32,
-                      2 * kQzStageBlocks, CU_TENSOR_MAP_SWIZZLE_128B);
+        ok = make_map(&tm_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, W0, 32, static_cast<uint64_t>(numel / 32), 32,
+                      kQzStageElems / 32, CU_TENSOR_MAP_SWIZZLE_128B);
     else
         ok = make_map(&tm_w,
                       dtype == NF4_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                      2, W0, 64, static_cast<uint64_t>(nb), 64, kQzStageBlocks, CU_TENSOR_MAP_SWIZZLE_128B);
+                      2, W0, 64, static_cast<uint64_t>(numel / 64), 64, kQzStageElems / 64,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok) return NF4_ERR_CUDA;
     // persistent: kQzCtasPerSm CTAs per SM walk the groups
     const int64_t grid = std::min<int64_t>(groups, int64_t(kQzCtasPerSm) * num_sms(current_device()));
-    auto kern = dtype == NF4_DTYPE_F32 ? nf4_quantize_kernel<kQzF32>
-                : dtype == NF4_DTYPE_BF16 ? nf4_quantize_kernel<kQzBF16> : nf4_quantize_kernel<kQzF16>;
+    void (*kern)(const CUtensorMap, int64_t, int, uint8_t *, float *, uint8_t *, float *);
+    if (w->block_size == 64)
+        kern = dtype == NF4_DTYPE_F32 ? nf4_quantize_kernel<kQzF32, 64>
+               : dtype == NF4_DTYPE_BF16 ? nf4_quantize_kernel<kQzBF16, 64> : nf4_quantize_kernel<kQzF16, 64>;
+    else
+        kern = dtype == NF4_DTYPE_F32 ? nf4_quantize_kernel<kQzF32, 128>
+               : dtype == NF4_DTYPE_BF16 ? nf4_quantize_kernel<kQzBF16, 128> : nf4_quantize_kernel<kQzF16, 128>;
     NF4_TRY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kQzSmemBytes));
     LaunchTimer t(KK_QUANTIZE, static_cast<cudaStream_t>(stream));
     kern<<<static_cast<unsigned>(grid), kQzThreads, kQzSmemBytes, static_cast<cudaStream_t>(stream)>>>(
@@ -886,12 +897,13 @@ nf4_status nf4_dequantize(const nf4_weight *w, void *out, int32_t out_bf16, void
     if (st != NF4_OK) return st;
     if (!out || (out_bf16 != 0 && out_bf16 != 1)) return NF4_ERR_INVALID_ARG;
     if (!aligned16(out)) return NF4_ERR_ALIGNMENT;
-    const int64_t nb = w->n * w->k / kBlock;
+    const int64_t nb = w->n * w->k / kBlock;       // 64-element steps
     const int dev = current_device();
     const int grid = static_cast<int>(std::min<int64_t>((nb + 255) / 256, int64_t(num_sms(dev)) * 16));
     LaunchTimer t(KK_DEQUANTIZE, static_cast<cudaStream_t>(stream));
     nf4_dequantize_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-        w->codes, w->absmax, w->absmax_q8, w->absmax_c, w->double_quant, nb, out_bf16, out);
+        w->codes, w->absmax, w->absmax_q8, w->absmax_c, w->double_quant, nb, block_shift_of(w->block_size),
+        out_bf16, out);
     t.stop();
     NF4_TRY_CUDA(cudaGetLastError());
     return NF4_OK;
@@ -920,6 +932,7 @@ nf4_status qlora_merge(const nf4_weight *w, const uint16_t *A, const uint16_t *B
     a.B = B;
     a.scale = alpha / static_cast<float>(r);
     a.out = out;
+    a.block = w->block_size;
     const dim3 grid(static_cast<unsigned>((w->k + kMgCols - 1) / kMgCols),
                     static_cast<unsigned>((w->n + kMgRows - 1) / kMgRows));
     const int smem = merge_smem_bytes(a.rp, out_is_bf16 != 0);

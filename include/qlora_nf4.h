@@ -32,9 +32,9 @@
  *     (non-finite weight values, a pipeline wait that ran out of time) are
  *     recorded in a per-device status word read by nf4_device_status().
  *   - Requirements (violations return an error and launch nothing):
- *       k % 64 == 0, n % 8 == 0, n >= 8, k >= 64, M >= 0,
- *       1 <= r <= 128 and r % 8 == 0, alpha finite,
- *       every pointer 16-byte aligned, block_size == 64.
+ *       block_size 64 or 128, k % block_size == 0, k >= block_size,
+ *       n % 8 == 0, n >= 8, M >= 0, 1 <= r <= 128 and r % 8 == 0,
+ *       alpha finite, every pointer 16-byte aligned.
  *   - No C++ exception crosses this boundary. Entry points are reentrant;
  *     calls on one stream are ordered, calls on different streams that share
  *     output or workspace buffers race.
@@ -72,10 +72,11 @@ typedef enum {
  *              index into the 16 NF4 levels; element 2j is the HIGH nibble of
  *              byte j ("Parameter-Efficient Fine-Tuning: From LoRA to QLoRA",
  *              Pillar 1, byte packing step of the numerical example).
- *   absmax     nb = n*k/64 fp32 block scales s_i = max |w| over each run of
- *              64 consecutive elements ("QLoRA Finetuner", section 2, absmax
- *              scale). Always written by nf4_quantize; read by the other
- *              entry points only when double_quant == 0.
+ *   absmax     nb = n*k/block_size fp32 block scales s_i = max |w| over each
+ *              run of block_size consecutive elements ("QLoRA Finetuner",
+ *              section 2: one absmax per block of 64 or 128 weights). Always
+ *              written by nf4_quantize; read by the other entry points only
+ *              when double_quant == 0.
  *   absmax_q8  nb bytes in [0, 127]: 8-bit codes of the block scales
  *              (double_quant == 1 only).
  *   absmax_c   ceil(nb/256) fp32 group constants: the largest s_i in each run
@@ -86,7 +87,7 @@ typedef enum {
 typedef struct {
     int64_t n;
     int64_t k;
-    int32_t block_size;   /* must be 64 */
+    int32_t block_size;   /* 64 or 128 elements per block; k % block_size == 0 */
     int32_t double_quant; /* 0 or 1 */
     uint8_t *codes;
     float *absmax;
@@ -95,8 +96,8 @@ typedef struct {
 } nf4_weight;
 
 /* Blockwise NF4 quantisation of W0 [n, k] fp32 into w ("QLoRA Finetuner",
- * section 2: absmax per 64-element block, normalise to [-1, 1], nearest of
- * the 16 NF4 quantiles; "Parameter-Efficient Fine-Tuning", Pillar 1 and the
+ * section 2: absmax per block of w->block_size (64 or 128) consecutive
+ * elements, normalise to [-1, 1], nearest of the 16 NF4 quantiles; "Parameter-Efficient Fine-Tuning", Pillar 1 and the
  * numerical step-by-step example; Pillar 2 for double quantisation).
  * Normalisation is one IEEE fp32 division w / s. A value exactly halfway
  * between two levels takes the lower level. An all-zero block stores s = 0

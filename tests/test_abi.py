@@ -132,7 +132,10 @@ def test_typed_quantize_and_merge_argument_checks(q):
     assert merge(bf16=2) == q.NF4_ERR_INVALID_ARG
     assert merge(out=None) == q.NF4_ERR_INVALID_ARG
     assert merge(A=FAKE + 8) == q.NF4_ERR_ALIGNMENT
-    assert merge(w=weight(q, block=128)) == q.NF4_ERR_INVALID_ARG
+    assert merge(w=weight(q, block=96)) == q.NF4_ERR_INVALID_ARG
+    # 128-element blocks need K to be a multiple of 128
+    assert merge(w=weight(q, block=128)) == q.NF4_ERR_UNSUPPORTED_SHAPE
+    assert L.nf4_quantize(FAKE, ctypes.byref(weight(q, k=192, block=128)), None) == q.NF4_ERR_UNSUPPORTED_SHAPE
 
 
 def test_multi_adapter_and_dropout_argument_checks(q):

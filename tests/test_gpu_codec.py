@@ -21,9 +21,9 @@ def q():
     return mod
 
 
-def quant_both(q, W: np.ndarray, dq: bool):
-    ref = oracle.quantize(W.reshape(-1), dq=dq)
-    qw = q.nf4_quantize(torch.from_numpy(np.ascontiguousarray(W)).cuda(), double_quant=dq)
+def quant_both(q, W: np.ndarray, dq: bool, block: int = 64):
+    ref = oracle.quantize(W.reshape(-1), block=block, dq=dq)
+    qw = q.nf4_quantize(torch.from_numpy(np.ascontiguousarray(W)).cuda(), double_quant=dq, block_size=block)
     torch.cuda.synchronize()
     assert q.device_status() == q.NF4_OK
     return ref, qw
@@ -131,10 +131,10 @@ def test_nonfinite_weight_sets_status(q):
 
 
 # ------------------------------------------------------------ 16-bit input --
-def quant_16(q, W16: torch.Tensor, dq: bool):
+def quant_16(q, W16: torch.Tensor, dq: bool, block: int = 64):
     """GPU quantisation of a 16-bit weight and the oracle's of its exact fp32 image."""
-    ref = oracle.quantize(W16.float().numpy().reshape(-1), dq=dq)
-    qw = q.nf4_quantize(W16.contiguous().cuda(), double_quant=dq)
+    ref = oracle.quantize(W16.float().numpy().reshape(-1), block=block, dq=dq)
+    qw = q.nf4_quantize(W16.contiguous().cuda(), double_quant=dq, block_size=block)
     torch.cuda.synchronize()
     assert q.device_status() == q.NF4_OK
     return ref, qw

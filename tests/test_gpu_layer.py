@@ -49,16 +49,16 @@ def rel_err(got: np.ndarray, ref: np.ndarray, ulp_allowance: bool = False) -> fl
 
 def oracle_weight(qw):
     """The GPU's quantised weight as an oracle Quantized record."""
-    return oracle.Quantized(qw.codes.cpu().numpy(), qw.absmax.cpu().numpy(),
-                            qw.absmax_q8.cpu().numpy()[: qw.n * qw.k // 64] if qw.double_quant else None,
-                            qw.absmax_c.cpu().numpy()[: (qw.n * qw.k // 64 + 255) // 256]
-                            if qw.double_quant else None,
-                            64, qw.double_quant, 256, qw.n * qw.k)
+    nb = qw.n * qw.k // qw.block_size
+    return oracle.Quantized(qw.codes.cpu().numpy(), qw.absmax.cpu().numpy()[:nb],
+                            qw.absmax_q8.cpu().numpy()[:nb] if qw.double_quant else None,
+                            qw.absmax_c.cpu().numpy()[: (nb + 255) // 256] if qw.double_quant else None,
+                            qw.block_size, qw.double_quant, 256, qw.n * qw.k)
 
 
-def run_layer(q, W0, A, B, x, dY, alpha, dq, rows=None, need_bwd=True):
+def run_layer(q, W0, A, B, x, dY, alpha, dq, rows=None, need_bwd=True, block=64):
     dev = "cuda"
-    qw = q.nf4_quantize(W0.to(dev), double_quant=dq)
+    qw = q.nf4_quantize(W0.to(dev), double_quant=dq, block_size=block)
     xd, Ad, Bd = x.to(dev), A.to(dev), B.to(dev)
     h, u = q.qlora_linear_fwd(qw, xd, Ad, Bd, alpha)
     out = {"qw": qw, "h": h, "u": u}
