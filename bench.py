@@ -724,9 +724,16 @@ def stack_leg(q, dev, peaks, warmup=2, steps=3):
             "steps": steps, "input_generation_s": gen_s}
 
 
-def cpu_baseline_leg(w, inp):
+def cpu_baseline_leg(w, inp, target_s=12.0):
+    """The oracle on a bounded sample of the workload's tokens: the sample grows
+    (at most 8x per try) until one try takes half of target_s or covers every
+    token, so the timed try takes roughly 5 to 20 s on the host."""
     tokens = 16
-    f, t = oracle_sample_step(w, inp, tokens)
+    while True:
+        f, t = oracle_sample_step(w, inp, tokens)
+        if t >= 0.5 * target_s or tokens >= w.M:
+            break
+        tokens = int(min(w.M, tokens * min(8.0, max(2.0, target_s / max(t, 1e-3)))))
     return {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
             "sample": f"{tokens} of {w.M} tokens: oracle forward+backward of those tokens "
                       f"({t:.1f} s on the host)"}
