@@ -198,7 +198,7 @@ def main():
     ap.add_argument("--skip-extras", action="store_true",
                     help="only the main fwd+bwd line (no decode/quantize/oracle/e2e legs)")
     ap.add_argument("--leg", default="all", choices=["all", "decode", "quantize", "stack", "mlp70b",
-                                                     "merge", "multi", "block128"],
+                                                     "merge", "multi", "block128", "dropout"],
                     help="run one secondary leg alone and print its JSON (for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -220,7 +220,7 @@ def main():
         if rank == 0:
             leg = {"decode": decode_leg, "quantize": quantize_leg, "stack": stack_leg,
                    "mlp70b": mlp70b_leg, "merge": merge_leg, "multi": multi_leg,
-                   "block128": block128_leg}[args.leg]
+                   "block128": block128_leg, "dropout": dropout_leg}[args.leg]
             print(json.dumps({"leg": args.leg, **leg(q, dev, load_peaks())}), flush=True)
         return
     if world > 1:
@@ -332,6 +332,7 @@ def main():
         line["merge"] = merge_leg(q, dev, peaks)
         line["multi_adapter"] = multi_leg(q, dev, peaks)
         line["block128"] = block128_leg(q, dev, peaks)
+        line["dropout"] = dropout_leg(q, dev, peaks)
         line["cpu_baseline"] = cpu_baseline_leg(w, inp)
     elif not args.skip_extras:
         e2e_leg(q, dp, qw, inp, w, args, dev, world)  # same collectives on every rank
@@ -570,6 +571,63 @@ def merge_leg(q, dev, peaks):
     del copies
     torch.cuda.empty_cache()
     return out
+
+
+def dropout_leg(q, dev, peaks, steps=50, p=0.05):
+    """The main workload's forward + backward with LoRA dropout p = 0.05 on the adapter input
+    (a seeded keep mask, drawn once): the rank-r kernels mask the landed x tiles, the dgrad
+    GEMM writes dY W~ in fp32 and the adapter-add kernel masks, adds and rounds dX once.
+    The adapter-add kernel is HBM-bound: it reads the fp32 base (4 B), writes dX (2 B) and
+    reads the mask (1/8 B) per element of dX."""
+    w = workloads.WORKLOADS[MAIN]
+    M, N, K, r, alpha = w.M, w.N, w.K, w.r, w.alpha
+    inp = workloads.make_inputs(w)
+    qw = q.nf4_quantize(inp["W0"].to(dev), double_quant=w.double_quant)
+    x, A, B, dY = (inp[k].to(dev) for k in ("x", "A", "B", "dY"))
+    g = torch.Generator(device="cpu").manual_seed(w.seed + 17)
+    keep = q.pack_keep((torch.rand(M, K, generator=g) >= p).to(dev))
+    h = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    dA = torch.empty(r, K, dtype=torch.bfloat16, device=dev)
+    dB = torch.empty(N, r, dtype=torch.bfloat16, device=dev)
+    ws_f = torch.empty(q.fwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(int(q.lib.qlora_bwd_dropout_workspace_bytes(M, N, K, r)), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        _, u = q.qlora_linear_fwd_dropout(qw, x, A, B, alpha, p, keep, h=h, workspace=ws_f)
+        q.qlora_linear_bwd_dropout(qw, x, A, B, alpha, p, keep, dY, u=u, workspace=ws_b, outs=(dX, dA, dB))
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for s, e in ev:
+        flush.zero_()
+        s.record()
+        step()
+        e.record()
+    torch.cuda.synchronize()
+    ms = statistics.mean(s.elapsed_time(e) for s, e in ev)
+    q.profiling(True)
+    for _ in range(steps):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    q.profiling(False)
+    prof = q.profile_read()
+    f_fwd, f_bwd = layer_flops(M, N, K, r)
+    add_n, add_t = prof.get("lora_dX_add", (0, 0.0))
+    add_us = 1e3 * add_t / max(add_n, 1)
+    add_bytes = M * K * 4 + M * K * 2 + M * K // 8
+    del qw, x, A, B, dY, keep, h, dX, dA, dB, ws_f, ws_b, flush, inp
+    torch.cuda.empty_cache()
+    return {"workload": f"{MAIN}: W0 {N}x{K} NF4 double quant, x {M}x{K}, r={r}, LoRA dropout p={p}, "
+                        f"fwd+bwd", "ms_per_step": ms, "tflops": (f_fwd + f_bwd) / (ms * 1e-3) / 1e12,
+            "kernels_us": {k: 1e3 * t / max(n, 1) for k, (n, t) in prof.items()},
+            "lora_dX_add": {"bytes": add_bytes, "kernel_us": add_us,
+                            "gbs": add_bytes / (add_us * 1e-6) / 1e9 if add_us > 0 else None,
+                            "frac": add_bytes / (add_us * 1e-6) / 1e9 / peaks["hbm_gbs"] if add_us > 0 else None}}
 
 
 def block128_leg(q, dev, peaks, steps=50):

@@ -338,13 +338,17 @@ def qlora_linear_fwd_dropout(qw: QuantizedWeight, x: torch.Tensor, A: torch.Tens
 def qlora_linear_bwd_dropout(qw: QuantizedWeight, x: torch.Tensor, A: torch.Tensor,
                              B: torch.Tensor, alpha: float, p: float, keep: torch.Tensor,
                              dY: torch.Tensor, u: Optional[torch.Tensor] = None,
-                             need_dX: bool = True, workspace: Optional[torch.Tensor] = None):
+                             need_dX: bool = True, workspace: Optional[torch.Tensor] = None,
+                             outs: Optional[tuple] = None):
     """(dX, dA, dB) with LoRA dropout (the mask of the forward)."""
     _need_cuda(x, A, B, dY, keep)
     M, r = x.shape[0], A.shape[0]
-    dX = torch.empty(M, qw.k, dtype=torch.bfloat16, device=x.device) if need_dX else None
-    dA = torch.empty(r, qw.k, dtype=torch.bfloat16, device=x.device)
-    dB = torch.empty(qw.n, r, dtype=torch.bfloat16, device=x.device)
+    if outs is not None:
+        dX, dA, dB = outs
+    else:
+        dX = torch.empty(M, qw.k, dtype=torch.bfloat16, device=x.device) if need_dX else None
+        dA = torch.empty(r, qw.k, dtype=torch.bfloat16, device=x.device)
+        dB = torch.empty(qw.n, r, dtype=torch.bfloat16, device=x.device)
     nbytes = int(lib.qlora_bwd_dropout_workspace_bytes(M, qw.n, qw.k, r))
     ws = workspace if workspace is not None else _workspace(nbytes, x.device)
     s = qw.struct()

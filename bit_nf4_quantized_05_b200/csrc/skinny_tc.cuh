@@ -196,22 +196,37 @@ skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a0,
     } else if ((warp == 2 || warp == 3) && J.mask_mode) {
         // dropout: zero the dropped elements of each landed A tile in place.
         // The tile is 128 rows of 128 bytes (64 consecutive k of one token,
-        // 128-byte swizzle); a 16-byte piece holds 8 k, i.e. one keep byte.
+        // 128-byte swizzle); a 16-byte piece holds 8 k, i.e. one keep byte,
+        // so a row's keep bits are one aligned 8-byte word (kx and the tile
+        // origins are multiples of 64). Thread t takes rows t and t + 64 and
+        // fetches their words before the tile lands.
         const int t64 = threadIdx.x - 64;
         for (int it = 0; it < nsteps; ++it) {
             const int st = it % kSkStages;
             const uint32_t ph = (it / kSkStages) & 1;
+            const int q0 = (s0 + it) * 64;
+            uint64_t kw[2];
+            bool rok[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int row = t64 + 64 * h;
+                const int64_t m = J.mask_mode == 1 ? p0 + row : q0 + (row & 63);
+                const int64_t k0 = J.mask_mode == 1 ? q0 : p0 + 64 * (row >> 6);
+                rok[h] = m < J.mx && k0 < J.kx;
+                kw[h] = rok[h] ? __ldg(reinterpret_cast<const unsigned long long *>(J.keep + ((m * J.kx + k0) >> 3)))
+                               : 0ull;
+            }
             if (!mbar_wait(&full[st], ph, abort_flag)) break;
             uint8_t *a = slot_a + st * Cfg::kABytes;
-            const int q0 = (s0 + it) * 64;
-#pragma unroll 4
-            for (int pc = t64; pc < 128 * 8; pc += 64) {
-                const int row = pc >> 3, c = pc & 7;
-                const int64_t m = J.mask_mode == 1 ? p0 + row : q0 + (row & 63);
-                const int64_t k0 = (J.mask_mode == 1 ? q0 : p0 + 64 * (row >> 6)) + 8 * c;
-                uint4 *piece = reinterpret_cast<uint4 *>(a + row * 128 + ((c ^ (row & 7)) << 4));
-                if (m < J.mx && k0 < J.kx) {
-                    const uint32_t kb = J.keep[(m * J.kx + k0) >> 3];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                if (!rok[h]) continue;
+                const int row = t64 + 64 * h;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint32_t kb = static_cast<uint32_t>(kw[h] >> (8 * c)) & 0xFFu;
+                    if (kb == 0xFFu) continue;                      // all eight kept
+                    uint4 *piece = reinterpret_cast<uint4 *>(a + row * 128 + ((c ^ (row & 7)) << 4));
                     uint4 v = *piece;
                     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
                     uint32_t o[4];
