@@ -24,7 +24,7 @@
 namespace nf4 {
 
 constexpr int kSkStages = 4;     // two CTAs fit on one SM
-constexpr int kSkThreads = 256;   // warp 0 TMA, warp 1 MMA, warps 4..7 epilogue
+constexpr int kSkThreads = 256;   // warp 0 TMA, warp 1 MMA, warps 4..7 dropout mask and epilogue
 constexpr int kSkMaxSplits = 8;   // portable cluster size
 
 // One product of a launch. A launch carries one or two products of the same
@@ -121,7 +121,7 @@ skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a0,
         for (int s = 0; s < kSkStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
-            mbar_init(&masked[s], 2);
+            mbar_init(&masked[s], 4);
         }
         mbar_init(done_bar, 1);
         *abort_flag = 0;
@@ -193,38 +193,30 @@ skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a0,
             umma_commit(&empty[st]);
         }
         if (ok) umma_commit(done_bar);
-    } else if ((warp == 2 || warp == 3) && J.mask_mode) {
-        // dropout: zero the dropped elements of each landed A tile in place.
-        // The tile is 128 rows of 128 bytes (64 consecutive k of one token,
-        // 128-byte swizzle); a 16-byte piece holds 8 k, i.e. one keep byte,
-        // so a row's keep bits are one aligned 8-byte word (kx and the tile
-        // origins are multiples of 64). Thread t takes rows t and t + 64 and
-        // fetches their words before the tile lands.
-        const int t64 = threadIdx.x - 64;
-        for (int it = 0; it < nsteps; ++it) {
-            const int st = it % kSkStages;
-            const uint32_t ph = (it / kSkStages) & 1;
-            const int q0 = (s0 + it) * 64;
-            uint64_t kw[2];
-            bool rok[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int row = t64 + 64 * h;
+    } else if (warp >= 4 && warp < 8) {
+        if (J.mask_mode) {
+            // dropout: zero the dropped elements of each landed A tile in place
+            // before the MMA reads it (these warps are idle until the last MMA).
+            // The tile is 128 rows of 128 bytes (64 consecutive k of one token,
+            // 128-byte swizzle); a 16-byte piece holds 8 k, i.e. one keep byte,
+            // so a row's keep bits are one aligned 8-byte word (kx and the tile
+            // origins are multiples of 64). Thread t takes row t and fetches its
+            // word before the tile lands.
+            const int row = threadIdx.x - 128;
+            for (int it = 0; it < nsteps; ++it) {
+                const int st = it % kSkStages;
+                const uint32_t ph = (it / kSkStages) & 1;
+                const int q0 = (s0 + it) * 64;
                 const int64_t m = J.mask_mode == 1 ? p0 + row : q0 + (row & 63);
                 const int64_t k0 = J.mask_mode == 1 ? q0 : p0 + 64 * (row >> 6);
-                rok[h] = m < J.mx && k0 < J.kx;
-                kw[h] = rok[h] ? __ldg(reinterpret_cast<const unsigned long long *>(J.keep + ((m * J.kx + k0) >> 3)))
-                               : 0ull;
-            }
-            if (!mbar_wait(&full[st], ph, abort_flag)) break;
-            uint8_t *a = slot_a + st * Cfg::kABytes;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                if (!rok[h]) continue;
-                const int row = t64 + 64 * h;
+                const bool rok = m < J.mx && k0 < J.kx;
+                const uint64_t kw =
+                    rok ? __ldg(reinterpret_cast<const unsigned long long *>(J.keep + ((m * J.kx + k0) >> 3))) : ~0ull;
+                if (!mbar_wait(&full[st], ph, abort_flag)) break;
+                uint8_t *a = slot_a + st * Cfg::kABytes;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    const uint32_t kb = static_cast<uint32_t>(kw[h] >> (8 * c)) & 0xFFu;
+                    const uint32_t kb = static_cast<uint32_t>(kw >> (8 * c)) & 0xFFu;
                     if (kb == 0xFFu) continue;                      // all eight kept
                     uint4 *piece = reinterpret_cast<uint4 *>(a + row * 128 + ((c ^ (row & 7)) << 4));
                     uint4 v = *piece;
@@ -236,12 +228,11 @@ skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a0,
                                        ((kb >> (2 * e + 1)) & 1u ? 0xffff0000u : 0u));
                     *piece = make_uint4(o[0], o[1], o[2], o[3]);
                 }
+                fence_proxy_async_smem();     // generic writes before the tensor core reads the tile
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&masked[st]);
             }
-            fence_proxy_async_smem();     // generic writes before the tensor core reads the tile
-            __syncwarp();
-            if ((threadIdx.x & 31) == 0) mbar_arrive(&masked[st]);
         }
-    } else if (warp >= 4 && warp < 8) {
         // accumulator -> this CTA's partial (the stage buffers are free once
         // the last MMA has completed: every load it waited for has landed)
         const int q = warp - 4;
