@@ -1,7 +1,7 @@
 """Compile the C oracle into oracle/_build/libnf4oracle.so.
 
-Test infrastructure: the oracle is a checker for the CUDA library and is never
-part of its product path. Building it is not using it.
+Test infrastructure: the oracle is the reference the CUDA library is tested
+against and is never part of its product path. Building it is not using it.
 """
 import os
 import subprocess
