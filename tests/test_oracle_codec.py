@@ -280,3 +280,17 @@ def test_zero_group():
     assert q.cg[0] == 0 and np.all(q.q8[:256] == 0)
     assert np.all(oracle.block_scales(q)[:256] == 0)
     assert q.cg[1] == 0.5 and q.q8[280] == 127
+
+
+def test_llama13b_storage_matches_page():
+    """Bytes per parameter of the stored format (codes, 8-bit scale codes and
+    group constants), measured on an oracle-quantised tensor, scaled to 13e9
+    parameters: the page's ~7 GB at 4-bit against 26 GB in 16 bits."""
+    g = read_golden_kv("llama13b_storage.txt")
+    n = float(g["params"])
+    W = np.random.default_rng(13).normal(0, 0.02, size=64 * 256 * 8).astype(np.float32)
+    q = oracle.quantize(W, dq=True)
+    per_param = (q.codes.nbytes + q.q8.nbytes + q.cg.nbytes) / W.size
+    assert per_param == 0.5 + 1 / 64 + 4 / (64 * 256)
+    assert round(n * 2 / 1e9) == int(g["bf16_gb"])
+    assert round(n * per_param / 1e9) == int(g["nf4_gb_approx"])       # 6.70 GB
