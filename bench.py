@@ -132,12 +132,18 @@ class ClockSampler:
 # --------------------------------------------------------------------------
 # CPU oracle on a bounded sample (the reported baseline and the reference arm)
 # --------------------------------------------------------------------------
-def oracle_sample_step(w, inp, tokens):
+def oracle_weight(w, inp):
+    """The workload's frozen weight quantised once by the oracle (not timed: it is
+    not part of a training step)."""
+    import oracle
+    return oracle.quantize(inp["W0"].numpy().reshape(-1), dq=w.double_quant)
+
+
+def oracle_sample_step(w, inp, tokens, qw):
     """Oracle forward+backward on the first `tokens` tokens of the workload.
     Returns (flops, seconds)."""
     import oracle
     bits = workloads.bf16_bits
-    qw = oracle.quantize(inp["W0"].numpy().reshape(-1), dq=w.double_quant)
     x, A, B = bits(inp["x"][:tokens]), bits(inp["A"]), bits(inp["B"])
     dY = bits(inp["dY"][:tokens])
     t0 = time.perf_counter()
@@ -162,11 +168,12 @@ def run_reference(args, rank, world):
     w = workloads.WORKLOADS[MAIN]
     tokens = 4
     inp = workloads.make_inputs(w, M=tokens)
+    qw = oracle_weight(w, inp)
     for _ in range(args.warmup):
-        oracle_sample_step(w, inp, tokens)
+        oracle_sample_step(w, inp, tokens, qw)
     tot_f, tot_t = 0, 0.0
     for _ in range(args.steps):
-        f, t = oracle_sample_step(w, inp, tokens)
+        f, t = oracle_sample_step(w, inp, tokens, qw)
         tot_f += f
         tot_t += t
     value = tot_f / tot_t / 1e12
@@ -787,8 +794,9 @@ def cpu_baseline_leg(w, inp, target_s=12.0):
     (at most 8x per try) until one try takes half of target_s or covers every
     token, so the timed try takes roughly 5 to 20 s on the host."""
     tokens = 16
+    qw = oracle_weight(w, inp)
     while True:
-        f, t = oracle_sample_step(w, inp, tokens)
+        f, t = oracle_sample_step(w, inp, tokens, qw)
         if t >= 0.5 * target_s or tokens >= w.M:
             break
         tokens = int(min(w.M, tokens * min(8.0, max(2.0, target_s / max(t, 1e-3)))))
