@@ -330,8 +330,14 @@ def main():
         "kernels": kernels,
     }
 
-    if rank == 0 and not args.skip_extras:
-        line["e2e"] = e2e_leg(q, dp, qw, inp, w, args, dev, world)
+    if not args.skip_extras:
+        # every rank takes the same collective steps in the end-to-end leg
+        e2e = e2e_leg(q, dp, qw, inp, w, args, dev, world)
+        if rank == 0:
+            line["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.skip_extras:
+        # single-GPU legs: at N > 1 the other ranks would wait in the closing
+        # barrier for minutes, beyond the process group's timeout
         line["decode"] = decode_leg(q, dev, peaks)
         line["quantize"] = quantize_leg(q, dev, peaks)
         line["mlp70b"] = mlp70b_leg(q, dev, peaks)
@@ -341,8 +347,6 @@ def main():
         line["block128"] = block128_leg(q, dev, peaks)
         line["dropout"] = dropout_leg(q, dev, peaks)
         line["cpu_baseline"] = cpu_baseline_leg(w, inp)
-    elif not args.skip_extras:
-        e2e_leg(q, dp, qw, inp, w, args, dev, world)  # same collectives on every rank
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
