@@ -123,6 +123,56 @@ def _need_cuda(*ts: torch.Tensor):
             raise ValueError("all tensors must be CUDA tensors (the library has no CPU path)")
 
 
+# The C entry points take raw pointers and the sizes below; they cannot see a
+# tensor's extent, so every tensor is checked here against the shape the call
+# implies before its pointer is passed on.
+def _check_t(name: str, t: torch.Tensor, shape, dtype, device) -> None:
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the weight on {device}")
+
+
+def _layer_args(qw: "QuantizedWeight", x: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
+                rank_cols: Optional[int] = None) -> Tuple[int, int]:
+    """(M, r) of x [M, k], A [r, k] and B [n, r] (B [n, rank_cols] when given)."""
+    if x.dim() != 2 or A.dim() != 2:
+        raise ValueError("x and A must be 2-D")
+    M, r = x.shape[0], A.shape[0]
+    _check_t("x", x, (M, qw.k), torch.bfloat16, qw.device)
+    _check_t("A", A, (r, qw.k), torch.bfloat16, qw.device)
+    _check_t("B", B, (qw.n, r if rank_cols is None else rank_cols), torch.bfloat16, qw.device)
+    return M, r
+
+
+def _check_ws(ws: Optional[torch.Tensor], device) -> None:
+    if ws is not None:
+        if ws.dtype != torch.uint8 or ws.dim() != 1 or not ws.is_contiguous() or ws.device != device:
+            raise ValueError("workspace must be a contiguous 1-D uint8 tensor on the weight's device")
+
+
+def _check_keep(keep: torch.Tensor, M: int, k: int, device) -> None:
+    _check_t("keep", keep, (M * k // 8,), torch.uint8, device)
+
+
+def _check_bwd(qw: "QuantizedWeight", M: int, r: int, dY: torch.Tensor, u: Optional[torch.Tensor],
+               outs: Optional[tuple], workspace: Optional[torch.Tensor]) -> None:
+    _check_t("dY", dY, (M, qw.n), torch.bfloat16, qw.device)
+    if u is not None:
+        _check_t("u", u, (M, r), torch.float32, qw.device)
+    if outs is not None:
+        dX, dA, dB = outs
+        if dX is not None:
+            _check_t("dX", dX, (M, qw.k), torch.bfloat16, qw.device)
+        _check_t("dA", dA, (r, qw.k), torch.bfloat16, qw.device)
+        _check_t("dB", dB, (qw.n, r), torch.bfloat16, qw.device)
+    _check_ws(workspace, qw.device)
+
+
 @dataclass
 class QuantizedWeight:
     """A frozen NF4 weight: device tensors owned by this object."""
@@ -136,6 +186,7 @@ class QuantizedWeight:
     block_size: int = BLOCK_SIZE         # 64 or 128 elements per block
 
     def struct(self) -> NF4WeightStruct:
+        self._check_arrays()
         return NF4WeightStruct(self.n, self.k, self.block_size, int(self.double_quant),
                                self.codes.data_ptr(), self.absmax.data_ptr(),
                                self.absmax_q8.data_ptr() if self.absmax_q8 is not None else None,
@@ -144,6 +195,23 @@ class QuantizedWeight:
     @property
     def device(self) -> torch.device:
         return self.codes.device
+
+    def _check_arrays(self) -> None:
+        """The arrays hold at least the entries the C library reads or writes."""
+        if self.block_size not in (64, 128):
+            raise ValueError("block_size must be 64 or 128")
+        nb = self.n * self.k // self.block_size
+        need = [("codes", self.codes, torch.uint8, self.n * self.k // 2),
+                ("absmax", self.absmax, torch.float32, nb)]
+        if self.double_quant:
+            need += [("absmax_q8", self.absmax_q8, torch.uint8, nb),
+                     ("absmax_c", self.absmax_c, torch.float32, (nb + 255) // 256)]
+        for name, t, dtype, count in need:
+            if t is None:
+                raise ValueError(f"{name} is required")
+            if t.dtype != dtype or not t.is_contiguous() or t.numel() < count or t.device != self.device:
+                raise ValueError(f"{name}: expected a contiguous {dtype} tensor of at least {count} "
+                                 f"entries on {self.device}")
 
     @staticmethod
     def empty(n: int, k: int, double_quant: bool, device, block_size: int = BLOCK_SIZE) -> "QuantizedWeight":
@@ -172,6 +240,9 @@ def nf4_quantize(W0: torch.Tensor, double_quant: bool = True,
     if W0.dtype not in _DTYPES or W0.dim() != 2 or not W0.is_contiguous():
         raise ValueError("W0 must be a contiguous 2-D float32, bfloat16 or float16 tensor")
     n, k = W0.shape
+    if out is not None and ((out.n, out.k) != (n, k) or bool(out.double_quant) != bool(double_quant)
+                            or out.device != W0.device):
+        raise ValueError("out must be a weight of W0's shape, double-quant flag and device")
     qw = out if out is not None else QuantizedWeight.empty(n, k, double_quant, W0.device, block_size)
     s = qw.struct()
     if W0.dtype == torch.float32:
@@ -207,9 +278,13 @@ def qlora_linear_fwd(qw: QuantizedWeight, x: torch.Tensor, A: torch.Tensor, B: t
                      workspace: Optional[torch.Tensor] = None, u: Optional[torch.Tensor] = None
                      ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """h = x W~^T + (alpha/r)(x A^T) B^T; also returns u = x A^T (fp32) if save_u."""
+    M, r = _layer_args(qw, x, A, B)
+    if h is not None:
+        _check_t("h", h, (M, qw.n), torch.bfloat16, qw.device)
+    if u is not None:
+        _check_t("u", u, (M, r), torch.float32, qw.device)
+    _check_ws(workspace, qw.device)
     _need_cuda(x, A, B)
-    M = x.shape[0]
-    r = A.shape[0]
     if h is None:
         h = torch.empty(M, qw.n, dtype=torch.bfloat16, device=x.device)
     if u is None and save_u:
@@ -231,9 +306,12 @@ def qlora_linear_fwd_noalloc(qw: QuantizedWeight, x: torch.Tensor, A: torch.Tens
     4 MiB device scratch, for callers that cannot allocate device memory while
     they run (see the C header for the token limit). Pass preallocated `h` and
     `u` to make the call itself allocation-free."""
+    M, r = _layer_args(qw, x, A, B)
+    if h is not None:
+        _check_t("h", h, (M, qw.n), torch.bfloat16, qw.device)
+    if u is not None:
+        _check_t("u", u, (M, r), torch.float32, qw.device)
     _need_cuda(x, A, B)
-    M = x.shape[0]
-    r = A.shape[0]
     if h is None:
         h = torch.empty(M, qw.n, dtype=torch.bfloat16, device=x.device)
     if u is None and save_u:
@@ -250,9 +328,9 @@ def qlora_linear_bwd(qw: QuantizedWeight, x: torch.Tensor, A: torch.Tensor, B: t
                      need_dX: bool = True, workspace: Optional[torch.Tensor] = None,
                      outs: Optional[tuple] = None):
     """(dX, dA, dB) of the layer; dX is None when need_dX is False."""
+    M, r = _layer_args(qw, x, A, B)
+    _check_bwd(qw, M, r, dY, u, outs, workspace)
     _need_cuda(x, A, B, dY)
-    M = x.shape[0]
-    r = A.shape[0]
     if outs is not None:
         dX, dA, dB = outs
     else:
@@ -276,11 +354,15 @@ def qlora_multi_lora_fwd(qw: QuantizedWeight, x: torch.Tensor, A_all: torch.Tens
     """h[m] = x[m] W~^T + (alphas[a]/r)(x[m] A_a^T) B_a^T with a = adapter_of_token[m]
     (int32 CUDA tensor; values outside [0, len(alphas)) mean no adapter). A_all stacks
     the adapters' A as [n_adapters * r, k], B_all their B as [n, n_adapters * r]."""
-    _need_cuda(x, A_all, B_all, adapter_of_token)
-    if adapter_of_token.dtype != torch.int32:
-        raise ValueError("adapter_of_token must be int32")
-    M = x.shape[0]
     n_ad = len(alphas)
+    if n_ad < 1 or A_all.dim() != 2 or A_all.shape[0] != n_ad * r:
+        raise ValueError("A_all must stack len(alphas) adapters of rank r: [len(alphas) * r, k]")
+    M, _ = _layer_args(qw, x, A_all, B_all)
+    _check_t("adapter_of_token", adapter_of_token, (M,), torch.int32, qw.device)
+    if h is not None:
+        _check_t("h", h, (M, qw.n), torch.bfloat16, qw.device)
+    _check_ws(workspace, qw.device)
+    _need_cuda(x, A_all, B_all, adapter_of_token)
     if h is None:
         h = torch.empty(M, qw.n, dtype=torch.bfloat16, device=x.device)
     nbytes = fwd_workspace_bytes(M, qw.n, qw.k, n_ad * r)
@@ -297,8 +379,14 @@ def qlora_merge(qw: QuantizedWeight, A: torch.Tensor, B: torch.Tensor, alpha: fl
                 bf16: bool = True, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """W~ + (alpha/r) B A as a [n, k] tensor (bf16, or fp32 for re-quantisation):
     the adapters folded into the dequantised frozen weight."""
-    _need_cuda(A, B)
+    if A.dim() != 2:
+        raise ValueError("A must be 2-D")
     r = A.shape[0]
+    _check_t("A", A, (r, qw.k), torch.bfloat16, qw.device)
+    _check_t("B", B, (qw.n, r), torch.bfloat16, qw.device)
+    if out is not None:
+        _check_t("out", out, (qw.n, qw.k), torch.bfloat16 if bf16 else torch.float32, qw.device)
+    _need_cuda(A, B)
     if out is None:
         out = torch.empty(qw.n, qw.k, dtype=torch.bfloat16 if bf16 else torch.float32,
                           device=qw.device)
@@ -322,8 +410,12 @@ def qlora_linear_fwd_dropout(qw: QuantizedWeight, x: torch.Tensor, A: torch.Tens
                              workspace: Optional[torch.Tensor] = None):
     """Forward with LoRA dropout; keep is the packed bit mask over x (see pack_keep).
     Returns (h, u) with u = (keep . x) A^T."""
+    M, r = _layer_args(qw, x, A, B)
+    _check_keep(keep, M, qw.k, qw.device)
+    if h is not None:
+        _check_t("h", h, (M, qw.n), torch.bfloat16, qw.device)
+    _check_ws(workspace, qw.device)
     _need_cuda(x, A, B, keep)
-    M, r = x.shape[0], A.shape[0]
     if h is None:
         h = torch.empty(M, qw.n, dtype=torch.bfloat16, device=x.device)
     u = torch.empty(M, r, dtype=torch.float32, device=x.device) if save_u else None
@@ -341,8 +433,10 @@ def qlora_linear_bwd_dropout(qw: QuantizedWeight, x: torch.Tensor, A: torch.Tens
                              need_dX: bool = True, workspace: Optional[torch.Tensor] = None,
                              outs: Optional[tuple] = None):
     """(dX, dA, dB) with LoRA dropout (the mask of the forward)."""
+    M, r = _layer_args(qw, x, A, B)
+    _check_keep(keep, M, qw.k, qw.device)
+    _check_bwd(qw, M, r, dY, u, outs, workspace)
     _need_cuda(x, A, B, dY, keep)
-    M, r = x.shape[0], A.shape[0]
     if outs is not None:
         dX, dA, dB = outs
     else:
