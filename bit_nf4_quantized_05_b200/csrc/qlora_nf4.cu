@@ -1013,7 +1013,8 @@ nf4_status qlora_linear_fwd_dropout(const nf4_weight *w, const uint16_t *x, int6
                                     const uint16_t *A, const uint16_t *B, int32_t r, float alpha,
                                     float p, const uint8_t *keep, uint16_t *h, float *u_out,
                                     void *workspace, size_t ws_bytes, void *stream) {
-    if (!keep) return NF4_ERR_INVALID_ARG;
+    // an empty batch has an empty mask: keep may be null only then
+    if ((M > 0 && !keep) || !(p >= 0.0f && p < 1.0f)) return NF4_ERR_INVALID_ARG;
     return fwd_impl(w, x, M, A, B, r, alpha, p, keep, h, u_out, workspace, ws_bytes, stream);
 }
 
@@ -1229,7 +1230,8 @@ nf4_status qlora_linear_bwd_dropout(const nf4_weight *w, const uint16_t *x, int6
                                     float p, const uint8_t *keep, const uint16_t *dY, const float *u,
                                     uint16_t *dX, uint16_t *dA, uint16_t *dB, void *workspace,
                                     size_t ws_bytes, void *stream) {
-    if (!keep) return NF4_ERR_INVALID_ARG;
+    // an empty batch has an empty mask: keep may be null only then
+    if ((M > 0 && !keep) || !(p >= 0.0f && p < 1.0f)) return NF4_ERR_INVALID_ARG;
     return bwd_impl(w, x, M, A, B, r, alpha, p, keep, dY, u, dX, dA, dB, workspace, ws_bytes, stream);
 }
 

@@ -183,8 +183,8 @@ QLORA_API nf4_status qlora_linear_fwd_noalloc(const nf4_weight *w, const uint16_
  * the masked adapter part added to it before the one rounding to bf16, so the
  * backward's workspace is qlora_bwd_dropout_workspace_bytes (M * k * 4 bytes
  * more than qlora_bwd_workspace_bytes). Otherwise as qlora_linear_fwd /
- * qlora_linear_bwd; a null keep or p outside [0, 1) returns
- * NF4_ERR_INVALID_ARG. */
+ * qlora_linear_bwd; a null keep (allowed only when M == 0) or p outside
+ * [0, 1) returns NF4_ERR_INVALID_ARG. */
 QLORA_API nf4_status qlora_linear_fwd_dropout(const nf4_weight *w, const uint16_t *x, int64_t M,
                                               const uint16_t *A, const uint16_t *B, int32_t r,
                                               float alpha, float p, const uint8_t *keep,

@@ -168,6 +168,8 @@ def test_multi_adapter_and_dropout_argument_checks(q):
     assert fwd_do(p=-0.1) == q.NF4_ERR_INVALID_ARG
     assert fwd_do(p=float("nan")) == q.NF4_ERR_INVALID_ARG
     assert fwd_do(keep=FAKE + 1) == q.NF4_ERR_ALIGNMENT
+    assert fwd_do(M=0, keep=None) == q.NF4_OK                 # an empty batch has an empty mask
+    assert fwd_do(M=0, keep=None, p=1.0) == q.NF4_ERR_INVALID_ARG
     assert fwd_do(wsb=16) == q.NF4_ERR_WORKSPACE
 
     def bwd_do(**kw):

@@ -105,3 +105,14 @@ def test_weight_arrays_are_checked(q):
     shape_refusal("block_size", q.QuantizedWeight(N, K, False, qw.codes, qw.absmax, None, None, 96).struct)
     with pytest.raises(ValueError):
         q.QuantizedWeight.empty(N, K, True, "cpu", block_size=32)
+
+
+def test_empty_batch_arguments_reach_the_device_check(q, args):
+    qw, A, B = args["qw"], args["A"], args["B"]
+    x, dY = bf16(0, K), bf16(0, N)
+    keep = torch.zeros(0, dtype=torch.uint8)
+    cuda_refusal(q.qlora_linear_fwd, qw, x, A, B, 16.0)
+    cuda_refusal(q.qlora_linear_bwd, qw, x, A, B, 16.0, dY, u=torch.zeros(0, R),
+                 outs=(bf16(0, K), bf16(R, K), bf16(N, R)))
+    cuda_refusal(q.qlora_linear_fwd_dropout, qw, x, A, B, 16.0, 0.1, keep)
+    cuda_refusal(q.qlora_linear_bwd_dropout, qw, x, A, B, 16.0, 0.1, keep, dY)

@@ -378,3 +378,33 @@ def test_dropout_full_size_attention_projection(q):
     errs = {"h": rel_err(to_f64(h)[rows], h_ref), "dX": rel_err(to_f64(dX)[rows], dX_ref),
             "dA": rel_err(to_f64(dA), dA_ref), "dB": rel_err(to_f64(dB), dB_ref)}
     assert all(v <= TOL for v in errs.values()), errs
+
+
+def test_empty_batch(q):
+    """M = 0: the forwards write nothing; the backwards write zero dA and dB (the
+    gradient of an empty batch), with or without dropout."""
+    N, K, r = 136, 640, 16
+    w = workloads.LayerWorkload("t", N, K, 1, r, 16.0, 0.02, True, 31)
+    inp = workloads.make_inputs(w)
+    qw = q.nf4_quantize(inp["W0"].cuda(), double_quant=True)
+    A, B = inp["A"].cuda(), inp["B"].cuda()
+    x = torch.empty(0, K, dtype=torch.bfloat16, device="cuda")
+    dY = torch.empty(0, N, dtype=torch.bfloat16, device="cuda")
+    keep = q.pack_keep(torch.ones(0, K, dtype=torch.bool, device="cuda"))
+
+    def nan_outs():
+        return (torch.empty(0, K, dtype=torch.bfloat16, device="cuda"),
+                torch.full((r, K), float("nan"), dtype=torch.bfloat16, device="cuda"),
+                torch.full((N, r), float("nan"), dtype=torch.bfloat16, device="cuda"))
+
+    h, u = q.qlora_linear_fwd(qw, x, A, B, 16.0)
+    outs = nan_outs()
+    q.qlora_linear_bwd(qw, x, A, B, 16.0, dY, u=u, outs=outs)
+    hd, ud = q.qlora_linear_fwd_dropout(qw, x, A, B, 16.0, 0.1, keep)
+    outs_d = nan_outs()
+    q.qlora_linear_bwd_dropout(qw, x, A, B, 16.0, 0.1, keep, dY, u=ud, outs=outs_d)
+    torch.cuda.synchronize()
+    assert q.device_status() == q.NF4_OK
+    assert h.shape == (0, N) and u.shape == (0, r) and hd.shape == (0, N)
+    for t in outs[1:] + outs_d[1:]:
+        assert int(torch.count_nonzero(t)) == 0
