@@ -294,3 +294,24 @@ def test_llama13b_storage_matches_page():
     assert per_param == 0.5 + 1 / 64 + 4 / (64 * 256)
     assert round(n * 2 / 1e9) == int(g["bf16_gb"])
     assert round(n * per_param / 1e9) == int(g["nf4_gb_approx"])       # 6.70 GB
+
+
+def test_quantize_brute_force_random_blocks_and_magnitudes():
+    """Random even block sizes and block magnitudes from 2^-120 to 2^120 (the
+    normalisation w / s is exact-rounded at every scale) against the brute-force
+    quantiser, including blocks that straddle zero with tiny elements."""
+    from hypothesis import given, settings, strategies as st
+
+    @settings(max_examples=60, deadline=None, derandomize=True)
+    @given(st.integers(1, 64).map(lambda h: 2 * h), st.integers(1, 4), st.integers(-120, 120),
+           st.integers(0, 2 ** 32 - 1))
+    def check(block, nblocks, exp, seed):
+        rng = np.random.default_rng(seed)
+        W = (rng.standard_normal(block * nblocks) * 2.0 ** exp).astype(np.float32)
+        W[rng.random(W.size) < 0.1] = 0.0
+        q = oracle.quantize(W, block=block)
+        bc, bs = brute_quantize(W, block)
+        assert np.array_equal(q.codes, bc)
+        assert np.array_equal(q.absmax, bs)
+
+    check()
