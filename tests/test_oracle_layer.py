@@ -284,3 +284,17 @@ def test_block128_with_equal_half_maxima_is_the_64_block_layer():
         assert np.array_equal(g128, g64)
     assert np.array_equal(oracle.qlora_merge(q128, N, K, A, B, r, alpha),
                           oracle.qlora_merge(q64, N, K, A, B, r, alpha))
+
+
+def test_keep_mask_bit_convention():
+    """Element e = m * k + kk of the mask is bit (e & 7) of byte e >> 3 (1 = kept),
+    for the oracle's packer and the binding's (run here on CPU tensors)."""
+    import bit_nf4_quantized_05_b200 as q
+    M, K = 3, 64
+    for e in (0, 1, 7, 8, 63, 64, 100, M * K - 1):
+        keep = np.zeros((M, K), dtype=bool)
+        keep.reshape(-1)[e] = True
+        expect = np.zeros(M * K // 8, dtype=np.uint8)
+        expect[e >> 3] = 1 << (e & 7)
+        assert np.array_equal(oracle.pack_keep(keep), expect)
+        assert np.array_equal(q.pack_keep(torch.from_numpy(keep)).numpy(), expect)
