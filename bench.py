@@ -7,13 +7,16 @@ gradients all-reduced across ranks when N > 1). Workload: the LLaMA-13B-like
 attention projection (W0 5120x5120 NF4 with double quantisation, 2048 tokens,
 r = 16, alpha = 32). value = algorithmic fwd+bwd FLOP/s over all ranks.
 
-Alongside it the same run reports, on rank 0: the decode-shaped forward
-(W0 13824x5120, M in {1,4,16}) as GB/s of 4-bit weight codes, the full-weight
-quantisation of the Llama-2-70B-like MLP weight (28672x8192) as GB/s moved,
-the CPU oracle's speed on a bounded sample, and the end-to-end speed through
-the public API with host buffers.
+Every rank also reports the end-to-end speed through the public API with host
+buffers. At N = 1 the same run adds: the decode-shaped forward (W0 13824x5120,
+M in {1,4,16}) as GB/s of 4-bit weight codes, the full-weight quantisation of
+the Llama-2-70B-like MLP weight (28672x8192) as GB/s moved, that MLP's
+fwd+bwd, the 160-projection stack, the adapter merge, the multi-adapter
+forward, the step with 128-element blocks, the step with LoRA dropout, and
+the CPU oracle's speed on a bounded sample.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                       [--skip-extras] [--leg decode|quantize|stack|mlp70b|merge|multi|block128|dropout]
        (N > 1: launch under torch.distributed.run, one rank per GPU)
 """
 import argparse
