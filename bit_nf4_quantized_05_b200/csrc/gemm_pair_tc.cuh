@@ -1,12 +1,17 @@
 // gemm_pair_tc.cuh -- fused NF4-dequantise + GEMM on CTA pairs
 // (tcgen05.mma.cta_group::2: one 256 x BN MMA spans the two CTAs of a cluster).
 //
-// Same products as gemm_tc.cuh,
+// It computes, in two directions of the QLoRA layer,
 //   forward: D = x W~^T + bf16((alpha/r) x A^T) B^T
 //   dgrad:   D = dY W~  + bf16((alpha/r) dY B) A
 // ("QLoRA explained", section "The LoRA adapter path", and the chain rule
-// through the frozen dequantised weight), but each output tile is 256 tokens
-// x BN columns computed by a pair of CTAs on two SMs:
+// through the frozen dequantised weight). The 4-bit codes stream into shared
+// memory through TMA and are dequantised in registers (a per-block lookup of
+// the 16 scaled levels) straight into the tensor core's 128-byte-swizzled
+// operand layout: K-major for the forward, MN-major for dgrad. The LoRA term
+// is ceil(r/64) extra reduction stages of the same accumulator (r
+// zero-padded to 64). Each output tile is 256 tokens x BN columns computed by
+// a pair of CTAs on two SMs:
 //   CTA v of the pair loads tokens [128v, 128v+128) of the tile (A operand),
 //   dequantises only half of the weight tile -- columns [v BN/2, v BN/2 + BN/2)
 //   of the MMA's B operand -- into its own shared memory, and keeps rows
@@ -29,9 +34,43 @@
 // taking every G-th stage).
 #pragma once
 
-#include "gemm_tc.cuh"
+#include "nf4_common.cuh"
 
 namespace nf4 {
+
+constexpr int kBM = 128;            // tokens per CTA of a pair tile (MMA M = 2 kBM)
+constexpr int kBK = 64;             // reduction per stage = one 64-element NF4 step
+constexpr int kEpiWarp0 = 0;
+constexpr int kTmaAWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kTmaCWarp = 6;
+constexpr int kDequantWarp0 = 7;
+
+struct GemmArgs {
+    int M;              // tokens
+    int red;            // reduction length (forward: K, dgrad: N)
+    int out;            // output columns   (forward: N, dgrad: K)
+    int main_steps;     // ceil(red / 64)
+    int lora_steps;     // ceil(r / 64)
+    int m_tiles, n_tiles;
+    int r;
+    // quantised weight (always the [N, K] weight)
+    int64_t Nw;         // rows of W
+    int64_t Kw;         // columns of W
+    int64_t kblocks;    // K / 64 (64-element steps per W row)
+    const float *absmax;
+    const uint8_t *q8;
+    const float *cg;
+    int dq;
+    const uint16_t *lora_b;   // forward: B [N, r]; dgrad: A [r, K]
+    uint16_t *D;        // [M, out] bf16
+    // stream-K schedule: 0 = whole tiles round-robin
+    int sk;
+    float *partial;     // [pairs][2][BN/32][128][32] fp32 partial tiles
+    int *flags;         // [pairs][2][4 epilogue warps], zero at launch; 1 = rows written
+    float *D32;         // when non-null: the fp32 result goes here instead of D
+    int bshift;         // log2(block size / 64): block of step j is j >> bshift
+};
 
 
 template <int BN, bool DGRAD, int G>

@@ -14,7 +14,6 @@
 #include <vector>
 
 #include "codec.cuh"
-#include "gemm_tc.cuh"
 #include "gemm_pair_tc.cuh"
 #include "skinny_tc.cuh"
 #include "decode_stream.cuh"
@@ -411,64 +410,6 @@ nf4_status skinny_product(int kind, const void *a, int64_t a_rows, int64_t a_col
     return skinny_launch(kind, &sp, 1, stream, zero_ints, zero_count);
 }
 
-template <int BN, bool DGRAD>
-nf4_status launch_gemm(const nf4_weight *w, const uint16_t *act, int64_t M, int64_t red,
-                       int64_t out, const uint16_t *la, int32_t r, const uint16_t *lb,
-                       uint16_t *D, cudaStream_t stream, float *D32 = nullptr) {
-    using Cfg = GemmCfg<BN, DGRAD>;
-    CUtensorMap tm_act, tm_codes, tm_la;
-    const int64_t N = w->n, K = w->k;
-    bool ok = make_map(&tm_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, act, red, M, kBK, kBM,
-                       CU_TENSOR_MAP_SWIZZLE_128B);
-    // 4-bit codes: one 32-byte block column per box (BN rows forward, 64 rows
-    // dgrad), 32-byte swizzle so that eight lanes reading eight rows hit
-    // distinct banks
-    ok = ok && make_map(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, K / 2, N, kBK / 2,
-                        DGRAD ? kBK : BN, CU_TENSOR_MAP_SWIZZLE_32B);
-    // no LoRA stage when la is null (the adapter term is added by another kernel)
-    if (la)
-        ok = ok && make_map(&tm_la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, la, r, M, kBK, kBM,
-                            CU_TENSOR_MAP_SWIZZLE_128B);
-    else
-        tm_la = tm_act;
-    if (!ok) return NF4_ERR_CUDA;
-
-    GemmArgs a{};
-    a.M = static_cast<int>(M);
-    a.red = static_cast<int>(red);
-    a.out = static_cast<int>(out);
-    a.main_steps = static_cast<int>((red + kBK - 1) / kBK);
-    a.lora_steps = la ? (r + kBK - 1) / kBK : 0;
-    a.m_tiles = static_cast<int>((M + kBM - 1) / kBM);
-    a.n_tiles = static_cast<int>((out + BN - 1) / BN);
-    a.r = r;
-    a.Nw = N;
-    a.Kw = K;
-    a.kblocks = K / kBlock;
-    a.bshift = block_shift_of(w->block_size);
-    a.absmax = w->absmax;
-    a.q8 = w->absmax_q8;
-    a.cg = w->absmax_c;
-    a.dq = w->double_quant;
-    a.lora_b = lb;
-    a.D = D;
-    a.D32 = D32;
-
-    const int dev = current_device();
-    const int tiles = a.m_tiles * a.n_tiles;
-    const int grid = std::min(tiles, num_sms(dev));
-    auto kern = qlora_gemm_kernel<BN, DGRAD>;
-    NF4_TRY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      Cfg::kSmemBytes));
-    LaunchTimer t(DGRAD ? KK_GEMM_DGRAD : KK_GEMM_FWD, stream);
-    const cudaError_t e = launch_ex(kern, dim3(grid), dim3(Cfg::kThreads), Cfg::kSmemBytes, stream,
-                                    0u, tm_act, tm_codes, tm_la, a);
-    t.stop();
-    if (e != cudaSuccess) return NF4_ERR_CUDA;
-    NF4_TRY_CUDA(cudaGetLastError());
-    return NF4_OK;
-}
-
 // Clusters of two CTAs of one pair-kernel configuration that can be resident
 // at once on the device (0 if the query fails).
 template <int BN, bool DGRAD, int G>
@@ -686,23 +627,6 @@ nf4_status launch_decode(const nf4_weight *w, const uint16_t *x, int64_t M, cons
     return NF4_OK;
 }
 
-// Output-column tile: the candidate with the smallest (rounds of tiles over
-// the SMs) x (tile width), i.e. the least per-SM time under even tiles.
-int pick_bn(int64_t M, int64_t out, int sms) {
-    const int64_t m_tiles = (M + kBM - 1) / kBM;
-    int best = 256;
-    int64_t best_cost = -1;
-    for (int bn : {256, 192}) {
-        const int64_t tiles = m_tiles * ((out + bn - 1) / bn);
-        const int64_t cost = ((tiles + sms - 1) / sms) * bn;
-        if (best_cost < 0 || cost < best_cost) {
-            best = bn;
-            best_cost = cost;
-        }
-    }
-    return best;
-}
-
 // Pair-tile width: the candidate with the smallest (rounds of 256-token
 // tiles over the resident pairs) x (time of one tile). A tile's time is
 // modelled as proportional to (width + 320): measured on B200, a stage costs
@@ -758,9 +682,8 @@ nf4_status launch_gemm_auto(const nf4_weight *w, const uint16_t *act, int64_t M,
             return launch_gemm_pair<256, DGRAD, kPairGroups>(w, act, M, red, out, la, r, lb, D, stream, nullptr, D32);
         }
     }
-    if (pick_bn(M, out, num_sms(dev)) == 192)
-        return launch_gemm<192, DGRAD>(w, act, M, red, out, la, r, lb, D, stream, D32);
-    return launch_gemm<256, DGRAD>(w, act, M, red, out, la, r, lb, D, stream, D32);
+    // no CTA pair of this kernel can be resident (not the case on a B200)
+    return NF4_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------------------
