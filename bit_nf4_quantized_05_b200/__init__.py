@@ -77,6 +77,8 @@ def _load() -> ctypes.CDLL:
         "qlora_bwd_workspace_bytes": ([i64, i64, i64, i32], sz),
         "qlora_linear_bwd": ([W, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, vp, vp, sz, vp],
                              ctypes.c_int),
+        "qlora_linear_bwd_f32grad": ([W, vp, i64, vp, vp, i32, f32, vp, vp, vp, vp, vp, vp, sz, vp],
+                                     ctypes.c_int),
         "qlora_linear_fwd_dropout": ([W, vp, i64, vp, vp, i32, f32, f32, vp, vp, vp, vp, sz, vp],
                                      ctypes.c_int),
         "qlora_bwd_dropout_workspace_bytes": ([i64, i64, i64, i32], sz),
@@ -168,8 +170,9 @@ def _check_bwd(qw: "QuantizedWeight", M: int, r: int, dY: torch.Tensor, u: Optio
         dX, dA, dB = outs
         if dX is not None:
             _check_t("dX", dX, (M, qw.k), torch.bfloat16, qw.device)
-        _check_t("dA", dA, (r, qw.k), torch.bfloat16, qw.device)
-        _check_t("dB", dB, (qw.n, r), torch.bfloat16, qw.device)
+        gdt = dA.dtype if dA.dtype in (torch.bfloat16, torch.float32) else torch.bfloat16
+        _check_t("dA", dA, (r, qw.k), gdt, qw.device)
+        _check_t("dB", dB, (qw.n, r), gdt, qw.device)
     _check_ws(workspace, qw.device)
 
 
@@ -326,24 +329,28 @@ def qlora_linear_fwd_noalloc(qw: QuantizedWeight, x: torch.Tensor, A: torch.Tens
 def qlora_linear_bwd(qw: QuantizedWeight, x: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
                      alpha: float, dY: torch.Tensor, u: Optional[torch.Tensor] = None,
                      need_dX: bool = True, workspace: Optional[torch.Tensor] = None,
-                     outs: Optional[tuple] = None):
-    """(dX, dA, dB) of the layer; dX is None when need_dX is False."""
+                     outs: Optional[tuple] = None, grad_dtype: torch.dtype = torch.bfloat16):
+    """(dX, dA, dB) of the layer; dX is None when need_dX is False. The adapter
+    gradients are bf16 (qlora_linear_bwd) or fp32 (qlora_linear_bwd_f32grad):
+    the dtype of the given outs, else grad_dtype."""
     M, r = _layer_args(qw, x, A, B)
     _check_bwd(qw, M, r, dY, u, outs, workspace)
     _need_cuda(x, A, B, dY)
     if outs is not None:
         dX, dA, dB = outs
     else:
+        if grad_dtype not in (torch.bfloat16, torch.float32):
+            raise ValueError("adapter gradients are bf16 or fp32")
         dX = torch.empty(M, qw.k, dtype=torch.bfloat16, device=x.device) if need_dX else None
-        dA = torch.empty(r, qw.k, dtype=torch.bfloat16, device=x.device)
-        dB = torch.empty(qw.n, r, dtype=torch.bfloat16, device=x.device)
+        dA = torch.empty(r, qw.k, dtype=grad_dtype, device=x.device)
+        dB = torch.empty(qw.n, r, dtype=grad_dtype, device=x.device)
     nbytes = bwd_workspace_bytes(M, qw.n, qw.k, r)
     ws = workspace if workspace is not None else _workspace(nbytes, x.device)
     s = qw.struct()
-    _check(lib.qlora_linear_bwd(ctypes.byref(s), _ptr(x), M, _ptr(A), _ptr(B), r, float(alpha),
-                                _ptr(dY), _ptr(u), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws),
-                                ws.numel(), _stream(x.device)),
-           "qlora_linear_bwd")
+    fn, name = ((lib.qlora_linear_bwd_f32grad, "qlora_linear_bwd_f32grad") if dA.dtype == torch.float32
+                else (lib.qlora_linear_bwd, "qlora_linear_bwd"))
+    _check(fn(ctypes.byref(s), _ptr(x), M, _ptr(A), _ptr(B), r, float(alpha), _ptr(dY), _ptr(u),
+              _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws), ws.numel(), _stream(x.device)), name)
     return dX, dA, dB
 
 

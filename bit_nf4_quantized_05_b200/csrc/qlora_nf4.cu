@@ -1054,10 +1054,12 @@ nf4_status lora_add(const float *base, const uint16_t *Vs, const uint16_t *A, co
 
 // Backward, with LoRA dropout when keep is non-null (u, when given, is the
 // forward's masked u = (keep . x) A^T).
+// Adapter gradients in bf16 (dA, dB) or, when grads32 is set, in fp32 (the
+// same pointers, as float).
 nf4_status bwd_impl(const nf4_weight *w, const uint16_t *x, int64_t M, const uint16_t *A,
                     const uint16_t *B, int32_t r, float alpha, float p, const uint8_t *keep,
-                    const uint16_t *dY, const float *u, uint16_t *dX, uint16_t *dA, uint16_t *dB,
-                    void *workspace, size_t ws_bytes, void *stream) {
+                    const uint16_t *dY, const float *u, uint16_t *dX, void *dA, void *dB,
+                    void *workspace, size_t ws_bytes, void *stream, bool grads32 = false) {
     nf4_status st = check_layer(w, x, M, A, B, r, alpha);
     if (st != NF4_OK) return st;
     if (keep && !(p >= 0.0f && p < 1.0f)) return NF4_ERR_INVALID_ARG;
@@ -1069,9 +1071,12 @@ nf4_status bwd_impl(const nf4_weight *w, const uint16_t *x, int64_t M, const uin
     const int64_t N = w->n, K = w->k;
     if (M == 0) {
         LaunchTimer t(KK_ZERO, s);
-        const cudaError_t e1 = launch_ex(zero_u16_kernel, dim3(64), dim3(256), 0, s, 0u, dA,
-                                         int64_t(r) * K);
-        const cudaError_t e2 = launch_ex(zero_u16_kernel, dim3(64), dim3(256), 0, s, 0u, dB, N * r);
+        // zero gradients: 2-byte words, twice as many for fp32
+        const int64_t per = grads32 ? 2 : 1;
+        const cudaError_t e1 = launch_ex(zero_u16_kernel, dim3(64), dim3(256), 0, s, 0u,
+                                         static_cast<uint16_t *>(dA), per * int64_t(r) * K);
+        const cudaError_t e2 = launch_ex(zero_u16_kernel, dim3(64), dim3(256), 0, s, 0u,
+                                         static_cast<uint16_t *>(dB), per * N * r);
         t.stop();
         if (e1 != cudaSuccess || e2 != cudaSuccess) return NF4_ERR_CUDA;
         NF4_TRY_CUDA(cudaGetLastError());
@@ -1114,8 +1119,15 @@ nf4_status bwd_impl(const nf4_weight *w, const uint16_t *x, int64_t M, const uin
     // dB = dY^T bf16(s u) ([N, r]) and dA = (x^T bf16(s v))^T ([r, K]) in one launch (under
     // dropout dA takes the masked x), which also clears the dgrad GEMM's stream-K flags
     {
-        SkinnySpec j[2] = {{dY, M, N, Major::MN, u_s, M, r, Major::MN, r, nullptr, dB, 1.0f, 0},
-                           {x, M, K, Major::MN, v_s, M, r, Major::MN, r, nullptr, dA, 1.0f, 1}};
+        SkinnySpec j[2] = {{dY, M, N, Major::MN, u_s, M, r, Major::MN, r, nullptr, nullptr, 1.0f, 0},
+                           {x, M, K, Major::MN, v_s, M, r, Major::MN, r, nullptr, nullptr, 1.0f, 1}};
+        if (grads32) {
+            j[0].out_f32 = static_cast<float *>(dB);
+            j[1].out_f32 = static_cast<float *>(dA);
+        } else {
+            j[0].out_bf16 = static_cast<uint16_t *>(dB);
+            j[1].out_bf16 = static_cast<uint16_t *>(dA);
+        }
         if (keep) {
             j[1].mask_mode = 2;
             j[1].keep = keep;
@@ -1140,6 +1152,14 @@ nf4_status qlora_linear_bwd(const nf4_weight *w, const uint16_t *x, int64_t M, c
                             void *workspace, size_t ws_bytes, void *stream) {
     return bwd_impl(w, x, M, A, B, r, alpha, 0.0f, nullptr, dY, u, dX, dA, dB, workspace, ws_bytes,
                     stream);
+}
+
+nf4_status qlora_linear_bwd_f32grad(const nf4_weight *w, const uint16_t *x, int64_t M,
+                                    const uint16_t *A, const uint16_t *B, int32_t r, float alpha,
+                                    const uint16_t *dY, const float *u, uint16_t *dX, float *dA,
+                                    float *dB, void *workspace, size_t ws_bytes, void *stream) {
+    return bwd_impl(w, x, M, A, B, r, alpha, 0.0f, nullptr, dY, u, dX, dA, dB, workspace, ws_bytes,
+                    stream, true);
 }
 
 size_t qlora_bwd_dropout_workspace_bytes(int64_t M, int64_t n, int64_t k, int32_t r) {

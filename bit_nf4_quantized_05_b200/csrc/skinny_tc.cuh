@@ -35,7 +35,7 @@ struct SkinnyJob {
     int steps;           // reduction steps of 64
     int steps_per_split;
     int r;               // output columns actually written (<= RN)
-    float *out_f32;      // [P][r] sum, or null
+    float *out_f32;      // the sum in fp32 (unscaled): [P][r], or [r][P] when transposed; or null
     uint16_t *out_bf16;  // bf16(scale * sum): [P][r], or [r][P] when transposed; or null
     float scale;
     int transposed;
@@ -278,7 +278,9 @@ skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a0,
             float acc = 0.0f;
             for (int s = 0; s < splits; ++s)
                 acc += ld_cluster_f32(mapa_shared(part_addr + off, static_cast<uint32_t>(s)));
-            if (J.out_f32) J.out_f32[static_cast<int64_t>(p) * r + j] = acc;
+            const int64_t o = J.transposed ? static_cast<int64_t>(j) * J.P + p
+                                           : static_cast<int64_t>(p) * r + j;
+            if (J.out_f32) J.out_f32[o] = acc;
             if (J.out_bf16) {
                 float sc = J.scale;
                 if (args.row_group) {
@@ -287,8 +289,6 @@ skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a0,
                     sc = keep ? args.gscale[gp] : 0.0f;
                 }
                 __nv_bfloat16 b = __float2bfloat16_rn(sc * acc);
-                const int64_t o = J.transposed ? static_cast<int64_t>(j) * J.P + p
-                                               : static_cast<int64_t>(p) * r + j;
                 J.out_bf16[o] = *reinterpret_cast<uint16_t *>(&b);
             }
         }

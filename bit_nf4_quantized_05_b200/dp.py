@@ -24,8 +24,12 @@ def shard_rows(M: int, rank: int, world: int) -> Tuple[int, int]:
     return start, start + base + (1 if rank < extra else 0)
 
 
-def grad_buffer(r: int, k: int, n: int, dtype=torch.bfloat16, device=None):
-    """One flat buffer holding dA [r, k] then dB [n, r]; returns (flat, dA, dB)."""
+def grad_buffer(r: int, k: int, n: int, dtype=torch.float32, device=None):
+    """One flat buffer holding dA [r, k] then dB [n, r]; returns (flat, dA, dB).
+
+    fp32 by default: the backward then writes the adapter gradients in fp32
+    (qlora_linear_bwd_f32grad) and the ranks sum them in fp32, so the reduced
+    gradient carries no bf16 rounding of the per-rank partial sums."""
     flat = torch.empty(r * k + n * r, dtype=dtype, device=device)
     return flat, flat[: r * k].view(r, k), flat[r * k:].view(n, r)
 

@@ -236,6 +236,19 @@ QLORA_API nf4_status qlora_linear_bwd(const nf4_weight *w, const uint16_t *x, in
                             const uint16_t *dY, const float *u, uint16_t *dX, uint16_t *dA,
                             uint16_t *dB, void *workspace, size_t ws_bytes, void *stream);
 
+/* qlora_linear_bwd with the adapter gradients written in fp32: dA [r, k] and
+ * dB [n, r] receive the fp32 sums of their products (the same sums that
+ * qlora_linear_bwd rounds to bf16), so that data-parallel ranks add their
+ * gradients in fp32 before the optimiser step (the adapters are the only
+ * trained parameters, "QLoRA explained", section "The LoRA adapter path").
+ * dX stays bf16. Same arguments, requirements and workspace as
+ * qlora_linear_bwd; M == 0 writes zeros. */
+QLORA_API nf4_status qlora_linear_bwd_f32grad(const nf4_weight *w, const uint16_t *x, int64_t M,
+                                              const uint16_t *A, const uint16_t *B, int32_t r,
+                                              float alpha, const uint16_t *dY, const float *u,
+                                              uint16_t *dX, float *dA, float *dB, void *workspace,
+                                              size_t ws_bytes, void *stream);
+
 /* Adapter merge for inference without adapters ("QLoRA explained", section
  * "Merging and deploying"; "How Fine-Tuning LLMs with LoRA and QLoRA Works",
  * FAQ on merging: W_new = W + (alpha/r) B A):

@@ -58,6 +58,14 @@ def lib() -> ctypes.CDLL:
         L.oracle_qlora_bwd.argtypes = [vp, vp, vp, vp, i32, i64, i64, vp, i64, vp, vp, i32,
                                        f64, vp, vp, i64, vp, vp, vp]
         L.oracle_qlora_bwd.restype = ctypes.c_int
+        L.oracle_dequant_operand.argtypes = [vp, vp, vp, vp, i64, i64, i32, vp]
+        L.oracle_dequant_operand.restype = None
+        L.oracle_qlora_fwd_rows_op.argtypes = [vp, i64, i64, vp, i64, vp, vp, i32, f64, vp, i64,
+                                               vp, vp]
+        L.oracle_qlora_fwd_rows_op.restype = ctypes.c_int
+        L.oracle_qlora_bwd_op.argtypes = [vp, i64, i64, vp, i64, vp, vp, i32, f64, vp, vp, i64,
+                                          vp, vp, vp]
+        L.oracle_qlora_bwd_op.restype = ctypes.c_int
         L.oracle_qlora_merge.argtypes = [vp, vp, vp, vp, i32, i64, i64, vp, vp, i32, f64, vp]
         L.oracle_qlora_merge.restype = ctypes.c_int
         L.oracle_qlora_multi_fwd_rows.argtypes = [vp, vp, vp, vp, i32, i64, i64, vp, i64, vp, vp,
@@ -263,6 +271,61 @@ def qlora_bwd(qw: Quantized, N: int, K: int, x: np.ndarray, A: np.ndarray, B: np
                                 _ptr(dA), _ptr(dB))
     if rc != 0:
         raise OracleError(f"oracle_qlora_bwd failed ({rc})")
+    return dX, dA, dB
+
+
+def dequant_operand(qw: Quantized, N: int, K: int) -> np.ndarray:
+    """The bf16 matmul operand RNE_bf16(fl32(scale * NF4[q])) of the whole
+    weight, as fp32 [N, K] (reading R6). The layer functions form it on every
+    call; forming it once lets a caller run many batches through one frozen
+    weight (the *_op functions below)."""
+    qw = _check_layer(qw, N, K)
+    out = np.zeros((N, K), dtype=np.float32)
+    lib().oracle_dequant_operand(_ptr(qw.codes), _ptr(qw.absmax), _ptr(qw.q8), _ptr(qw.cg),
+                                 N, K, int(qw.dq), _ptr(out))
+    return out
+
+
+def qlora_fwd_rows_op(Wt: np.ndarray, x: np.ndarray, A: np.ndarray, B: np.ndarray, r: int,
+                      alpha: float, rows: Optional[Sequence[int]] = None):
+    """qlora_fwd_rows with the dequantised operand Wt [N, K] given."""
+    Wt = np.ascontiguousarray(Wt, dtype=np.float32)
+    N, K = Wt.shape
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    A = np.ascontiguousarray(A, dtype=np.uint16)
+    B = np.ascontiguousarray(B, dtype=np.uint16)
+    M = x.shape[0]
+    assert x.shape == (M, K) and A.shape == (r, K) and B.shape == (N, r)
+    rows = np.arange(M, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    h = np.zeros((rows.size, N), dtype=np.float64)
+    u = np.zeros((rows.size, r), dtype=np.float64)
+    rc = lib().oracle_qlora_fwd_rows_op(_ptr(Wt), N, K, _ptr(x), M, _ptr(A), _ptr(B), r,
+                                        float(alpha), _ptr(rows), rows.size, _ptr(h), _ptr(u))
+    if rc != 0:
+        raise OracleError(f"oracle_qlora_fwd_rows_op failed ({rc})")
+    return h, u
+
+
+def qlora_bwd_op(Wt: np.ndarray, x: np.ndarray, A: np.ndarray, B: np.ndarray, r: int,
+                 alpha: float, dY: np.ndarray, dx_rows: Optional[Sequence[int]] = None):
+    """qlora_bwd with the dequantised operand Wt [N, K] given."""
+    Wt = np.ascontiguousarray(Wt, dtype=np.float32)
+    N, K = Wt.shape
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    A = np.ascontiguousarray(A, dtype=np.uint16)
+    B = np.ascontiguousarray(B, dtype=np.uint16)
+    dY = np.ascontiguousarray(dY, dtype=np.uint16)
+    M = x.shape[0]
+    assert dY.shape == (M, N)
+    rows = np.arange(M, dtype=np.int64) if dx_rows is None else np.ascontiguousarray(dx_rows, dtype=np.int64)
+    dX = np.zeros((rows.size, K), dtype=np.float64)
+    dA = np.zeros((r, K), dtype=np.float64)
+    dB = np.zeros((N, r), dtype=np.float64)
+    rc = lib().oracle_qlora_bwd_op(_ptr(Wt), N, K, _ptr(x), M, _ptr(A), _ptr(B), r, float(alpha),
+                                   _ptr(dY), _ptr(rows), rows.size, _ptr(dX) if rows.size else None,
+                                   _ptr(dA), _ptr(dB))
+    if rc != 0:
+        raise OracleError(f"oracle_qlora_bwd_op failed ({rc})")
     return dX, dA, dB
 
 

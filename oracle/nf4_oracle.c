@@ -256,18 +256,24 @@ static double *widen_bf16(const uint16_t *p, int64_t n)
 /* Dequantised weight as the bf16 matmul operand (R6), held as fp32 (every
  * bf16 value is exact in fp32) and widened to fp64 where it is used:
  * Wt[n][k] = RNE_bf16(fl32(scale * NF4[q])). */
-static float *dequant_operand(const uint8_t *codes, const float *absmax,
-                               const uint8_t *q8, const float *cg, int64_t N,
-                               int64_t K, int32_t dq)
+void oracle_dequant_operand(const uint8_t *codes, const float *absmax, const uint8_t *q8,
+                            const float *cg, int64_t N, int64_t K, int32_t dq, float *w)
 {
     int64_t numel = N * K;
-    float *w = (float *)malloc(sizeof(float) * (size_t)numel);
-    if (!w)
-        return NULL;
     oracle_nf4_dequantize(codes, absmax, q8, cg, numel, 64, dq, 256, w);
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < numel; ++i)
         w[i] = (float)oracle_bf16_to_f64(oracle_f32_to_bf16(w[i]));
+}
+
+static float *dequant_operand(const uint8_t *codes, const float *absmax,
+                               const uint8_t *q8, const float *cg, int64_t N,
+                               int64_t K, int32_t dq)
+{
+    float *w = (float *)malloc(sizeof(float) * (size_t)(N * K));
+    if (!w)
+        return NULL;
+    oracle_dequant_operand(codes, absmax, q8, cg, N, K, dq, w);
     return w;
 }
 
@@ -279,19 +285,17 @@ static float *dequant_operand(const uint8_t *codes, const float *absmax,
  *   h_out       nrows x N fp64
  *   u_out       nrows x r fp64 (u = x A^T), may be NULL
  * Returns 0, or ORACLE_ERR_ARG on allocation failure / bad shapes. */
-int oracle_qlora_fwd_rows(const uint8_t *codes, const float *absmax, const uint8_t *q8,
-                          const float *cg, int32_t dq, int64_t N, int64_t K,
-                          const uint16_t *x, int64_t M, const uint16_t *A,
-                          const uint16_t *B, int32_t r, double alpha,
-                          const int64_t *rows, int64_t nrows, double *h_out, double *u_out)
+int oracle_qlora_fwd_rows_op(const float *Wt, int64_t N, int64_t K,
+                             const uint16_t *x, int64_t M, const uint16_t *A,
+                             const uint16_t *B, int32_t r, double alpha,
+                             const int64_t *rows, int64_t nrows, double *h_out, double *u_out)
 {
-    if (N <= 0 || K <= 0 || K % 64 != 0 || r <= 0 || M < 0)
+    if (N <= 0 || K <= 0 || K % 64 != 0 || r <= 0 || M < 0 || !Wt)
         return ORACLE_ERR_ARG;
-    float *Wt = dequant_operand(codes, absmax, q8, cg, N, K, dq);
     double *Ad = widen_bf16(A, (int64_t)r * K);
     double *Bd = widen_bf16(B, N * r);
-    if (!Wt || !Ad || !Bd) {
-        free(Wt); free(Ad); free(Bd);
+    if (!Ad || !Bd) {
+        free(Ad); free(Bd);
         return ORACLE_ERR_ARG;
     }
     const double s = alpha / (double)r;
@@ -330,8 +334,26 @@ int oracle_qlora_fwd_rows(const uint8_t *codes, const float *absmax, const uint8
         free(xr);
         free(u);
     }
-    free(Wt); free(Ad); free(Bd);
+    free(Ad); free(Bd);
     return err ? ORACLE_ERR_ARG : ORACLE_OK;
+}
+
+/* The forward from the quantised weight: its dequantised operand is formed
+ * (oracle_dequant_operand) and the forward above runs on it. */
+int oracle_qlora_fwd_rows(const uint8_t *codes, const float *absmax, const uint8_t *q8,
+                          const float *cg, int32_t dq, int64_t N, int64_t K,
+                          const uint16_t *x, int64_t M, const uint16_t *A,
+                          const uint16_t *B, int32_t r, double alpha,
+                          const int64_t *rows, int64_t nrows, double *h_out, double *u_out)
+{
+    if (N <= 0 || K <= 0 || K % 64 != 0 || r <= 0 || M < 0)
+        return ORACLE_ERR_ARG;
+    float *Wt = dequant_operand(codes, absmax, q8, cg, N, K, dq);
+    if (!Wt)
+        return ORACLE_ERR_ARG;
+    int rc = oracle_qlora_fwd_rows_op(Wt, N, K, x, M, A, B, r, alpha, rows, nrows, h_out, u_out);
+    free(Wt);
+    return rc;
 }
 
 /* Backward of the layer (chain rule; the frozen weight gets no gradient:
@@ -344,12 +366,11 @@ int oracle_qlora_fwd_rows(const uint8_t *codes, const float *absmax, const uint8
  *   dB = s dY^T u                  (N x r, full)
  * All in fp64 from bf16 inputs. dx_out is ndx x K; dA_out r x K; dB_out N x r.
  * Any output pointer may be NULL to skip it. */
-int oracle_qlora_bwd(const uint8_t *codes, const float *absmax, const uint8_t *q8,
-                     const float *cg, int32_t dq, int64_t N, int64_t K,
-                     const uint16_t *x, int64_t M, const uint16_t *A,
-                     const uint16_t *B, int32_t r, double alpha, const uint16_t *dY,
-                     const int64_t *dx_rows, int64_t ndx, double *dx_out,
-                     double *dA_out, double *dB_out)
+int oracle_qlora_bwd_op(const float *Wt, int64_t N, int64_t K,
+                        const uint16_t *x, int64_t M, const uint16_t *A,
+                        const uint16_t *B, int32_t r, double alpha, const uint16_t *dY,
+                        const int64_t *dx_rows, int64_t ndx, double *dx_out,
+                        double *dA_out, double *dB_out)
 {
     if (N <= 0 || K <= 0 || K % 64 != 0 || r <= 0 || M < 0)
         return ORACLE_ERR_ARG;
@@ -381,7 +402,6 @@ int oracle_qlora_bwd(const uint8_t *codes, const float *absmax, const uint8_t *q
 
     int err = 0;
     if (dx_out && ndx > 0) {
-        float *Wt = dequant_operand(codes, absmax, q8, cg, N, K, dq);
         if (!Wt) {
             err = 1;
         } else {
@@ -407,7 +427,6 @@ int oracle_qlora_bwd(const uint8_t *codes, const float *absmax, const uint8_t *q
                     row[k] += s * acc;
                 }
             }
-            free(Wt);
         }
     }
 
@@ -444,6 +463,26 @@ int oracle_qlora_bwd(const uint8_t *codes, const float *absmax, const uint8_t *q
 
     free(Ad); free(Bd); free(v); free(u);
     return err ? ORACLE_ERR_ARG : ORACLE_OK;
+}
+
+/* The backward from the quantised weight: the dequantised operand is formed
+ * only when dX rows are asked for. */
+int oracle_qlora_bwd(const uint8_t *codes, const float *absmax, const uint8_t *q8,
+                     const float *cg, int32_t dq, int64_t N, int64_t K,
+                     const uint16_t *x, int64_t M, const uint16_t *A,
+                     const uint16_t *B, int32_t r, double alpha, const uint16_t *dY,
+                     const int64_t *dx_rows, int64_t ndx, double *dx_out,
+                     double *dA_out, double *dB_out)
+{
+    if (N <= 0 || K <= 0 || K % 64 != 0 || r <= 0 || M < 0)
+        return ORACLE_ERR_ARG;
+    float *Wt = NULL;
+    if (dx_out && ndx > 0)
+        Wt = dequant_operand(codes, absmax, q8, cg, N, K, dq);
+    int rc = oracle_qlora_bwd_op(Wt, N, K, x, M, A, B, r, alpha, dY, dx_rows, ndx, dx_out,
+                                 dA_out, dB_out);
+    free(Wt);
+    return rc;
 }
 
 /* Adapter merge ([P3] "Merging and deploying": the adapters are folded into

@@ -134,6 +134,31 @@ def test_b_zero_is_base_only(q):
     assert float(res["dA"].float().abs().max()) == 0.0   # v = dY B = 0
 
 
+@pytest.mark.parametrize("N,K,M,r,alpha,dq", [SMALL[0], SMALL[2], SMALL[4],
+                                              (5120, 5120, 2048, 16, 32.0, True)])
+def test_fp32_adapter_gradients(q, N, K, M, r, alpha, dq):
+    """qlora_linear_bwd_f32grad: dA and dB in fp32 against the oracle at the
+    bar, and their bf16 rounding is the bf16 entry point's result bit for bit
+    (both round the same fp32 sums; dX is the same launch sequence)."""
+    w = workloads.LayerWorkload("t", N, K, M, r, alpha, 0.02, dq, 999 + N + K + M + r)
+    inp = workloads.make_inputs(w)
+    dev = "cuda"
+    qw = q.nf4_quantize(inp["W0"].to(dev), double_quant=dq)
+    x, A, B, dY = (inp[k].to(dev) for k in ("x", "A", "B", "dY"))
+    h, u = q.qlora_linear_fwd(qw, x, A, B, alpha)
+    dX16, dA16, dB16 = q.qlora_linear_bwd(qw, x, A, B, alpha, dY, u=u)
+    dX32, dA32, dB32 = q.qlora_linear_bwd(qw, x, A, B, alpha, dY, u=u, grad_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert q.device_status() == q.NF4_OK
+    assert dA32.dtype == torch.float32 and dB32.dtype == torch.float32
+    assert torch.equal(dA32.to(torch.bfloat16), dA16) and torch.equal(dB32.to(torch.bfloat16), dB16)
+    assert torch.equal(dX32, dX16)
+    ow = oracle_weight(qw)
+    _, dA_ref, dB_ref = oracle.qlora_bwd(ow, N, K, bits(inp["x"]), bits(inp["A"]), bits(inp["B"]), r,
+                                         alpha, bits(inp["dY"]), dx_rows=[])
+    assert rel_err(to_f64(dA32), dA_ref) <= TOL and rel_err(to_f64(dB32), dB_ref) <= TOL
+
+
 def test_single_1024_workload(q):
     w = workloads.WORKLOADS["single_1024"]
     inp = workloads.make_inputs(w)

@@ -298,3 +298,22 @@ def test_keep_mask_bit_convention():
         expect[e >> 3] = 1 << (e & 7)
         assert np.array_equal(oracle.pack_keep(keep), expect)
         assert np.array_equal(q.pack_keep(torch.from_numpy(keep)).numpy(), expect)
+
+
+@pytest.mark.parametrize("block", [64, 128])
+def test_operand_given_layer_functions_equal_the_plain_ones(block):
+    """The forward and backward run on a dequantised operand formed once equal
+    the functions that form it themselves, bit for bit; the operand is the
+    bf16 image of the codec's dequantised weight."""
+    rng = np.random.default_rng(41)
+    N, K, M, r, alpha = 72, 256, 6, 16, 32.0
+    qw, x, A, B, dY = random_layer(rng, N, K, M, r, True, block=block)
+    Wt = oracle.dequant_operand(qw, N, K)
+    assert np.array_equal(Wt.astype(np.float64), operand(qw, N, K))
+    h, u = oracle.qlora_fwd_rows(qw, N, K, x, A, B, r, alpha)
+    h2, u2 = oracle.qlora_fwd_rows_op(Wt, x, A, B, r, alpha)
+    assert np.array_equal(h, h2) and np.array_equal(u, u2)
+    g = oracle.qlora_bwd(qw, N, K, x, A, B, r, alpha, dY, dx_rows=[5, 1])
+    g2 = oracle.qlora_bwd_op(Wt, x, A, B, r, alpha, dY, dx_rows=[5, 1])
+    for a, b in zip(g, g2):
+        assert np.array_equal(a, b)
