@@ -58,6 +58,13 @@ def lib() -> ctypes.CDLL:
         L.oracle_qlora_bwd.argtypes = [vp, vp, vp, vp, i32, i64, i64, vp, i64, vp, vp, i32,
                                        f64, vp, vp, i64, vp, vp, vp]
         L.oracle_qlora_bwd.restype = ctypes.c_int
+        L.oracle_philox4x32_10.argtypes = [vp, vp, vp]
+        L.oracle_philox4x32_10.restype = None
+        L.oracle_dropout_threshold.argtypes = [ctypes.c_float]
+        L.oracle_dropout_threshold.restype = ctypes.c_uint32
+        L.oracle_dropout_keep_mask.argtypes = [i64, i64, ctypes.c_float, ctypes.c_uint64,
+                                               ctypes.c_uint64, vp]
+        L.oracle_dropout_keep_mask.restype = None
         L.oracle_dequant_operand.argtypes = [vp, vp, vp, vp, i64, i64, i32, vp]
         L.oracle_dequant_operand.restype = None
         L.oracle_qlora_fwd_rows_op.argtypes = [vp, i64, i64, vp, i64, vp, vp, i32, f64, vp, i64,
@@ -430,3 +437,32 @@ def qlora_bwd_dropout(qw: Quantized, N: int, K: int, x: np.ndarray, A: np.ndarra
 def pack_keep(keep_bool: np.ndarray) -> np.ndarray:
     """Bit mask (uint8, bit e & 7 of byte e >> 3) of a boolean keep array, row-major."""
     return np.packbits(np.ascontiguousarray(keep_bool, dtype=bool).reshape(-1), bitorder="little")
+
+
+# --------------------------------------------------------------------------
+# dropout mask drawn from Philox4x32-10 (counter-based; regenerated, not stored)
+# --------------------------------------------------------------------------
+def philox4x32_10(counter: Sequence[int], key: Sequence[int]) -> np.ndarray:
+    """The four 32-bit outputs of Philox4x32-10 for one counter and key."""
+    c = np.ascontiguousarray(counter, dtype=np.uint32)
+    k = np.ascontiguousarray(key, dtype=np.uint32)
+    assert c.size == 4 and k.size == 2
+    out = np.zeros(4, dtype=np.uint32)
+    lib().oracle_philox4x32_10(_ptr(c), _ptr(k), _ptr(out))
+    return out
+
+
+def dropout_threshold(p: float) -> int:
+    """floor(p * 2^32) for an fp32 p: elements whose draw is below it are dropped."""
+    return int(lib().oracle_dropout_threshold(ctypes.c_float(float(np.float32(p)))))
+
+
+def dropout_keep_mask(M: int, K: int, p: float, seed: int, offset: int) -> np.ndarray:
+    """Keep bit mask (pack_keep's convention) of x [M, K] drawn for (seed, offset):
+    element e = m K + k is kept when word e mod 4 of Philox4x32-10 at counter
+    (e div 4 as two 32-bit halves, offset as two halves), key (seed halves) is at
+    least dropout_threshold(p)."""
+    out = np.zeros((M * K + 7) // 8, dtype=np.uint8)
+    lib().oracle_dropout_keep_mask(M, K, ctypes.c_float(float(np.float32(p))), int(seed) & (2 ** 64 - 1),
+                                   int(offset) & (2 ** 64 - 1), _ptr(out))
+    return out

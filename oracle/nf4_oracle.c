@@ -760,3 +760,84 @@ int oracle_qlora_bwd_dropout(const uint8_t *codes, const float *absmax, const ui
     free(Ad); free(Bd); free(v); free(u);
     return err ? ORACLE_ERR_ARG : ORACLE_OK;
 }
+
+/* ------------------------------------------------------------------------ */
+/* LoRA dropout with the mask drawn from a counter-based generator.          */
+/* ------------------------------------------------------------------------ */
+/* [P1] section 1 puts dropout on the LoRA input and [P3]'s recipe uses
+ * lora_dropout = 0.05; the pages name no random generator. Reading: the
+ * draw comes from Philox4x32-10, the counter-based generator of Salmon,
+ * Moraes, Dror and Shaw ("Parallel random numbers: as easy as 1, 2, 3",
+ * SC'11), so that the backward can regenerate the forward's mask from
+ * (seed, offset) instead of storing it.
+ *
+ * One Philox round on the counter (c0, c1, c2, c3) with round key (k0, k1):
+ * the two 32x32 -> 64-bit products hi0:lo0 = 0xD2511F53 * c0 and
+ * hi1:lo1 = 0xCD9E8D57 * c2 give the new counter
+ * (hi1 ^ c1 ^ k0, lo1, hi0 ^ c3 ^ k1, lo0). Ten rounds; the key is bumped by
+ * the Weyl constants (0x9E3779B9, 0xBB67AE85) between rounds. */
+void oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4])
+{
+    uint32_t c0 = ctr[0], c1 = ctr[1], c2 = ctr[2], c3 = ctr[3];
+    uint32_t k0 = key[0], k1 = key[1];
+    for (int round = 0; round < 10; ++round) {
+        if (round > 0) {
+            k0 += 0x9E3779B9u;
+            k1 += 0xBB67AE85u;
+        }
+        uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+        uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+        uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+        uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+        c0 = hi1 ^ c1 ^ k0;
+        c1 = lo1;
+        c2 = hi0 ^ c3 ^ k1;
+        c3 = lo0;
+    }
+    out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+}
+
+/* Drop threshold of probability p: the element is dropped when its 32-bit
+ * draw is below t = floor(p * 2^32), so P(drop) = t / 2^32 (within 2^-32 of
+ * p). p * 2^32 is exact in fp64 for an fp32 p. */
+uint32_t oracle_dropout_threshold(float p)
+{
+    double t = floor((double)p * 4294967296.0);
+    if (!(t > 0.0))
+        return 0u;
+    if (t > 4294967295.0)
+        return 4294967295u;
+    return (uint32_t)t;
+}
+
+/* Keep mask of x [M, K] for one (seed, offset): element e = m*K + k takes
+ * word (e mod 4) of Philox4x32-10 at counter (g_lo, g_hi, offset_lo,
+ * offset_hi), g = e div 4, key (seed_lo, seed_hi); it is kept when that word
+ * is >= oracle_dropout_threshold(p). Written as the bit mask the keep-mask
+ * functions above read: bit (e & 7) of byte e >> 3, 1 = kept; keep holds
+ * ceil(M*K/8) bytes. */
+void oracle_dropout_keep_mask(int64_t M, int64_t K, float p, uint64_t seed, uint64_t offset,
+                              uint8_t *keep)
+{
+    const int64_t n = M * K;
+    const uint32_t t = oracle_dropout_threshold(p);
+    const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    memset(keep, 0, (size_t)((n + 7) / 8));
+#pragma omp parallel for schedule(static)
+    for (int64_t byte = 0; byte < (n + 7) / 8; ++byte) {
+        uint8_t bits = 0;
+        for (int b = 0; b < 8; ++b) {
+            const int64_t e = byte * 8 + b;
+            if (e >= n)
+                break;
+            const uint64_t g = (uint64_t)e >> 2;
+            const uint32_t ctr[4] = {(uint32_t)g, (uint32_t)(g >> 32), (uint32_t)offset,
+                                     (uint32_t)(offset >> 32)};
+            uint32_t w[4];
+            oracle_philox4x32_10(ctr, key, w);
+            if (w[e & 3] >= t)
+                bits |= (uint8_t)(1u << b);
+        }
+        keep[byte] = bits;
+    }
+}
