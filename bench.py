@@ -2,25 +2,30 @@
 """Benchmark of the QLoRA linear layer (NF4 frozen weight + LoRA adapters) on B200.
 
 One step = the layer's forward and backward on one batch of synthetic tokens,
-i.e. h = x W~^T + (alpha/r)(x A^T)B^T, then dX, dA, dB (with the adapter
-gradients all-reduced across ranks when N > 1). Workload: the LLaMA-13B-like
-attention projection (W0 5120x5120 NF4 with double quantisation, 2048 tokens,
-r = 16, alpha = 32). value = algorithmic fwd+bwd FLOP/s over all ranks.
+i.e. h = x W~^T + (alpha/r)(x A^T)B^T, then dX, dA, dB (the adapter gradients
+in fp32, all-reduced across ranks when N > 1). Headline workload: the
+Llama-2-70B-like MLP projection (W0 28672x8192 NF4 with double quantisation,
+8192 tokens per rank, r = 64, alpha = 16), the largest configuration that fits
+one GPU. value = algorithmic fwd+bwd FLOP/s over all ranks.
 
 Every rank also reports the end-to-end speed through the public API with host
-buffers. At N = 1 the same run adds: the decode-shaped forward (W0 13824x5120,
-M in {1,4,16}) as GB/s of 4-bit weight codes, the full-weight quantisation of
-the Llama-2-70B-like MLP weight (28672x8192) as GB/s moved, that MLP's
-fwd+bwd, the 160-projection stack, the adapter merge, the multi-adapter
-forward, the step with 128-element blocks, the step with LoRA dropout, and
-the CPU oracle's speed on a bounded sample.
+buffers. At N = 1 the same run adds, as compact entries of "legs": the
+LLaMA-13B-like attention projection's step (5120x5120, 2048 tokens), the
+160-projection adapter stack, the decode-shaped forward (W0 13824x5120, M in
+{1,4,16}) as GB/s of 4-bit weight codes, the full-weight quantisation of the
+70B MLP weight, the adapter merge, the multi-adapter forward, the step with
+128-element blocks, the steps with LoRA dropout (keep mask given, and drawn in
+the kernels from a counter-based generator), and the CPU oracle's speed on a
+bounded sample of the headline workload. Per-kernel details go to stderr as
+one more JSON line.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                       [--skip-extras] [--leg decode|quantize|stack|mlp70b|merge|multi|block128|dropout]
+                       [--skip-extras] [--leg NAME]
        (N > 1: launch under torch.distributed.run, one rank per GPU)
 """
 import argparse
 import json
+import math
 import os
 import statistics
 import sys
@@ -37,15 +42,17 @@ import torch  # noqa: E402
 import workloads  # noqa: E402
 
 METRIC = "QLoRA linear fwd+bwd TFLOP/s (large M) & NF4 weight GB/s (decode) vs roofline"
-# DRAM bytes (read + write) per launch of the fused GEMM on this workload, mean of the forward and
-# dgrad launches, from one ncu capture of the kernels as they are now (summary and command under
-# profiles/). None whenever the kernel has changed since that capture.
-GEMM_TRAFFIC_BYTES = 42.3e6
-MAIN = "llama13b_attn_5120"
+MAIN = "llama2_70b_mlp_28672x8192"
+ATTN = "llama13b_attn_5120"
 DECODE = "decode_mlp_up_13824x5120"
 QUANT = "llama2_70b_mlp_28672x8192"
 STACK = "llama13b_stack_40x4"
 L2_FLUSH_BYTES = 512 << 20
+# DRAM bytes (read + write) per launch of the fused GEMM, mean of the forward
+# and dgrad launches, per workload, from one ncu capture of the kernels as they
+# are now (summary and command under profiles/). None whenever the kernel has
+# changed since that capture.
+GEMM_TRAFFIC_BYTES = {MAIN: None, ATTN: None}
 
 
 def layer_flops(M, N, K, r):
@@ -53,6 +60,19 @@ def layer_flops(M, N, K, r):
     fwd = 2 * M * N * K + 2 * M * r * (K + N)
     bwd = 2 * M * N * K + 4 * M * N * r + 4 * M * K * r
     return fwd, bwd
+
+
+def gemm_flops(M, N, K, r):
+    """Algorithmic FLOPs of the fused GEMM launches of one step: the forward
+    (x W~^T plus the up-projection stage) and dgrad (dY W~ plus s v A)."""
+    return (2 * M * N * K + 2 * M * N * r) + (2 * M * N * K + 2 * M * K * r)
+
+
+def sig(v, n=4):
+    """v rounded to n significant digits (compact JSON)."""
+    if v is None or not isinstance(v, (int, float)) or v == 0 or not math.isfinite(v):
+        return v
+    return round(v, -int(math.floor(math.log10(abs(v)))) + n - 1)
 
 
 def load_peaks():
@@ -64,6 +84,15 @@ def load_peaks():
                 "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
             "source": "fallback"}
+
+
+def main_config(w, world):
+    """The headline workload as the JSON line's config (both arms)."""
+    return {"workload": f"{w.name}: W0 {w.N}x{w.K} NF4 (blocks of 64, double quant), "
+                        f"x {w.M}x{w.K} bf16 per rank, r={w.r}, alpha={w.alpha:g}, fwd+bwd",
+            "global_batch_tokens": w.M * world, "parallelism": f"dp{world}",
+            "l2": "512 MiB buffer written before every timed step (outside the events); "
+                  "every operand is larger than L2 as well"}
 
 
 # --------------------------------------------------------------------------
@@ -135,28 +164,6 @@ class ClockSampler:
 # --------------------------------------------------------------------------
 # CPU oracle on a bounded sample (the reported baseline and the reference arm)
 # --------------------------------------------------------------------------
-def oracle_weight(w, inp):
-    """The workload's frozen weight quantised once by the oracle (not timed: it is
-    not part of a training step)."""
-    import oracle
-    return oracle.quantize(inp["W0"].numpy().reshape(-1), dq=w.double_quant)
-
-
-def oracle_sample_step(w, inp, tokens, qw):
-    """Oracle forward+backward on the first `tokens` tokens of the workload.
-    Returns (flops, seconds)."""
-    import oracle
-    bits = workloads.bf16_bits
-    x, A, B = bits(inp["x"][:tokens]), bits(inp["A"]), bits(inp["B"])
-    dY = bits(inp["dY"][:tokens])
-    t0 = time.perf_counter()
-    oracle.qlora_fwd_rows(qw, w.N, w.K, x, A, B, w.r, w.alpha)
-    oracle.qlora_bwd(qw, w.N, w.K, x, A, B, w.r, w.alpha, dY)
-    dt = time.perf_counter() - t0
-    f, b = layer_flops(tokens, w.N, w.K, w.r)
-    return f + b, dt
-
-
 def cpu_cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -164,52 +171,161 @@ def cpu_cores():
         return os.cpu_count()
 
 
+class OracleSample:
+    """The oracle on the headline workload, on a few tokens per step. The frozen
+    weight is quantised and dequantised to its bf16 operand once, before any
+    step (the GPU path quantises once too); a step is the oracle's full forward
+    and backward of `tokens` tokens (h and dX rows, and their dA/dB terms)."""
+
+    def __init__(self, w, tokens):
+        import oracle
+        self.w, self.tokens = w, tokens
+        inp = workloads.make_inputs(w, M=tokens)
+        qw = oracle.quantize(inp["W0"].numpy().reshape(-1), dq=w.double_quant)
+        del inp["W0"]
+        self.Wt = oracle.dequant_operand(qw, w.N, w.K)
+        bits = workloads.bf16_bits
+        self.x, self.A, self.B, self.dY = (bits(inp[k]) for k in ("x", "A", "B", "dY"))
+        f, b = layer_flops(tokens, w.N, w.K, w.r)
+        self.flops = f + b
+
+    def step(self):
+        """One step; returns its seconds."""
+        import oracle
+        w = self.w
+        t0 = time.perf_counter()
+        oracle.qlora_fwd_rows_op(self.Wt, self.x, self.A, self.B, w.r, w.alpha)
+        oracle.qlora_bwd_op(self.Wt, self.x, self.A, self.B, w.r, w.alpha, self.dY)
+        return time.perf_counter() - t0
+
+    def describe(self):
+        return (f"{self.tokens} of the {self.w.M} tokens per step: the oracle's forward and "
+                f"backward of those tokens (h and dX rows, dA and dB over them), the weight "
+                f"quantised and dequantised to its bf16 operand once before the steps")
+
+
+def sample_tokens():
+    """Tokens per oracle step: about one per host core (its rows run in parallel)."""
+    return int(min(64, max(8, cpu_cores())))
+
+
 def run_reference(args, rank, world):
     """The oracle as it stands, timed on the host cores (rank 0 only)."""
     if rank != 0:
         return
     w = workloads.WORKLOADS[MAIN]
-    tokens = 4
-    inp = workloads.make_inputs(w, M=tokens)
-    qw = oracle_weight(w, inp)
+    smp = OracleSample(w, sample_tokens())
     for _ in range(args.warmup):
-        oracle_sample_step(w, inp, tokens, qw)
-    tot_f, tot_t = 0, 0.0
+        smp.step()
+    tot_t = 0.0
     for _ in range(args.steps):
-        f, t = oracle_sample_step(w, inp, tokens, qw)
-        tot_f += f
-        tot_t += t
-    value = tot_f / tot_t / 1e12
-    sample = (f"{tokens} of the {w.M} tokens per step: full forward and backward of those "
-              f"tokens (h, dX rows, and their dA/dB contributions), W0 dequantised each step")
+        tot_t += smp.step()
+    value = smp.flops * args.steps / tot_t / 1e12
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{MAIN}: W0 5120x5120 NF4 double-quant, x {w.M}x5120 bf16, "
-                               f"r=16, alpha=32, forward+backward", "parallelism": "cpu-oracle"},
+        "config": main_config(w, world),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
-                         "sample": sample},
+                         "sample": smp.describe()},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
+def cpu_baseline_leg(target_s=12.0):
+    """The oracle on the headline workload, timed like the reference arm: steps of
+    sample_tokens() tokens until about target_s seconds of steps have run."""
+    w = workloads.WORKLOADS[MAIN]
+    smp = OracleSample(w, sample_tokens())
+    smp.step()                                   # warm-up
+    n, t = 0, 0.0
+    while n < 2 or t < target_s:
+        t += smp.step()
+        n += 1
+    return {"value": smp.flops * n / t / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(),
+            "kind": "oracle", "sample": f"{n} steps ({t:.1f} s); " + smp.describe()}
+
+
 # --------------------------------------------------------------------------
 # our arm
 # --------------------------------------------------------------------------
+class LayerRun:
+    """One workload's layer on the device: quantised weight, inputs, outputs,
+    workspaces and the flat fp32 adapter-gradient buffer."""
+
+    def __init__(self, q, dp, w, dev, block=64):
+        self.q, self.dp, self.w = q, dp, w
+        inp = workloads.make_inputs(w)
+        self.qw = q.nf4_quantize(inp.pop("W0").to(dev), double_quant=w.double_quant, block_size=block)
+        self.x, self.A, self.B, self.dY = (inp[k].to(dev) for k in ("x", "A", "B", "dY"))
+        self.inp = inp
+        M, N, K, r = w.M, w.N, w.K, w.r
+        self.h = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        self.u = torch.empty(M, r, dtype=torch.float32, device=dev)
+        self.dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+        self.flat, self.dA, self.dB = dp.grad_buffer(r, K, N, device=dev)
+        self.ws_f = torch.empty(q.fwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
+        self.ws_b = torch.empty(q.bwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
+
+    def step(self, world=1):
+        q, w = self.q, self.w
+        q.qlora_linear_fwd(self.qw, self.x, self.A, self.B, w.alpha, h=self.h, u=self.u, workspace=self.ws_f)
+        q.qlora_linear_bwd(self.qw, self.x, self.A, self.B, w.alpha, self.dY, u=self.u,
+                           workspace=self.ws_b, outs=(self.dX, self.dA, self.dB))
+        self.dp.allreduce_adapter_grads(self.flat, world)
+
+
+def event_steps(step, steps, flush):
+    """Per-step device times (ms): `steps` steps, each bracketed by its own two
+    events, the L2 flush between them outside the events."""
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for s, e in ev:
+        flush.zero_()
+        s.record()
+        step()
+        e.record()
+    torch.cuda.synchronize()
+    return [s.elapsed_time(e) for s, e in ev]
+
+
+def profiled_steps(q, step, steps, flush):
+    """The same steps with the library's per-launch events: {kind: (launches, ms)}."""
+    q.profiling(True)
+    for _ in range(steps):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    q.profiling(False)
+    return q.profile_read()
+
+
+def gemm_roofline(prof, w, steps, peaks):
+    g_launch = sum(prof.get(k, (0, 0.0))[0] for k in ("qlora_gemm_fwd", "qlora_gemm_dgrad"))
+    g_ms = sum(prof.get(k, (0, 0.0))[1] for k in ("qlora_gemm_fwd", "qlora_gemm_dgrad"))
+    g_tflops = steps * gemm_flops(w.M, w.N, w.K, w.r) / (g_ms * 1e-3) / 1e12 if g_ms > 0 else None
+    return {"bound": "tensor", "achieved": g_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": (g_tflops / peaks["bf16_tflops"]) if g_tflops else None,
+            "traffic": GEMM_TRAFFIC_BYTES.get(w.name),
+            "kernel": "qlora_gemm_pair_kernel (forward and dgrad launches)",
+            "peak_source": peaks["source"] + " bf16 burst",
+            "avg_launch_us": 1e3 * g_ms / max(g_launch, 1)}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--skip-extras", action="store_true",
-                    help="only the main fwd+bwd line (no decode/quantize/oracle/e2e legs)")
-    ap.add_argument("--leg", default="all", choices=["all", "decode", "quantize", "stack", "mlp70b",
-                                                     "merge", "multi", "block128", "dropout"],
-                    help="run one secondary leg alone and print its JSON (for profiling)")
+                    help="only the headline fwd+bwd line (no legs, no end-to-end, no oracle)")
+    ap.add_argument("--leg", default="all",
+                    choices=["all", "attn5120", "decode", "quantize", "stack", "merge", "multi",
+                             "block128", "dropout", "dropout_philox", "cpu"],
+                    help="run one leg alone and print its JSON (for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -226,37 +342,24 @@ def main():
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
+    peaks = load_peaks()
     if args.leg != "all":
         if rank == 0:
-            leg = {"decode": decode_leg, "quantize": quantize_leg, "stack": stack_leg,
-                   "mlp70b": mlp70b_leg, "merge": merge_leg, "multi": multi_leg,
-                   "block128": block128_leg, "dropout": dropout_leg}[args.leg]
-            print(json.dumps({"leg": args.leg, **leg(q, dev, load_peaks())}), flush=True)
+            print(json.dumps({"leg": args.leg, **run_leg(args.leg, q, dp, dev, peaks)}), flush=True)
         return
     if world > 1:
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
-    peaks = load_peaks()
 
     w = workloads.WORKLOADS[MAIN]
-    M, N, K, r, alpha = w.M, w.N, w.K, w.r, w.alpha
-    inp = workloads.make_inputs(w)
-    qw = q.nf4_quantize(inp["W0"].to(dev), double_quant=w.double_quant)
-    x, A, B, dY = (inp[k].to(dev) for k in ("x", "A", "B", "dY"))
-    h = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-    u = torch.empty(M, r, dtype=torch.float32, device=dev)
-    dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
-    flat, dA, dB = dp.grad_buffer(r, K, N, device=dev)
-    ws_f = torch.empty(q.fwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
-    ws_b = torch.empty(q.bwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
+    M, N, K, r = w.M, w.N, w.K, w.r
+    run = LayerRun(q, dp, w, dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
-    def step(xx=x, dYY=dY):
-        q.qlora_linear_fwd(qw, xx, A, B, alpha, h=h, u=u, workspace=ws_f)
-        q.qlora_linear_bwd(qw, xx, A, B, alpha, dYY, u=u, workspace=ws_b, outs=(dX, dA, dB))
-        dp.allreduce_adapter_grads(flat, world)
+    def step():
+        run.step(world)
 
     def barrier():
         if world > 1:
@@ -269,32 +372,18 @@ def main():
     if st != q.NF4_OK:
         raise RuntimeError(f"device status after warm-up: {q.status_string(st)}")
 
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
     # Timed region: K steps with only the two step events each (per-launch
     # events would sit between the kernels and stop each launch from
     # overlapping the tail of the one before).
     with ClockSampler(local_rank) as clk:
-        for i in range(args.steps):
-            flush.zero_()                      # L2 flush between timed steps (untimed)
-            starts[i].record()
-            step()
-            ends[i].record()
-        torch.cuda.synchronize()
+        per_step = event_steps(step, args.steps, flush)
     barrier()
     # Kernel durations: the same K steps again with the library's per-launch
     # CUDA events (recorded on the stream each kernel is launched on).
-    q.profiling(True)
-    for i in range(args.steps):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize()
+    prof = profiled_steps(q, step, args.steps, flush)
     barrier()
-    q.profiling(False)
-    prof = q.profile_read()
-    per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     ms = statistics.mean(per_step)
     if world > 1:
         t = torch.tensor([ms], device=dev)
@@ -302,71 +391,123 @@ def main():
         ms = float(t.item())
     f_fwd, f_bwd = layer_flops(M, N, K, r)
     value = world * (f_fwd + f_bwd) / (ms * 1e-3) / 1e12
-
-    # roofline of the dominant kernel: the fused dequant-GEMM (forward + dgrad launches)
-    g_launch = sum(prof.get(k, (0, 0.0))[0] for k in ("qlora_gemm_fwd", "qlora_gemm_dgrad"))
-    g_ms = sum(prof.get(k, (0, 0.0))[1] for k in ("qlora_gemm_fwd", "qlora_gemm_dgrad"))
-    g_flops = args.steps * ((2 * M * N * K + 2 * M * N * r) + (2 * M * N * K + 2 * M * K * r))
-    g_tflops = g_flops / (g_ms * 1e-3) / 1e12 if g_ms > 0 else None
-    roofline = {"bound": "tensor", "achieved": g_tflops, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": (g_tflops / peaks["bf16_tflops"]) if g_tflops else None,
-                "traffic": GEMM_TRAFFIC_BYTES, "traffic_unit": "bytes per launch (ncu dram read + write)",
-                "kernel": "qlora_gemm (forward + dgrad launches)",
-                "peak_source": peaks["source"] + " bf16 burst",
-                "avg_launch_us": 1e3 * g_ms / max(g_launch, 1)}
-    kernels = {k: {"launches": n, "avg_us": 1e3 * t / max(n, 1), "share": t / max(
-        sum(v[1] for v in prof.values()), 1e-12)} for k, (n, t) in prof.items()}
+    roofline = gemm_roofline(prof, w, args.steps, peaks)
     gpu_launches = sum(n for n, _ in prof.values())
+    kernels = {k: {"launches": n, "avg_us": 1e3 * t / max(n, 1)} for k, (n, t) in prof.items()}
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic",
-        "config": {"workload": f"{MAIN}: W0 {N}x{K} NF4 (blocks of 64, double quant), "
-                               f"x {M}x{K} bf16 per rank, r={r}, alpha={alpha:g}, fwd+bwd",
-                   "global_batch_tokens": M * world, "parallelism": f"dp{world}",
-                   "l2": "512 MiB buffer written before every timed step (outside the events)"},
-        "roofline": roofline,
+        "data": "synthetic (seeded; shapes and distributions of the pages' workloads)",
+        "config": main_config(w, world),
+        "roofline": {k: sig(v) for k, v in roofline.items()},
         "gpu_launches": gpu_launches,
         "clocks": clk.summary(),
-        "kernels": kernels,
     }
+    detail = {"main_kernels_us": kernels}
 
     if not args.skip_extras:
         # every rank takes the same collective steps in the end-to-end leg
-        e2e = e2e_leg(q, dp, qw, inp, w, args, dev, world)
+        e2e = e2e_leg(q, dp, run, args, dev, world)
         if rank == 0:
-            line["e2e"] = e2e
+            line["e2e"] = {k: sig(v) for k, v in e2e.items()}
+    del run, flush
+    torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.skip_extras:
         # single-GPU legs: at N > 1 the other ranks would wait in the closing
         # barrier for minutes, beyond the process group's timeout
-        line["decode"] = decode_leg(q, dev, peaks)
-        line["quantize"] = quantize_leg(q, dev, peaks)
-        line["mlp70b"] = mlp70b_leg(q, dev, peaks)
-        line["stack"] = stack_leg(q, dev, peaks)
-        line["merge"] = merge_leg(q, dev, peaks)
-        line["multi_adapter"] = multi_leg(q, dev, peaks)
-        line["block128"] = block128_leg(q, dev, peaks)
-        line["dropout"] = dropout_leg(q, dev, peaks)
-        line["cpu_baseline"] = cpu_baseline_leg(w, inp)
+        legs = {}
+        for name in ("attn5120", "stack", "decode", "quantize", "dropout", "dropout_philox",
+                     "block128", "merge", "multi"):
+            res = run_leg(name, q, dp, dev, peaks)
+            detail[name] = res
+            legs[name] = compact_leg(name, res)
+        line["legs"] = legs
+        line["cpu_baseline"] = cpu_baseline_leg()
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
     if rank == 0:
+        print(json.dumps({"detail": detail}), file=sys.stderr, flush=True)
         print(json.dumps(line), flush=True)
 
 
-def e2e_leg(q, dp, qw, inp, w, args, dev, world):
+def run_leg(name, q, dp, dev, peaks):
+    if name == "cpu":
+        return cpu_baseline_leg()
+    fn = {"attn5120": attn_leg, "decode": decode_leg, "quantize": quantize_leg, "stack": stack_leg,
+          "merge": merge_leg, "multi": multi_leg, "block128": block128_leg, "dropout": dropout_leg,
+          "dropout_philox": dropout_philox_leg}[name]
+    out = fn(q, dev, peaks)
+    torch.cuda.synchronize()
+    st = q.device_status(dev)
+    if st != q.NF4_OK:
+        raise RuntimeError(f"device status after the {name} leg: {q.status_string(st)}")
+    return out
+
+
+def compact_leg(name, res):
+    """The few figures of a leg that go on the JSON line."""
+    if name == "decode":
+        return {m: {"us": sig(v["graph_call_us"]), "gbs": sig(v["gbs_graph_call"]),
+                    "frac": sig(v["frac_graph_call"], 3)}
+                for m, v in res.items() if m.startswith("M")}
+    if name == "quantize":
+        return {"us": sig(res["kernel_us"]), "gbs": sig(res["gbs"]), "frac": sig(res["frac"], 3),
+                "bf16_in_us": sig(res["bf16_input"]["kernel_us"])}
+    if name in ("attn5120", "stack"):
+        return {k: sig(res[k], 4 if k != "frac" and k != "gemm_frac" else 3)
+                for k in ("ms_per_step", "tflops", "frac", "gemm_frac") if k in res}
+    if name in ("dropout", "dropout_philox"):
+        return {"ms_per_step": sig(res["ms_per_step"]), "tflops": sig(res["tflops"])}
+    if name == "block128":
+        return {"step_ms": sig(res["step"]["ms_per_step"]),
+                "decode_M1_us": sig(res["decode"]["M1"]["graph_call_us"]),
+                "quantize_us": sig(res["quantize"]["kernel_us"])}
+    if name == "merge":
+        return {"bf16_frac": sig(res["bf16"]["frac"], 3), "fp32_frac": sig(res["fp32"]["frac"], 3)}
+    if name == "multi":
+        return {"us": sig(res["graph_call_us"]), "frac": sig(res["frac_graph_call"], 3)}
+    return {}
+
+
+def attn_leg(q, dev, peaks, warmup=3, steps=50):
+    """The LLaMA-13B-like attention projection's fwd+bwd step (W0 5120x5120 NF4 with
+    double quant, 2048 tokens, r = 16, alpha = 32), timed like the headline step."""
+    from bit_nf4_quantized_05_b200 import dp
+    w = workloads.WORKLOADS[ATTN]
+    run = LayerRun(q, dp, w, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(warmup):
+        run.step()
+    torch.cuda.synchronize()
+    ms = statistics.mean(event_steps(run.step, steps, flush))
+    prof = profiled_steps(q, run.step, steps, flush)
+    f, b = layer_flops(w.M, w.N, w.K, w.r)
+    roof = gemm_roofline(prof, w, steps, peaks)
+    del run, flush
+    torch.cuda.empty_cache()
+    tflops = (f + b) / (ms * 1e-3) / 1e12
+    return {"workload": f"{w.name}: W0 {w.N}x{w.K} NF4 double quant, x {w.M}x{w.K} bf16, r={w.r}, "
+                        f"alpha={w.alpha:g}, forward+backward",
+            "ms_per_step": ms, "tflops": tflops, "frac": tflops / peaks["bf16_tflops"],
+            "gemm_tflops": roof["achieved"], "gemm_frac": roof["frac"], "gemm_traffic": roof["traffic"],
+            "kernel_avg_us": {k: 1e3 * t / max(n, 1) for k, (n, t) in prof.items()}}
+
+
+def e2e_leg(q, dp, run, args, dev, world):
     """Same metric through the public API with host buffers: every step copies
-    x and dY in from pinned host memory and h, dX, dA, dB back out."""
+    x and dY in from pinned host memory and h, dX and the fp32 adapter
+    gradients back out (the frozen weight and the adapters stay resident)."""
+    w = run.w
     M, N, K, r, alpha = w.M, w.N, w.K, w.r, w.alpha
-    hx = inp["x"].pin_memory()
-    hdY = inp["dY"].pin_memory()
+    hx = run.inp["x"].pin_memory()
+    hdY = run.inp["dY"].pin_memory()
     oh = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
     odX = torch.empty(M, K, dtype=torch.bfloat16).pin_memory()
-    ograd = torch.empty(r * K + N * r, dtype=torch.bfloat16).pin_memory()
-    A, B = inp["A"].to(dev), inp["B"].to(dev)
+    ograd = torch.empty(r * K + N * r, dtype=torch.float32).pin_memory()
+    qw, A, B = run.qw, run.A, run.B
     x = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
     dY = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
     flat, dA, dB = dp.grad_buffer(r, K, N, device=dev)
@@ -399,6 +540,8 @@ def e2e_leg(q, dp, qw, inp, w, args, dev, world):
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms = float(t.item())
     f, b = layer_flops(M, N, K, r)
+    del x, dY, flat, dA, dB
+    torch.cuda.empty_cache()
     return {"value": world * (f + b) / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
             "ms_per_step": ms, "h2d_bytes_per_step": hx.nbytes + hdY.nbytes,
             "d2h_bytes_per_step": oh.nbytes + odX.nbytes + ograd.nbytes}
@@ -556,14 +699,14 @@ def merge_leg(q, dev, peaks):
     bf16 and to an fp32 weight. GB/s counts the bytes a merge must move: codes, 8-bit scale
     codes and group constants in, the merged weight out (the adapters are 0.3 MB). Four
     weight copies and outputs are rotated so that no launch finds its operands in L2."""
-    w = workloads.WORKLOADS[MAIN]
+    w = workloads.WORKLOADS[ATTN]
     inp = workloads.make_inputs(w, M=0, with_dy=False)
     W0 = inp["W0"].to(dev)
     copies = [q.nf4_quantize(W0, double_quant=True) for _ in range(4)]
     del W0
     A, B = inp["A"].to(dev), inp["B"].to(dev)
     nb = w.N * w.K // 64
-    out = {"workload": f"{MAIN}: W0 {w.N}x{w.K} NF4 double quant, r={w.r}, alpha={w.alpha:g}",
+    out = {"workload": f"{ATTN}: W0 {w.N}x{w.K} NF4 double quant, r={w.r}, alpha={w.alpha:g}",
            "peak_gbs": peaks["hbm_gbs"]}
     for name, bf16 in (("bf16", True), ("fp32", False)):
         outs = [torch.empty(w.N, w.K, dtype=torch.bfloat16 if bf16 else torch.float32, device=dev)
@@ -593,7 +736,7 @@ def dropout_leg(q, dev, peaks, steps=50, p=0.05):
     GEMM writes dY W~ in fp32 and the adapter-add kernel masks, adds and rounds dX once.
     The adapter-add kernel is HBM-bound: it reads the fp32 base (4 B), writes dX (2 B) and
     reads the mask (1/8 B) per element of dX."""
-    w = workloads.WORKLOADS[MAIN]
+    w = workloads.WORKLOADS[ATTN]
     M, N, K, r, alpha = w.M, w.N, w.K, w.r, w.alpha
     inp = workloads.make_inputs(w)
     qw = q.nf4_quantize(inp["W0"].to(dev), double_quant=w.double_quant)
@@ -636,7 +779,7 @@ def dropout_leg(q, dev, peaks, steps=50, p=0.05):
     add_bytes = M * K * 4 + M * K * 2 + M * K // 8
     del qw, x, A, B, dY, keep, h, dX, dA, dB, ws_f, ws_b, flush, inp
     torch.cuda.empty_cache()
-    return {"workload": f"{MAIN}: W0 {N}x{K} NF4 double quant, x {M}x{K}, r={r}, LoRA dropout p={p}, "
+    return {"workload": f"{ATTN}: W0 {N}x{K} NF4 double quant, x {M}x{K}, r={r}, LoRA dropout p={p}, "
                         f"fwd+bwd", "ms_per_step": ms, "tflops": (f_fwd + f_bwd) / (ms * 1e-3) / 1e12,
             "kernels_us": {k: 1e3 * t / max(n, 1) for k, (n, t) in prof.items()},
             "lora_dX_add": {"bytes": add_bytes, "kernel_us": add_us,
@@ -644,12 +787,52 @@ def dropout_leg(q, dev, peaks, steps=50, p=0.05):
                             "frac": add_bytes / (add_us * 1e-6) / 1e9 / peaks["hbm_gbs"] if add_us > 0 else None}}
 
 
+def dropout_philox_leg(q, dev, peaks, steps=50, p=0.05):
+    """The main workload's forward + backward with LoRA dropout p = 0.05 whose mask the
+    kernels draw from Philox4x32-10 (a new offset every step; the backward regenerates the
+    forward's mask, nothing is stored): the rank-r kernels draw and apply the mask to the
+    landed x tiles, the dgrad GEMM writes dY W~ in fp32 and the adapter-add kernel draws,
+    masks, adds and rounds dX once."""
+    w = workloads.WORKLOADS[ATTN]
+    M, N, K, r, alpha = w.M, w.N, w.K, w.r, w.alpha
+    inp = workloads.make_inputs(w)
+    qw = q.nf4_quantize(inp["W0"].to(dev), double_quant=w.double_quant)
+    x, A, B, dY = (inp[k].to(dev) for k in ("x", "A", "B", "dY"))
+    h = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    dA = torch.empty(r, K, dtype=torch.bfloat16, device=dev)
+    dB = torch.empty(N, r, dtype=torch.bfloat16, device=dev)
+    ws_f = torch.empty(q.fwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(int(q.lib.qlora_bwd_dropout_workspace_bytes(M, N, K, r)), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    seed, offset = 20241202, [0]
+
+    def step():
+        offset[0] += 1
+        _, u = q.qlora_linear_fwd_dropout_philox(qw, x, A, B, alpha, p, seed, offset[0], h=h, workspace=ws_f)
+        q.qlora_linear_bwd_dropout_philox(qw, x, A, B, alpha, p, seed, offset[0], dY, u=u, workspace=ws_b,
+                                          outs=(dX, dA, dB))
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    ms = statistics.mean(event_steps(step, steps, flush))
+    prof = profiled_steps(q, step, steps, flush)
+    f_fwd, f_bwd = layer_flops(M, N, K, r)
+    del qw, x, A, B, dY, h, dX, dA, dB, ws_f, ws_b, flush, inp
+    torch.cuda.empty_cache()
+    return {"workload": f"{ATTN}: W0 {N}x{K} NF4 double quant, x {M}x{K}, r={r}, LoRA dropout p={p} "
+                        f"drawn in the kernels (Philox4x32-10), fwd+bwd",
+            "ms_per_step": ms, "tflops": (f_fwd + f_bwd) / (ms * 1e-3) / 1e12,
+            "kernels_us": {k: 1e3 * t / max(n, 1) for k, (n, t) in prof.items()}}
+
+
 def block128_leg(q, dev, peaks, steps=50):
     """The main workload's fused forward + backward, the decode forward and the
     quantiser with 128-element blocks (the pages' other block size): the same
     kernels with two 64-element steps per scale."""
     from bit_nf4_quantized_05_b200 import dp
-    w = workloads.WORKLOADS[MAIN]
+    w = workloads.WORKLOADS[ATTN]
     M, N, K, r, alpha = w.M, w.N, w.K, w.r, w.alpha
     inp = workloads.make_inputs(w)
     qw = q.nf4_quantize(inp["W0"].to(dev), double_quant=w.double_quant, block_size=128)
@@ -680,7 +863,7 @@ def block128_leg(q, dev, peaks, steps=50):
     f_fwd, f_bwd = layer_flops(M, N, K, r)
     del qw, x, A, B, dY, h, u, dX, ws_f, ws_b, flush, inp
     torch.cuda.empty_cache()
-    return {"step": {"workload": f"{MAIN}: W0 {N}x{K} NF4 (blocks of 128, double quant), x {M}x{K}, "
+    return {"step": {"workload": f"{ATTN}: W0 {N}x{K} NF4 (blocks of 128, double quant), x {M}x{K}, "
                                  f"r={r}, fwd+bwd", "ms_per_step": ms,
                      "tflops": (f_fwd + f_bwd) / (ms * 1e-3) / 1e12},
             "decode": decode_leg(q, dev, peaks, block=128, tokens=(1, 16)),
@@ -699,50 +882,6 @@ def _time_steps(step, warmup, steps):
     e.record()
     torch.cuda.synchronize()
     return s.elapsed_time(e) / steps
-
-
-def mlp70b_leg(q, dev, peaks, warmup=3, steps=5):
-    """Forward + backward of the Llama-2-70B-like MLP projection (W0 28672x8192 NF4 with
-    double quant, 8192 tokens, r = 64, alpha = 16). Every operand is larger than L2."""
-    from bit_nf4_quantized_05_b200 import dp
-    w = workloads.WORKLOADS[QUANT]
-    M, N, K, r, alpha = w.M, w.N, w.K, w.r, w.alpha
-    inp = workloads.make_inputs(w)
-    qw = q.nf4_quantize(inp["W0"].to(dev), double_quant=True)
-    x, A, B, dY = (inp[k].to(dev) for k in ("x", "A", "B", "dY"))
-    del inp
-    h = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-    u = torch.empty(M, r, dtype=torch.float32, device=dev)
-    dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
-    flat, dA, dB = dp.grad_buffer(r, K, N, device=dev)
-    ws_f = torch.empty(q.fwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
-    ws_b = torch.empty(q.bwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
-
-    def step():
-        q.qlora_linear_fwd(qw, x, A, B, alpha, h=h, u=u, workspace=ws_f)
-        q.qlora_linear_bwd(qw, x, A, B, alpha, dY, u=u, workspace=ws_b, outs=(dX, dA, dB))
-
-    ms = _time_steps(step, warmup, steps)
-    q.profiling(True)
-    for _ in range(steps):
-        step()
-    torch.cuda.synchronize()
-    q.profiling(False)
-    prof = q.profile_read()
-    f, b = layer_flops(M, N, K, r)
-    g_ms = sum(prof.get(k, (0, 0.0))[1] for k in ("qlora_gemm_fwd", "qlora_gemm_dgrad")) / steps
-    g_flops = (2 * M * N * K + 2 * M * N * r) + (2 * M * N * K + 2 * M * K * r)
-    del qw, x, A, B, dY, h, u, dX, flat, ws_f, ws_b
-    torch.cuda.empty_cache()
-    tflops = (f + b) / (ms * 1e-3) / 1e12
-    gemm_tflops = g_flops / (g_ms * 1e-3) / 1e12 if g_ms > 0 else None
-    return {"workload": f"{QUANT}: W0 {N}x{K} NF4 double quant, x {M}x{K} bf16, r={r}, "
-                        f"alpha={alpha:g}, forward+backward",
-            "ms_per_step": ms, "tflops": tflops, "frac": tflops / peaks["bf16_tflops"],
-            "gemm_tflops": gemm_tflops,
-            "gemm_frac": gemm_tflops / peaks["bf16_tflops"] if gemm_tflops else None,
-            "peak_tflops": peaks["bf16_tflops"], "steps": steps,
-            "kernel_avg_us": {k: 1e3 * t / max(n, 1) for k, (n, t) in prof.items()}}
 
 
 def stack_leg(q, dev, peaks, warmup=2, steps=3):
@@ -794,22 +933,6 @@ def stack_leg(q, dev, peaks, warmup=2, steps=3):
             "ms_per_step": ms, "tflops": tflops, "frac": tflops / peaks["bf16_tflops"],
             "peak_tflops": peaks["bf16_tflops"], "algorithmic_tflop": total / 1e12,
             "steps": steps, "input_generation_s": gen_s}
-
-
-def cpu_baseline_leg(w, inp, target_s=12.0):
-    """The oracle on a bounded sample of the workload's tokens: the sample grows
-    (at most 8x per try) until one try takes half of target_s or covers every
-    token, so the timed try takes roughly 5 to 20 s on the host."""
-    tokens = 16
-    qw = oracle_weight(w, inp)
-    while True:
-        f, t = oracle_sample_step(w, inp, tokens, qw)
-        if t >= 0.5 * target_s or tokens >= w.M:
-            break
-        tokens = int(min(w.M, tokens * min(8.0, max(2.0, target_s / max(t, 1e-3)))))
-    return {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
-            "sample": f"{tokens} of {w.M} tokens: oracle forward+backward of those tokens "
-                      f"({t:.1f} s on the host)"}
 
 
 if __name__ == "__main__":

@@ -66,6 +66,7 @@ def _load() -> ctypes.CDLL:
             "(nvcc, sm_100a). There is no fallback implementation.")
     L = ctypes.CDLL(LIB_PATH)
     vp, i64, i32, f32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    u64 = ctypes.c_uint64
     W = ctypes.POINTER(NF4WeightStruct)
     sig = {
         "nf4_quantize": ([vp, W, vp], ctypes.c_int),
@@ -82,6 +83,10 @@ def _load() -> ctypes.CDLL:
         "qlora_linear_fwd_dropout": ([W, vp, i64, vp, vp, i32, f32, f32, vp, vp, vp, vp, sz, vp],
                                      ctypes.c_int),
         "qlora_bwd_dropout_workspace_bytes": ([i64, i64, i64, i32], sz),
+        "qlora_linear_fwd_dropout_philox": ([W, vp, i64, vp, vp, i32, f32, f32, u64, u64, vp, vp, vp,
+                                             sz, vp], ctypes.c_int),
+        "qlora_linear_bwd_dropout_philox": ([W, vp, i64, vp, vp, i32, f32, f32, u64, u64, vp, vp, vp,
+                                             vp, vp, vp, sz, vp], ctypes.c_int),
         "qlora_linear_bwd_dropout": ([W, vp, i64, vp, vp, i32, f32, f32, vp, vp, vp, vp, vp, vp, vp,
                                       sz, vp], ctypes.c_int),
         "qlora_merge": ([W, vp, vp, i32, f32, vp, i32, vp], ctypes.c_int),
@@ -446,6 +451,8 @@ def qlora_linear_bwd_dropout(qw: QuantizedWeight, x: torch.Tensor, A: torch.Tens
     _need_cuda(x, A, B, dY, keep)
     if outs is not None:
         dX, dA, dB = outs
+        if dA.dtype != torch.bfloat16:
+            raise ValueError("the dropout backward writes bf16 adapter gradients")
     else:
         dX = torch.empty(M, qw.k, dtype=torch.bfloat16, device=x.device) if need_dX else None
         dA = torch.empty(r, qw.k, dtype=torch.bfloat16, device=x.device)
@@ -457,6 +464,62 @@ def qlora_linear_bwd_dropout(qw: QuantizedWeight, x: torch.Tensor, A: torch.Tens
                                         float(p), _ptr(keep), _ptr(dY), _ptr(u), _ptr(dX), _ptr(dA),
                                         _ptr(dB), _ptr(ws), ws.numel(), _stream(x.device)),
            "qlora_linear_bwd_dropout")
+    return dX, dA, dB
+
+
+def qlora_linear_fwd_dropout_philox(qw: QuantizedWeight, x: torch.Tensor, A: torch.Tensor,
+                                    B: torch.Tensor, alpha: float, p: float, seed: int,
+                                    offset: int, save_u: bool = True,
+                                    h: Optional[torch.Tensor] = None,
+                                    workspace: Optional[torch.Tensor] = None):
+    """Forward with LoRA dropout whose mask the kernels draw from Philox4x32-10
+    at (seed, offset). Returns (h, u) with u = (keep . x) A^T."""
+    M, r = _layer_args(qw, x, A, B)
+    if h is not None:
+        _check_t("h", h, (M, qw.n), torch.bfloat16, qw.device)
+    _check_ws(workspace, qw.device)
+    _need_cuda(x, A, B)
+    if h is None:
+        h = torch.empty(M, qw.n, dtype=torch.bfloat16, device=x.device)
+    u = torch.empty(M, r, dtype=torch.float32, device=x.device) if save_u else None
+    ws = workspace if workspace is not None else _workspace(fwd_workspace_bytes(M, qw.n, qw.k, r), x.device)
+    s = qw.struct()
+    _check(lib.qlora_linear_fwd_dropout_philox(ctypes.byref(s), _ptr(x), M, _ptr(A), _ptr(B), r,
+                                               float(alpha), float(p), int(seed) & (2 ** 64 - 1),
+                                               int(offset) & (2 ** 64 - 1), _ptr(h), _ptr(u), _ptr(ws),
+                                               ws.numel(), _stream(x.device)),
+           "qlora_linear_fwd_dropout_philox")
+    return h, u
+
+
+def qlora_linear_bwd_dropout_philox(qw: QuantizedWeight, x: torch.Tensor, A: torch.Tensor,
+                                    B: torch.Tensor, alpha: float, p: float, seed: int,
+                                    offset: int, dY: torch.Tensor,
+                                    u: Optional[torch.Tensor] = None, need_dX: bool = True,
+                                    workspace: Optional[torch.Tensor] = None,
+                                    outs: Optional[tuple] = None):
+    """(dX, dA, dB) with LoRA dropout, the mask regenerated from the forward's
+    (p, seed, offset)."""
+    M, r = _layer_args(qw, x, A, B)
+    _check_bwd(qw, M, r, dY, u, outs, workspace)
+    _need_cuda(x, A, B, dY)
+    if outs is not None:
+        dX, dA, dB = outs
+        if dA.dtype != torch.bfloat16:
+            raise ValueError("the dropout backward writes bf16 adapter gradients")
+    else:
+        dX = torch.empty(M, qw.k, dtype=torch.bfloat16, device=x.device) if need_dX else None
+        dA = torch.empty(r, qw.k, dtype=torch.bfloat16, device=x.device)
+        dB = torch.empty(qw.n, r, dtype=torch.bfloat16, device=x.device)
+    nbytes = int(lib.qlora_bwd_dropout_workspace_bytes(M, qw.n, qw.k, r))
+    ws = workspace if workspace is not None else _workspace(nbytes, x.device)
+    s = qw.struct()
+    _check(lib.qlora_linear_bwd_dropout_philox(ctypes.byref(s), _ptr(x), M, _ptr(A), _ptr(B), r,
+                                               float(alpha), float(p), int(seed) & (2 ** 64 - 1),
+                                               int(offset) & (2 ** 64 - 1), _ptr(dY), _ptr(u),
+                                               _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws), ws.numel(),
+                                               _stream(x.device)),
+           "qlora_linear_bwd_dropout_philox")
     return dX, dA, dB
 
 

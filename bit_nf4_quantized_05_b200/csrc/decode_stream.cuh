@@ -537,7 +537,7 @@ constexpr int kDsUParkBytes = 256 * 32 * 4;
 
 template <int TG>
 __global__ void __launch_bounds__(kDsThreads, 1)
-qlora_decode_u_kernel(const DecodeArgs a, const uint8_t *__restrict__ keep) {
+qlora_decode_u_kernel(const DecodeArgs a, const uint8_t *__restrict__ keep, const DropRng rng) {
     extern __shared__ __align__(16) float upark[];     // [256][32]
     // x may come from the kernel before this one
     griddep_wait();
@@ -576,11 +576,15 @@ qlora_decode_u_kernel(const DecodeArgs a, const uint8_t *__restrict__ keep) {
                     const uint4 *px = reinterpret_cast<const uint4 *>(xrow[tg] + kb * 64);
                     xa[tg] = __ldg(px);
                     xb[tg] = __ldg(px + 1);
-                    if (keep) {
-                        // LoRA dropout: zero the dropped tokens' elements (16 k, two keep bytes)
+                    if (keep || rng.on) {
+                        // LoRA dropout: zero the dropped tokens' elements (16 k: two keep
+                        // bytes of the mask, or drawn from the generator)
                         const int m = tg * 8 + g;
                         const int64_t e = static_cast<int64_t>(m) * a.K + kb * 64 + 16 * t;
-                        const uint32_t kbits = keep[e >> 3] | (static_cast<uint32_t>(keep[(e >> 3) + 1]) << 8);
+                        const uint32_t kbits =
+                            rng.on ? (drop_keep8(rng, static_cast<uint64_t>(e)) |
+                                      (drop_keep8(rng, static_cast<uint64_t>(e) + 8) << 8))
+                                   : (keep[e >> 3] | (static_cast<uint32_t>(keep[(e >> 3) + 1]) << 8));
                         uint32_t w[8] = {xa[tg].x, xa[tg].y, xa[tg].z, xa[tg].w,
                                          xb[tg].x, xb[tg].y, xb[tg].z, xb[tg].w};
 #pragma unroll

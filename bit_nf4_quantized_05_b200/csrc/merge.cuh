@@ -201,7 +201,8 @@ struct LoraAddArgs {
     int r, rp;
     const uint16_t *Vs;        // [M, r]
     const uint16_t *A;         // [r, K]
-    const uint8_t *keep;       // bit mask over [M, K]
+    const uint8_t *keep;       // bit mask over [M, K] (when rng.on is 0)
+    DropRng rng;               // the mask drawn from the generator (rng.on)
     const float *base;         // [M, K] fp32: dY W~
     uint16_t *dX;              // [M, K] bf16 result
 };
@@ -276,7 +277,8 @@ __global__ void __launch_bounds__(kMgThreads, 4) qlora_lora_add_kernel(const Lor
         const int64_t m = m0 + rw + rl;
         if (m >= a.M) continue;
         const int64_t k = k0 + cw + 8 * ch;
-        const uint32_t kb = a.keep[(m * a.K + k) >> 3];
+        const uint32_t kb = a.rng.on ? drop_keep8(a.rng, static_cast<uint64_t>(m * a.K + k))
+                                     : a.keep[(m * a.K + k) >> 3];
         uint4 *px = reinterpret_cast<uint4 *>(a.dX + m * a.K + k);
         const float4 b0 = *reinterpret_cast<const float4 *>(a.base + m * a.K + k);
         const float4 b1 = *reinterpret_cast<const float4 *>(a.base + m * a.K + k + 4);

@@ -396,4 +396,59 @@ __device__ __forceinline__ void dequant8(const BlockLut &L, uint32_t w, uint32_t
     }
 }
 
+// ---------------------------------------------------------------------------
+// LoRA dropout drawn in the kernels ("QLoRA Finetuner -- Juan Martos",
+// section 1: dropout on the adapter input). The draw is Philox4x32-10, the
+// counter-based generator of Salmon et al. ("Parallel random numbers: as easy
+// as 1, 2, 3", SC'11): element e of x [M, k] takes word e % 4 of the
+// generator at counter (e / 4 as two 32-bit words, offset as two words) with
+// key (seed as two words), and is dropped when that word is below
+// floor(p * 2^32). Any kernel that needs the mask of some elements computes
+// exactly those words, so the backward regenerates the forward's mask and no
+// mask is stored.
+// ---------------------------------------------------------------------------
+struct DropRng {
+    uint32_t k0, k1;       // key: the seed's low and high words
+    uint32_t o0, o1;       // counter words 2 and 3: the offset's low and high words
+    uint32_t thresh;       // an element is dropped when its word is below this
+    int on;                // 0: no generated mask
+};
+
+__device__ __forceinline__ uint4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
+                                               uint32_t k0, uint32_t k1) {
+#pragma unroll
+    for (int round = 0; round < 10; ++round) {
+        if (round > 0) {
+            k0 += 0x9E3779B9u;     // Weyl sequence of the round keys
+            k1 += 0xBB67AE85u;
+        }
+        const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * c0;
+        const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * c2;
+        const uint32_t n0 = static_cast<uint32_t>(p1 >> 32) ^ c1 ^ k0;
+        const uint32_t n2 = static_cast<uint32_t>(p0 >> 32) ^ c3 ^ k1;
+        c1 = static_cast<uint32_t>(p1);
+        c3 = static_cast<uint32_t>(p0);
+        c0 = n0;
+        c2 = n2;
+    }
+    return make_uint4(c0, c1, c2, c3);
+}
+
+// Keep bits of the eight elements [e0, e0 + 8) of x (e0 % 8 == 0): bit i is 1
+// when element e0 + i is kept.
+__device__ __forceinline__ uint32_t drop_keep8(const DropRng &d, uint64_t e0) {
+    uint32_t bits = 0;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint64_t g = (e0 >> 2) + h;
+        const uint4 v = philox4x32_10(static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), d.o0, d.o1,
+                                      d.k0, d.k1);
+        bits |= (v.x >= d.thresh ? 1u : 0u) << (4 * h);
+        bits |= (v.y >= d.thresh ? 1u : 0u) << (4 * h + 1);
+        bits |= (v.z >= d.thresh ? 1u : 0u) << (4 * h + 2);
+        bits |= (v.w >= d.thresh ? 1u : 0u) << (4 * h + 3);
+    }
+    return bits;
+}
+
 }  // namespace nf4

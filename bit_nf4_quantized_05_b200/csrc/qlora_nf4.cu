@@ -290,6 +290,7 @@ struct SkinnySpec {
     int mask_mode = 0;                 // dropout on x as the A operand (see SkinnyJob)
     const uint8_t *keep = nullptr;
     int64_t mx = 0, kx = 0;
+    DropRng rng{};                     // the mask drawn from the generator instead of keep
 };
 
 // Tensor maps and job fields of one product; splits is the launch's split count.
@@ -318,6 +319,7 @@ bool skinny_job(const SkinnySpec &sp, int RN, int splits, CUtensorMap *ta, CUten
     job->transposed = sp.transposed;
     job->mask_mode = sp.mask_mode;
     job->keep = sp.keep;
+    job->rng = sp.rng;
     job->mx = sp.mx;
     job->kx = sp.kx;
     return ok;
@@ -562,7 +564,7 @@ bool decode_shape(const nf4_weight *w, int64_t M, int32_t r) {
 nf4_status launch_decode(const nf4_weight *w, const uint16_t *x, int64_t M, const uint16_t *A,
                          const uint16_t *B, int32_t r, float scale, uint16_t *h, float *u_out,
                          float *upart, cudaStream_t stream, const RowGroups *groups = nullptr,
-                         const uint8_t *keep = nullptr) {
+                         const uint8_t *keep = nullptr, const DropRng &rng = DropRng{}) {
     // each of the 16 warps takes rb blocks of every 32-row tile, fetched in
     // chunks of cb blocks (the largest divisor of rb that is at most 5)
     const int64_t kblocks = w->k / kBlock;
@@ -605,7 +607,7 @@ nf4_status launch_decode(const nf4_weight *w, const uint16_t *x, int64_t M, cons
         LaunchTimer t(KK_DECODE_U, stream);
         auto ku = tg == 1 ? qlora_decode_u_kernel<1> : qlora_decode_u_kernel<2>;
         NF4_TRY_CUDA(cudaFuncSetAttribute(ku, cudaFuncAttributeMaxDynamicSharedMemorySize, kDsUParkBytes));
-        const cudaError_t e = launch_ex(ku, dim3(kDsUCtas), dim3(kDsThreads), kDsUParkBytes, stream, 0u, a, keep);
+        const cudaError_t e = launch_ex(ku, dim3(kDsUCtas), dim3(kDsThreads), kDsUParkBytes, stream, 0u, a, keep, rng);
         t.stop();
         if (e != cudaSuccess) return NF4_ERR_CUDA;
     }
@@ -885,15 +887,17 @@ size_t qlora_fwd_workspace_bytes(int64_t M, int64_t n, int64_t k, int32_t r) {
     return fwd_layout(M, r, num_sms(current_device())).total;
 }
 
-// Forward, with LoRA dropout when keep is non-null (inverted dropout on the
-// adapter input with the keep mask given; the branch is scaled by
-// (alpha/r)/(1-p)).
+// Forward, with LoRA dropout when keep is non-null or rng.on (inverted dropout
+// on the adapter input with the keep mask given, or drawn in the kernels; the
+// branch is scaled by (alpha/r)/(1-p)).
 nf4_status fwd_impl(const nf4_weight *w, const uint16_t *x, int64_t M, const uint16_t *A,
                     const uint16_t *B, int32_t r, float alpha, float p, const uint8_t *keep,
-                    uint16_t *h, float *u_out, void *workspace, size_t ws_bytes, void *stream) {
+                    uint16_t *h, float *u_out, void *workspace, size_t ws_bytes, void *stream,
+                    const DropRng &rng = DropRng{}) {
     nf4_status st = check_layer(w, x, M, A, B, r, alpha);
     if (st != NF4_OK) return st;
-    if (keep && !(p >= 0.0f && p < 1.0f)) return NF4_ERR_INVALID_ARG;
+    const bool masked = keep != nullptr || rng.on;
+    if (masked && !(p >= 0.0f && p < 1.0f)) return NF4_ERR_INVALID_ARG;
     if (M == 0) return NF4_OK;
     if (!h) return NF4_ERR_INVALID_ARG;
     if (!aligned16(h) || !aligned16(u_out) || !aligned16(keep)) return NF4_ERR_ALIGNMENT;
@@ -907,17 +911,18 @@ nf4_status fwd_impl(const nf4_weight *w, const uint16_t *x, int64_t M, const uin
     const SkBuf sk{reinterpret_cast<float *>(ws + L.partial), reinterpret_cast<int *>(ws + L.flags),
                    sk_pairs_max(sms)};
     float scale = alpha / static_cast<float>(r);
-    if (keep) scale = scale / (1.0f - p);
+    if (masked) scale = scale / (1.0f - p);
     if (decode_shape(w, M, r))
         return launch_decode(w, x, M, A, B, r, scale, h, u_out, reinterpret_cast<float *>(ws + L.upart), s,
-                             nullptr, keep);
+                             nullptr, keep, rng);
     // u = x A^T (fp32, optional; under dropout the dropped elements of x are
     // zero) and bf16(scale u) for the up-projection stage; this kernel also
     // clears the GEMM's stream-K flags
     SkinnySpec su{x, M, w->k, Major::K, A, r, w->k, Major::K, r, u_out, u_s, scale, 0};
-    if (keep) {
+    if (masked) {
         su.mask_mode = 1;
         su.keep = keep;
+        su.rng = rng;
         su.mx = M;
         su.kx = w->k;
     }
@@ -1017,7 +1022,7 @@ size_t qlora_bwd_workspace_bytes(int64_t M, int64_t n, int64_t k, int32_t r) {
 
 // dX += keep . (Vs A) on the tensor cores (the adapter part of dX under dropout).
 nf4_status lora_add(const float *base, const uint16_t *Vs, const uint16_t *A, const uint8_t *keep,
-                    int64_t M, int64_t K, int32_t r, uint16_t *dX, cudaStream_t s) {
+                    const DropRng &rng, int64_t M, int64_t K, int32_t r, uint16_t *dX, cudaStream_t s) {
     LoraAddArgs a{};
     a.base = base;
     a.M = M;
@@ -1027,6 +1032,7 @@ nf4_status lora_add(const float *base, const uint16_t *Vs, const uint16_t *A, co
     a.Vs = Vs;
     a.A = A;
     a.keep = keep;
+    a.rng = rng;
     a.dX = dX;
     if ((M + kMgRows - 1) / kMgRows > 65535) return NF4_ERR_UNSUPPORTED_SHAPE;
     const dim3 grid(static_cast<unsigned>((K + kMgCols - 1) / kMgCols), static_cast<unsigned>((M + kMgRows - 1) / kMgRows));
@@ -1052,17 +1058,19 @@ nf4_status lora_add(const float *base, const uint16_t *Vs, const uint16_t *A, co
     return NF4_OK;
 }
 
-// Backward, with LoRA dropout when keep is non-null (u, when given, is the
-// forward's masked u = (keep . x) A^T).
+// Backward, with LoRA dropout when keep is non-null or rng.on (u, when given,
+// is the forward's masked u = (keep . x) A^T).
 // Adapter gradients in bf16 (dA, dB) or, when grads32 is set, in fp32 (the
 // same pointers, as float).
 nf4_status bwd_impl(const nf4_weight *w, const uint16_t *x, int64_t M, const uint16_t *A,
                     const uint16_t *B, int32_t r, float alpha, float p, const uint8_t *keep,
                     const uint16_t *dY, const float *u, uint16_t *dX, void *dA, void *dB,
-                    void *workspace, size_t ws_bytes, void *stream, bool grads32 = false) {
+                    void *workspace, size_t ws_bytes, void *stream, bool grads32 = false,
+                    const DropRng &rng = DropRng{}) {
     nf4_status st = check_layer(w, x, M, A, B, r, alpha);
     if (st != NF4_OK) return st;
-    if (keep && !(p >= 0.0f && p < 1.0f)) return NF4_ERR_INVALID_ARG;
+    const bool masked = keep != nullptr || rng.on;
+    if (masked && !(p >= 0.0f && p < 1.0f)) return NF4_ERR_INVALID_ARG;
     if (!dA || !dB || (M > 0 && !dY)) return NF4_ERR_INVALID_ARG;
     if (!aligned16(dY) || !aligned16(u) || !aligned16(dX) || !aligned16(dA) || !aligned16(dB) ||
         !aligned16(keep))
@@ -1085,7 +1093,7 @@ nf4_status bwd_impl(const nf4_weight *w, const uint16_t *x, int64_t M, const uin
     const int sms = num_sms(current_device());
     const BwdLayout L = bwd_layout(M, r, sms);
     // under dropout the workspace also holds dY W~ in fp32 ([M, k]) for the masked add
-    const size_t need = keep ? L.total + align256(size_t(M) * size_t(K) * 4) : L.total;
+    const size_t need = masked ? L.total + align256(size_t(M) * size_t(K) * 4) : L.total;
     if (!workspace || ws_bytes < need) return NF4_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return NF4_ERR_ALIGNMENT;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -1095,15 +1103,16 @@ nf4_status bwd_impl(const nf4_weight *w, const uint16_t *x, int64_t M, const uin
     const SkBuf sk{reinterpret_cast<float *>(ws + L.partial), reinterpret_cast<int *>(ws + L.flags),
                    sk_pairs_max(sms)};
     float scale = alpha / static_cast<float>(r);
-    if (keep) scale = scale / (1.0f - p);
+    if (masked) scale = scale / (1.0f - p);
 
     // bf16(s u): recomputed from x here (masked under dropout), or converted from
     // the saved u by the v launch
     if (!u) {
         SkinnySpec su{x, M, K, Major::K, A, r, K, Major::K, r, nullptr, u_s, scale, 0};
-        if (keep) {
+        if (masked) {
             su.mask_mode = 1;
             su.keep = keep;
+            su.rng = rng;
             su.mx = M;
             su.kx = K;
         }
@@ -1128,9 +1137,10 @@ nf4_status bwd_impl(const nf4_weight *w, const uint16_t *x, int64_t M, const uin
             j[0].out_bf16 = static_cast<uint16_t *>(dB);
             j[1].out_bf16 = static_cast<uint16_t *>(dA);
         }
-        if (keep) {
+        if (masked) {
             j[1].mask_mode = 2;
             j[1].keep = keep;
+            j[1].rng = rng;
             j[1].mx = M;
             j[1].kx = K;
         }
@@ -1140,10 +1150,10 @@ nf4_status bwd_impl(const nf4_weight *w, const uint16_t *x, int64_t M, const uin
     if (!dX) return NF4_OK;
     // dX = dY W~ + bf16(s v) A; under dropout the adapter part is masked
     // element-wise, so it is added by its own kernel after the GEMM
-    if (!keep) return launch_gemm_auto<true>(w, dY, M, N, K, v_s, r, A, dX, s, &sk);
+    if (!masked) return launch_gemm_auto<true>(w, dY, M, N, K, v_s, r, A, dX, s, &sk);
     st = launch_gemm_auto<true>(w, dY, M, N, K, nullptr, r, A, dX, s, &sk, base32);
     if (st != NF4_OK) return st;
-    return lora_add(base32, v_s, A, keep, M, K, r, dX, s);
+    return lora_add(base32, v_s, A, keep, rng, M, K, r, dX, s);
 }
 
 nf4_status qlora_linear_bwd(const nf4_weight *w, const uint16_t *x, int64_t M, const uint16_t *A,
@@ -1176,6 +1186,41 @@ nf4_status qlora_linear_bwd_dropout(const nf4_weight *w, const uint16_t *x, int6
     // an empty batch has an empty mask: keep may be null only then
     if ((M > 0 && !keep) || !(p >= 0.0f && p < 1.0f)) return NF4_ERR_INVALID_ARG;
     return bwd_impl(w, x, M, A, B, r, alpha, p, keep, dY, u, dX, dA, dB, workspace, ws_bytes, stream);
+}
+
+// The generator's parameters of one (p, seed, offset): the drop threshold is
+// floor(p * 2^32), exact in fp64 for an fp32 p.
+DropRng make_drop_rng(float p, uint64_t seed, uint64_t offset) {
+    DropRng d{};
+    d.k0 = static_cast<uint32_t>(seed);
+    d.k1 = static_cast<uint32_t>(seed >> 32);
+    d.o0 = static_cast<uint32_t>(offset);
+    d.o1 = static_cast<uint32_t>(offset >> 32);
+    const double t = std::floor(static_cast<double>(p) * 4294967296.0);
+    d.thresh = t > 0.0 ? (t < 4294967295.0 ? static_cast<uint32_t>(t) : 0xFFFFFFFFu) : 0u;
+    d.on = 1;
+    return d;
+}
+
+nf4_status qlora_linear_fwd_dropout_philox(const nf4_weight *w, const uint16_t *x, int64_t M,
+                                           const uint16_t *A, const uint16_t *B, int32_t r,
+                                           float alpha, float p, uint64_t seed, uint64_t offset,
+                                           uint16_t *h, float *u_out, void *workspace,
+                                           size_t ws_bytes, void *stream) {
+    if (!(p >= 0.0f && p < 1.0f)) return NF4_ERR_INVALID_ARG;
+    return fwd_impl(w, x, M, A, B, r, alpha, p, nullptr, h, u_out, workspace, ws_bytes, stream,
+                    make_drop_rng(p, seed, offset));
+}
+
+nf4_status qlora_linear_bwd_dropout_philox(const nf4_weight *w, const uint16_t *x, int64_t M,
+                                           const uint16_t *A, const uint16_t *B, int32_t r,
+                                           float alpha, float p, uint64_t seed, uint64_t offset,
+                                           const uint16_t *dY, const float *u, uint16_t *dX,
+                                           uint16_t *dA, uint16_t *dB, void *workspace,
+                                           size_t ws_bytes, void *stream) {
+    if (!(p >= 0.0f && p < 1.0f)) return NF4_ERR_INVALID_ARG;
+    return bwd_impl(w, x, M, A, B, r, alpha, p, nullptr, dY, u, dX, dA, dB, workspace, ws_bytes,
+                    stream, false, make_drop_rng(p, seed, offset));
 }
 
 }  // extern "C"

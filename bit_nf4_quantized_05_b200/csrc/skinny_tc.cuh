@@ -40,12 +40,14 @@ struct SkinnyJob {
     float scale;
     int transposed;
     // dropout on x as the A operand (LoRA dropout: the keep mask is an input,
-    // bit (e & 7) of byte e >> 3 for element e = m * kx + k of x [mx, kx]):
+    // bit (e & 7) of byte e >> 3 for element e = m * kx + k of x [mx, kx], or,
+    // when rng.on, drawn here from the counter-based generator):
     // 0 = none, 1 = A is x K-major (tile rows are tokens), 2 = A is x
     // MN-major (tile rows are tokens of two 64-column halves)
     int mask_mode;
     const uint8_t *keep;
     int64_t mx, kx;
+    DropRng rng;
 };
 
 struct SkinnyArgs {
@@ -210,8 +212,19 @@ skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a0,
                 const int64_t m = J.mask_mode == 1 ? p0 + row : q0 + (row & 63);
                 const int64_t k0 = J.mask_mode == 1 ? q0 : p0 + 64 * (row >> 6);
                 const bool rok = m < J.mx && k0 < J.kx;
-                const uint64_t kw =
-                    rok ? __ldg(reinterpret_cast<const unsigned long long *>(J.keep + ((m * J.kx + k0) >> 3))) : ~0ull;
+                uint64_t kw = ~0ull;
+                if (rok) {
+                    if (J.rng.on) {
+                        // the row's 64 keep bits from the generator
+                        kw = 0;
+#pragma unroll 1
+                        for (int c = 0; c < 8; ++c)
+                            kw |= static_cast<uint64_t>(drop_keep8(J.rng, static_cast<uint64_t>(m * J.kx + k0) + 8 * c))
+                                  << (8 * c);
+                    } else {
+                        kw = __ldg(reinterpret_cast<const unsigned long long *>(J.keep + ((m * J.kx + k0) >> 3)));
+                    }
+                }
                 if (!mbar_wait(&full[st], ph, abort_flag)) break;
                 uint8_t *a = slot_a + st * Cfg::kABytes;
 #pragma unroll

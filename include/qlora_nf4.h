@@ -198,6 +198,34 @@ QLORA_API nf4_status qlora_linear_bwd_dropout(const nf4_weight *w, const uint16_
                                               uint16_t *dA, uint16_t *dB, void *workspace,
                                               size_t ws_bytes, void *stream);
 
+/* The same forward and backward with the dropout mask drawn inside the
+ * kernels instead of passed in. The pages fix no random generator; the draw is
+ * the counter-based Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel
+ * random numbers: as easy as 1, 2, 3", SC'11): element e = m * k + kk of x
+ * takes word (e mod 4) of Philox4x32-10 at counter (e div 4 as two 32-bit
+ * words, low first; offset as two words) with key (seed as two words) and is
+ * dropped when that word is below floor(p * 2^32). Each kernel that needs the
+ * mask computes the words of the elements it touches, so no mask is stored:
+ * the backward, given the forward's (p, seed, offset), regenerates exactly the
+ * forward's mask. Use a new offset (or seed) for every training step. All else
+ * (scaling, rounding, u, workspace sizes, requirements) is as in
+ * qlora_linear_fwd_dropout / qlora_linear_bwd_dropout; p outside [0, 1)
+ * returns NF4_ERR_INVALID_ARG. */
+QLORA_API nf4_status qlora_linear_fwd_dropout_philox(const nf4_weight *w, const uint16_t *x,
+                                                     int64_t M, const uint16_t *A,
+                                                     const uint16_t *B, int32_t r, float alpha,
+                                                     float p, uint64_t seed, uint64_t offset,
+                                                     uint16_t *h, float *u_out, void *workspace,
+                                                     size_t ws_bytes, void *stream);
+QLORA_API nf4_status qlora_linear_bwd_dropout_philox(const nf4_weight *w, const uint16_t *x,
+                                                     int64_t M, const uint16_t *A,
+                                                     const uint16_t *B, int32_t r, float alpha,
+                                                     float p, uint64_t seed, uint64_t offset,
+                                                     const uint16_t *dY, const float *u,
+                                                     uint16_t *dX, uint16_t *dA, uint16_t *dB,
+                                                     void *workspace, size_t ws_bytes,
+                                                     void *stream);
+
 /* Forward of one NF4 base with several adapters, one chosen per token, as a
  * server keeps one quantised base resident and applies each request's own
  * adapter ("Parameter-Efficient Fine-Tuning: From LoRA to QLoRA", "The PEFT

@@ -182,3 +182,36 @@ def test_multi_adapter_and_dropout_argument_checks(q):
     plain = q.bwd_workspace_bytes(4, 64, 64, 8)
     assert bwd_do(wsb=plain) == q.NF4_ERR_WORKSPACE
     assert L.qlora_bwd_dropout_workspace_bytes(4, 64, 64, 8) >= plain + 4 * 64 * 4
+
+
+def test_drawn_mask_dropout_argument_checks(q):
+    L = q.lib
+    w = weight(q)
+
+    def fwd(**kw):
+        return L.qlora_linear_fwd_dropout_philox(ctypes.byref(w), FAKE, kw.get("M", 4), FAKE, FAKE, 8,
+                                                 16.0, kw.get("p", 0.05), 1, 2, FAKE, None, FAKE,
+                                                 kw.get("wsb", 1 << 30), None)
+    assert fwd(p=1.0) == q.NF4_ERR_INVALID_ARG
+    assert fwd(p=-0.1) == q.NF4_ERR_INVALID_ARG
+    assert fwd(p=float("nan")) == q.NF4_ERR_INVALID_ARG
+    assert fwd(M=0) == q.NF4_OK
+    assert fwd(wsb=16) == q.NF4_ERR_WORKSPACE
+
+    def bwd(**kw):
+        return L.qlora_linear_bwd_dropout_philox(ctypes.byref(w), FAKE, 4, FAKE, FAKE, 8, 16.0,
+                                                 kw.get("p", 0.05), 1, 2, FAKE, None, None, FAKE, FAKE,
+                                                 FAKE, kw.get("wsb", 16), None)
+    assert bwd(p=1.5) == q.NF4_ERR_INVALID_ARG
+    plain = q.bwd_workspace_bytes(4, 64, 64, 8)
+    assert bwd(wsb=plain) == q.NF4_ERR_WORKSPACE
+
+    # the fp32-gradient backward takes the plain backward's workspace
+    def bwd32(**kw):
+        return L.qlora_linear_bwd_f32grad(ctypes.byref(w), FAKE, 4, FAKE, FAKE, kw.get("r", 8), 16.0,
+                                          FAKE, None, None, kw.get("dA", FAKE), FAKE, FAKE,
+                                          kw.get("wsb", 16), None)
+    assert bwd32(r=4) == q.NF4_ERR_UNSUPPORTED_SHAPE
+    assert bwd32(dA=None) == q.NF4_ERR_INVALID_ARG
+    assert bwd32(dA=FAKE + 4) == q.NF4_ERR_ALIGNMENT
+    assert bwd32(wsb=16) == q.NF4_ERR_WORKSPACE

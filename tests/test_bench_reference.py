@@ -28,3 +28,8 @@ def test_reference_arm_prints_contract_line():
     assert d["e2e"] == {"value": d["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
     assert "workload" in d["config"]
+    # the same workload description as the GPU arm's line (the headline workload)
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads
+    assert d["config"] == bench.main_config(workloads.WORKLOADS[bench.MAIN], 1)
