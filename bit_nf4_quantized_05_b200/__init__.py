@@ -83,6 +83,7 @@ def _load() -> ctypes.CDLL:
         "qlora_linear_fwd_dropout": ([W, vp, i64, vp, vp, i32, f32, f32, vp, vp, vp, vp, sz, vp],
                                      ctypes.c_int),
         "qlora_bwd_dropout_workspace_bytes": ([i64, i64, i64, i32], sz),
+        "nf4_debug_flag_wait": ([i32, i64], ctypes.c_int),
         "qlora_linear_fwd_dropout_philox": ([W, vp, i64, vp, vp, i32, f32, f32, u64, u64, vp, vp, vp,
                                              sz, vp], ctypes.c_int),
         "qlora_linear_bwd_dropout_philox": ([W, vp, i64, vp, vp, i32, f32, f32, u64, u64, vp, vp, vp,

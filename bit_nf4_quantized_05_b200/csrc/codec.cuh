@@ -91,14 +91,6 @@ __device__ __forceinline__ uint32_t nf4_code_exact(float w, float s, const float
     return c;
 }
 
-// Bounded wait that ignores the abort flag: used only to let copies already
-// issued land before the CTA exits.
-__device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity) {
-    const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity))
-        if (clock64() - t0 > kWaitLimitCycles) return;
-}
-
 // tm_w views W0 as 128-byte rows: fp32 [numel / 32, 32] with box {32, 128},
 // or 16-bit [numel / 64, 64] with box {64, 64}; either way a stage is 4096
 // elements. BS (64 or 128) elements per block: BS / 16 lanes code a block.

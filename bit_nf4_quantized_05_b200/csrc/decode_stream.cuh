@@ -508,14 +508,12 @@ qlora_decode_stream_kernel(const __grid_constant__ CUtensorMap tm_codes,   // [N
         if (kParkBufs == 1) __syncthreads();
     }
 done:
-    // leave no copy in flight into shared memory this CTA is about to release
-    if (lane == 0) {
-        for (int q = 0; q < 2; ++q) {
-            const int cq = c + q;           // chunks issued but not consumed: c and c + 1
-            if (cq < nchunks && cq >= 0)
-                mbar_wait(&bars[warp * 2 + (cq & 1)], static_cast<uint32_t>(cq >> 1) & 1u, abort_flag);
-        }
-    }
+    // Leave no copy in flight into shared memory this CTA is about to release.
+    // The only wait of the loop is on chunk c, and chunk c + 1 is issued only
+    // after it succeeds, so after giving up there, chunk c is the one copy
+    // that may still be landing (after a normal end, c == nchunks).
+    if (lane == 0 && c < nchunks)
+        mbar_drain(&bars[warp * 2 + (c & 1)], static_cast<uint32_t>(c >> 1) & 1u);
     __syncwarp();
 }
 

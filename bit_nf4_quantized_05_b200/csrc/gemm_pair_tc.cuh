@@ -99,31 +99,58 @@ struct PairCfg {
 };
 
 // The work of one pair: segments of stages [k0, k1) of a tile.
-//   Whole-tile schedule: tiles p, p + P, p + 2P, ... with every stage.
-//   Stream-K schedule: the units (tile, stage), numbered tile-major, are cut
-//   into P contiguous runs [W p / P, W (p + 1) / P) with W = T S; with T > P
-//   every run spans more than one tile, so a tile is split between at most
-//   two consecutive pairs: its head (stages [0, k)) is the last segment of
-//   pair p and its tail (stages [k, S)) the first segment of pair p + 1.
+//   Whole-tile schedule (sk = 0): tiles p, p + P, p + 2P, ... with every stage.
+//   Data-parallel waves + stream-K (sk = 1): the first (floor(T / P) - 1) P
+//   tiles go round-robin (pair p takes tiles p, p + P, ...) with every stage;
+//   the units (tile, stage) of the remaining P + (T mod P) tiles, numbered
+//   tile-major, are cut into P contiguous runs [W p / P, W (p + 1) / P) with
+//   W = (P + T mod P) S. Every run spans at least one tile, so a tile there is
+//   split between at most two consecutive pairs: its head (stages [0, k)) is
+//   the last segment of pair p and its tail (stages [k, S)) the first segment
+//   of pair p + 1. The round-robin waves keep the tiles in flight at one time
+//   consecutive in the raster order below (operands shared in L2), and the
+//   stream-K tail keeps the last wave from leaving pairs idle.
 struct PairSeg {
     int tile, k0, k1;
 };
 
 struct PairSched {
     int S, T, P, p, sk;
-    int64_t u0, u1;
+    int n_dp;          // tiles of the round-robin waves
+    int dp_count;      // this pair's round-robin tiles
+    int64_t u0, u1;    // this pair's stream-K units, as tile * S + stage
 
     __device__ __forceinline__ void init(int S_, int T_, int P_, int p_, int sk_) {
         S = S_; T = T_; P = P_; p = p_; sk = sk_;
-        const int64_t W = static_cast<int64_t>(T) * S;
-        u0 = sk ? (W * p) / P : 0;
-        u1 = sk ? (W * (p + 1)) / P : 0;
-    }
-    __device__ __forceinline__ bool first(PairSeg &g) const {
         if (!sk) {
-            g = {p, 0, S};
-            return p < T;
+            n_dp = T;
+            u0 = u1 = 0;
+        } else {
+            n_dp = (T / P - 1) * P;
+            const int64_t W = static_cast<int64_t>(T - n_dp) * S;
+            const int64_t base = static_cast<int64_t>(n_dp) * S;
+            u0 = base + (W * p) / P;
+            u1 = base + (W * (p + 1)) / P;
         }
+        dp_count = p < n_dp ? (n_dp - p + P - 1) / P : 0;
+    }
+    // units of this pair, in schedule order
+    __device__ __forceinline__ int units() const {
+        return dp_count * S + static_cast<int>(u1 - u0);
+    }
+    // the i-th unit of this pair (0 <= i < units())
+    __device__ __forceinline__ void unit(int i, int &tile, int &it) const {
+        if (i < dp_count * S) {
+            const int j = i / S;
+            tile = p + j * P;
+            it = i - j * S;
+        } else {
+            const int64_t u = u0 + (i - dp_count * S);
+            tile = static_cast<int>(u / S);
+            it = static_cast<int>(u - static_cast<int64_t>(tile) * S);
+        }
+    }
+    __device__ __forceinline__ bool sk_first(PairSeg &g) const {
         if (u0 >= u1) return false;
         const int t = static_cast<int>(u0 / S);
         const int k0 = static_cast<int>(u0 - static_cast<int64_t>(t) * S);
@@ -131,10 +158,20 @@ struct PairSched {
         g = {t, k0, rest < S ? static_cast<int>(rest) : S};
         return true;
     }
+    __device__ __forceinline__ bool first(PairSeg &g) const {
+        if (dp_count > 0) {
+            g = {p, 0, S};
+            return true;
+        }
+        return sk_first(g);
+    }
     __device__ __forceinline__ bool next(PairSeg &g) const {
-        if (!sk) {
-            g = {g.tile + P, 0, S};
-            return g.tile < T;
+        if (g.tile < n_dp) {
+            if (g.tile + P < n_dp) {
+                g = {g.tile + P, 0, S};
+                return true;
+            }
+            return sk_first(g);
         }
         const int t = g.tile + 1;
         const int64_t rest = u1 - static_cast<int64_t>(t) * S;
@@ -144,18 +181,38 @@ struct PairSched {
     }
 };
 
+// Raster order of the output tiles (256 tokens x BN columns): groups of
+// kRasterGroup token tiles, within a group column tile by column tile with
+// the token tiles fastest. The tiles of one wave (the pairs' current tiles,
+// consecutive in this order) then read about kRasterGroup activation slices
+// and P / kRasterGroup weight column tiles, a working set that stays in L2.
+constexpr int kRasterGroup = 4;
+
+__device__ __forceinline__ void tile_coords(int tile, int m_pairs, int n_tiles, int &mi, int &ni) {
+    const int per_group = kRasterGroup * n_tiles;
+    const int g = tile / per_group;
+    const int r = tile - g * per_group;
+    const int gm = min(kRasterGroup, m_pairs - g * kRasterGroup);   // token tiles in this group
+    ni = r / gm;
+    mi = g * kRasterGroup + (r - ni * gm);
+}
+
 // Bounded wait until a flag in global memory becomes non-zero (acquire, GPU
-// scope). On timeout the kernel's status is set and the caller gives up.
+// scope). It returns false if the CTA is giving up, or when the wait runs out
+// of time: then NF4_ERR_TIMEOUT is recorded in the device status and the
+// caller finishes its tile without what the flag guards (a wait on global
+// memory has no copy in flight, so nothing needs to unwind). The cycle limit
+// is the pipeline's unless a test has set g_dbg_flag_wait_limit.
 __device__ __forceinline__ bool wait_flag_gpu(const int *flag, volatile int *abort_flag) {
     const long long t0 = clock64();
+    const long long lim = g_dbg_flag_wait_limit > 0 ? g_dbg_flag_wait_limit : kWaitLimitCycles;
     while (true) {
         int v;
         asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
         if (v != 0) return true;
         if (*abort_flag) return false;
-        if (clock64() - t0 > kWaitLimitCycles) {
+        if (clock64() - t0 > lim) {
             record_status(NF4_ERR_TIMEOUT);
-            *abort_flag = 1;
             return false;
         }
     }
@@ -190,8 +247,12 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
     uint64_t *b_empty = b_full + SB;         // MMA done (pair commit)
     uint64_t *acc_full = b_empty + SB;       // [2] accumulator complete (pair commit)
     uint64_t *acc_empty = acc_full + 2;      // [2] even CTA: drained (epilogue warps of both)
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
+    uint64_t *mma_drain = acc_empty + 2;     // even CTA: the MMAs issued before giving up completed
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    // even CTA, read only after giving up: activation stages issued by each
+    // CTA's producer, and stages the MMA issuer consumed
+    volatile int *progress = reinterpret_cast<volatile int *>(tmem_slot + 2);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();             // 0 or 1 within the pair
@@ -215,6 +276,7 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
             mbar_init(&acc_full[b], 1);
             mbar_init(&acc_empty[b], 8);
         }
+        mbar_init(mma_drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tm_act);
@@ -243,6 +305,8 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
     PairSched sched;
     sched.init(nsteps, total_tiles, npairs, pair, args.sk);
     PairSeg sg;
+    // progress of the producers and of the MMA issuer (read after giving up)
+    int na = 0, nc = 0, cm = 0;
 
     if (warp == kTmaAWarp) {
         // ------------------------------------------------ TMA: activations
@@ -252,21 +316,23 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
             uint32_t pa = 0;
             bool la_ready = false;     // the rank-r activations are written by the kernel before
             for (bool more = sched.first(sg); more; more = sched.next(sg)) {
-                const int m0 = (sg.tile % m_pairs) * (2 * kBM) + static_cast<int>(rank) * kBM;
+                int mi, ni;
+                tile_coords(sg.tile, m_pairs, args.n_tiles, mi, ni);
+                const int m0 = mi * (2 * kBM) + static_cast<int>(rank) * kBM;
                 for (int it = sg.k0; it < sg.k1; ++it) {
                     if (!mbar_wait_cluster(&a_empty[sa], pa ^ 1, abort_flag)) goto done;
+                    if (it >= args.main_steps && !la_ready) {
+                        griddep_wait();
+                        la_ready = true;
+                    }
                     if (rank == 0) mbar_arrive_expect_tx(&a_full[sa], 2 * Cfg::kABytes);
                     if (it < args.main_steps)
                         tma_load_2d_pair(slot_a + sa * Cfg::kABytes, &tm_act, full0 + 8u * sa,
                                          it * kBK, m0);
-                    else {
-                        if (!la_ready) {
-                            griddep_wait();
-                            la_ready = true;
-                        }
+                    else
                         tma_load_2d_pair(slot_a + sa * Cfg::kABytes, &tm_la, full0 + 8u * sa,
                                          (it - args.main_steps) * kBK, m0);
-                    }
+                    ++na;
                     if (++sa == SA) { sa = 0; pa ^= 1; }
                 }
             }
@@ -277,7 +343,9 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
             int sc = 0;
             uint32_t pc = 0;
             for (bool more = sched.first(sg); more; more = sched.next(sg)) {
-                const int nh = (sg.tile / m_pairs) * BN + static_cast<int>(rank) * BH;
+                int mi, ni;
+                tile_coords(sg.tile, m_pairs, args.n_tiles, mi, ni);
+                const int nh = ni * BN + static_cast<int>(rank) * BH;
                 for (int it = sg.k0; it < sg.k1; ++it) {
                     if (!mbar_wait(&c_empty[sc], pc ^ 1, abort_flag)) goto done;
                     uint8_t *c = slot_c + sc * Cfg::kCBytes;
@@ -294,6 +362,7 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
                     } else {
                         mbar_arrive(&c_full[sc]);      // LoRA stage: no codes
                     }
+                    ++nc;
                     if (++sc == SC) { sc = 0; pc ^= 1; }
                 }
             }
@@ -324,6 +393,7 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
                     }
                     umma_commit_pair(&a_empty[sa], 0x3);
                     umma_commit_pair(&b_empty[sb], 0x3);
+                    ++cm;
                     if (++sa == SA) { sa = 0; pa ^= 1; }
                     if (++sb == SB) { sb = 0; pb ^= 1; }
                 }
@@ -346,8 +416,10 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
         int ab = 0;
         uint32_t aph = 0;
         for (bool more = sched.first(sg); more; more = sched.next(sg)) {
-            const int m0 = (sg.tile % m_pairs) * (2 * kBM) + static_cast<int>(rank) * kBM;
-            const int n0 = (sg.tile / m_pairs) * BN;
+            int mi, ni;
+            tile_coords(sg.tile, m_pairs, args.n_tiles, mi, ni);
+            const int m0 = mi * (2 * kBM) + static_cast<int>(rank) * kBM;
+            const int n0 = ni * BN;
             const bool tail = sg.k0 > 0;
             const bool head = !tail && sg.k1 < nsteps;
             const int rloc = q * 32 + lane;               // row within this CTA's 128
@@ -372,15 +444,17 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
                 if (lane == 0) {
                     mbar_arrive_cluster(empty0 + 8u * ab);
                     __threadfence();
-                    set_flag_gpu(args.flags + (pair * 2 + rank) * 4 + q);
+                    if (!g_dbg_skip_flag_set) set_flag_gpu(args.flags + (pair * 2 + rank) * 4 + q);
                 }
             } else {
                 const float *pp = nullptr;
+                bool add_partial = false;
                 if (head) {
                     // rows rloc of the partial were written by warp q of the
                     // same-rank CTA of the next pair
                     const int src = (pair + 1) * 2 + static_cast<int>(rank);
-                    if (!wait_flag_gpu(args.flags + src * 4 + q, abort_flag)) goto done;
+                    add_partial = wait_flag_gpu(args.flags + src * 4 + q, abort_flag);
+                    if (*abort_flag) goto done;
                     pp = args.partial + static_cast<int64_t>(src) * kChunks * (128 * 32) + rloc * 32;
                 }
                 const int row = m0 + rloc;
@@ -398,7 +472,7 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
                                 float f[8];
 #pragma unroll
                                 for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[g * 8 + e]);
-                                if (head) {
+                                if (add_partial) {
                                     const float4 *pv = reinterpret_cast<const float4 *>(
                                         pp + c * (128 * 32) + g * 8);
                                     const float4 p0 = pv[0], p1 = pv[1];
@@ -461,35 +535,34 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
             int tile, it;
             int64_t item;      // W row (forward) or W block column (dgrad); -1 outside W
         };
-        auto set_tile = [&](Pos &p) {
-            p.item = -1;
-            if (p.tile >= total_tiles) return;
-            const int64_t nh = static_cast<int64_t>(p.tile / m_pairs) * BN + rank * BH;
-            if (!DGRAD) {
-                if (nh + i < args.Nw) p.item = nh + i;
-            } else {
-                if (nh / 64 + kb < args.kblocks) p.item = nh / 64 + kb;
-            }
+        auto item_of = [&](int tile) -> int64_t {
+            int mi, ni;
+            tile_coords(tile, m_pairs, args.n_tiles, mi, ni);
+            const int64_t nh = static_cast<int64_t>(ni) * BN + rank * BH;
+            if (!DGRAD) return nh + i < args.Nw ? nh + i : -1;
+            return nh / 64 + kb < args.kblocks ? nh / 64 + kb : -1;
         };
-        const int tile_step = args.sk ? 1 : npairs;
-        auto step = [&](Pos &p, int n) {
-            p.it += n;
+        const int nunits = sched.units();
+        const int dp_units = sched.dp_count * nsteps;
+        // move from unit u to unit u + G (u + G < nunits): within the round-robin
+        // tiles or within the stream-K run by stepping, across the boundary
+        // between them by the schedule's unit()
+        auto advance = [&](Pos &p, int u) {
+            const int un = u + G;
+            if (u < dp_units && un >= dp_units) {
+                sched.unit(un, p.tile, p.it);
+                p.item = item_of(p.tile);
+                return;
+            }
+            const int tstep = un < dp_units ? npairs : 1;
+            p.it += G;
             bool moved = false;
             while (p.it >= nsteps) {
                 p.it -= nsteps;
-                p.tile += tile_step;
+                p.tile += tstep;
                 moved = true;
             }
-            if (moved) set_tile(p);
-        };
-        // the walk ends at unit (end_tile, end_it)
-        int end_tile = total_tiles, end_it = 0;
-        if (args.sk) {
-            end_tile = static_cast<int>(sched.u1 / nsteps);
-            end_it = static_cast<int>(sched.u1 - static_cast<int64_t>(end_tile) * nsteps);
-        }
-        auto alive = [&](const Pos &p) -> bool {
-            return p.tile < end_tile || (p.tile == end_tile && p.it < end_it);
+            if (moved) p.item = item_of(p.tile);
         };
         auto block_of = [&](const Pos &p) -> int64_t {
             if (p.tile >= total_tiles || p.it >= args.main_steps || p.item < 0) return -1;
@@ -512,19 +585,18 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
             return rs;
         };
 
-        Pos cur{pair, 0, -1};
-        if (args.sk) {
-            cur.tile = static_cast<int>(sched.u0 / nsteps);
-            cur.it = static_cast<int>(sched.u0 - static_cast<int64_t>(cur.tile) * nsteps);
+        int u = grp;
+        Pos cur{0, 0, -1};
+        if (u < nunits) {
+            sched.unit(u, cur.tile, cur.it);
+            cur.item = item_of(cur.tile);
         }
-        set_tile(cur);
-        step(cur, grp);
         // The scale of the next item is loaded after this item's last fence,
         // so that no load is outstanding across a proxy fence.
-        RawScale cs = load_scale(block_of(cur));
+        RawScale cs = load_scale(u < nunits ? block_of(cur) : -1);
         int sb = grp, sc = grp;
         uint32_t pb = 0, pc = 0;
-        while (alive(cur)) {
+        while (u < nunits) {
             const bool main = cur.it < args.main_steps;
 
             if (!mbar_wait(&c_full[sc], pc, abort_flag)) goto done;
@@ -598,13 +670,65 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
             if (sb >= SB) { sb -= SB; pb ^= 1; }
             sc += G;
             if (sc >= SC) { sc -= SC; pc ^= 1; }
-            step(cur, G);
-            cs = load_scale(block_of(cur));
+            if (u + G < nunits) {
+                advance(cur, u);
+                cs = load_scale(block_of(cur));
+            }
+            u += G;
         }
     }
 done:
+    // ---- giving up: leave no copy or MMA in flight. A role that gave up has
+    // raised this CTA's abort flag; pass it to the other CTA of the pair, whose
+    // roles then leave their waits too.
+    if (*abort_flag && lane == 0) {
+        const uint32_t peer = mapa_shared(smem_u32(const_cast<int *>(abort_flag)), rank ^ 1u);
+        asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(peer), "r"(1) : "memory");
+    }
+    if (lane == 0 && warp == kMmaWarp && rank == 0) {
+        if (*abort_flag) {
+            // the MMAs already issued complete before the operands are released
+            umma_commit_pair(mma_drain, 0x1);
+            mbar_drain(mma_drain, 0);
+        }
+        progress[2] = cm;
+    }
+    if (lane == 0 && warp == kTmaAWarp) {
+        // activation stages issued by this CTA, kept in the even CTA
+        if (rank == 0) {
+            progress[0] = na;
+        } else {
+            const uint32_t dst = mapa_shared(smem_u32(const_cast<int *>(progress)) + 4u, 0u);
+            asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(dst), "r"(na) : "memory");
+        }
+    }
+    if (lane == 0 && warp == kTmaCWarp) {
+        // code tiles land in this CTA only: wait for the ones still in flight
+        for (int it = nc > SC ? nc - SC : 0; it < nc; ++it)
+            mbar_drain(&c_full[it % SC], static_cast<uint32_t>(it / SC) & 1u);
+    }
     __syncthreads();
     cluster_sync();            // neither CTA leaves while the other may still use its memory
+    if (*abort_flag) {
+        // Both CTAs' activation copies complete on the even CTA's barriers,
+        // which expect the two halves of a stage once the even producer has
+        // issued its own. Stages the MMA issuer did not consume may still be in
+        // flight; where only one producer issued a stage, the even CTA supplies
+        // the other half's arrival or bytes so that the phase can complete,
+        // then waits for it. (At most SA stages are outstanding, one per slot.)
+        if (rank == 0 && warp == kTmaAWarp && lane == 0) {
+            const int n0 = progress[0], n1 = progress[1];
+            const int hi = n0 > n1 ? n0 : n1;
+            for (int st = progress[2]; st < hi; ++st) {
+                uint64_t *bar = &a_full[st % SA];
+                if (st < n0 && st >= n1) mbar_complete_tx(bar, Cfg::kABytes);
+                if (st >= n0 && st < n1) mbar_arrive_expect_tx(bar, Cfg::kABytes);
+                mbar_drain(bar, static_cast<uint32_t>(st / SA) & 1u);
+            }
+        }
+        __syncthreads();
+        cluster_sync();        // the odd CTA's activation copies have landed too
+    }
     if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc_pair(tmem_base, Cfg::kTmemCols);

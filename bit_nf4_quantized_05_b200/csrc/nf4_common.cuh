@@ -130,6 +130,29 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
+// Bounded wait that ignores the abort flag: used on the way out of a kernel
+// that gave up, so that the copies (or tensor-core operations) it has already
+// issued land before its shared memory and tensor memory are released.
+__device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity))
+        if (clock64() - t0 > kWaitLimitCycles) return;
+}
+
+// complete_tx of `bytes` on an mbarrier of this CTA (bytes that will never be
+// copied: lets a phase whose copy was never issued complete).
+__device__ __forceinline__ void mbar_complete_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+// Test hooks of the stream-K flag wait (set through nf4_debug_flag_wait):
+// when g_dbg_skip_flag_set is nonzero the tails of split tiles do not raise
+// their flags, and a nonzero g_dbg_flag_wait_limit replaces the flag wait's
+// cycle limit, so a test can make that one wait run out.
+__device__ int g_dbg_skip_flag_set;
+__device__ long long g_dbg_flag_wait_limit;
+
 // ---------------------------------------------------------------------------
 // Programmatic dependent launch. Every kernel of this library that is launched
 // as a programmatic dependent first waits for the grid before it in the stream

@@ -765,6 +765,15 @@ int32_t nf4_profile_read(nf4_kernel_time *out, int32_t max) {
     return cnt;
 }
 
+nf4_status nf4_debug_flag_wait(int32_t skip_flag_set, int64_t limit_cycles) {
+    if (limit_cycles < 0 || (skip_flag_set != 0 && skip_flag_set != 1)) return NF4_ERR_INVALID_ARG;
+    const int skip = skip_flag_set;
+    const long long lim = limit_cycles;
+    NF4_TRY_CUDA(cudaMemcpyToSymbol(g_dbg_skip_flag_set, &skip, sizeof skip));
+    NF4_TRY_CUDA(cudaMemcpyToSymbol(g_dbg_flag_wait_limit, &lim, sizeof lim));
+    return NF4_OK;
+}
+
 nf4_status nf4_device_status(void *stream) {
     NF4_TRY_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
     unsigned int v = 0, zero = 0;

@@ -153,10 +153,12 @@ skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a0,
     }
 
     if (warp == 0 && lane == 0) {
+        int issued = 0;
         for (int it = 0; it < nsteps; ++it) {
             const int st = it % kSkStages;
             const uint32_t ph = (it / kSkStages) & 1;
             if (!mbar_wait(&empty[st], ph ^ 1, abort_flag)) break;
+            ++issued;
             uint8_t *a = slot_a + st * Cfg::kABytes;
             uint8_t *b = slot_b + st * Cfg::kBBytes;
             const int q0 = (s0 + it) * 64;
@@ -175,6 +177,11 @@ skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a0,
                     tma_load_2d(b + ja * 8192, tm_b, &full[st], ja * 64, q0);
             }
         }
+        // every copy issued has landed before the stage buffers are reused or
+        // released (at most one stage per slot can still be in flight; after
+        // a normal run all of them were consumed, so these return at once)
+        for (int it = issued > kSkStages ? issued - kSkStages : 0; it < issued; ++it)
+            mbar_drain(&full[it % kSkStages], static_cast<uint32_t>(it / kSkStages) & 1u);
     } else if (warp == 1 && lane == 0) {
         const uint32_t a_base = smem_u32(slot_a), b_base = smem_u32(slot_b);
         bool ok = true;
@@ -194,7 +201,10 @@ skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a0,
             }
             umma_commit(&empty[st]);
         }
-        if (ok) umma_commit(done_bar);
+        // after giving up, the MMAs already issued must complete before the
+        // stage buffers and tensor memory are released
+        umma_commit(done_bar);
+        if (!ok) mbar_drain(done_bar, 0);
     } else if (warp >= 4 && warp < 8) {
         if (J.mask_mode) {
             // dropout: zero the dropped elements of each landed A tile in place

@@ -295,6 +295,19 @@ QLORA_API nf4_status qlora_merge(const nf4_weight *w, const uint16_t *A, const u
  * kernels of the current device set (NF4_OK if nothing was recorded). */
 QLORA_API nf4_status nf4_device_status(void *stream);
 
+/* Test hook of the failure-detection path (no counterpart on the pages).
+ * Every wait inside the kernels is bounded: a pipeline wait that runs out
+ * records NF4_ERR_TIMEOUT, lets the copies and tensor-core operations already
+ * issued complete, and returns; the wait of a split tile's first half for the
+ * partial sum of its second half (computed by the next CTA pair) records
+ * NF4_ERR_TIMEOUT and finishes the tile without it. With skip_flag_set = 1 the
+ * second halves do not signal their partial sums, and limit_cycles > 0
+ * replaces that one wait's limit (SM clock cycles), so a test can make it run
+ * out in microseconds and check the status and a following clean call.
+ * (0, 0) restores normal operation. Applies to the current device, between
+ * calls (it is not ordered with kernels in flight: synchronise first). */
+QLORA_API nf4_status nf4_debug_flag_wait(int32_t skip_flag_set, int64_t limit_cycles);
+
 /* Per-kernel timing, for benchmarks. While enabled, every kernel the library
  * launches is bracketed by two CUDA events recorded on the stream it is
  * launched on; nf4_profile_read() synchronises those events and reports, per

@@ -215,3 +215,9 @@ def test_drawn_mask_dropout_argument_checks(q):
     assert bwd32(dA=None) == q.NF4_ERR_INVALID_ARG
     assert bwd32(dA=FAKE + 4) == q.NF4_ERR_ALIGNMENT
     assert bwd32(wsb=16) == q.NF4_ERR_WORKSPACE
+
+
+def test_debug_flag_wait_hook_argument_checks(q):
+    L = q.lib
+    assert L.nf4_debug_flag_wait(2, 0) == q.NF4_ERR_INVALID_ARG
+    assert L.nf4_debug_flag_wait(0, -1) == q.NF4_ERR_INVALID_ARG
