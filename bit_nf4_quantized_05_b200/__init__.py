@@ -39,7 +39,10 @@ DQ_GROUP = 256
 class NF4Error(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = code
-        super().__init__(f"{where}: {status_string(code)} (status {code})")
+        detail = ""
+        if code == NF4_ERR_CUDA:
+            detail = ": " + lib.nf4_last_cuda_error().decode(errors="replace")
+        super().__init__(f"{where}: {status_string(code)} (status {code}){detail}")
 
 
 class NF4WeightStruct(ctypes.Structure):
@@ -84,6 +87,7 @@ def _load() -> ctypes.CDLL:
                                      ctypes.c_int),
         "qlora_bwd_dropout_workspace_bytes": ([i64, i64, i64, i32], sz),
         "nf4_debug_flag_wait": ([i32, i64], ctypes.c_int),
+        "nf4_last_cuda_error": ([], ctypes.c_char_p),
         "qlora_linear_fwd_dropout_philox": ([W, vp, i64, vp, vp, i32, f32, f32, u64, u64, vp, vp, vp,
                                              sz, vp], ctypes.c_int),
         "qlora_linear_bwd_dropout_philox": ([W, vp, i64, vp, vp, i32, f32, f32, u64, u64, vp, vp, vp,

@@ -580,8 +580,7 @@ qlora_decode_u_kernel(const DecodeArgs a, const uint8_t *__restrict__ keep, cons
                         const int m = tg * 8 + g;
                         const int64_t e = static_cast<int64_t>(m) * a.K + kb * 64 + 16 * t;
                         const uint32_t kbits =
-                            rng.on ? (drop_keep8(rng, static_cast<uint64_t>(e)) |
-                                      (drop_keep8(rng, static_cast<uint64_t>(e) + 8) << 8))
+                            rng.on ? static_cast<uint32_t>(drop_keep_bits<4>(rng, static_cast<uint64_t>(e)))
                                    : (keep[e >> 3] | (static_cast<uint32_t>(keep[(e >> 3) + 1]) << 8));
                         uint32_t w[8] = {xa[tg].x, xa[tg].y, xa[tg].z, xa[tg].w,
                                          xb[tg].x, xb[tg].y, xb[tg].z, xb[tg].w};

@@ -457,21 +457,37 @@ __device__ __forceinline__ uint4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_
     return make_uint4(c0, c1, c2, c3);
 }
 
-// Keep bits of the eight elements [e0, e0 + 8) of x (e0 % 8 == 0): bit i is 1
-// when element e0 + i is kept.
-__device__ __forceinline__ uint32_t drop_keep8(const DropRng &d, uint64_t e0) {
-    uint32_t bits = 0;
+// Keep bits of the 4 * CALLS elements [e0, e0 + 4 CALLS) of x (e0 % 4 == 0):
+// bit i is 1 when element e0 + i is kept. The generator calls are independent
+// and computed four at a time, so that their multiply chains overlap.
+template <int CALLS>
+__device__ __forceinline__ uint64_t drop_keep_bits(const DropRng &d, uint64_t e0) {
+    static_assert(CALLS >= 1 && CALLS <= 16, "at most 64 bits");
+    constexpr int kBatch = CALLS < 4 ? CALLS : 4;
+    uint64_t bits = 0;
+    const uint64_t g0 = e0 >> 2;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const uint64_t g = (e0 >> 2) + h;
-        const uint4 v = philox4x32_10(static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), d.o0, d.o1,
-                                      d.k0, d.k1);
-        bits |= (v.x >= d.thresh ? 1u : 0u) << (4 * h);
-        bits |= (v.y >= d.thresh ? 1u : 0u) << (4 * h + 1);
-        bits |= (v.z >= d.thresh ? 1u : 0u) << (4 * h + 2);
-        bits |= (v.w >= d.thresh ? 1u : 0u) << (4 * h + 3);
+    for (int q = 0; q < CALLS; q += kBatch) {
+        uint4 v[kBatch];
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) {
+            const uint64_t g = g0 + q + j;
+            v[j] = philox4x32_10(static_cast<uint32_t>(g), static_cast<uint32_t>(g >> 32), d.o0, d.o1, d.k0,
+                                 d.k1);
+        }
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) {
+            const uint64_t nib = (v[j].x >= d.thresh ? 1u : 0u) | (v[j].y >= d.thresh ? 2u : 0u) |
+                                 (v[j].z >= d.thresh ? 4u : 0u) | (v[j].w >= d.thresh ? 8u : 0u);
+            bits |= nib << (4 * (q + j));
+        }
     }
     return bits;
+}
+
+// Keep bits of the eight elements [e0, e0 + 8) of x (e0 % 8 == 0).
+__device__ __forceinline__ uint32_t drop_keep8(const DropRng &d, uint64_t e0) {
+    return static_cast<uint32_t>(drop_keep_bits<2>(d, e0));
 }
 
 }  // namespace nf4

@@ -9,6 +9,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -26,9 +27,24 @@ namespace {
 constexpr int kMaxDevices = 64;
 constexpr int kMaxAdapters = 16;   // stacked adapters of one multi-adapter forward
 
-#define NF4_TRY_CUDA(expr)                          \
-    do {                                            \
-        if ((expr) != cudaSuccess) return NF4_ERR_CUDA; \
+// The description of the last NF4_ERR_CUDA returned on this thread: the
+// failing CUDA call's error string and where it came from.
+thread_local char t_last_error[256] = "";
+
+nf4_status cuda_fail(cudaError_t e, int line) {
+    std::snprintf(t_last_error, sizeof t_last_error, "%s (qlora_nf4.cu line %d)", cudaGetErrorString(e), line);
+    return NF4_ERR_CUDA;
+}
+
+nf4_status map_fail(int line) {
+    std::snprintf(t_last_error, sizeof t_last_error, "tensor map encoding failed (qlora_nf4.cu line %d)", line);
+    return NF4_ERR_CUDA;
+}
+
+#define NF4_TRY_CUDA(expr)                                  \
+    do {                                                    \
+        const cudaError_t nf4_e_ = (expr);                  \
+        if (nf4_e_ != cudaSuccess) return cuda_fail(nf4_e_, __LINE__); \
     } while (0)
 
 // ---------------------------------------------------------------------------
@@ -358,7 +374,7 @@ nf4_status skinny_launch(int kind, const SkinnySpec *sp, int n, cudaStream_t str
     SkinnyArgs args{};
     CUtensorMap ta[2], tb[2];
     for (int i = 0; i < n; ++i)
-        if (!skinny_job(sp[i], RN, splits, &ta[i], &tb[i], &args.job[i])) return NF4_ERR_CUDA;
+        if (!skinny_job(sp[i], RN, splits, &ta[i], &tb[i], &args.job[i])) return map_fail(__LINE__);
     if (n == 1) {
         ta[1] = ta[0];
         tb[1] = tb[0];
@@ -399,7 +415,7 @@ nf4_status skinny_launch(int kind, const SkinnySpec *sp, int n, cudaStream_t str
 #undef NF4_SKINNY_CASE
         t.stop();
     }
-    if (e != cudaSuccess) return NF4_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_fail(e, __LINE__);
     NF4_TRY_CUDA(cudaGetLastError());
     return NF4_OK;
 }
@@ -467,7 +483,7 @@ nf4_status launch_gemm_pair(const nf4_weight *w, const uint16_t *act, int64_t M,
                             CU_TENSOR_MAP_SWIZZLE_128B);
     else
         tm_la = tm_act;
-    if (!ok) return NF4_ERR_CUDA;
+    if (!ok) return map_fail(__LINE__);
 
     GemmArgs a{};
     a.M = static_cast<int>(M);
@@ -492,7 +508,10 @@ nf4_status launch_gemm_pair(const nf4_weight *w, const uint16_t *act, int64_t M,
 
     const int dev = current_device();
     const int cap = pair_capacity<BN, DGRAD, G>(dev);
-    if (cap <= 0) return NF4_ERR_CUDA;
+    if (cap <= 0) {
+        std::snprintf(t_last_error, sizeof t_last_error, "no CTA pair of the fused GEMM can be resident");
+        return NF4_ERR_CUDA;
+    }
     const int64_t m_pairs = (M + 2 * kBM - 1) / (2 * kBM);
     const int64_t tiles = m_pairs * a.n_tiles;
     const bool use_sk = BN == 256 && sk && sk->partial && sk->flags && cap <= sk->pairs_max &&
@@ -513,7 +532,7 @@ nf4_status launch_gemm_pair(const nf4_weight *w, const uint16_t *act, int64_t M,
             : launch_ex(qlora_gemm_pair_kernel<BN, DGRAD, G, false>, dim3(static_cast<unsigned>(2 * pairs)),
                         dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, 2u, tm_act, tm_codes, tm_la, a);
     t.stop();
-    if (e != cudaSuccess) return NF4_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_fail(e, __LINE__);
     NF4_TRY_CUDA(cudaGetLastError());
     return NF4_OK;
 }
@@ -596,7 +615,7 @@ nf4_status launch_decode(const nf4_weight *w, const uint16_t *x, int64_t M, cons
     CUtensorMap tm_codes;
     if (!make_map(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, w->k / 2, w->n,
                   static_cast<uint32_t>(32 * cb), kDsRows, CU_TENSOR_MAP_SWIZZLE_NONE))
-        return NF4_ERR_CUDA;
+        return map_fail(__LINE__);
     const int64_t tiles = (w->n + kDsRows - 1) / kDsRows;
     // the decode grid leaves kDsUCtas SMs to the u kernel
     const int sms = num_sms(current_device());
@@ -609,7 +628,7 @@ nf4_status launch_decode(const nf4_weight *w, const uint16_t *x, int64_t M, cons
         NF4_TRY_CUDA(cudaFuncSetAttribute(ku, cudaFuncAttributeMaxDynamicSharedMemorySize, kDsUParkBytes));
         const cudaError_t e = launch_ex(ku, dim3(kDsUCtas), dim3(kDsThreads), kDsUParkBytes, stream, 0u, a, keep, rng);
         t.stop();
-        if (e != cudaSuccess) return NF4_ERR_CUDA;
+        if (e != cudaSuccess) return cuda_fail(e, __LINE__);
     }
     LaunchTimer t(KK_DECODE, stream);
     cudaError_t e;
@@ -624,7 +643,7 @@ nf4_status launch_decode(const nf4_weight *w, const uint16_t *x, int64_t M, cons
         e = launch_decode_stream(tg, cb, grid, stream, tm_codes, a, DsNoGroups{});
     }
     t.stop();
-    if (e != cudaSuccess) return NF4_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_fail(e, __LINE__);
     NF4_TRY_CUDA(cudaGetLastError());
     return NF4_OK;
 }
@@ -685,6 +704,7 @@ nf4_status launch_gemm_auto(const nf4_weight *w, const uint16_t *act, int64_t M,
         }
     }
     // no CTA pair of this kernel can be resident (not the case on a B200)
+    std::snprintf(t_last_error, sizeof t_last_error, "no CTA pair of the fused GEMM can be resident");
     return NF4_ERR_CUDA;
 }
 
@@ -717,6 +737,8 @@ void *static_scratch_on_current_device() {
 }  // namespace
 
 extern "C" {
+
+const char *nf4_last_cuda_error(void) { return t_last_error; }
 
 const char *nf4_status_string(nf4_status s) {
     switch (s) {
@@ -803,7 +825,7 @@ nf4_status nf4_quantize_typed(const void *W0, int32_t dtype, const nf4_weight *w
                       dtype == NF4_DTYPE_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
                       2, W0, 64, static_cast<uint64_t>(numel / 64), 64, kQzStageElems / 64,
                       CU_TENSOR_MAP_SWIZZLE_128B);
-    if (!ok) return NF4_ERR_CUDA;
+    if (!ok) return map_fail(__LINE__);
     // persistent: kQzCtasPerSm CTAs per SM walk the groups
     const int64_t grid = std::min<int64_t>(groups, int64_t(kQzCtasPerSm) * num_sms(current_device()));
     void (*kern)(const CUtensorMap, int64_t, int, uint8_t *, float *, uint8_t *, float *);
@@ -886,7 +908,7 @@ nf4_status qlora_merge(const nf4_weight *w, const uint16_t *A, const uint16_t *B
     LaunchTimer t(KK_MERGE, s);
     const cudaError_t e = launch_ex(kern, grid, dim3(kMgThreads), static_cast<size_t>(smem), s, 0u, a);
     t.stop();
-    if (e != cudaSuccess) return NF4_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_fail(e, __LINE__);
     NF4_TRY_CUDA(cudaGetLastError());
     return NF4_OK;
 }
@@ -1011,7 +1033,10 @@ nf4_status qlora_linear_fwd_noalloc(const nf4_weight *w, const uint16_t *x, int6
     const FwdLayout L = fwd_layout(M, r, 0, false);   // whole-tile schedule: no stream-K scratch
     if (L.total > kStaticScratchBytes) return NF4_ERR_UNSUPPORTED_SHAPE;
     uint8_t *ws = static_cast<uint8_t *>(static_scratch_on_current_device());
-    if (!ws) return NF4_ERR_CUDA;
+    if (!ws) {
+        std::snprintf(t_last_error, sizeof t_last_error, "the scratch array's device address was not found");
+        return NF4_ERR_CUDA;
+    }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint16_t *u_s = reinterpret_cast<uint16_t *>(ws + L.us);
     const float scale = alpha / static_cast<float>(r);
@@ -1062,7 +1087,7 @@ nf4_status lora_add(const float *base, const uint16_t *Vs, const uint16_t *A, co
     LaunchTimer t(KK_LORA_ADD, s);
     const cudaError_t e = launch_ex(kern, grid, dim3(kMgThreads), static_cast<size_t>(smem), s, 0u, a);
     t.stop();
-    if (e != cudaSuccess) return NF4_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_fail(e, __LINE__);
     NF4_TRY_CUDA(cudaGetLastError());
     return NF4_OK;
 }
@@ -1095,7 +1120,7 @@ nf4_status bwd_impl(const nf4_weight *w, const uint16_t *x, int64_t M, const uin
         const cudaError_t e2 = launch_ex(zero_u16_kernel, dim3(64), dim3(256), 0, s, 0u,
                                          static_cast<uint16_t *>(dB), per * N * r);
         t.stop();
-        if (e1 != cudaSuccess || e2 != cudaSuccess) return NF4_ERR_CUDA;
+        if (e1 != cudaSuccess || e2 != cudaSuccess) return cuda_fail(e1 != cudaSuccess ? e1 : e2, __LINE__);
         NF4_TRY_CUDA(cudaGetLastError());
         return NF4_OK;
     }

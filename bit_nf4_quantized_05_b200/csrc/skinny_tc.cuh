@@ -226,11 +226,7 @@ skinny_cluster_kernel(const __grid_constant__ CUtensorMap tm_a0,
                 if (rok) {
                     if (J.rng.on) {
                         // the row's 64 keep bits from the generator
-                        kw = 0;
-#pragma unroll 1
-                        for (int c = 0; c < 8; ++c)
-                            kw |= static_cast<uint64_t>(drop_keep8(J.rng, static_cast<uint64_t>(m * J.kx + k0) + 8 * c))
-                                  << (8 * c);
+                        kw = drop_keep_bits<16>(J.rng, static_cast<uint64_t>(m * J.kx + k0));
                     } else {
                         kw = __ldg(reinterpret_cast<const unsigned long long *>(J.keep + ((m * J.kx + k0) >> 3)));
                     }

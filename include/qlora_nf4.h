@@ -328,6 +328,12 @@ QLORA_API nf4_status nf4_profiling(int32_t enable);
  * (or -1 if reading an event failed). */
 QLORA_API int32_t nf4_profile_read(nf4_kernel_time *out, int32_t max);
 
+/* When an entry point returned NF4_ERR_CUDA: the failing CUDA call's error
+ * string and where in the library it came from (the last such failure on the
+ * calling thread; empty if none). Never NULL; valid until the thread's next
+ * failing call. */
+QLORA_API const char *nf4_last_cuda_error(void);
+
 /* Static description of a status code. Never NULL. */
 QLORA_API const char *nf4_status_string(nf4_status s);
 

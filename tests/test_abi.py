@@ -221,3 +221,8 @@ def test_debug_flag_wait_hook_argument_checks(q):
     L = q.lib
     assert L.nf4_debug_flag_wait(2, 0) == q.NF4_ERR_INVALID_ARG
     assert L.nf4_debug_flag_wait(0, -1) == q.NF4_ERR_INVALID_ARG
+
+
+def test_last_cuda_error_is_a_string(q):
+    s = q.lib.nf4_last_cuda_error()
+    assert isinstance(s, bytes)
