@@ -110,6 +110,39 @@ def test_layer_small_shapes(q, N, K, M, r, alpha, dq):
                          tag=f"{N}x{K} M={M} r={r}", edge=M < 16)
 
 
+# More 256 x 256 output tiles than resident CTA pairs (74 on a B200): round-
+# robin waves, then the last tiles split between pairs (stream-K); ragged
+# token and feature tails, one and two LoRA stages, blocks of 64 and 128.
+STREAM_K_SHAPES = [
+    # (N, K, M, r, alpha, dq, block)
+    (8000, 576, 600, 16, 32.0, True, 64),
+    (8000, 512, 520, 128, 16.0, False, 64),
+    (7944, 1152, 700, 64, 16.0, True, 128),
+]
+
+
+@pytest.mark.parametrize("N,K,M,r,alpha,dq,block", STREAM_K_SHAPES)
+def test_layer_stream_k_ragged(q, N, K, M, r, alpha, dq, block):
+    w = workloads.LayerWorkload("t", N, K, M, r, alpha, 0.02, dq, 3131 + N + K + M + r)
+    inp = workloads.make_inputs(w)
+    res = run_layer(q, inp["W0"], inp["A"], inp["B"], inp["x"], inp["dY"], alpha, dq, block=block)
+    check_against_oracle(q, res, inp["A"], inp["B"], inp["x"], inp["dY"], alpha,
+                         rows=sampled_rows(M, 40, 7), tag=f"{N}x{K} M={M} r={r} b{block}")
+
+
+def test_stream_k_lora_branch_alone(q):
+    """W0 = 0 on a stream-K forward: h is the up-projection stage alone, also in
+    the tiles split between two CTA pairs."""
+    N, K, M, r, alpha = 8000, 512, 520, 64, 16.0
+    w = workloads.LayerWorkload("t", N, K, M, r, alpha, 0.02, True, 6262)
+    inp = workloads.make_inputs(w)
+    res = run_layer(q, torch.zeros(N, K), inp["A"], inp["B"], inp["x"], inp["dY"], alpha, True,
+                    need_bwd=False)
+    check_against_oracle(q, res, inp["A"], inp["B"], inp["x"], None, alpha, need_bwd=False,
+                         rows=sampled_rows(M, 40, 9), tag="stream-K lora-only")
+    assert float(res["h"].float().abs().max()) > 0
+
+
 @pytest.mark.parametrize("r", [8, 64])
 def test_lora_branch_alone(q, r):
     """W0 = 0: every code is the zero level, h and dX are the LoRA terms only."""
