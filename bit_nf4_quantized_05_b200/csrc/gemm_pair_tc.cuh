@@ -429,13 +429,14 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
                 float *pp = args.partial +
                             (static_cast<int64_t>(pair) * 2 + rank) * kChunks * (128 * 32) + rloc * 32;
 #pragma unroll 1
-                for (int c = 0; c < kChunks; ++c) {
-                    uint32_t v[32];
-                    tmem_ld_32x32b_x32(tmem_base + ((q * 32) << 16) + ab * BN + c * 32, v);
+                for (int c2 = 0; c2 < 2 * kChunks; ++c2) {      // 16 columns at a time
+                    uint32_t v[16];
+                    tmem_ld_32x32b_x16(tmem_base + ((q * 32) << 16) + ab * BN + c2 * 16, v);
                     tmem_ld_wait();
+                    float *dst = pp + (c2 >> 1) * (128 * 32) + (c2 & 1) * 16;
 #pragma unroll
-                    for (int e = 0; e < 32; e += 4)
-                        *reinterpret_cast<float4 *>(pp + c * (128 * 32) + e) =
+                    for (int e = 0; e < 16; e += 4)
+                        *reinterpret_cast<float4 *>(dst + e) =
                             make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
                                         __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
                 }
@@ -460,18 +461,20 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
                 const int row = m0 + rloc;
                 uint16_t *drow = args.D + static_cast<int64_t>(row) * args.out;
 #pragma unroll 1
-                for (int c = 0; c < kChunks; ++c) {
-                    uint32_t v[32];
-                    tmem_ld_32x32b_x32(tmem_base + ((q * 32) << 16) + ab * BN + c * 32, v);
+                for (int c2 = 0; c2 < 2 * kChunks; ++c2) {      // 16 columns at a time
+                    const int c = c2 >> 1;
+                    uint32_t v[16];
+                    tmem_ld_32x32b_x16(tmem_base + ((q * 32) << 16) + ab * BN + c2 * 16, v);
                     tmem_ld_wait();
                     if (row < args.M) {
 #pragma unroll
-                        for (int g = 0; g < 4; ++g) {
+                        for (int gg = 0; gg < 2; ++gg) {
+                            const int g = 2 * (c2 & 1) + gg;       // 8-column group of the 32-column chunk
                             const int col = n0 + c * 32 + g * 8;
                             if (col < args.out) {
                                 float f[8];
 #pragma unroll
-                                for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[g * 8 + e]);
+                                for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[gg * 8 + e]);
                                 if (add_partial) {
                                     const float4 *pv = reinterpret_cast<const float4 *>(
                                         pp + c * (128 * 32) + g * 8);
@@ -600,24 +603,36 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
             const bool main = cur.it < args.main_steps;
 
             if (!mbar_wait(&c_full[sc], pc, abort_flag)) goto done;
-            uint32_t out[32];
+            // this item's 64 codes go to registers, which frees the code slot
+            uint4 h0 = make_uint4(0, 0, 0, 0), h1 = h0;
+            float s = 0.0f;          // blocks outside W get scale 0: every level maps to +-0
             if (main) {
                 const uint8_t *cp = slot_c + sc * Cfg::kCBytes + code_off;
-                const uint4 h0 = *reinterpret_cast<const uint4 *>(cp + 16 * cswz);
-                const uint4 h1 = *reinterpret_cast<const uint4 *>(cp + 16 * (cswz ^ 1));
-                // blocks outside W get scale 0: every level maps to +-0
-                float s = 0.0f;
+                h0 = *reinterpret_cast<const uint4 *>(cp + 16 * cswz);
+                h1 = *reinterpret_cast<const uint4 *>(cp + 16 * (cswz ^ 1));
                 if (cs.b >= 0)
                     s = args.dq ? __fmul_rn(static_cast<float>(cs.q8), __fdiv_rn(cs.v, 127.0f))
                                 : cs.v;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&c_empty[sc]);
+
+            // Each 8-code word becomes one 16-byte piece of the row and is stored
+            // at once, so at most one piece is live in registers (no spills at
+            // the 72 registers a thread has).
+            if (!mbar_wait_cluster(&b_empty[sb], pb ^ 1, abort_flag)) goto done;
+            uint8_t *brow = slot_b + sb * Cfg::kBBytes + row_off;
+            auto put = [&](int c, uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
+                *reinterpret_cast<uint4 *>(brow + ((c ^ swz) << 4)) = make_uint4(w0, w1, w2, w3);
+            };
+            if (main) {
                 const BlockLut L = make_block_lut(s);
                 const uint32_t words[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
 #pragma unroll
                 for (int wd = 0; wd < 8; ++wd) {
                     uint32_t o[4];
                     dequant8(L, words[wd], o);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) out[4 * wd + e] = o[e];
+                    put(wd, o[0], o[1], o[2], o[3]);
                 }
             } else {
                 // LoRA stage: the adapter tile comes straight from global memory
@@ -646,22 +661,9 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
                 for (int c = 0; c < 8; ++c) {
                     uint4 v = make_uint4(0, 0, 0, 0);
                     if (c < nvalid) v = __ldg(reinterpret_cast<const uint4 *>(src) + c);
-                    out[4 * c] = v.x;
-                    out[4 * c + 1] = v.y;
-                    out[4 * c + 2] = v.z;
-                    out[4 * c + 3] = v.w;
+                    put(c, v.x, v.y, v.z, v.w);
                 }
             }
-            // codes and scales are consumed (out depends on them): release the slot
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&c_empty[sc]);
-
-            if (!mbar_wait_cluster(&b_empty[sb], pb ^ 1, abort_flag)) goto done;
-            uint8_t *brow = slot_b + sb * Cfg::kBBytes + row_off;
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                *reinterpret_cast<uint4 *>(brow + ((c ^ swz) << 4)) =
-                    make_uint4(out[4 * c], out[4 * c + 1], out[4 * c + 2], out[4 * c + 3]);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(full0 + 8u * sb);
