@@ -24,7 +24,10 @@
 //
 // Synchronisation across the pair:
 //   a_full  (even CTA)   both CTAs' activation loads credit their bytes here
-//   b_full  (even CTA)   the dequant warps of both CTAs arrive here
+//   b_full  (even CTA)   the dequant warps of both CTAs arrive here; the even
+//                        CTA's warps arrive only once the stage's a_full phase
+//                        has completed, so the MMA issuer waits on b_full alone
+//                        (one barrier probe per stage on its critical path)
 //   acc_empty (even CTA) the epilogue warps of both CTAs arrive here
 //   a_empty, b_empty, acc_full (both CTAs)  one multicast tcgen05.commit
 // The code-tile ring is private to each CTA.
@@ -95,6 +98,10 @@ struct PairCfg {
     static_assert(kBBytes % 1024 == 0 && kCBytes % 1024 == 0, "stage alignment");
     static_assert(kSC % G == 0 && kSB % G == 0, "each dequant group owns every G-th slot");
     static_assert(kSA >= 3, "pipeline depth");
+    // The even CTA's dequant warps wait on a_full of stage u while the MMA may
+    // still hold stage u - kSB; with kSA >= kSB the phase of stage u - kSA has
+    // completed by then, so the parity they wait on names stage u alone.
+    static_assert(kSA >= kSB, "activation ring at least as deep as the weight ring");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
@@ -210,7 +217,7 @@ __device__ __forceinline__ bool wait_flag_gpu(const int *flag, volatile int *abo
         int v;
         asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
         if (v != 0) return true;
-        if (*abort_flag) return false;
+        if (abort_raised(abort_flag)) return false;
         if (clock64() - t0 > lim) {
             record_status(NF4_ERR_TIMEOUT);
             return false;
@@ -320,7 +327,7 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
                 tile_coords(sg.tile, m_pairs, args.n_tiles, mi, ni);
                 const int m0 = mi * (2 * kBM) + static_cast<int>(rank) * kBM;
                 for (int it = sg.k0; it < sg.k1; ++it) {
-                    if (!mbar_wait_cluster(&a_empty[sa], pa ^ 1, abort_flag)) goto done;
+                    if (!mbar_wait(&a_empty[sa], pa ^ 1, abort_flag)) goto done;
                     if (it >= args.main_steps && !la_ready) {
                         griddep_wait();
                         la_ready = true;
@@ -371,15 +378,15 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
         // ------------------------------------------------------------ MMA
         if (lane == 0 && rank == 0) {
             int sa = 0, sb = 0, ab = 0;
-            uint32_t pa = 0, pb = 0, aph = 0;
+            uint32_t pb = 0, aph = 0;
             const uint32_t a_base = smem_u32(slot_a), b_base = smem_u32(slot_b);
             for (bool more = sched.first(sg); more; more = sched.next(sg)) {
-                if (!mbar_wait_cluster(&acc_empty[ab], aph ^ 1, abort_flag)) goto done;
+                if (!mbar_wait(&acc_empty[ab], aph ^ 1, abort_flag)) goto done;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + ab * BN;
                 for (int it = sg.k0; it < sg.k1; ++it) {
-                    if (!mbar_wait_cluster(&a_full[sa], pa, abort_flag)) goto done;
-                    if (!mbar_wait_cluster(&b_full[sb], pb, abort_flag)) goto done;
+                    // b_full implies a_full (see the dequant role)
+                    if (!mbar_wait(&b_full[sb], pb, abort_flag)) goto done;
                     tc_fence_after();
                     const uint32_t a_addr = a_base + sa * Cfg::kABytes;
                     const uint32_t b_addr = b_base + sb * Cfg::kBBytes;
@@ -394,7 +401,7 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
                     umma_commit_pair(&a_empty[sa], 0x3);
                     umma_commit_pair(&b_empty[sb], 0x3);
                     ++cm;
-                    if (++sa == SA) { sa = 0; pa ^= 1; }
+                    if (++sa == SA) sa = 0;
                     if (++sb == SB) { sb = 0; pb ^= 1; }
                 }
                 umma_commit_pair(&acc_full[ab], 0x3);
@@ -423,7 +430,7 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
             const bool tail = sg.k0 > 0;
             const bool head = !tail && sg.k1 < nsteps;
             const int rloc = q * 32 + lane;               // row within this CTA's 128
-            if (!mbar_wait_cluster(&acc_full[ab], aph, abort_flag)) goto done;
+            if (!mbar_wait(&acc_full[ab], aph, abort_flag)) goto done;
             tc_fence_after();
             if (tail) {
                 float *pp = args.partial +
@@ -443,7 +450,7 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
                 tc_fence_before();
                 __syncwarp();                 // this warp's 32 rows of the partial are written
                 if (lane == 0) {
-                    mbar_arrive_cluster(empty0 + 8u * ab);
+                    mbar_arrive_remote(empty0 + 8u * ab);
                     __threadfence();
                     if (!g_dbg_skip_flag_set) set_flag_gpu(args.flags + (pair * 2 + rank) * 4 + q);
                 }
@@ -503,7 +510,7 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(empty0 + 8u * ab);
+                if (lane == 0) mbar_arrive_remote(empty0 + 8u * ab);
             }
             if (++ab == 2) { ab = 0; aph ^= 1; }
         }
@@ -620,7 +627,7 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
             // Each 8-code word becomes one 16-byte piece of the row and is stored
             // at once, so at most one piece is live in registers (no spills at
             // the 72 registers a thread has).
-            if (!mbar_wait_cluster(&b_empty[sb], pb ^ 1, abort_flag)) goto done;
+            if (!mbar_wait(&b_empty[sb], pb ^ 1, abort_flag)) goto done;
             uint8_t *brow = slot_b + sb * Cfg::kBBytes + row_off;
             auto put = [&](int c, uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
                 *reinterpret_cast<uint4 *>(brow + ((c ^ swz) << 4)) = make_uint4(w0, w1, w2, w3);
@@ -664,9 +671,13 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
                     put(c, v.x, v.y, v.z, v.w);
                 }
             }
+            // the even CTA vouches for the activation tile of this stage too
+            if (rank == 0 &&
+                !mbar_wait(&a_full[u % SA], static_cast<uint32_t>(u / SA) & 1u, abort_flag))
+                goto done;
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(full0 + 8u * sb);
+            if (lane == 0) mbar_arrive_remote(full0 + 8u * sb);
 
             sb += G;
             if (sb >= SB) { sb -= SB; pb ^= 1; }
