@@ -29,7 +29,10 @@
 //                        has completed, so the MMA issuer waits on b_full alone
 //                        (one barrier probe per stage on its critical path)
 //   acc_empty (even CTA) the epilogue warps of both CTAs arrive here
-//   a_empty, b_empty, acc_full (both CTAs)  one multicast tcgen05.commit
+//   consumed, acc_full (both CTAs)  one multicast tcgen05.commit; consumed[u mod
+//                        kConsumedBars] completes when the MMAs of stage u have, and
+//                        frees that stage's activation slot and weight slot alike:
+//                        one commit per stage on the MMA issuer's critical path
 // The code-tile ring is private to each CTA.
 //
 // Warp roles per CTA: 0..3 epilogue, 4 TMA activations, 5 TMEM owner and (even
@@ -43,6 +46,7 @@ namespace nf4 {
 
 constexpr int kBM = 128;            // tokens per CTA of a pair tile (MMA M = 2 kBM)
 constexpr int kBK = 64;             // reduction per stage = one 64-element NF4 step
+constexpr int kConsumedBars = 16;   // ring of stage-consumed barriers (a power of two)
 constexpr int kEpiWarp0 = 0;
 constexpr int kTmaAWarp = 4;
 constexpr int kMmaWarp = 5;
@@ -102,6 +106,15 @@ struct PairCfg {
     // still hold stage u - kSB; with kSA >= kSB the phase of stage u - kSA has
     // completed by then, so the parity they wait on names stage u alone.
     static_assert(kSA >= kSB, "activation ring at least as deep as the weight ring");
+    // A producer of stage u waits on consumed[(u - S) mod R] (S = kSA or kSB):
+    // that barrier's next phase needs stage u - S + R consumed, which needs
+    // stage u itself when R > S, and its previous phase (stage u - S - R) was
+    // waited for already when R >= G (the dequant group's previous stage).
+    static_assert(kConsumedBars > kSA && kConsumedBars > kSB && kConsumedBars >= G,
+                  "stage-consumed ring deeper than either operand ring");
+    // barriers, then the TMEM address, the abort flag and three progress counters
+    static_assert((kSA + kConsumedBars + 2 * kSC + kSB + 2 + 2 + 1) * 8 + 4 + 4 + 12 <= 512,
+                  "barrier area");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
@@ -247,12 +260,11 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
     uint8_t *slot_c = slot_b + SB * Cfg::kBBytes;        // [SC][kCBytes]
     uint64_t *bars = reinterpret_cast<uint64_t *>(slot_c + SC * Cfg::kCBytes);
     uint64_t *a_full = bars;                 // even CTA: both loads landed (1 + tx)
-    uint64_t *a_empty = a_full + SA;         // MMA done (pair commit)
-    uint64_t *c_full = a_empty + SA;         // code TMA landed (1 + tx) or LoRA stage (1)
+    uint64_t *consumed = a_full + SA;        // [kConsumedBars] MMAs of a stage done (pair commit)
+    uint64_t *c_full = consumed + kConsumedBars;   // code TMA landed (1 + tx) or LoRA stage (1)
     uint64_t *c_empty = c_full + SC;         // codes read (one dequant group of this CTA)
     uint64_t *b_full = c_empty + SC;         // even CTA: halves written (groups of both CTAs)
-    uint64_t *b_empty = b_full + SB;         // MMA done (pair commit)
-    uint64_t *acc_full = b_empty + SB;       // [2] accumulator complete (pair commit)
+    uint64_t *acc_full = b_full + SB;        // [2] accumulator complete (pair commit)
     uint64_t *acc_empty = acc_full + 2;      // [2] even CTA: drained (epilogue warps of both)
     uint64_t *mma_drain = acc_empty + 2;     // even CTA: the MMAs issued before giving up completed
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_drain + 1);
@@ -267,17 +279,14 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
     const int npairs = static_cast<int>(cluster_count_x());
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < SA; ++s) {
-            mbar_init(&a_full[s], 1);
-            mbar_init(&a_empty[s], 1);
-        }
+        for (int s = 0; s < SA; ++s) mbar_init(&a_full[s], 1);
+        for (int s = 0; s < kConsumedBars; ++s) mbar_init(&consumed[s], 1);
         for (int s = 0; s < SC; ++s) {
             mbar_init(&c_full[s], 1);
             mbar_init(&c_empty[s], Cfg::kGroupWarps);
         }
         for (int s = 0; s < SB; ++s) {
             mbar_init(&b_full[s], 2 * Cfg::kGroupWarps);
-            mbar_init(&b_empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
@@ -320,14 +329,18 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
         if (lane == 0) {
             const uint32_t full0 = mapa_shared(smem_u32(a_full), 0);
             int sa = 0;
-            uint32_t pa = 0;
             bool la_ready = false;     // the rank-r activations are written by the kernel before
             for (bool more = sched.first(sg); more; more = sched.next(sg)) {
                 int mi, ni;
                 tile_coords(sg.tile, m_pairs, args.n_tiles, mi, ni);
                 const int m0 = mi * (2 * kBM) + static_cast<int>(rank) * kBM;
                 for (int it = sg.k0; it < sg.k1; ++it) {
-                    if (!mbar_wait(&a_empty[sa], pa ^ 1, abort_flag)) goto done;
+                    if (na >= SA) {               // the slot's previous stage, na - SA, consumed
+                        const int v = na - SA;
+                        if (!mbar_wait(&consumed[v & (kConsumedBars - 1)],
+                                       static_cast<uint32_t>(v / kConsumedBars) & 1u, abort_flag))
+                            goto done;
+                    }
                     if (it >= args.main_steps && !la_ready) {
                         griddep_wait();
                         la_ready = true;
@@ -340,7 +353,7 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
                         tma_load_2d_pair(slot_a + sa * Cfg::kABytes, &tm_la, full0 + 8u * sa,
                                          (it - args.main_steps) * kBK, m0);
                     ++na;
-                    if (++sa == SA) { sa = 0; pa ^= 1; }
+                    if (++sa == SA) sa = 0;
                 }
             }
         }
@@ -398,8 +411,7 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
                         umma_bf16_ss_pair(d_tmem, ad, bd, Cfg::kIdesc,
                                           (it > sg.k0 || kk > 0) ? 1u : 0u);
                     }
-                    umma_commit_pair(&a_empty[sa], 0x3);
-                    umma_commit_pair(&b_empty[sb], 0x3);
+                    umma_commit_pair(&consumed[cm & (kConsumedBars - 1)], 0x3);
                     ++cm;
                     if (++sa == SA) sa = 0;
                     if (++sb == SB) { sb = 0; pb ^= 1; }
@@ -605,7 +617,7 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
         // so that no load is outstanding across a proxy fence.
         RawScale cs = load_scale(u < nunits ? block_of(cur) : -1);
         int sb = grp, sc = grp;
-        uint32_t pb = 0, pc = 0;
+        uint32_t pc = 0;
         while (u < nunits) {
             const bool main = cur.it < args.main_steps;
 
@@ -627,7 +639,12 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
             // Each 8-code word becomes one 16-byte piece of the row and is stored
             // at once, so at most one piece is live in registers (no spills at
             // the 72 registers a thread has).
-            if (!mbar_wait(&b_empty[sb], pb ^ 1, abort_flag)) goto done;
+            if (u >= SB) {                    // the slot's previous stage, u - SB, consumed
+                const int v = u - SB;
+                if (!mbar_wait(&consumed[v & (kConsumedBars - 1)],
+                               static_cast<uint32_t>(v / kConsumedBars) & 1u, abort_flag))
+                    goto done;
+            }
             uint8_t *brow = slot_b + sb * Cfg::kBBytes + row_off;
             auto put = [&](int c, uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
                 *reinterpret_cast<uint4 *>(brow + ((c ^ swz) << 4)) = make_uint4(w0, w1, w2, w3);
@@ -680,7 +697,7 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
             if (lane == 0) mbar_arrive_remote(full0 + 8u * sb);
 
             sb += G;
-            if (sb >= SB) { sb -= SB; pb ^= 1; }
+            if (sb >= SB) sb -= SB;
             sc += G;
             if (sc >= SC) { sc -= SC; pc ^= 1; }
             if (u + G < nunits) {
