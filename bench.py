@@ -509,40 +509,75 @@ def attn_leg(q, dev, peaks, warmup=3, steps=50):
 def e2e_leg(q, dp, run, args, dev, world):
     """Same metric through the public API with host buffers: every step copies
     x and dY in from pinned host memory and h, dX and the fp32 adapter
-    gradients back out (the frozen weight and the adapters stay resident)."""
+    gradients back out (the frozen weight and the adapters stay resident).
+    The copies run as a training input pipeline would: two sets of device
+    buffers, step i + 1's inputs copied in on one copy stream while step i
+    computes, step i's outputs copied out on another (the other direction of
+    the host link). Every step's copies are inside the timed region."""
     w = run.w
     M, N, K, r, alpha = w.M, w.N, w.K, w.r, w.alpha
     hx = run.inp["x"].pin_memory()
     hdY = run.inp["dY"].pin_memory()
-    oh = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
-    odX = torch.empty(M, K, dtype=torch.bfloat16).pin_memory()
-    ograd = torch.empty(r * K + N * r, dtype=torch.float32).pin_memory()
+    oh = [torch.empty(M, N, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    odX = [torch.empty(M, K, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    ograd = [torch.empty(r * K + N * r, dtype=torch.float32).pin_memory() for _ in range(2)]
     qw, A, B = run.qw, run.A, run.B
-    x = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
-    dY = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-    flat, dA, dB = dp.grad_buffer(r, K, N, device=dev)
+    xs = [torch.empty(M, K, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    dYs = [torch.empty(M, N, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    hs = [torch.empty(M, N, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    dXs = [torch.empty(M, K, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    grads = [dp.grad_buffer(r, K, N, device=dev) for _ in range(2)]
+    main = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]     # set k's inputs landed
+    ev_used = [torch.cuda.Event() for _ in range(2)]   # the step on set k has computed
+    ev_out = [torch.cuda.Event() for _ in range(2)]    # set k's outputs copied out
+    for k in range(2):
+        ev_used[k].record(main)
+        ev_out[k].record(main)
 
-    def step():
-        x.copy_(hx, non_blocking=True)
-        dY.copy_(hdY, non_blocking=True)
-        h, u = q.qlora_linear_fwd(qw, x, A, B, alpha)
-        dX, _, _ = q.qlora_linear_bwd(qw, x, A, B, alpha, dY, u=u, outs=(torch.empty_like(x), dA, dB))
+    def copy_in(i):
+        k = i % 2
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev_used[k])                # the step two back is done with set k
+            xs[k].copy_(hx, non_blocking=True)
+            dYs[k].copy_(hdY, non_blocking=True)
+            ev_in[k].record(s_in)
+
+    def compute(i):
+        k = i % 2
+        main.wait_event(ev_in[k])
+        main.wait_event(ev_out[k])                     # set k's previous outputs are out
+        flat, dA, dB = grads[k]
+        _, u = q.qlora_linear_fwd(qw, xs[k], A, B, alpha, h=hs[k])
+        q.qlora_linear_bwd(qw, xs[k], A, B, alpha, dYs[k], u=u, outs=(dXs[k], dA, dB))
         dp.allreduce_adapter_grads(flat, world)
-        oh.copy_(h, non_blocking=True)
-        odX.copy_(dX, non_blocking=True)
-        ograd.copy_(flat, non_blocking=True)
+        ev_used[k].record(main)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_used[k])
+            oh[k].copy_(hs[k], non_blocking=True)
+            odX[k].copy_(dXs[k], non_blocking=True)
+            ograd[k].copy_(flat, non_blocking=True)
+            ev_out[k].record(s_out)
+
+    def run_steps(n):
+        copy_in(0)
+        for i in range(n):
+            if i + 1 < n:
+                copy_in(i + 1)
+            compute(i)
+        main.wait_stream(s_out)
 
     steps = max(5, min(args.steps, 20))
-    for _ in range(3):
-        step()
+    run_steps(3)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record()
-    for _ in range(steps):
-        step()
-    e.record()
+    s.record(main)
+    s_in.wait_stream(main)
+    run_steps(steps)
+    e.record(main)
     torch.cuda.synchronize()
     ms = s.elapsed_time(e) / steps
     if world > 1:
@@ -550,11 +585,11 @@ def e2e_leg(q, dp, run, args, dev, world):
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms = float(t.item())
     f, b = layer_flops(M, N, K, r)
-    del x, dY, flat, dA, dB
+    nbytes_in, nbytes_out = hx.nbytes + hdY.nbytes, oh[0].nbytes + odX[0].nbytes + ograd[0].nbytes
+    del xs, dYs, hs, dXs, grads
     torch.cuda.empty_cache()
     return {"value": world * (f + b) / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-            "ms_per_step": ms, "h2d_bytes_per_step": hx.nbytes + hdY.nbytes,
-            "d2h_bytes_per_step": oh.nbytes + odX.nbytes + ograd.nbytes}
+            "ms_per_step": ms, "h2d_bytes_per_step": nbytes_in, "d2h_bytes_per_step": nbytes_out}
 
 
 def decode_leg(q, dev, peaks, block=64, tokens=(1, 4, 16)):
