@@ -11,12 +11,14 @@
 // multiply-add with w~ and one rounding to the output type (bf16 for the
 // 16-bit merged model, fp32 for re-quantisation with nf4_quantize).
 //
-// One CTA writes a 64-row x 128-column tile of out. Warp w takes rows
-// [16 (w % 4), +16) and the 64 columns (one NF4 block per row)
-// [64 (w / 4), +64) of the tile. The tile's rows of B, its columns of A
-// (stored transposed, so that each MMA's B fragment is one 32-bit word) and
-// its 4-bit codes are staged in shared memory; each warp's results go through
-// a padded shared buffer so that every row leaves as 16-byte stores.
+// A CTA owns one 128-column stripe of out and walks its 64-row tiles (every
+// gridDim.y-th): the stripe's columns of A (stored transposed, so that each
+// MMA's B fragment is one 32-bit word) are staged once, and the next tile's
+// rows of B and 4-bit codes arrive by cp.async while the current tile is
+// computed (two buffers). Warp w takes rows [16 (w % 4), +16) and the 64
+// columns (one NF4 block per row) [64 (w / 4), +64) of a tile; each warp's
+// results go through a padded shared buffer so that every row leaves as
+// 16-byte stores.
 #pragma once
 
 #include "nf4_common.cuh"
@@ -47,42 +49,53 @@ struct MergeArgs {
 // Shared-memory layout of one CTA (bytes), for padded rank rp.
 __host__ __device__ constexpr int merge_bs_stride(int rp) { return rp + 8; }    // bf16 per B row
 __host__ __device__ inline int merge_smem_bytes(int rp, bool out_bf16) {
-    return kMgRows * merge_bs_stride(rp) * 2          // B rows
-           + kMgCols * merge_bs_stride(rp) * 2        // A columns (transposed)
-           + kMgRows * kMgCodeStride                  // codes
+    return kMgCols * merge_bs_stride(rp) * 2          // A columns (transposed)
+           + 2 * kMgRows * merge_bs_stride(rp) * 2    // B rows, two buffers
+           + 2 * kMgRows * kMgCodeStride              // codes, two buffers
            + 16 * 4                                   // levels
            + 8 * 16 * (out_bf16 ? (64 + 8) * 2 : (64 + 4) * 4);   // per-warp output staging
 }
-
 // RQ = padded rank / 16 (1..8), a compile-time constant so that the rank
 // loops unroll without guards.
 template <bool OUT_BF16, int RQ>
 __global__ void __launch_bounds__(kMgThreads, 4) qlora_merge_kernel(const MergeArgs a) {
     extern __shared__ __align__(16) uint8_t msm[];
     constexpr int rs = merge_bs_stride(16 * RQ);
-    uint16_t *Bs = reinterpret_cast<uint16_t *>(msm);                       // [64][rs]
-    uint16_t *Ats = Bs + kMgRows * rs;                                      // [128][rs]
-    uint8_t *cs = reinterpret_cast<uint8_t *>(Ats + kMgCols * rs);          // [64][kMgCodeStride]
-    float *lv = reinterpret_cast<float *>(cs + kMgRows * kMgCodeStride);    // [16]
+    uint16_t *Ats = reinterpret_cast<uint16_t *>(msm);                      // [128][rs]
+    uint16_t *Bs2 = Ats + kMgCols * rs;                                     // [2][64][rs]
+    uint8_t *cs2 = reinterpret_cast<uint8_t *>(Bs2 + 2 * kMgRows * rs);     // [2][64][kMgCodeStride]
+    float *lv = reinterpret_cast<float *>(cs2 + 2 * kMgRows * kMgCodeStride);    // [16]
     uint8_t *stage = reinterpret_cast<uint8_t *>(lv + 16);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
-    const int64_t n0 = static_cast<int64_t>(blockIdx.y) * kMgRows;
     const int64_t k0 = static_cast<int64_t>(blockIdx.x) * kMgCols;
+    const int row_tiles = static_cast<int>((a.N + kMgRows - 1) / kMgRows);
 
     griddep_wait();
     griddep_launch_dependents();
 
+    // tile rt's rows of B (zero beyond N and r) and codes into buffer buf
+    auto prefetch = [&](int rt, int buf) {
+        const int64_t n0 = static_cast<int64_t>(rt) * kMgRows;
+        uint16_t *Bs = Bs2 + buf * kMgRows * rs;
+        for (int idx = tid; idx < kMgRows * (a.rp / 8); idx += kMgThreads) {
+            const int row = idx / (a.rp / 8), ch = idx % (a.rp / 8);
+            const bool ok = n0 + row < a.N && ch * 8 < a.r;
+            cp_async16(Bs + row * rs + ch * 8, ok ? a.B + (n0 + row) * a.r + ch * 8 : a.B, ok);
+        }
+        {
+            const int row = tid >> 2, ch = tid & 3;
+            const bool ok = n0 + row < a.N && k0 + ch * 32 < a.K;
+            cp_async16(cs2 + buf * kMgRows * kMgCodeStride + row * kMgCodeStride + ch * 16,
+                       ok ? a.codes + (n0 + row) * (a.K / 2) + k0 / 2 + ch * 16 : a.codes, ok);
+        }
+        cp_async_commit();
+    };
+    int rt = static_cast<int>(blockIdx.y);
+    if (rt < row_tiles) prefetch(rt, 0);
+
     if (tid < 16) lv[tid] = c_levels[tid];
-    // B rows n0..n0+63, zero beyond N and beyond r (8 bf16 per 16-byte chunk)
-    for (int idx = tid; idx < kMgRows * (a.rp / 8); idx += kMgThreads) {
-        const int row = idx / (a.rp / 8), ch = idx % (a.rp / 8);
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (n0 + row < a.N && ch * 8 < a.r)
-            v = __ldg(reinterpret_cast<const uint4 *>(a.B + (n0 + row) * a.r) + ch);
-        *reinterpret_cast<uint4 *>(Bs + row * rs + ch * 8) = v;
-    }
     // A columns k0..k0+127 as rows of Ats (Ats[c][j] = A[j][k0 + c]), zero beyond K and r;
     // consecutive threads take consecutive j, so each 16-bit store of a warp
     // lands on consecutive addresses
@@ -96,89 +109,94 @@ __global__ void __launch_bounds__(kMgThreads, 4) qlora_merge_kernel(const MergeA
         for (int e = 0; e < 8; ++e)
             Ats[(ch * 8 + e) * rs + j] = static_cast<uint16_t>(w[e >> 1] >> (16 * (e & 1)));
     }
-    // codes of the tile: 64 rows x 64 bytes
-    {
-        const int row = tid >> 2, ch = tid & 3;
-        uint4 v = make_uint4(0x77777777u, 0x77777777u, 0x77777777u, 0x77777777u);
-        if (n0 + row < a.N && k0 + ch * 32 < a.K)
-            v = __ldg(reinterpret_cast<const uint4 *>(a.codes + (n0 + row) * (a.K / 2) + k0 / 2) + ch);
-        *reinterpret_cast<uint4 *>(cs + row * kMgCodeStride + ch * 16) = v;
-    }
-    __syncthreads();
 
     const int rw = 16 * (warp & 3);          // first tile row of this warp
     const int cw = 64 * (warp >> 2);         // first tile column of this warp
     const bool cols_ok = k0 + cw < a.K;      // K is a multiple of 64: a warp's block is all in or all out
-
-    // block scales of rows rw + g and rw + g + 8 (a warp's 64 columns lie in one block)
-    float sc[2] = {0.0f, 0.0f};
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int64_t n = n0 + rw + g + 8 * h;
-        if (n < a.N && cols_ok) {
-            const int64_t b = n * (a.K / a.block) + (k0 + cw) / a.block;
-            sc[h] = a.dq ? __fmul_rn(static_cast<float>(__ldg(a.q8 + b)), __fdiv_rn(__ldg(a.cg + (b >> 8)), 127.0f))
-                         : __ldg(a.absmax + b);
-        }
-    }
-
-    // rows rw + g, rw + g + 8 of B as MMA A fragments, one set per 16 ranks
-    uint32_t af[RQ][4];
-#pragma unroll
-    for (int q = 0; q < RQ; ++q) {
-        const int ks = 16 * q;
-        af[q][0] = *reinterpret_cast<const uint32_t *>(Bs + (rw + g) * rs + ks + 2 * t);
-        af[q][1] = *reinterpret_cast<const uint32_t *>(Bs + (rw + g + 8) * rs + ks + 2 * t);
-        af[q][2] = *reinterpret_cast<const uint32_t *>(Bs + (rw + g) * rs + ks + 2 * t + 8);
-        af[q][3] = *reinterpret_cast<const uint32_t *>(Bs + (rw + g + 8) * rs + ks + 2 * t + 8);
-    }
-
-    // per 8-column tile i: the rank-r product, then out = fma(s, BA, w~) for
-    // elements (row, 8 i + 2 t) and (row, 8 i + 2 t + 1), rows g and g + 8
     uint8_t *st = stage + warp * 16 * (OUT_BF16 ? (64 + 8) * 2 : (64 + 4) * 4);
-    const uint8_t *crow0 = cs + (rw + g) * kMgCodeStride + cw / 2;
-    const uint8_t *crow1 = crow0 + 8 * kMgCodeStride;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        const uint16_t *bc = Ats + (cw + 8 * i + g) * rs + 2 * t;
-#pragma unroll
-        for (int q = 0; q < RQ; ++q)
-            mma_bf16_16816(acc, af[q], *reinterpret_cast<const uint32_t *>(bc + 16 * q),
-                           *reinterpret_cast<const uint32_t *>(bc + 16 * q + 8));
+
+    for (int buf = 0; rt < row_tiles; rt += static_cast<int>(gridDim.y), buf ^= 1) {
+        // this tile's rows of B and codes have landed (the only copies in
+        // flight), and every warp is done with the previous tile and its
+        // buffer, which takes the next tile now
+        cp_async_wait_all();
+        __syncthreads();
+        if (rt + static_cast<int>(gridDim.y) < row_tiles) prefetch(rt + static_cast<int>(gridDim.y), buf ^ 1);
+        const int64_t n0 = static_cast<int64_t>(rt) * kMgRows;
+        const uint16_t *Bs = Bs2 + buf * kMgRows * rs;
+        const uint8_t *cs = cs2 + buf * kMgRows * kMgCodeStride;
+
+        // block scales of rows rw + g and rw + g + 8 (a warp's 64 columns lie in one block)
+        float sc[2] = {0.0f, 0.0f};
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            const uint32_t byte = (h ? crow1 : crow0)[4 * i + t];
-            const float w0 = __fmul_rn(sc[h], lv[byte >> 4]);
-            const float w1 = __fmul_rn(sc[h], lv[byte & 15u]);
-            const float o0 = fmaf(a.scale, acc[2 * h], w0);
-            const float o1 = fmaf(a.scale, acc[2 * h + 1], w1);
-            const int rl = g + 8 * h, cl = 8 * i + 2 * t;
-            if (OUT_BF16) {
-                __nv_bfloat162 p = __floats2bfloat162_rn(o0, o1);
-                *reinterpret_cast<__nv_bfloat162 *>(st + (rl * (64 + 8) + cl) * 2) = p;
-            } else {
-                *reinterpret_cast<float2 *>(st + (rl * (64 + 4) + cl) * 4) = make_float2(o0, o1);
+            const int64_t n = n0 + rw + g + 8 * h;
+            if (n < a.N && cols_ok) {
+                const int64_t b = n * (a.K / a.block) + (k0 + cw) / a.block;
+                sc[h] = a.dq ? __fmul_rn(static_cast<float>(__ldg(a.q8 + b)), __fdiv_rn(__ldg(a.cg + (b >> 8)), 127.0f))
+                             : __ldg(a.absmax + b);
             }
         }
-    }
-    __syncwarp();
-    if (!cols_ok) return;
-    // 16 rows of 64 outputs leave as 16-byte stores, consecutive lanes along a row
-    constexpr int kChunksPerRow = OUT_BF16 ? 8 : 16;
+
+        // rows rw + g, rw + g + 8 of B as MMA A fragments, one set per 16 ranks
+        uint32_t af[RQ][4];
 #pragma unroll
-    for (int c = lane; c < 16 * kChunksPerRow; c += 32) {
-        const int rl = c / kChunksPerRow, ch = c % kChunksPerRow;
-        const int64_t n = n0 + rw + rl;
-        if (n >= a.N) continue;
-        const int64_t col = k0 + cw + ch * (OUT_BF16 ? 8 : 4);
-        if (OUT_BF16) {
-            const uint4 v = *reinterpret_cast<const uint4 *>(st + (rl * (64 + 8) + ch * 8) * 2);
-            *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(a.out) + n * a.K + col) = v;
-        } else {
-            const uint4 v = *reinterpret_cast<const uint4 *>(st + (rl * (64 + 4) + ch * 4) * 4);
-            *reinterpret_cast<uint4 *>(static_cast<float *>(a.out) + n * a.K + col) = v;
+        for (int q = 0; q < RQ; ++q) {
+            const int ks = 16 * q;
+            af[q][0] = *reinterpret_cast<const uint32_t *>(Bs + (rw + g) * rs + ks + 2 * t);
+            af[q][1] = *reinterpret_cast<const uint32_t *>(Bs + (rw + g + 8) * rs + ks + 2 * t);
+            af[q][2] = *reinterpret_cast<const uint32_t *>(Bs + (rw + g) * rs + ks + 2 * t + 8);
+            af[q][3] = *reinterpret_cast<const uint32_t *>(Bs + (rw + g + 8) * rs + ks + 2 * t + 8);
         }
+
+        // per 8-column tile i: the rank-r product, then out = fma(s, BA, w~) for
+        // elements (row, 8 i + 2 t) and (row, 8 i + 2 t + 1), rows g and g + 8
+        const uint8_t *crow0 = cs + (rw + g) * kMgCodeStride + cw / 2;
+        const uint8_t *crow1 = crow0 + 8 * kMgCodeStride;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            const uint16_t *bc = Ats + (cw + 8 * i + g) * rs + 2 * t;
+#pragma unroll
+            for (int q = 0; q < RQ; ++q)
+                mma_bf16_16816(acc, af[q], *reinterpret_cast<const uint32_t *>(bc + 16 * q),
+                               *reinterpret_cast<const uint32_t *>(bc + 16 * q + 8));
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t byte = (h ? crow1 : crow0)[4 * i + t];
+                const float w0 = __fmul_rn(sc[h], lv[byte >> 4]);
+                const float w1 = __fmul_rn(sc[h], lv[byte & 15u]);
+                const float o0 = fmaf(a.scale, acc[2 * h], w0);
+                const float o1 = fmaf(a.scale, acc[2 * h + 1], w1);
+                const int rl = g + 8 * h, cl = 8 * i + 2 * t;
+                if (OUT_BF16) {
+                    __nv_bfloat162 p = __floats2bfloat162_rn(o0, o1);
+                    *reinterpret_cast<__nv_bfloat162 *>(st + (rl * (64 + 8) + cl) * 2) = p;
+                } else {
+                    *reinterpret_cast<float2 *>(st + (rl * (64 + 4) + cl) * 4) = make_float2(o0, o1);
+                }
+            }
+        }
+        __syncwarp();
+        if (cols_ok) {
+            // 16 rows of 64 outputs leave as 16-byte stores, consecutive lanes along a row
+            constexpr int kChunksPerRow = OUT_BF16 ? 8 : 16;
+#pragma unroll
+            for (int c = lane; c < 16 * kChunksPerRow; c += 32) {
+                const int rl = c / kChunksPerRow, ch = c % kChunksPerRow;
+                const int64_t n = n0 + rw + rl;
+                if (n >= a.N) continue;
+                const int64_t col = k0 + cw + ch * (OUT_BF16 ? 8 : 4);
+                if (OUT_BF16) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(st + (rl * (64 + 8) + ch * 8) * 2);
+                    *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(a.out) + n * a.K + col) = v;
+                } else {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(st + (rl * (64 + 4) + ch * 4) * 4);
+                    *reinterpret_cast<uint4 *>(static_cast<float *>(a.out) + n * a.K + col) = v;
+                }
+            }
+        }
+        __syncwarp();            // the staging buffer is read before the next tile writes it
     }
 }
 

@@ -889,8 +889,6 @@ nf4_status qlora_merge(const nf4_weight *w, const uint16_t *A, const uint16_t *B
     a.scale = alpha / static_cast<float>(r);
     a.out = out;
     a.block = w->block_size;
-    const dim3 grid(static_cast<unsigned>((w->k + kMgCols - 1) / kMgCols),
-                    static_cast<unsigned>((w->n + kMgRows - 1) / kMgRows));
     const int smem = merge_smem_bytes(a.rp, out_is_bf16 != 0);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     void (*kern)(const MergeArgs) = nullptr;
@@ -905,6 +903,14 @@ nf4_status qlora_merge(const nf4_weight *w, const uint16_t *A, const uint16_t *B
     }
 #undef NF4_MERGE_CASE
     NF4_TRY_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    // one wave: the column stripes times enough CTAs per stripe to fill the
+    // resident CTA slots, each walking every gy-th row tile of its stripe
+    int per_sm = 0;
+    NF4_TRY_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kMgThreads, static_cast<size_t>(smem)));
+    const int64_t gx = (w->k + kMgCols - 1) / kMgCols, row_tiles = (w->n + kMgRows - 1) / kMgRows;
+    const int64_t slots = static_cast<int64_t>(std::max(1, per_sm)) * num_sms(current_device());
+    const int64_t gy = std::max<int64_t>(1, std::min<int64_t>(row_tiles, slots / gx));
+    const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
     LaunchTimer t(KK_MERGE, s);
     const cudaError_t e = launch_ex(kern, grid, dim3(kMgThreads), static_cast<size_t>(smem), s, 0u, a);
     t.stop();
