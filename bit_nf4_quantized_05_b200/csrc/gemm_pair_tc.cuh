@@ -482,6 +482,14 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
 #pragma unroll 1
                 for (int c2 = 0; c2 < 2 * kChunks; ++c2) {      // 16 columns at a time
                     const int c = c2 >> 1;
+                    // the partial's 16 values are requested before the tensor-memory
+                    // load and its wait, so that the two latencies overlap
+                    float4 pv4[4] = {};
+                    if (add_partial) {
+                        const float4 *pv = reinterpret_cast<const float4 *>(pp + c * (128 * 32) + (c2 & 1) * 16);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) pv4[i] = pv[i];
+                    }
                     uint32_t v[16];
                     tmem_ld_32x32b_x16(tmem_base + ((q * 32) << 16) + ab * BN + c2 * 16, v);
                     tmem_ld_wait();
@@ -495,9 +503,7 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
 #pragma unroll
                                 for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[gg * 8 + e]);
                                 if (add_partial) {
-                                    const float4 *pv = reinterpret_cast<const float4 *>(
-                                        pp + c * (128 * 32) + g * 8);
-                                    const float4 p0 = pv[0], p1 = pv[1];
+                                    const float4 p0 = pv4[2 * gg], p1 = pv4[2 * gg + 1];
                                     f[0] += p0.x; f[1] += p0.y; f[2] += p0.z; f[3] += p0.w;
                                     f[4] += p1.x; f[5] += p1.y; f[6] += p1.z; f[7] += p1.w;
                                 }
