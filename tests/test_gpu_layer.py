@@ -262,6 +262,10 @@ MERGE_SHAPES = [
     (64, 128, 8, 16.0, False),
     (136, 576, 64, 16.0, True),
     (72, 192, 128, 32.0, False),
+    # 64 column stripes leave ~9 CTAs per stripe for 16 row tiles (the last one 40 rows): CTAs walk
+    # several tiles with the next tile's operands in flight, and end on a ragged tile
+    (1000, 8192, 16, 32.0, True),
+    (1000, 8192, 64, 16.0, False),
 ]
 
 
