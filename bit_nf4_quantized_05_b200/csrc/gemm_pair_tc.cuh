@@ -389,17 +389,19 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA
-        if (lane == 0 && rank == 0) {
+        // The whole warp walks the schedule and waits; the elected lane
+        // issues every MMA and commit (so its commits track all of them).
+        if (rank == 0) {
             int sa = 0, sb = 0, ab = 0;
             uint32_t pb = 0, aph = 0;
             const uint32_t a_base = smem_u32(slot_a), b_base = smem_u32(slot_b);
             for (bool more = sched.first(sg); more; more = sched.next(sg)) {
-                if (!mbar_wait(&acc_empty[ab], aph ^ 1, abort_flag)) goto done;
+                if (!mbar_wait_warp(&acc_empty[ab], aph ^ 1, abort_flag)) goto done;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + ab * BN;
                 for (int it = sg.k0; it < sg.k1; ++it) {
                     // b_full implies a_full (see the dequant role)
-                    if (!mbar_wait(&b_full[sb], pb, abort_flag)) goto done;
+                    if (!mbar_wait_warp(&b_full[sb], pb, abort_flag)) goto done;
                     tc_fence_after();
                     const uint32_t a_addr = a_base + sa * Cfg::kABytes;
                     const uint32_t b_addr = b_base + sb * Cfg::kBBytes;
@@ -408,15 +410,15 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,    // [M, red
                         const uint64_t ad = smem_desc_sw128(a_addr + kk * 32, 16, 1024);
                         const uint64_t bd = DGRAD ? smem_desc_sw128(b_addr + kk * 2048, 8192, 1024)
                                                   : smem_desc_sw128(b_addr + kk * 32, 16, 1024);
-                        umma_bf16_ss_pair(d_tmem, ad, bd, Cfg::kIdesc,
-                                          (it > sg.k0 || kk > 0) ? 1u : 0u);
+                        umma_bf16_ss_pair_warp(d_tmem, ad, bd, Cfg::kIdesc,
+                                               (it > sg.k0 || kk > 0) ? 1u : 0u);
                     }
-                    umma_commit_pair(&consumed[cm & (kConsumedBars - 1)], 0x3);
+                    umma_commit_pair_warp(&consumed[cm & (kConsumedBars - 1)], 0x3);
                     ++cm;
                     if (++sa == SA) sa = 0;
                     if (++sb == SB) { sb = 0; pb ^= 1; }
                 }
-                umma_commit_pair(&acc_full[ab], 0x3);
+                umma_commit_pair_warp(&acc_full[ab], 0x3);
                 if (++ab == 2) { ab = 0; aph ^= 1; }
             }
         }
@@ -721,13 +723,16 @@ done:
         const uint32_t peer = mapa_shared(smem_u32(const_cast<int *>(abort_flag)), rank ^ 1u);
         asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(peer), "r"(1) : "memory");
     }
-    if (lane == 0 && warp == kMmaWarp && rank == 0) {
-        if (*abort_flag) {
+    if (warp == kMmaWarp && rank == 0) {
+        // the warp left its loop together (its waits vote), so it is converged
+        // and elect.sync picks the lane that issued the MMAs
+        __syncwarp();
+        if (__any_sync(0xffffffffu, *abort_flag != 0)) {
             // the MMAs already issued complete before the operands are released
-            umma_commit_pair(mma_drain, 0x1);
-            mbar_drain(mma_drain, 0);
+            umma_commit_pair_warp(mma_drain, 0x1);
+            if (lane == 0) mbar_drain(mma_drain, 0);
         }
-        progress[2] = cm;
+        if (lane == 0) progress[2] = cm;
     }
     if (lane == 0 && warp == kTmaAWarp) {
         // activation stages issued by this CTA, kept in the even CTA

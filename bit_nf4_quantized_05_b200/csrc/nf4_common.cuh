@@ -117,6 +117,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
+// mbar_wait by every lane of a converged warp; the lanes agree on the outcome
+// (any lane that gave up makes the whole warp give up), so the warp stays
+// converged on both paths.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag)) != 0;
+}
+
 // Bounded wait that ignores the abort flag: used on the way out of a kernel
 // that gave up, so that the copies (or tensor-core operations) it has already
 // issued land before its shared memory and tensor memory are released.
@@ -295,12 +302,38 @@ __device__ __forceinline__ void umma_bf16_ss_pair(uint32_t d_tmem, uint64_t ades
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// The same MMA executed by a whole converged warp with warp-uniform operands
+// and issued by the lane that elect.sync picks (the same lane every time the
+// full warp executes it). A lone thread issuing from divergent code is slowed
+// by the other warps sharing its scheduler; the converged, elected form keeps
+// the tensor pipe fed under that load.
+__device__ __forceinline__ void umma_bf16_ss_pair_warp(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                       uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
 // Arrive once on the mbarrier at this offset in each CTA of `mask` when the
 // pair MMAs issued so far by this thread have completed.
 __device__ __forceinline__ void umma_commit_pair(uint64_t *bar, uint16_t mask) {
     asm volatile(
         "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
         " [%0], %1;" ::"r"(smem_u32(bar)),
+        "h"(mask)
+        : "memory");
+}
+// umma_commit_pair executed by a converged warp: the elected lane (the one
+// that issued the warp's MMAs) commits.
+__device__ __forceinline__ void umma_commit_pair_warp(uint64_t *bar, uint16_t mask) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;\n\t}" ::"r"(smem_u32(bar)),
         "h"(mask)
         : "memory");
 }
